@@ -1,0 +1,28 @@
+"""CPU oracle for the W8A8 ConvRot expert-choice MoE block.
+
+This package is TEST INFRASTRUCTURE. Only the test suite, the smoke check in
+``__graft_entry__`` and the ``cpu_baseline`` / ``--impl reference`` legs of
+``bench.py`` may import it. The product path (the CUDA library and its Python
+binding) never imports, links or executes anything in here, and nothing in
+here imports the product package.
+
+Everything is plain NumPy: fp64 for the rotation, exact integer GEMMs, and
+fp32 only where the method's definition is fp32 (the scales, the dequantised
+outputs, SwiGLU, the router-weighted combine).
+"""
+
+from .convrot_oracle import (  # noqa: F401
+    bf16_round,
+    block_rotate,
+    dequant,
+    expert_choice_topc,
+    hadamard,
+    int_gemm,
+    moe_block,
+    quantize_rows,
+    rotation_matrix,
+    rotquant,
+    router_softmax,
+    silu_f32,
+    w8a8_linear,
+)

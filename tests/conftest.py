@@ -1,0 +1,24 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
+    config.addinivalue_line("markers", "slow: full-size cases (minutes)")
+
+
+def to_np(t):
+    """bf16/float CPU tensor -> float32 NumPy array (exact for bf16)."""
+    return t.float().numpy()
+
+
+@pytest.fixture
+def rng():
+    import numpy as np
+    return np.random.default_rng(1234)
