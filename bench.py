@@ -1,0 +1,431 @@
+"""Benchmark of the W8A8 ConvRot expert-choice MoE block on B200.
+
+One step = one pass of the whole hot path (router softmax, activation
+rotate+quantise, expert-choice top-C, gather, gate/up GEMM + SwiGLU, h
+rotate+requantise, down GEMM + router-weighted scatter, bf16 store) over one
+batch of synthetic tokens, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config moe_T8192]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+Multi-GPU (launched by torch.distributed.run): every rank runs its own batch
+of T tokens against the same weights (weak scaling, no data-path
+collective); the barrier and the max-over-ranks timing use the process group.
+`--impl reference` times the CPU oracle (the only reference there is) on a
+bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synthetic import MOE_CONFIGS, moe_inputs  # noqa: E402
+
+METRIC = "W8A8 ConvRot MoE block tokens/s"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def algorithmic_work(cfg, t):
+    """Ops and compulsory bytes of one block call and of its two GEMM launches."""
+    e, c, d, f = cfg.n_exp, cfg.c, cfg.d, cfg.f
+    w_bytes = e * (2 * f * d + d * f)
+    s_bytes = e * (2 * f + d) * 4
+    block_bytes = w_bytes + s_bytes + t * d * 2 + t * e * 2 + t * d * 2
+    ops = 2 * e * c * (d * 2 * f + f * d)
+    gateup = {
+        "ops": 2 * e * c * d * 2 * f,
+        # weights + their scales + gathered codes and scales in + h (fp32) out
+        "bytes": e * 2 * f * d + e * 2 * f * 4 + e * c * (d + 4) + e * c * f * 4,
+    }
+    down = {
+        "ops": 2 * e * c * f * d,
+        # weights + scales + h codes and scales in + fp32 red-add of the combine
+        "bytes": e * d * f + e * d * 4 + e * c * (f + 4) + e * c * d * 4,
+    }
+    return {"ops": ops, "block_bytes": block_bytes, "gateup": gateup, "down": down}
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.tmp.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world):
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ CPU oracle ----
+def oracle_sample(cfg, inp, n_experts):
+    """Time the oracle on all routing + the first n_experts experts' FFN and
+    extrapolate the block time to all experts. Returns (seconds per block, info)."""
+    import threadpoolctl
+
+    import oracle as O
+    x = inp["x"].float().numpy()
+    logits = inp["logits"].float().numpy()
+    wgu_q = np.zeros((cfg.n_exp, 2 * cfg.f, cfg.d), np.int8)
+    s_gu = np.zeros((cfg.n_exp, 2 * cfg.f), np.float32)
+    wd_q = np.zeros((cfg.n_exp, cfg.d, cfg.f), np.int8)
+    s_d = np.zeros((cfg.n_exp, cfg.d), np.float32)
+    for e in range(n_experts):  # offline weight quantisation: not timed
+        wgu_q[e], s_gu[e] = O.rotquant(inp["wgu"][e].float().numpy(), cfg.g_gu)
+        wd_q[e], s_d[e] = O.rotquant(inp["wd"][e].float().numpy(), cfg.g_d)
+    t0 = time.perf_counter()
+    O.moe_block(x, logits, wgu_q, s_gu, wd_q, s_d, cfg.c, cfg.g_gu, cfg.g_d, experts=[])
+    t_route = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.moe_block(x, logits, wgu_q, s_gu, wd_q, s_d, cfg.c, cfg.g_gu, cfg.g_d,
+                experts=list(range(n_experts)))
+    t_sample = time.perf_counter() - t0
+    per_expert = max(t_sample - t_route, 0.0) / n_experts
+    block_s = t_route + per_expert * cfg.n_exp
+    threads = max((i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()), default=1)
+    cores = min(threads, len(os.sched_getaffinity(0)))
+    info = {"kind": "oracle", "cores": cores,
+            "sample": (f"oracle block on {cfg.name} inputs: all routing + FFN of experts "
+                       f"0..{n_experts - 1} of {cfg.n_exp} timed ({t_sample:.1f} s), "
+                       f"extrapolated per expert to the full block")}
+    return block_s, info
+
+
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return
+    inp = moe_inputs(cfg)
+    times = []
+    info = None
+    for _ in range(args.warmup + args.steps):
+        block_s, info = oracle_sample(cfg, inp, n_experts=1)
+        times.append(block_s)
+    timed = times[args.warmup:]
+    block_s = statistics.mean(timed)
+    value = cfg.t / block_s
+    info["value"] = value
+    info["unit"] = UNIT
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": block_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64/int64",
+            "data": "synthetic (seeded; stands in for real prompts and trained weights)",
+            "config": {"workload": cfg.name, "tokens": cfg.t, "d": cfg.d, "experts": cfg.n_exp,
+                       "f": cfg.f, "capacity": cfg.c},
+            "cpu_baseline": info,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------- GPU path ----
+def stage_times(W, ws_views, inp_dev, wq, cfg, t, reps, flush_buf):
+    """Device time of every stage, launched through its own C-ABI entry with
+    the block's real intermediates, CUDA events on the launching stream."""
+    v = ws_views
+    wgu_q, s_gu, wd_q, s_d = wq
+    stream = torch.cuda.current_stream()
+    stages = {
+        "router_softmax": lambda: W.binding.lib().convrot_router_softmax(
+            W.binding._p(inp_dev["logits"]), t, cfg.n_exp, W.binding._p(v["s_t"]),
+            W.binding._stream()),
+        "rotquant_x": lambda: W.convrot_rotquant(inp_dev["x"], cfg.g_gu, q=v["x_q"], scale=v["s_x"]),
+        "topc": lambda: W.binding.lib().convrot_topc(
+            W.binding._p(v["s_t"]), t, cfg.n_exp, cfg.c, W.binding._p(v["idx"]),
+            W.binding._p(v["w"]), W.binding._stream()),
+        "gather": lambda: W.binding.lib().convrot_gather_rows(
+            W.binding._p(v["x_q"]), W.binding._p(v["s_x"]), t, W.binding._p(v["idx"]),
+            cfg.n_exp * cfg.c, cfg.d, W.binding._p(v["x_g"]), W.binding._p(v["s_g"]),
+            W.binding._stream()),
+        "gemm_gateup_swiglu": lambda: W.binding.lib().convrot_i8_gemm_swiglu(
+            W.binding._p(v["x_g"]), W.binding._p(v["s_g"]), W.binding._p(wgu_q),
+            W.binding._p(s_gu), cfg.n_exp, cfg.c, cfg.f, cfg.d, W.binding._p(v["h"]),
+            W.binding._stream()),
+        "rotquant_h": lambda: W.convrot_rotquant(v["h"].view(-1, cfg.f), cfg.g_d,
+                                                 q=v["h_q"].view(-1, cfg.f), scale=v["s_h"].view(-1)),
+        "gemm_down_scatter": lambda: W.binding.lib().convrot_i8_gemm_scatter(
+            W.binding._p(v["h_q"]), W.binding._p(v["s_h"]), W.binding._p(wd_q),
+            W.binding._p(s_d), W.binding._p(v["idx"]), W.binding._p(v["w"]), cfg.n_exp, cfg.c,
+            cfg.d, cfg.f, W.binding._p(v["out32"]), t, W.binding._stream()),
+        "f32_to_bf16": lambda: W.binding.lib().convrot_f32_to_bf16(
+            W.binding._p(v["out32"]), t * cfg.d, W.binding._p(inp_dev["y"]), W.binding._stream()),
+    }
+    out = {}
+    for name, fn in stages.items():
+        ts = []
+        for i in range(reps + 1):
+            flush_buf.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            rc = fn()
+            b.record(stream)
+            if isinstance(rc, int) and rc != 0:
+                raise RuntimeError(f"stage {name} failed: {rc}")
+            torch.cuda.synchronize()
+            if i > 0:
+                ts.append(a.elapsed_time(b) * 1e-3)
+        out[name] = statistics.median(ts)
+    return out
+
+
+def run_ours(args, cfg, world, rank, local):
+    import w8a8_rotated_int8_b200 as W
+    W.load_library()
+    W.convrot_device_check()
+    dev = torch.device("cuda", local)
+    t = cfg.t
+    inp = moe_inputs(cfg)
+    if rank > 0:  # every rank gets its own batch of tokens; weights are shared
+        gen = torch.Generator().manual_seed(cfg.seed * 1000 + rank)
+        inp["x"] = (torch.randn(t, cfg.d, generator=gen) * inp["x"].float().std()).to(torch.bfloat16)
+        inp["logits"] = torch.randn(t, cfg.n_exp, generator=gen).to(torch.bfloat16)
+    wgu_q, s_gu = W.convrot_quantize_weights(inp["wgu"].to(dev), cfg.g_gu)
+    wd_q, s_d = W.convrot_quantize_weights(inp["wd"].to(dev), cfg.g_d)
+    wq = (wgu_q, s_gu, wd_q, s_d)
+    x = inp["x"].to(dev)
+    logits = inp["logits"].to(dev)
+    y = torch.empty((t, cfg.d), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(W.moe_workspace_size(t, cfg.d, cfg.f, cfg.n_exp, cfg.c), dtype=torch.uint8,
+                     device=dev)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(xx, ll, yy):
+        W.moe_expert_choice_forward(xx, ll, wgu_q, s_gu, wd_q, s_d, cfg.c, cfg.g_gu, cfg.g_d,
+                                    y=yy, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush_buf.zero_()
+        step(x, logits, y)
+    torch.cuda.synchronize()
+    if W.convrot_check_device_error() != 0:
+        raise RuntimeError("device-side wait timed out during warm-up")
+
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush_buf.zero_()  # L2 flush, outside the timed events
+        starts[i].record(stream)
+        step(x, logits, y)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop()
+    step_s = [s.elapsed_time(e) * 1e-3 for s, e in zip(starts, ends)]
+    mean_step = max_over_ranks(statistics.mean(step_s), world)
+
+    # end to end through the C ABI with host buffers: pinned inputs in, result out
+    x_h = inp["x"].pin_memory()
+    l_h = inp["logits"].pin_memory()
+    y_h = torch.empty((t, cfg.d), dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        flush_buf.zero_()
+        x.copy_(x_h, non_blocking=True)
+        logits.copy_(l_h, non_blocking=True)
+        step(x, logits, y)
+        y_h.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_t = []
+    for _ in range(args.steps):
+        flush_buf.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        x.copy_(x_h, non_blocking=True)
+        logits.copy_(l_h, non_blocking=True)
+        step(x, logits, y)
+        y_h.copy_(y, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        e2e_t.append(a.elapsed_time(b) * 1e-3)
+    e2e_step = max_over_ranks(statistics.mean(e2e_t), world)
+
+    # per-stage device times (dominant kernel for the roofline)
+    views = W.moe_stage_views(ws, t, cfg.d, cfg.f, cfg.n_exp, cfg.c)
+    st = stage_times(W, views, {"x": x, "logits": logits, "y": y}, wq, cfg, t, 5, flush_buf)
+    flags = W.convrot_check_device_error()
+    if flags != 0:
+        raise RuntimeError(f"device error flags {flags:#x}")
+
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    work = algorithmic_work(cfg, t)
+    dom = max(("gemm_gateup_swiglu", "gemm_down_scatter"), key=lambda k: st[k])
+    dk = work["gateup"] if dom == "gemm_gateup_swiglu" else work["down"]
+    int8_peak_tops = 2.0 * peaks["bf16_tflops"]  # int8 dense = 2x bf16 dense (nominal ratio)
+    t_hbm = dk["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = dk["ops"] / (int8_peak_tops * 1e12)
+    if t_hbm >= t_tc:
+        achieved = dk["bytes"] / st[dom] / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = dk["ops"] / st[dom] / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak_tops, "unit": "TOPS"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dom
+    roof["algorithmic_bytes"] = dk["bytes"]
+    roof["algorithmic_ops"] = dk["ops"]
+    roof["peak_source"] = (f"{peaks['source']} (HBM copy; int8 = 2 x measured bf16 burst)")
+    roof["traffic"] = args.traffic_bytes
+    block_roof_t = max(work["block_bytes"] / (peaks["hbm_gbs"] * 1e9),
+                       work["ops"] / (int8_peak_tops * 1e12))
+
+    value = world * t / mean_step
+    launches_per_step = 8 if cfg.c > 0 else 3
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": mean_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8 (int32 acc, fp32 epilogue)",
+        "data": "synthetic (seeded; stands in for real prompts and trained weights)",
+        "config": {"workload": cfg.name, "tokens_per_gpu": t, "d": cfg.d, "experts": cfg.n_exp,
+                   "f": cfg.f, "capacity": cfg.c, "g_gu": cfg.g_gu, "g_d": cfg.g_d,
+                   "parallelism": f"replicas x{world} (independent batches)",
+                   "l2": "flushed before every step (256 MiB write outside the timed events)"},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": world * t / e2e_step, "unit": UNIT,
+                "h2d_bytes_per_step": int(x_h.numel() * 2 + l_h.numel() * 2),
+                "d2h_bytes_per_step": int(y_h.numel() * 2)},
+        "roofline": roof,
+        "block_roofline": {"time_us": block_roof_t * 1e6, "frac": block_roof_t / mean_step,
+                           "algorithmic_bytes": work["block_bytes"], "ops": work["ops"],
+                           "effective_tops": work["ops"] / mean_step / 1e12},
+        "stage_us": {k: v * 1e6 for k, v in st.items()},
+        "clocks": clk,
+        "wall_s": wall,
+    }
+    if args.cpu_baseline and world == 1:
+        block_s, info = oracle_sample(cfg, inp, n_experts=1)
+        info["value"] = cfg.t / block_s
+        info["unit"] = UNIT
+        line["cpu_baseline"] = info
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="moe_T8192", choices=sorted(MOE_CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="dram bytes per launch of the dominant kernel from an ncu capture")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = MOE_CONFIGS[args.config]
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, cfg, world, rank)
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_ours(args, cfg, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,218 @@
+/*
+ * convrot.h -- C ABI of the B200 (sm_100a) W8A8 ConvRot expert-choice MoE library.
+ *
+ * What the calls compute (web pages, cited by title and section):
+ *  - "Nucleus-Image INT8 Convrot Experts + FP8 Text Encoder", section
+ *    "Quantization": every routed-expert matrix is rotated (ConvRot), then
+ *    quantised to symmetric INT8 with nearest rounding and one FP32 scale per
+ *    output row; rotation groups are 256 for gate/up and 64 for down;
+ *    inference uses W8A8 ConvRot linears with BF16 outputs.
+ *  - "NitroFusion2 for ComfyUI: int8, W6A8, W4A8", section "How they were
+ *    made": int8 ConvRot = block Hadamard rotation, one scale per row, 8-bit
+ *    activations.
+ *  - "MLX Nucleus-Image", opening paragraph: 64 routed experts with
+ *    expert-choice routing; table "Conversion notes": each expert picks its
+ *    top-C tokens, outputs are scattered back; experts compute
+ *    silu(gate) * up with gate in the first half.
+ *
+ * Readings fixed by this library where the pages are silent:
+ *  - rotation: Sylvester Hadamard in natural order, normalised by 1/sqrt(g),
+ *    applied to contiguous groups of g along K; g in {1, 4, 16, 64, 256};
+ *  - quantiser: s = fp32(absmax / 127), q = clamp(rint(v / s), -127, 127)
+ *    (ties to even), codes and scale 0 for an all-zero row;
+ *  - activations (and the SwiGLU output h) use per-row dynamic scales;
+ *  - router score: per-token softmax over the experts (fp64, rounded to
+ *    fp32); top-C ties go to the lower token index; each expert's tokens are
+ *    listed in ascending order;
+ *  - dequant y = fp32(acc) * (s_w * s_x); h = silu(g) * u in fp32; combine
+ *    out32[t] += w * z in fp32, one bf16 rounding at the end.
+ *
+ * Conventions for every call:
+ *  - All buffers are owned by the caller; the library allocates nothing.
+ *    Pointers marked "device" must be device memory of the current CUDA
+ *    device and 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream). They return a status code and never throw or abort.
+ *  - Arguments are checked before anything is launched; on any error nothing
+ *    is launched. A kernel that gives up on a bounded device-side wait sets a
+ *    flag that convrot_check_device_error() reports (CONVROT_ERR_TIMEOUT).
+ *  - Layouts are row-major; "K-contiguous" means the last index is K.
+ */
+#ifndef CONVROT_H_
+#define CONVROT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  CONVROT_OK = 0,
+  CONVROT_ERR_INVALID_ARG = 1,        /* a size, group or pointer is not acceptable */
+  CONVROT_ERR_UNSUPPORTED_DEVICE = 2, /* current device is not sm_100 / no device */
+  CONVROT_ERR_WORKSPACE_TOO_SMALL = 3,
+  CONVROT_ERR_MISALIGNED = 4,         /* a pointer is not 16-byte aligned */
+  CONVROT_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+  CONVROT_ERR_TIMEOUT = 6             /* a device-side wait ran out (see check call) */
+};
+
+enum { CONVROT_DTYPE_BF16 = 0, CONVROT_DTYPE_F32 = 1 };
+
+/* Version of this ABI (incremented on incompatible changes). */
+int convrot_abi_version(void);
+
+/* Static description of a status code. Never NULL. */
+const char* convrot_status_string(int status);
+
+/* Checks that the current device is an sm_100 part the kernels were built for.
+ * Returns CONVROT_OK or CONVROT_ERR_UNSUPPORTED_DEVICE. */
+int convrot_device_check(void);
+
+/* Synchronises `stream`, then reads and clears the device error word.
+ * *flags (may be NULL) receives the raw bits. Returns CONVROT_ERR_TIMEOUT if a
+ * bounded wait ran out since the last check, CONVROT_ERR_CUDA if the
+ * synchronisation failed, else CONVROT_OK. */
+int convrot_check_device_error(void* stream, unsigned* flags);
+
+/* Diagnostic: launches one CTA that waits `limit_ns` on an mbarrier nothing
+ * arrives on, through the same bounded wait the GEMM pipeline uses. It must
+ * give up and record a flag; *result_dev (device int) receives 0 when it gave
+ * up. Used to test the failure path without faulting the GPU. */
+int convrot_wait_selftest(unsigned long long limit_ns, int* result_dev, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Rotate + quantise rows (offline weights, run-time activations, and the
+ * SwiGLU output h before the down projection). "Nucleus-Image INT8 Convrot
+ * Experts + FP8 Text Encoder", section "Quantization".
+ *   x      device, [rows, K] bf16 (x_dtype = CONVROT_DTYPE_BF16) or fp32
+ *   rows   >= 0;  K: multiple of 16 and of `group`, 16 <= K <= 8192
+ *   group  rotation group g in {1, 4, 16, 64, 256}
+ *   q      device, [rows, K] int8 codes (K-contiguous)
+ *   scale  device, [rows] fp32 per-row scales
+ * rows == 0 launches nothing and returns CONVROT_OK.
+ * ------------------------------------------------------------------------- */
+int convrot_rotquant(const void* x, int x_dtype, int64_t rows, int64_t K, int group, int8_t* q,
+                     float* scale, void* stream);
+
+/* Offline weight quantisation: the same operation on bf16 weight rows. A
+ * stack of expert matrices [E, N, K] is passed as rows = E * N (the rotation
+ * is per row, so the 3-D packed layout needs no other entry point). */
+int convrot_quantize_weights(const void* w_bf16, int64_t rows, int64_t K, int group,
+                             int8_t* w_q, float* row_scale, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Router softmax. "MLX Nucleus-Image", opening paragraph (expert-choice).
+ *   logits  device, [T, E] bf16;  1 <= E <= 256
+ *   s_t     device, [E, T] fp32: s_t[e, t] = softmax_e(logits[t, :]) (transposed)
+ * ------------------------------------------------------------------------- */
+int convrot_router_softmax(const void* logits_bf16, int64_t T, int E, float* s_t, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Expert-choice top-C. "MLX Nucleus-Image", table "Conversion notes".
+ *   s_t   device, [E, T] fp32 scores (no NaN)
+ *   C     0 <= C <= T
+ *   idx   device, [E, C] int32: the C tokens with the largest score, ties to
+ *         the lower token index, in ascending token order
+ *   w     device, [E, C] fp32: w[e, c] = s_t[e, idx[e, c]]
+ * ------------------------------------------------------------------------- */
+int convrot_topc(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float* w,
+                 void* stream);
+
+/* Gather rows: dst[r, :] = src[idx[r], :], s_dst[r] = s_src[idx[r]].
+ *   src [n_src, K] int8, s_src [n_src] fp32, idx [n_rows] int32 (each in
+ *   [0, n_src)), dst [n_rows, K] int8, s_dst [n_rows] fp32; K % 16 == 0. */
+int convrot_gather_rows(const int8_t* src, const float* s_src, int64_t n_src, const int32_t* idx,
+                        int64_t n_rows, int64_t K, int8_t* dst, float* s_dst, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Grouped INT8 GEMMs on the tcgen05 tensor cores (exact int32 accumulation).
+ * For every group g: acc[g, m, n] = sum_k a[g, m, k] * b[g, n, k].
+ *   a  device, [G, M, K] int8;  b device, [G, N, K] int8 (K-contiguous)
+ *   K % 16 == 0, 16 <= K;  N % 16 == 0;  G, M, N < 2^31
+ * ------------------------------------------------------------------------- */
+
+/* acc stored as int32 d [G, M, N]. */
+int convrot_i8_gemm_i32(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t N,
+                        int64_t K, int32_t* d, void* stream);
+
+/* y[g, m, n] = bf16(fp32(acc) * (s_b[g, n] * s_a[g, m])); s_a [G, M], s_b [G, N]. */
+int convrot_i8_gemm_bf16(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
+                         int64_t G, int64_t M, int64_t N, int64_t K, void* y_bf16, void* stream);
+
+/* SwiGLU epilogue: b = [G, 2F, K] with gate rows 0..F-1 and up rows F..2F-1,
+ * s_b [G, 2F]. h[g, m, f] = silu(y[g, m, f]) * y[g, m, F + f] in fp32 with
+ * y = fp32(acc) * (s_b * s_a); h device [G, M, F] fp32; F % 16 == 0. */
+int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
+                           int64_t G, int64_t M, int64_t F, int64_t K, float* h, void* stream);
+
+/* Router-weighted scatter epilogue:
+ * out32[idx[g, m], n] += w[g, m] * (fp32(acc) * (s_b[g, n] * s_a[g, m])).
+ * out32 device [T, N] fp32 (accumulated with fp32 atomics, order not fixed);
+ * idx [G, M] int32 in [0, T); w [G, M] fp32. */
+int convrot_i8_gemm_scatter(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
+                            const int32_t* idx, const float* w, int64_t G, int64_t M, int64_t N,
+                            int64_t K, float* out32, int64_t T, void* stream);
+
+/* y = bf16(x) (nearest even), n elements, n % 4 == 0. */
+int convrot_f32_to_bf16(const float* x, int64_t n, void* y_bf16, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * W8A8 ConvRot linear. "Nucleus-Image INT8 Convrot Experts + FP8 Text
+ * Encoder", section "Quantization" (W8A8 with BF16 outputs).
+ *   x       device, [M, K] bf16 activations (rotated and quantised per token)
+ *   w_q     device, [N, K] int8 rotated weight codes (convrot_quantize_weights)
+ *   w_scale device, [N] fp32
+ *   y       device, [M, N] bf16: bf16(fp32(acc) * (w_scale[n] * s_x[m]))
+ *   workspace device, >= convrot_linear_workspace_size(M, K) bytes
+ * ------------------------------------------------------------------------- */
+size_t convrot_linear_workspace_size(int64_t M, int64_t K);
+int w8a8_convrot_linear(const void* x_bf16, int64_t M, int64_t K, const int8_t* w_q,
+                        const float* w_scale, int64_t N, int group, void* y_bf16, void* workspace,
+                        size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Expert-choice W8A8 ConvRot MoE block (one call = the whole hot path).
+ * "MLX Nucleus-Image", opening paragraph and table "Conversion notes";
+ * "Nucleus-Image INT8 Convrot Experts + FP8 Text Encoder", "Quantization".
+ *   x       device, [T, d] bf16;  logits device, [T, E] bf16
+ *   w_gu    device, [E, 2f, d] int8 (rows 0..f-1 gate, f..2f-1 up), rotated g_gu
+ *   s_gu    device, [E, 2f] fp32
+ *   w_d     device, [E, d, f] int8, rotated g_d;  s_d device, [E, d] fp32
+ *   C       tokens per expert, 0 <= C <= T
+ *   y       device, [T, d] bf16 = bf16(sum over experts that chose t of
+ *           w[e, c] * down_e(requant(silu(gate_e) * up_e)))
+ *   Sizes: d % 16 == 0, d % g_gu == 0, 16 <= d <= 8192; f % 16 == 0,
+ *   f % g_d == 0, 16 <= f <= 8192; 1 <= E <= 256.
+ * The workspace holds every intermediate; its layout is reported by
+ * moe_workspace_layout so a caller can inspect each stage after the call.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  size_t x_q;      /* [T, d] int8     rotated activation codes      */
+  size_t s_x;      /* [T] fp32        token scales                  */
+  size_t s_t;      /* [E, T] fp32     router scores, transposed     */
+  size_t idx;      /* [E, C] int32    chosen tokens                 */
+  size_t w;        /* [E, C] fp32     router weights of the choices */
+  size_t x_g;      /* [E, C, d] int8  gathered codes                */
+  size_t s_g;      /* [E, C] fp32     gathered scales               */
+  size_t h;        /* [E, C, f] fp32  silu(gate) * up               */
+  size_t h_q;      /* [E, C, f] int8  rotated, requantised h        */
+  size_t s_h;      /* [E, C] fp32     scales of h                   */
+  size_t out32;    /* [T, d] fp32     combine accumulator           */
+  size_t total;    /* bytes required                                */
+} convrot_moe_layout_t;
+
+int moe_workspace_layout(int64_t T, int64_t d, int64_t f, int E, int64_t C,
+                         convrot_moe_layout_t* layout);
+size_t moe_workspace_size(int64_t T, int64_t d, int64_t f, int E, int64_t C);
+int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const int8_t* w_gu,
+                              const float* s_gu, const int8_t* w_d, const float* s_d, int64_t T,
+                              int64_t d, int64_t f, int E, int64_t C, int g_gu, int g_d,
+                              void* y_bf16, void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONVROT_H_ */

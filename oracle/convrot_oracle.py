@@ -206,14 +206,16 @@ def silu_f32(g: np.ndarray) -> np.ndarray:
 
 # -------------------------------------------------------------- MoE block ---
 def moe_block(x, logits, wgu_q, s_gu, wd_q, s_d, c, g_gu=256, g_d=64,
-              experts=None, keep=False):
+              experts=None, keep=False, out_tokens=None):
     """Expert-choice W8A8 ConvRot MoE block.
 
     x: [T, d] bf16 values; logits: [T, E] bf16 values;
     wgu_q: [E, 2f, d] int8 (rows 0..f-1 gate, f..2f-1 up), s_gu: [E, 2f];
     wd_q: [E, d, f] int8, s_d: [E, d]; c: tokens per expert.
     ``experts`` restricts the combine to a subset of experts (used to time a
-    bounded sample); ``keep`` returns the intermediates as a dict.
+    bounded sample); ``out_tokens`` evaluates only the output rows of those
+    tokens (each row depends only on its own token, so the others are simply
+    skipped and left 0); ``keep`` returns the intermediates as a dict.
 
     Returns Y as fp32 holding bf16 values [T, d] (and the dict if keep).
     """
@@ -229,13 +231,18 @@ def moe_block(x, logits, wgu_q, s_gu, wd_q, s_d, c, g_gu=256, g_d=64,
              "h": {}, "h_q": {}, "s_h": {}}
     for e in (range(n_exp) if experts is None else experts):
         rows = idx[e]
+        if out_tokens is not None:
+            rows = rows[np.isin(rows, out_tokens)]
+            if rows.size == 0:
+                continue
+        sel = np.searchsorted(idx[e], rows)
         y = dequant(int_gemm(x_q[rows], wgu_q[e]), s_gu[e], s_x[rows])
         gate, up = y[:, :f], y[:, f:]
         h = (silu_f32(gate) * up).astype(np.float32)
         h_q, s_h = rotquant(h, g_d)
         z = dequant(int_gemm(h_q, wd_q[e]), s_d[e], s_h)
         # rows are distinct within an expert, so fancy-index += is exact
-        out32[rows] = out32[rows] + (w[e][:, None] * z).astype(np.float32)
+        out32[rows] = out32[rows] + (w[e][sel][:, None] * z).astype(np.float32)
         if keep:
             inter["h"][e], inter["h_q"][e], inter["s_h"][e] = h, h_q, s_h
     y_out = bf16_round(out32)

@@ -1,0 +1,89 @@
+"""The C-ABI library loads without a GPU, exports every declared symbol, and
+rejects bad arguments on the host before touching the device (no GPU)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from w8a8_rotated_int8_b200 import binding
+from w8a8_rotated_int8_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "convrot.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("convrot_quantize_weights", "w8a8_convrot_linear",
+                     "moe_expert_choice_forward", "convrot_rotquant", "convrot_topc",
+                     "convrot_i8_gemm_i32"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(binding._SIGNATURES) == set(declared_functions())
+
+
+def test_abi_version_and_strings(lib):
+    assert lib.convrot_abi_version() == 1
+    for code in range(7):
+        assert binding.status_string(code)
+    assert binding.status_string(99) == "unknown status"
+
+
+def test_argument_checks_need_no_gpu(lib):
+    al = ctypes.c_void_p(4096)       # 16-byte aligned placeholder, never dereferenced
+    mis = ctypes.c_void_p(4096 + 8)
+    INVALID, MISALIGNED = binding.CONVROT_ERR_INVALID_ARG, binding.CONVROT_ERR_MISALIGNED
+    # unsupported rotation group / K not a multiple of the group / K % 16
+    assert lib.convrot_rotquant(al, 0, 4, 256, 128, al, al, None) == INVALID
+    assert lib.convrot_rotquant(al, 0, 4, 96, 64, al, al, None) == INVALID
+    assert lib.convrot_rotquant(al, 0, 4, 40, 4, al, al, None) == INVALID
+    assert lib.convrot_rotquant(al, 7, 4, 256, 256, al, al, None) == INVALID
+    assert lib.convrot_rotquant(mis, 0, 4, 256, 256, al, al, None) == MISALIGNED
+    # top-C capacity beyond T
+    assert lib.convrot_topc(al, 10, 4, 11, al, al, None) == INVALID
+    # GEMM: K not a multiple of 16, N not a multiple of 16, int32 overflow bound
+    assert lib.convrot_i8_gemm_i32(al, al, 1, 8, 16, 40, al, None) == INVALID
+    assert lib.convrot_i8_gemm_i32(al, al, 1, 8, 24, 64, al, None) == INVALID
+    assert lib.convrot_i8_gemm_i32(al, al, 1, 8, 16, 1 << 20, al, None) == INVALID
+    # MoE: C > T, bad group, d not a multiple of g_gu, workspace too small
+    args = [al] * 6
+    assert lib.moe_expert_choice_forward(*args, 8, 256, 64, 4, 9, 256, 64, al, al, 1 << 30, None) == INVALID
+    assert lib.moe_expert_choice_forward(*args, 8, 256, 64, 4, 2, 32, 64, al, al, 1 << 30, None) == INVALID
+    assert lib.moe_expert_choice_forward(*args, 8, 320, 64, 4, 2, 256, 64, al, al, 1 << 30, None) == INVALID
+    assert (lib.moe_expert_choice_forward(*args, 8, 256, 64, 4, 2, 256, 64, al, al, 16, None)
+            == binding.CONVROT_ERR_WORKSPACE_TOO_SMALL)
+
+
+def test_no_device_is_reported_not_crashed(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert lib.convrot_device_check() == binding.CONVROT_ERR_UNSUPPORTED_DEVICE
+
+
+def test_workspace_layout_is_disjoint_and_aligned(lib):
+    lay = binding.moe_workspace_layout(8192, 2048, 1536, 64, 256)
+    names = [n for n in lay if n != "total"]
+    offs = sorted(lay[n] for n in names)
+    assert all(o % 256 == 0 for o in offs)
+    assert len(set(offs)) == len(offs)
+    assert lay["total"] >= lay["out32"] + 8192 * 2048 * 4

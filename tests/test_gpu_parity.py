@@ -1,0 +1,360 @@
+"""GPU parity: every stage of the CUDA path through the C ABI against the oracle.
+
+Bar: bit-exact codes, scales, int32 accumulators, top-C index sets and
+dequantised outputs; the SwiGLU output and the fp32 combine within the bounds
+their arithmetic allows (CUDA expf vs a correctly rounded exp; atomic
+accumulation order); the block output within the 1e-2 max-relative budget.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from synthetic import LINEAR_CONFIGS, MOE_CONFIGS, linear_inputs, moe_inputs
+from tests.golden import read_fixture
+
+pytestmark = pytest.mark.gpu
+
+W = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def gpu_lib():
+    global W
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import w8a8_rotated_int8_b200 as lib_mod
+    lib_mod.load_library()
+    lib_mod.convrot_device_check()
+    W = lib_mod
+    yield
+    W.convrot_check_device_error()
+
+
+@pytest.fixture(autouse=True)
+def no_device_errors():
+    yield
+    assert W.convrot_check_device_error() == 0
+
+
+def np32(t):
+    return t.detach().float().cpu().numpy()
+
+
+def bf16_activations(rows, k, seed, outliers=True):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(rows, k, generator=g)
+    if outliers:
+        ch = torch.randperm(k, generator=g)[: max(1, round(0.01 * k))]
+        x[:, ch] *= 20
+    return x.to(torch.bfloat16)
+
+
+# ----------------------------------------------------------- rotate+quant --
+@pytest.mark.parametrize("rows,k,g", [
+    (64, 256, 256), (300, 768, 256), (257, 2048, 256), (5, 8192, 256), (33, 320, 64),
+    (100, 1536, 64), (77, 512, 16), (50, 256, 4), (40, 64, 1), (3, 16, 16), (1, 4096, 64),
+])
+def test_rotquant_bf16_bit_exact(rows, k, g):
+    x = bf16_activations(rows, k, seed=rows * 7 + k)
+    q, s = W.convrot_rotquant(x.cuda(), g)
+    q_ref, s_ref = O.rotquant(np32(x), g)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+@pytest.mark.parametrize("rows,k,g", [(160, 320, 64), (513, 1536, 64), (64, 2048, 256)])
+def test_rotquant_f32_bit_exact(rows, k, g):
+    gen = torch.Generator().manual_seed(k)
+    a = torch.randn(rows, k, generator=gen)
+    b = torch.randn(rows, k, generator=gen)
+    h = (torch.nn.functional.silu(a) * b).float()  # SwiGLU-shaped fp32 rows
+    q, s = W.convrot_rotquant(h.cuda(), g)
+    q_ref, s_ref = O.rotquant(h.numpy(), g)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def test_rotquant_worked_examples_and_degenerate_rows():
+    ties = read_fixture("quant_ties.txt")
+    rot = read_fixture("rotation_g4.txt")
+    x = torch.zeros(4, 16)
+    x[0, :8] = torch.tensor(ties["input"][0])
+    x[1, :8] = torch.tensor(rot["input"][0])
+    x[3, :] = 0.75  # constant row
+    xb = x.to(torch.bfloat16)
+    q1, s1 = W.convrot_rotquant(xb.cuda(), 1)
+    assert q1[0, :8].tolist() == ties["codes"][0] and s1[0].item() == 1.0
+    assert q1[2].abs().sum().item() == 0 and s1[2].item() == 0.0  # zero row
+    q4, s4 = W.convrot_rotquant(xb.cuda(), 4)
+    assert q4[1, :8].tolist() == rot["codes"][0]
+    assert s4[1].item() == np.float32(13.0 / 127.0)
+    assert q4[2].abs().sum().item() == 0
+
+
+def test_weight_quantisation_3d_stack():
+    cfg = MOE_CONFIGS["moe_small"]
+    inp = moe_inputs(cfg)
+    q, s = W.convrot_quantize_weights(inp["wd"].cuda(), cfg.g_d)
+    for e in range(cfg.n_exp):
+        q_ref, s_ref = O.rotquant(np32(inp["wd"][e]), cfg.g_d)
+        assert np.array_equal(q[e].cpu().numpy(), q_ref)
+        assert np.array_equal(s[e].cpu().numpy(), s_ref)
+
+
+# ----------------------------------------------------------------- routing --
+def _ulp_diff(a, b):
+    ai = a.view(np.int32).astype(np.int64)
+    bi = b.view(np.int32).astype(np.int64)
+    return np.abs(ai - bi)
+
+
+@pytest.mark.parametrize("t,e", [(8192, 64), (1000, 8), (33, 256), (1, 1)])
+def test_router_softmax(t, e):
+    gen = torch.Generator().manual_seed(t + e)
+    logits = torch.randn(t, e, generator=gen).to(torch.bfloat16)
+    s_t = W.convrot_router_softmax(logits.cuda()).cpu().numpy()
+    ref = O.router_softmax(np32(logits)).T
+    d = _ulp_diff(s_t, ref)
+    assert d.max() <= 1
+    assert (d != 0).mean() <= 1e-4
+
+
+@pytest.mark.parametrize("t,e,c", [(8192, 64, 256), (2048, 64, 64), (1000, 8, 100),
+                                   (300, 5, 300), (50, 3, 1), (1, 2, 1), (64, 4, 0)])
+def test_topc_exact_given_scores(t, e, c):
+    gen = torch.Generator().manual_seed(t * 3 + c)
+    s = torch.softmax(torch.randn(t, e, generator=gen), dim=1).numpy().astype(np.float32)
+    if t == 1000:
+        s = (np.floor(s * 16) / 16).astype(np.float32)  # heavy ties
+    idx, w = W.convrot_topc(torch.from_numpy(np.ascontiguousarray(s.T)).cuda(), c)
+    idx_ref, w_ref = O.expert_choice_topc(s, c)
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert np.array_equal(w.cpu().numpy(), w_ref)
+
+
+def test_gather_rows():
+    src = torch.randint(-127, 128, (100, 64), dtype=torch.int8)
+    s_src = torch.rand(100)
+    idx = torch.tensor([5, 0, 99, 5, 42], dtype=torch.int32)
+    dst, s_dst = W.convrot_gather_rows(src.cuda(), s_src.cuda(), idx.cuda())
+    assert torch.equal(dst.cpu(), src[idx.long()])
+    assert torch.equal(s_dst.cpu(), s_src[idx.long()])
+
+
+# -------------------------------------------------------------------- GEMM --
+GEMM_SHAPES = [(1, 64, 256, 256), (3, 160, 320, 768), (2, 40, 48, 2048), (1, 128, 256, 128),
+               (1, 300, 272, 1536), (4, 256, 3072, 2048), (1, 1, 16, 16), (2, 129, 512, 64)]
+
+
+def _codes(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(-127, 128, shape, generator=g, dtype=torch.int8)
+
+
+@pytest.mark.parametrize("g,m,n,k", GEMM_SHAPES)
+def test_gemm_int32_bit_exact(g, m, n, k):
+    a = _codes((g, m, k), 1 + m)
+    b = _codes((g, n, k), 2 + n)
+    d = W.convrot_i8_gemm_i32(a.cuda(), b.cuda()).cpu().numpy()
+    for gi in range(g):
+        assert np.array_equal(d[gi], O.int_gemm(a[gi].numpy(), b[gi].numpy()))
+
+
+def test_gemm_int32_extremes():
+    k = 2048
+    a = torch.full((1, 128, k), 127, dtype=torch.int8)
+    b = torch.full((1, 256, k), -127, dtype=torch.int8)
+    b[0, 1] = 127
+    d = W.convrot_i8_gemm_i32(a.cuda(), b.cuda()).cpu()
+    assert int(d[0, 0, 0]) == -k * 127 * 127 and int(d[0, 5, 1]) == k * 127 * 127
+
+
+@pytest.mark.parametrize("g,m,n,k", [(1, 64, 256, 256), (2, 200, 320, 512), (1, 513, 528, 1536)])
+def test_gemm_bf16_dequant_bit_exact(g, m, n, k):
+    a = _codes((g, m, k), 3)
+    b = _codes((g, n, k), 4)
+    s_a = torch.rand(g, m) * 0.05 + 1e-3
+    s_b = torch.rand(g, n) * 1e-3 + 1e-5
+    y = W.convrot_i8_gemm_bf16(a.cuda(), s_a.cuda(), b.cuda(), s_b.cuda()).cpu()
+    for gi in range(g):
+        ref = O.bf16_round(O.dequant(O.int_gemm(a[gi].numpy(), b[gi].numpy()),
+                                     s_b[gi].numpy(), s_a[gi].numpy()))
+        assert np.array_equal(np32(y[gi]), ref)
+
+
+def _fp32_ulps(x, ref):
+    return np.abs(x.astype(np.float64) - ref) / np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
+
+
+@pytest.mark.parametrize("g,m,f,k", [(2, 160, 320, 768), (1, 64, 1536, 2048), (3, 40, 192, 512)])
+def test_gemm_swiglu(g, m, f, k):
+    a = _codes((g, m, k), 5)
+    b = _codes((g, 2 * f, k), 6)
+    s_a = torch.rand(g, m) * 0.05 + 1e-3
+    s_b = torch.rand(g, 2 * f) * 1e-4 + 1e-6
+    h = W.convrot_i8_gemm_swiglu(a.cuda(), s_a.cuda(), b.cuda(), s_b.cuda()).cpu().numpy()
+    for gi in range(g):
+        y = O.dequant(O.int_gemm(a[gi].numpy(), b[gi].numpy()), s_b[gi].numpy(), s_a[gi].numpy())
+        ref = (O.silu_f32(y[:, :f]) * y[:, f:]).astype(np.float32)
+        ulps = _fp32_ulps(h[gi], ref)
+        # CUDA expf is within 2 ulp of exp: silu(g)*u within a few ulp
+        assert ulps.max() <= 4
+        assert (ulps == 0).mean() > 0.9
+
+
+def test_gemm_scatter():
+    g, m, n, k, t = 4, 100, 320, 512, 150
+    a = _codes((g, m, k), 7)
+    b = _codes((g, n, k), 8)
+    s_a = torch.rand(g, m) * 0.05 + 1e-3
+    s_b = torch.rand(g, n) * 1e-4 + 1e-6
+    gen = torch.Generator().manual_seed(9)
+    idx = torch.stack([torch.sort(torch.randperm(t, generator=gen)[:m]).values for _ in range(g)])
+    idx = idx.to(torch.int32)
+    w = torch.rand(g, m)
+    out = torch.zeros(t, n)
+    ref = np.zeros((t, n), np.float32)
+    for gi in range(g):
+        z = O.dequant(O.int_gemm(a[gi].numpy(), b[gi].numpy()), s_b[gi].numpy(), s_a[gi].numpy())
+        ref[idx[gi].numpy()] += w[gi].numpy()[:, None] * z
+    out_gpu = W.convrot_i8_gemm_scatter(a.cuda(), s_a.cuda(), b.cuda(), s_b.cuda(), idx.cuda(),
+                                        w.cuda(), out.cuda()).cpu().numpy()
+    # fp32 sums of <= 4 terms in another order: within 4 ulps of the largest term
+    assert np.max(np.abs(out_gpu - ref)) <= 4 * np.spacing(np.float32(np.abs(ref).max()))
+
+
+# ------------------------------------------------------------------ linear --
+@pytest.mark.parametrize("name", ["linear_64x256x256", "gateup_4096x3072x2048",
+                                  "down_4096x2048x1536"])
+def test_w8a8_linear_bit_exact(name):
+    cfg = LINEAR_CONFIGS[name]
+    x, w = linear_inputs(cfg)
+    w_q, s_w = W.convrot_quantize_weights(w.cuda(), cfg.group)
+    y = W.w8a8_convrot_linear(x.cuda(), w_q, s_w, cfg.group).cpu()
+    w_q_ref, s_w_ref = O.rotquant(np32(w), cfg.group)
+    assert np.array_equal(w_q.cpu().numpy(), w_q_ref) and np.array_equal(s_w.cpu().numpy(), s_w_ref)
+    y_ref = O.w8a8_linear(np32(x), w_q_ref, s_w_ref, cfg.group)
+    assert np.array_equal(np32(y), y_ref)
+
+
+def test_linear_empty_batch():
+    w = torch.randn(32, 256).to(torch.bfloat16).cuda()
+    w_q, s_w = W.convrot_quantize_weights(w, 256)
+    y = W.w8a8_convrot_linear(torch.empty(0, 256, dtype=torch.bfloat16, device="cuda"), w_q, s_w, 256)
+    assert y.shape == (0, 32)
+
+
+# -------------------------------------------------------------- MoE block --
+def _quantise_moe_on_gpu(inp, cfg):
+    wgu_q, s_gu = W.convrot_quantize_weights(inp["wgu"].cuda(), cfg.g_gu)
+    wd_q, s_d = W.convrot_quantize_weights(inp["wd"].cuda(), cfg.g_d)
+    return wgu_q, s_gu, wd_q, s_d
+
+
+def _oracle_weights(inp, cfg, experts):
+    e_n, f, d = cfg.n_exp, cfg.f, cfg.d
+    wgu_q = np.zeros((e_n, 2 * f, d), np.int8)
+    s_gu = np.zeros((e_n, 2 * f), np.float32)
+    wd_q = np.zeros((e_n, d, f), np.int8)
+    s_d = np.zeros((e_n, d), np.float32)
+    for e in experts:
+        wgu_q[e], s_gu[e] = O.rotquant(np32(inp["wgu"][e]), cfg.g_gu)
+        wd_q[e], s_d[e] = O.rotquant(np32(inp["wd"][e]), cfg.g_d)
+    return wgu_q, s_gu, wd_q, s_d
+
+
+def _run_moe(inp, cfg, t=None):
+    t = cfg.t if t is None else t
+    wgu_q, s_gu, wd_q, s_d = _quantise_moe_on_gpu(inp, cfg)
+    ws = torch.empty(W.moe_workspace_size(t, cfg.d, cfg.f, cfg.n_exp, cfg.c), dtype=torch.uint8,
+                     device="cuda")
+    y = W.moe_expert_choice_forward(inp["x"].cuda(), inp["logits"].cuda(), wgu_q, s_gu, wd_q, s_d,
+                                    cfg.c, cfg.g_gu, cfg.g_d, workspace=ws)
+    torch.cuda.synchronize()
+    views = W.moe_stage_views(ws, t, cfg.d, cfg.f, cfg.n_exp, cfg.c)
+    return y, views, (wgu_q, s_gu, wd_q, s_d)
+
+
+def _max_rel(y, ref):
+    return float(np.max(np.abs(y - ref)) / max(np.max(np.abs(ref)), 1e-30))
+
+
+@pytest.mark.parametrize("name", ["moe_small", "moe_small_c40"])
+def test_moe_block_small_end_to_end(name):
+    cfg = MOE_CONFIGS[name]
+    inp = moe_inputs(cfg)
+    y, v, wq = _run_moe(inp, cfg)
+    ow = _oracle_weights(inp, cfg, range(cfg.n_exp))
+    for got, ref in zip(wq, ow):
+        assert np.array_equal(got.cpu().numpy(), ref)
+    y_ref, it = O.moe_block(np32(inp["x"]), np32(inp["logits"]), *ow, c=cfg.c, g_gu=cfg.g_gu,
+                            g_d=cfg.g_d, keep=True)
+    # stage by stage
+    assert np.array_equal(v["x_q"].cpu().numpy(), it["x_q"])
+    assert np.array_equal(v["s_x"].cpu().numpy(), it["s_x"])
+    assert _ulp_diff(v["s_t"].cpu().numpy(), it["scores"].T).max() <= 1
+    assert np.array_equal(v["idx"].cpu().numpy(), it["idx"])
+    assert np.array_equal(v["w"].cpu().numpy(), it["w"])
+    h_q_diff = 0
+    n_codes = 0
+    for e in range(cfg.n_exp):
+        assert _fp32_ulps(v["h"][e].cpu().numpy(), it["h"][e]).max() <= 4
+        dq = np.abs(v["h_q"][e].cpu().numpy().astype(np.int32) - it["h_q"][e].astype(np.int32))
+        assert dq.max() <= 1
+        h_q_diff += int((dq != 0).sum())
+        n_codes += dq.size
+    assert h_q_diff <= max(2, 1e-4 * n_codes)
+    y_np = np32(y)
+    assert _max_rel(y_np, y_ref) <= 1e-2
+    assert (y_np != y_ref).mean() < 0.01
+    unchosen = np.setdiff1d(np.arange(cfg.t), np.unique(it["idx"]))
+    assert np.all(y_np[unchosen] == 0)
+
+
+def test_moe_block_capacity_extremes():
+    base = MOE_CONFIGS["moe_small_c40"]
+    for c in (0, 1, base.t):
+        cfg = base.__class__(**{**base.__dict__, "c": c})
+        inp = moe_inputs(cfg)
+        y, _, _ = _run_moe(inp, cfg)
+        ow = _oracle_weights(inp, cfg, range(cfg.n_exp))
+        y_ref = O.moe_block(np32(inp["x"]), np32(inp["logits"]), *ow, c=c, g_gu=cfg.g_gu,
+                            g_d=cfg.g_d)
+        assert _max_rel(np32(y), y_ref) <= 1e-2 if c > 0 else np.all(np32(y) == 0)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["moe_T8192", "moe_T2048"])
+def test_moe_block_full_size_sampled_rows(name):
+    """Full-size block as the bench runs it; the oracle evaluates sampled rows."""
+    cfg = MOE_CONFIGS[name]
+    inp = moe_inputs(cfg)
+    y, v, wq = _run_moe(inp, cfg)
+    x_np, logits_np = np32(inp["x"]), np32(inp["logits"])
+    scores = O.router_softmax(logits_np)
+    idx_ref, _ = O.expert_choice_topc(scores, cfg.c)
+    assert np.array_equal(v["idx"].cpu().numpy(), idx_ref)
+    counts = np.bincount(idx_ref.ravel(), minlength=cfg.t)
+    rng = np.random.default_rng(0)
+    busy = np.argsort(-counts, kind="stable")[:8]
+    sample = np.unique(np.concatenate([np.arange(8), rng.choice(cfg.t, 16, replace=False), busy]))
+    experts = sorted({e for e in range(cfg.n_exp) if np.isin(idx_ref[e], sample).any()})
+    ow = _oracle_weights(inp, cfg, experts)
+    for e in experts[:4]:
+        assert np.array_equal(wq[0][e].cpu().numpy(), ow[0][e])
+        assert np.array_equal(wq[2][e].cpu().numpy(), ow[2][e])
+    y_ref = O.moe_block(x_np, logits_np, *ow, c=cfg.c, g_gu=cfg.g_gu, g_d=cfg.g_d,
+                        out_tokens=sample)
+    y_np = np32(y)
+    assert _max_rel(y_np[sample], y_ref[sample]) <= 1e-2
+    assert np.array_equal(v["x_q"].cpu().numpy()[sample], O.rotquant(x_np[sample], cfg.g_gu)[0])
+
+
+# ---------------------------------------------------------- failure path --
+def test_bounded_wait_gives_up_and_reports():
+    assert W.convrot_wait_selftest(2_000_000) == 0   # 2 ms limit, nothing arrives
+    flags = W.convrot_check_device_error()
+    assert flags & (1 << 5)
+    assert W.convrot_check_device_error() == 0       # cleared by the read

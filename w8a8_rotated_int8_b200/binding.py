@@ -1,0 +1,353 @@
+"""Thin Python binding of libconvrot.so (the C ABI in include/convrot.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI. PyTorch is used for device memory (output and
+workspace tensors) and for the current CUDA stream. There is no CPU or
+PyTorch fallback: if the library is missing or the device is not an sm_100
+part, the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libconvrot.so")
+
+CONVROT_OK = 0
+CONVROT_ERR_INVALID_ARG = 1
+CONVROT_ERR_UNSUPPORTED_DEVICE = 2
+CONVROT_ERR_WORKSPACE_TOO_SMALL = 3
+CONVROT_ERR_MISALIGNED = 4
+CONVROT_ERR_CUDA = 5
+CONVROT_ERR_TIMEOUT = 6
+DTYPE_BF16 = 0
+DTYPE_F32 = 1
+
+
+class ConvrotError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class MoeLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("x_q", "s_x", "s_t", "idx", "w", "x_g", "s_g", "h", "h_q", "s_h", "out32", "total")]
+
+
+_lib = None
+_lock = threading.Lock()
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+_SIGNATURES = {
+    "convrot_abi_version": (_I, []),
+    "convrot_status_string": (ctypes.c_char_p, [_I]),
+    "convrot_device_check": (_I, []),
+    "convrot_check_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
+    "convrot_wait_selftest": (_I, [ctypes.c_ulonglong, _P, _P]),
+    "convrot_rotquant": (_I, [_P, _I, _I64, _I64, _I, _P, _P, _P]),
+    "convrot_quantize_weights": (_I, [_P, _I64, _I64, _I, _P, _P, _P]),
+    "convrot_router_softmax": (_I, [_P, _I64, _I, _P, _P]),
+    "convrot_topc": (_I, [_P, _I64, _I, _I64, _P, _P, _P]),
+    "convrot_gather_rows": (_I, [_P, _P, _I64, _P, _I64, _I64, _P, _P, _P]),
+    "convrot_i8_gemm_i32": (_I, [_P, _P, _I64, _I64, _I64, _I64, _P, _P]),
+    "convrot_i8_gemm_bf16": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P]),
+    "convrot_i8_gemm_swiglu": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P]),
+    "convrot_i8_gemm_scatter": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _I64, _P]),
+    "convrot_f32_to_bf16": (_I, [_P, _I64, _P, _P]),
+    "convrot_linear_workspace_size": (_SZ, [_I64, _I64]),
+    "w8a8_convrot_linear": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _P, _P, _SZ, _P]),
+    "moe_workspace_layout": (_I, [_I64, _I64, _I64, _I, _I64, ctypes.POINTER(MoeLayout)]),
+    "moe_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I64]),
+    "moe_expert_choice_forward": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I64, _I, _I,
+                                       _P, _P, _SZ, _P]),
+}
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libconvrot.so and declares every C signature. Raises if missing."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise ImportError(
+                f"{path} is missing: build it with `python -m w8a8_rotated_int8_b200.build` "
+                "(there is no fallback implementation)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+def lib() -> ctypes.CDLL:
+    return _lib if _lib is not None else load_library()
+
+
+def status_string(status: int) -> str:
+    return lib().convrot_status_string(status).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != CONVROT_OK:
+        raise ConvrotError(rc, where)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ------------------------------------------------------------- diagnostics --
+def convrot_device_check():
+    _check(lib().convrot_device_check(), "convrot_device_check")
+
+
+def convrot_check_device_error(stream=None) -> int:
+    """Synchronises and returns the device error bits (0 = none); clears them."""
+    flags = ctypes.c_uint(0)
+    rc = lib().convrot_check_device_error(_stream(stream), ctypes.byref(flags))
+    if rc not in (CONVROT_OK, CONVROT_ERR_TIMEOUT):
+        raise ConvrotError(rc, "convrot_check_device_error")
+    return int(flags.value)
+
+
+def convrot_wait_selftest(limit_ns: int, stream=None) -> int:
+    """Runs the bounded-wait self-test; returns 0 when the wait gave up."""
+    res = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    _check(lib().convrot_wait_selftest(limit_ns, _p(res), _stream(stream)), "convrot_wait_selftest")
+    return int(res.item())
+
+
+# ------------------------------------------------------------------ stages --
+def convrot_rotquant(x, group, q=None, scale=None, stream=None):
+    """Rotate rows of x ([rows, K] bf16 or fp32) in groups of `group`, then
+    quantise per row. Returns (codes int8 [rows, K], scales fp32 [rows])."""
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("x must be bf16 or fp32")
+    _need(x, x.dtype, "x")
+    rows, k = x.shape
+    q = torch.empty((rows, k), dtype=torch.int8, device=x.device) if q is None else q
+    scale = torch.empty((rows,), dtype=torch.float32, device=x.device) if scale is None else scale
+    dt = DTYPE_BF16 if x.dtype == torch.bfloat16 else DTYPE_F32
+    _check(lib().convrot_rotquant(_p(x), dt, rows, k, group, _p(q), _p(scale), _stream(stream)),
+           "convrot_rotquant")
+    return q, scale
+
+
+def convrot_quantize_weights(w, group, stream=None):
+    """Offline quantisation of bf16 weight rows; [..., K] -> (codes, scales [...])."""
+    _need(w, torch.bfloat16, "w")
+    k = w.shape[-1]
+    rows = w.numel() // k
+    q = torch.empty(w.shape, dtype=torch.int8, device=w.device)
+    s = torch.empty(w.shape[:-1], dtype=torch.float32, device=w.device)
+    _check(lib().convrot_quantize_weights(_p(w), rows, k, group, _p(q), _p(s), _stream(stream)),
+           "convrot_quantize_weights")
+    return q, s
+
+
+def convrot_router_softmax(logits, stream=None):
+    """[T, E] bf16 logits -> transposed scores [E, T] fp32."""
+    _need(logits, torch.bfloat16, "logits")
+    t, e = logits.shape
+    s_t = torch.empty((e, t), dtype=torch.float32, device=logits.device)
+    _check(lib().convrot_router_softmax(_p(logits), t, e, _p(s_t), _stream(stream)),
+           "convrot_router_softmax")
+    return s_t
+
+
+def convrot_topc(s_t, c, stream=None):
+    """[E, T] fp32 scores -> (idx int32 [E, C], w fp32 [E, C])."""
+    _need(s_t, torch.float32, "s_t")
+    e, t = s_t.shape
+    idx = torch.empty((e, c), dtype=torch.int32, device=s_t.device)
+    w = torch.empty((e, c), dtype=torch.float32, device=s_t.device)
+    _check(lib().convrot_topc(_p(s_t), t, e, c, _p(idx), _p(w), _stream(stream)), "convrot_topc")
+    return idx, w
+
+
+def convrot_gather_rows(src, s_src, idx, stream=None):
+    _need(src, torch.int8, "src")
+    _need(s_src, torch.float32, "s_src")
+    _need(idx, torch.int32, "idx")
+    n_src, k = src.shape
+    n = idx.numel()
+    dst = torch.empty((n, k), dtype=torch.int8, device=src.device)
+    s_dst = torch.empty((n,), dtype=torch.float32, device=src.device)
+    _check(lib().convrot_gather_rows(_p(src), _p(s_src), n_src, _p(idx), n, k, _p(dst), _p(s_dst),
+                                     _stream(stream)), "convrot_gather_rows")
+    return dst, s_dst
+
+
+def _gemm_dims(a, b):
+    _need(a, torch.int8, "a")
+    _need(b, torch.int8, "b")
+    if a.dim() == 2:
+        a, b = a[None], b[None]
+    g, m, k = a.shape
+    gb, n, kb = b.shape
+    if gb != g or kb != k:
+        raise ValueError("a [G,M,K] and b [G,N,K] disagree")
+    return g, m, n, k
+
+
+def convrot_i8_gemm_i32(a, b, stream=None):
+    """Exact int32 acc[g, m, n] = sum_k a[g, m, k] b[g, n, k]."""
+    g, m, n, k = _gemm_dims(a, b)
+    d = torch.empty((g, m, n), dtype=torch.int32, device=a.device)
+    _check(lib().convrot_i8_gemm_i32(_p(a), _p(b), g, m, n, k, _p(d), _stream(stream)),
+           "convrot_i8_gemm_i32")
+    return d if a.dim() == 3 else d[0]
+
+
+def convrot_i8_gemm_bf16(a, s_a, b, s_b, stream=None):
+    g, m, n, k = _gemm_dims(a, b)
+    _need(s_a, torch.float32, "s_a")
+    _need(s_b, torch.float32, "s_b")
+    y = torch.empty((g, m, n), dtype=torch.bfloat16, device=a.device)
+    _check(lib().convrot_i8_gemm_bf16(_p(a), _p(s_a), _p(b), _p(s_b), g, m, n, k, _p(y),
+                                      _stream(stream)), "convrot_i8_gemm_bf16")
+    return y if a.dim() == 3 else y[0]
+
+
+def convrot_i8_gemm_swiglu(a, s_a, b, s_b, stream=None):
+    """b = [G, 2F, K] (gate rows then up rows) -> h [G, M, F] fp32."""
+    g, m, n2, k = _gemm_dims(a, b)
+    _need(s_a, torch.float32, "s_a")
+    _need(s_b, torch.float32, "s_b")
+    f = n2 // 2
+    h = torch.empty((g, m, f), dtype=torch.float32, device=a.device)
+    _check(lib().convrot_i8_gemm_swiglu(_p(a), _p(s_a), _p(b), _p(s_b), g, m, f, k, _p(h),
+                                        _stream(stream)), "convrot_i8_gemm_swiglu")
+    return h if a.dim() == 3 else h[0]
+
+
+def convrot_i8_gemm_scatter(a, s_a, b, s_b, idx, w, out32, stream=None):
+    """out32[idx[g, m], n] += w[g, m] * dequant(acc)[g, m, n] (in place)."""
+    g, m, n, k = _gemm_dims(a, b)
+    for t, nm in ((s_a, "s_a"), (s_b, "s_b"), (w, "w"), (out32, "out32")):
+        _need(t, torch.float32, nm)
+    _need(idx, torch.int32, "idx")
+    _check(lib().convrot_i8_gemm_scatter(_p(a), _p(s_a), _p(b), _p(s_b), _p(idx), _p(w), g, m, n,
+                                         k, _p(out32), out32.shape[0], _stream(stream)),
+           "convrot_i8_gemm_scatter")
+    return out32
+
+
+def convrot_f32_to_bf16(x, stream=None):
+    _need(x, torch.float32, "x")
+    y = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    _check(lib().convrot_f32_to_bf16(_p(x), x.numel(), _p(y), _stream(stream)),
+           "convrot_f32_to_bf16")
+    return y
+
+
+# ---------------------------------------------------------------- linears --
+def convrot_linear_workspace_size(m, k) -> int:
+    return int(lib().convrot_linear_workspace_size(m, k))
+
+
+def w8a8_convrot_linear(x, w_q, w_scale, group, y=None, workspace=None, stream=None):
+    """Y[M, N] bf16 = W8A8 ConvRot linear of x [M, K] bf16 with rotated codes w_q [N, K]."""
+    _need(x, torch.bfloat16, "x")
+    _need(w_q, torch.int8, "w_q")
+    _need(w_scale, torch.float32, "w_scale")
+    m, k = x.shape
+    n = w_q.shape[0]
+    ws_bytes = convrot_linear_workspace_size(m, k)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=x.device)
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    _check(lib().w8a8_convrot_linear(_p(x), m, k, _p(w_q), _p(w_scale), n, group, _p(y),
+                                     _p(workspace), workspace.numel(), _stream(stream)),
+           "w8a8_convrot_linear")
+    return y
+
+
+# -------------------------------------------------------------- MoE block --
+def moe_workspace_layout(t, d, f, e, c) -> dict:
+    lay = MoeLayout()
+    _check(lib().moe_workspace_layout(t, d, f, e, c, ctypes.byref(lay)), "moe_workspace_layout")
+    return {name: int(getattr(lay, name)) for name, _ in MoeLayout._fields_}
+
+
+def moe_workspace_size(t, d, f, e, c) -> int:
+    return int(lib().moe_workspace_size(t, d, f, e, c))
+
+
+def moe_expert_choice_forward(x, logits, w_gu, s_gu, w_d, s_d, c, g_gu=256, g_d=64, y=None,
+                              workspace=None, stream=None):
+    """Expert-choice W8A8 ConvRot MoE block. x [T, d] bf16, logits [T, E] bf16,
+    w_gu [E, 2f, d] int8, s_gu [E, 2f], w_d [E, d, f] int8, s_d [E, d] -> y [T, d] bf16."""
+    _need(x, torch.bfloat16, "x")
+    _need(logits, torch.bfloat16, "logits")
+    _need(w_gu, torch.int8, "w_gu")
+    _need(w_d, torch.int8, "w_d")
+    _need(s_gu, torch.float32, "s_gu")
+    _need(s_d, torch.float32, "s_d")
+    t, d = x.shape
+    e, two_f, _ = w_gu.shape
+    f = two_f // 2
+    size = moe_workspace_size(t, d, f, e, c)
+    if workspace is None:
+        workspace = torch.empty((max(size, 16),), dtype=torch.uint8, device=x.device)
+    if y is None:
+        y = torch.empty((t, d), dtype=torch.bfloat16, device=x.device)
+    _check(lib().moe_expert_choice_forward(_p(x), _p(logits), _p(w_gu), _p(s_gu), _p(w_d), _p(s_d),
+                                           t, d, f, e, c, g_gu, g_d, _p(y), _p(workspace),
+                                           workspace.numel(), _stream(stream)),
+           "moe_expert_choice_forward")
+    return y
+
+
+def moe_stage_views(workspace, t, d, f, e, c) -> dict:
+    """Typed views of every intermediate the MoE call leaves in its workspace."""
+    lay = moe_workspace_layout(t, d, f, e, c)
+
+    def view(name, dtype, shape):
+        n = 1
+        for s in shape:
+            n *= s
+        nbytes = n * torch.tensor([], dtype=dtype).element_size()
+        return workspace[lay[name]:lay[name] + nbytes].view(dtype).view(shape)
+
+    return {
+        "x_q": view("x_q", torch.int8, (t, d)),
+        "s_x": view("s_x", torch.float32, (t,)),
+        "s_t": view("s_t", torch.float32, (e, t)),
+        "idx": view("idx", torch.int32, (e, c)),
+        "w": view("w", torch.float32, (e, c)),
+        "x_g": view("x_g", torch.int8, (e, c, d)),
+        "s_g": view("s_g", torch.float32, (e, c)),
+        "h": view("h", torch.float32, (e, c, f)),
+        "h_q": view("h_q", torch.int8, (e, c, f)),
+        "s_h": view("s_h", torch.float32, (e, c)),
+        "out32": view("out32", torch.float32, (t, d)),
+    }

@@ -1,0 +1,553 @@
+// Host side of the C ABI declared in include/convrot.h: argument checks,
+// TMA tensor-map encoding, launch configuration, and the composition of the
+// W8A8 ConvRot linear and the expert-choice MoE block from the kernels.
+//
+// All kernels live in this one translation unit (the device error word is a
+// single __device__ variable without relocatable device code).
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/convrot.h"
+#include "common.cuh"
+#include "gemm_tcgen05.cuh"
+#include "rotquant.cuh"
+#include "routing.cuh"
+
+using namespace convrot;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  bool supported = false;
+  int sm_count = 0;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+template <typename InT, int G>
+void set_rq_attr() {
+  cudaFuncSetAttribute(rotquant_kernel<InT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       96 * 1024);
+}
+
+template <typename InT>
+void set_rq_attrs() {
+  set_rq_attr<InT, 1>();
+  set_rq_attr<InT, 4>();
+  set_rq_attr<InT, 16>();
+  set_rq_attr<InT, 64>();
+  set_rq_attr<InT, 256>();
+}
+
+// Per-device one-time setup: capability check, SM count, kernel attributes.
+int device_setup(int* sm_count) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return CONVROT_ERR_UNSUPPORTED_DEVICE;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return CONVROT_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return CONVROT_ERR_UNSUPPORTED_DEVICE;
+    }
+    d.supported = (major == 10 && minor == 0);
+    d.sm_count = sms;
+    if (d.supported) {
+      cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiI32>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+      cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiBf16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+      cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiSwiglu>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+      cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiScatter>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+      set_rq_attrs<__nv_bfloat16>();
+      set_rq_attrs<float>();
+      if (cudaGetLastError() != cudaSuccess) return CONVROT_ERR_CUDA;
+    }
+    d.ready = true;
+  }
+  if (!d.supported) return CONVROT_ERR_UNSUPPORTED_DEVICE;
+  if (sm_count) *sm_count = d.sm_count;
+  return CONVROT_OK;
+}
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool valid_group(int g) { return g == 1 || g == 4 || g == 16 || g == 64 || g == 256; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+// --------------------------------------------------------------- rotquant --
+template <typename InT, int G>
+void launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, cudaStream_t st) {
+  const int nch = K / 16;
+  int tpr;
+  if (nch <= 32) {
+    tpr = 1;
+    while (tpr < nch) tpr <<= 1;
+  } else {
+    tpr = (nch + 31) / 32 * 32;
+  }
+  const int threads = std::max(kRqThreads, tpr);
+  const int rpc = threads / tpr;
+  const size_t smem = 128 + (G >= 64 ? (size_t)rpc * K * 9 : 0);
+  const int64_t grid = (rows + rpc - 1) / rpc;
+  rotquant_kernel<InT, G><<<(unsigned)grid, threads, smem, st>>>(
+      reinterpret_cast<const InT*>(x), rows, K, tpr, q, s);
+}
+
+template <typename InT>
+void dispatch_rq(int group, const void* x, int64_t rows, int K, int8_t* q, float* s,
+                 cudaStream_t st) {
+  switch (group) {
+    case 1: launch_rq<InT, 1>(x, rows, K, q, s, st); break;
+    case 4: launch_rq<InT, 4>(x, rows, K, q, s, st); break;
+    case 16: launch_rq<InT, 16>(x, rows, K, q, s, st); break;
+    case 64: launch_rq<InT, 64>(x, rows, K, q, s, st); break;
+    default: launch_rq<InT, 256>(x, rows, K, q, s, st); break;
+  }
+}
+
+int check_rq_args(const void* x, int x_dtype, int64_t rows, int64_t K, int group, const int8_t* q,
+                  const float* s) {
+  if (x_dtype != CONVROT_DTYPE_BF16 && x_dtype != CONVROT_DTYPE_F32) return CONVROT_ERR_INVALID_ARG;
+  if (rows < 0 || rows >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
+  if (!valid_group(group)) return CONVROT_ERR_INVALID_ARG;
+  if (K < 16 || K > 8192 || K % 16 != 0 || K % group != 0) return CONVROT_ERR_INVALID_ARG;
+  if (rows > 0 && (!x || !q || !s)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(x) || !al16(q) || !al16(s)) return CONVROT_ERR_MISALIGNED;
+  return CONVROT_OK;
+}
+
+int rotquant_impl(const void* x, int x_dtype, int64_t rows, int64_t K, int group, int8_t* q,
+                  float* s, cudaStream_t st) {
+  if (rows == 0) return CONVROT_OK;
+  if (x_dtype == CONVROT_DTYPE_BF16)
+    dispatch_rq<__nv_bfloat16>(group, x, rows, (int)K, q, s, st);
+  else
+    dispatch_rq<float>(group, x, rows, (int)K, q, s, st);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ GEMM --
+int encode_3d_i8(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint64_t groups,
+                 uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return CONVROT_ERR_CUDA;
+  const cuuint64_t dims[3] = {K, rows, groups};
+  const cuuint64_t strides[2] = {K, K * rows};
+  const cuuint32_t box[3] = {(cuuint32_t)gemm::BK, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+int check_gemm_shape(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t NB,
+                     int64_t K) {
+  if (G < 0 || M < 0 || NB < 0 || K < 16) return CONVROT_ERR_INVALID_ARG;
+  if (G >= ((int64_t)1 << 31) || M >= ((int64_t)1 << 31) || NB >= ((int64_t)1 << 31))
+    return CONVROT_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K >= ((int64_t)1 << 31) || NB % 16 != 0) return CONVROT_ERR_INVALID_ARG;
+  if (K * 127 * 127 >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;  // int32 accumulator
+  if (G * M > 0 && (!a || !b)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(a) || !al16(b)) return CONVROT_ERR_MISALIGNED;
+  return CONVROT_OK;
+}
+
+template <int EPI>
+int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t NB, int64_t K,
+                int64_t n_out, GemmArgs args, cudaStream_t st) {
+  int sms = 0;
+  int rc = device_setup(&sms);
+  if (rc != CONVROT_OK) return rc;
+  if (G == 0 || M == 0 || n_out == 0) return CONVROT_OK;
+  CUtensorMap ta, tb;
+  const uint32_t box_a = (uint32_t)std::min<int64_t>(gemm::BM, M);
+  const uint32_t box_b = (uint32_t)std::min<int64_t>(gemm::BN / 2, NB);
+  if ((rc = encode_3d_i8(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)G, box_a)) != CONVROT_OK)
+    return rc;
+  if ((rc = encode_3d_i8(&tb, b, (uint64_t)K, (uint64_t)NB, (uint64_t)G, box_b)) != CONVROT_OK)
+    return rc;
+  args.G = (int)G;
+  args.M = (int)M;
+  args.NB = (int)NB;
+  args.K = (int)K;
+  args.n_out = (int)n_out;
+  args.m_blocks = (int)((M + gemm::BM - 1) / gemm::BM);
+  const int64_t n_tile = (EPI == kEpiSwiglu) ? gemm::BN / 2 : gemm::BN;
+  args.n_blocks = (int)((n_out + n_tile - 1) / n_tile);
+  args.k_blocks = (int)((K + gemm::BK - 1) / gemm::BK);
+  const int64_t tiles = G * args.m_blocks * args.n_blocks;
+  if (tiles >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
+  args.num_tiles = (int)tiles;
+  args.box_bytes = (int)((box_a + 2 * box_b) * gemm::BK);
+  const int grid = (int)std::min<int64_t>(tiles, sms);
+  gemm_s8_tcgen05_kernel<EPI><<<grid, gemm::THREADS, gemm::SMEM_BYTES, st>>>(ta, tb, args);
+  return launch_status();
+}
+
+int topc_impl(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float* w,
+              cudaStream_t st) {
+  if (C == 0 || E == 0) return CONVROT_OK;
+  topc_kernel<<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w);
+  return launch_status();
+}
+
+int softmax_impl(const void* logits, int64_t T, int E, float* s_t, float* clear,
+                 int64_t clear_cols, cudaStream_t st) {
+  if (T == 0) return CONVROT_OK;
+  const int64_t grid = (T + kSmTokens - 1) / kSmTokens;
+  router_softmax_kernel<<<(unsigned)grid, 256, (size_t)E * kSmTokens * sizeof(float), st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(logits), (int)T, E, s_t, clear, clear_cols);
+  return launch_status();
+}
+
+int gather_impl(const int8_t* src, const float* s_src, int64_t n_src, const int32_t* idx,
+                int64_t n_rows, int64_t K, int8_t* dst, float* s_dst, cudaStream_t st) {
+  if (n_rows == 0) return CONVROT_OK;
+  const int64_t grid = (n_rows + 7) / 8;
+  gather_rows_kernel<<<(unsigned)grid, 256, 0, st>>>(src, s_src, n_src, idx, n_rows, (int)K, dst,
+                                                      s_dst);
+  return launch_status();
+}
+
+int convert_impl(const float* x, int64_t n, void* y, int sms, cudaStream_t st) {
+  if (n == 0) return CONVROT_OK;
+  const int64_t n4 = n / 4;
+  const int64_t grid = std::min<int64_t>((n4 + 255) / 256, (int64_t)sms * 16);
+  f32_to_bf16_kernel<<<(unsigned)grid, 256, 0, st>>>(x, n4,
+                                                     reinterpret_cast<__nv_bfloat16*>(y));
+  return launch_status();
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+// ===================================================================== ABI ==
+extern "C" {
+
+int convrot_abi_version(void) { return 1; }
+
+const char* convrot_status_string(int status) {
+  switch (status) {
+    case CONVROT_OK: return "ok";
+    case CONVROT_ERR_INVALID_ARG: return "invalid argument";
+    case CONVROT_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs sm_100)";
+    case CONVROT_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case CONVROT_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case CONVROT_ERR_CUDA: return "CUDA error";
+    case CONVROT_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int convrot_device_check(void) { return device_setup(nullptr); }
+
+int convrot_check_device_error(void* stream, unsigned* flags) {
+  int rc = device_setup(nullptr);
+  if (rc != CONVROT_OK) return rc;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return CONVROT_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return CONVROT_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  if (flags) *flags = v;
+  return v ? CONVROT_ERR_TIMEOUT : CONVROT_OK;
+}
+
+int convrot_wait_selftest(unsigned long long limit_ns, int* result_dev, void* stream) {
+  int rc = device_setup(nullptr);
+  if (rc != CONVROT_OK) return rc;
+  if (!result_dev || limit_ns > 10000000000ull) return CONVROT_ERR_INVALID_ARG;
+  wait_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(limit_ns, result_dev);
+  return launch_status();
+}
+
+int convrot_rotquant(const void* x, int x_dtype, int64_t rows, int64_t K, int group, int8_t* q,
+                     float* scale, void* stream) {
+  int rc = check_rq_args(x, x_dtype, rows, K, group, q, scale);
+  if (rc != CONVROT_OK) return rc;
+  if ((rc = device_setup(nullptr)) != CONVROT_OK) return rc;
+  return rotquant_impl(x, x_dtype, rows, K, group, q, scale, as_stream(stream));
+}
+
+int convrot_quantize_weights(const void* w_bf16, int64_t rows, int64_t K, int group, int8_t* w_q,
+                             float* row_scale, void* stream) {
+  return convrot_rotquant(w_bf16, CONVROT_DTYPE_BF16, rows, K, group, w_q, row_scale, stream);
+}
+
+int convrot_router_softmax(const void* logits_bf16, int64_t T, int E, float* s_t, void* stream) {
+  if (T < 0 || T >= ((int64_t)1 << 31) || E < 1 || E > 256) return CONVROT_ERR_INVALID_ARG;
+  if (T > 0 && (!logits_bf16 || !s_t)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(logits_bf16) || !al16(s_t)) return CONVROT_ERR_MISALIGNED;
+  int rc = device_setup(nullptr);
+  if (rc != CONVROT_OK) return rc;
+  return softmax_impl(logits_bf16, T, E, s_t, nullptr, 0, as_stream(stream));
+}
+
+int convrot_topc(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float* w,
+                 void* stream) {
+  if (T < 0 || T >= ((int64_t)1 << 31) || E < 0 || E > 65535 || C < 0 || C > T)
+    return CONVROT_ERR_INVALID_ARG;
+  if (C > 0 && E > 0 && (!s_t || !idx || !w)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(s_t) || !al16(idx) || !al16(w)) return CONVROT_ERR_MISALIGNED;
+  int rc = device_setup(nullptr);
+  if (rc != CONVROT_OK) return rc;
+  return topc_impl(s_t, T, E, C, idx, w, as_stream(stream));
+}
+
+int convrot_gather_rows(const int8_t* src, const float* s_src, int64_t n_src, const int32_t* idx,
+                        int64_t n_rows, int64_t K, int8_t* dst, float* s_dst, void* stream) {
+  if (n_src < 0 || n_rows < 0 || K < 16 || K % 16 != 0 || K >= ((int64_t)1 << 31))
+    return CONVROT_ERR_INVALID_ARG;
+  if (n_rows > 0 && (!src || !s_src || !idx || !dst || !s_dst || n_src == 0))
+    return CONVROT_ERR_INVALID_ARG;
+  if (!al16(src) || !al16(dst)) return CONVROT_ERR_MISALIGNED;
+  int rc = device_setup(nullptr);
+  if (rc != CONVROT_OK) return rc;
+  return gather_impl(src, s_src, n_src, idx, n_rows, K, dst, s_dst, as_stream(stream));
+}
+
+int convrot_i8_gemm_i32(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t N,
+                        int64_t K, int32_t* d, void* stream) {
+  int rc = check_gemm_shape(a, b, G, M, N, K);
+  if (rc != CONVROT_OK) return rc;
+  if (G * M * N > 0 && !d) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(d)) return CONVROT_ERR_MISALIGNED;
+  GemmArgs args{};
+  args.out = d;
+  return launch_gemm<kEpiI32>(a, b, G, M, N, K, N, args, as_stream(stream));
+}
+
+int convrot_i8_gemm_bf16(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
+                         int64_t G, int64_t M, int64_t N, int64_t K, void* y_bf16, void* stream) {
+  int rc = check_gemm_shape(a, b, G, M, N, K);
+  if (rc != CONVROT_OK) return rc;
+  if (G * M * N > 0 && (!s_a || !s_b || !y_bf16)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(s_a) || !al16(s_b) || !al16(y_bf16)) return CONVROT_ERR_MISALIGNED;
+  GemmArgs args{};
+  args.s_a = s_a;
+  args.s_b = s_b;
+  args.out = y_bf16;
+  return launch_gemm<kEpiBf16>(a, b, G, M, N, K, N, args, as_stream(stream));
+}
+
+int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
+                           int64_t G, int64_t M, int64_t F, int64_t K, float* h, void* stream) {
+  if (F < 0 || F % 16 != 0) return CONVROT_ERR_INVALID_ARG;
+  int rc = check_gemm_shape(a, b, G, M, 2 * F, K);
+  if (rc != CONVROT_OK) return rc;
+  if (G * M * F > 0 && (!s_a || !s_b || !h)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(s_a) || !al16(s_b) || !al16(h)) return CONVROT_ERR_MISALIGNED;
+  GemmArgs args{};
+  args.s_a = s_a;
+  args.s_b = s_b;
+  args.out = h;
+  return launch_gemm<kEpiSwiglu>(a, b, G, M, 2 * F, K, F, args, as_stream(stream));
+}
+
+int convrot_i8_gemm_scatter(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
+                            const int32_t* idx, const float* w, int64_t G, int64_t M, int64_t N,
+                            int64_t K, float* out32, int64_t T, void* stream) {
+  int rc = check_gemm_shape(a, b, G, M, N, K);
+  if (rc != CONVROT_OK) return rc;
+  if (T < 0) return CONVROT_ERR_INVALID_ARG;
+  if (G * M * N > 0 && (!s_a || !s_b || !idx || !w || !out32 || T == 0))
+    return CONVROT_ERR_INVALID_ARG;
+  if (!al16(s_a) || !al16(s_b) || !al16(out32)) return CONVROT_ERR_MISALIGNED;
+  GemmArgs args{};
+  args.s_a = s_a;
+  args.s_b = s_b;
+  args.out = out32;
+  args.idx = idx;
+  args.w = w;
+  if (T >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
+  args.out_rows = (int)T;
+  return launch_gemm<kEpiScatter>(a, b, G, M, N, K, N, args, as_stream(stream));
+}
+
+int convrot_f32_to_bf16(const float* x, int64_t n, void* y_bf16, void* stream) {
+  if (n < 0 || n % 4 != 0) return CONVROT_ERR_INVALID_ARG;
+  if (n > 0 && (!x || !y_bf16)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(x) || ((uintptr_t)y_bf16 & 7u) != 0) return CONVROT_ERR_MISALIGNED;
+  int sms = 0;
+  int rc = device_setup(&sms);
+  if (rc != CONVROT_OK) return rc;
+  return convert_impl(x, n, y_bf16, sms, as_stream(stream));
+}
+
+size_t convrot_linear_workspace_size(int64_t M, int64_t K) {
+  if (M < 0 || K < 0) return 0;
+  return align256((size_t)M * (size_t)K) + align256((size_t)M * sizeof(float));
+}
+
+int w8a8_convrot_linear(const void* x_bf16, int64_t M, int64_t K, const int8_t* w_q,
+                        const float* w_scale, int64_t N, int group, void* y_bf16, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  int rc = check_rq_args(x_bf16, CONVROT_DTYPE_BF16, M, K, group, (const int8_t*)workspace,
+                         (const float*)workspace);
+  if (rc != CONVROT_OK) return rc;
+  if ((rc = check_gemm_shape(w_q, w_q, 1, M, N, K)) != CONVROT_OK) return rc;
+  if (M > 0 && N > 0 && (!w_scale || !y_bf16 || !workspace)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(w_scale) || !al16(y_bf16) || !al16(workspace)) return CONVROT_ERR_MISALIGNED;
+  if (ws_bytes < convrot_linear_workspace_size(M, K)) return CONVROT_ERR_WORKSPACE_TOO_SMALL;
+  if ((rc = device_setup(nullptr)) != CONVROT_OK) return rc;
+  if (M == 0 || N == 0) return CONVROT_OK;
+  cudaStream_t st = as_stream(stream);
+  int8_t* x_q = reinterpret_cast<int8_t*>(workspace);
+  float* s_x = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
+                                        align256((size_t)M * (size_t)K));
+  if ((rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, M, K, group, x_q, s_x, st)) != CONVROT_OK)
+    return rc;
+  GemmArgs args{};
+  args.s_a = s_x;
+  args.s_b = w_scale;
+  args.out = y_bf16;
+  return launch_gemm<kEpiBf16>(x_q, w_q, 1, M, N, K, N, args, st);
+}
+
+int moe_workspace_layout(int64_t T, int64_t d, int64_t f, int E, int64_t C,
+                         convrot_moe_layout_t* lay) {
+  if (!lay || T < 0 || d < 0 || f < 0 || E < 0 || C < 0) return CONVROT_ERR_INVALID_ARG;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t ec = (size_t)E * (size_t)C;
+  lay->x_q = take((size_t)T * d);
+  lay->s_x = take((size_t)T * 4);
+  lay->s_t = take((size_t)E * T * 4);
+  lay->idx = take(ec * 4);
+  lay->w = take(ec * 4);
+  lay->x_g = take(ec * d);
+  lay->s_g = take(ec * 4);
+  lay->h = take(ec * f * 4);
+  lay->h_q = take(ec * f);
+  lay->s_h = take(ec * 4);
+  lay->out32 = take((size_t)T * d * 4);
+  lay->total = off;
+  return CONVROT_OK;
+}
+
+size_t moe_workspace_size(int64_t T, int64_t d, int64_t f, int E, int64_t C) {
+  convrot_moe_layout_t lay;
+  if (moe_workspace_layout(T, d, f, E, C, &lay) != CONVROT_OK) return 0;
+  return lay.total;
+}
+
+int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const int8_t* w_gu,
+                              const float* s_gu, const int8_t* w_d, const float* s_d, int64_t T,
+                              int64_t d, int64_t f, int E, int64_t C, int g_gu, int g_d,
+                              void* y_bf16, void* workspace, size_t ws_bytes, void* stream) {
+  if (T < 0 || T >= ((int64_t)1 << 31) || E < 1 || E > 256 || C < 0 || C > T)
+    return CONVROT_ERR_INVALID_ARG;
+  if (!valid_group(g_gu) || !valid_group(g_d)) return CONVROT_ERR_INVALID_ARG;
+  if (d < 16 || d > 8192 || d % 16 != 0 || d % g_gu != 0) return CONVROT_ERR_INVALID_ARG;
+  if (f < 16 || f > 8192 || f % 16 != 0 || f % g_d != 0) return CONVROT_ERR_INVALID_ARG;
+  if ((int64_t)E * C >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
+  if (T > 0 && (!x_bf16 || !logits_bf16 || !w_gu || !s_gu || !w_d || !s_d || !y_bf16 ||
+                !workspace))
+    return CONVROT_ERR_INVALID_ARG;
+  if (!al16(x_bf16) || !al16(logits_bf16) || !al16(w_gu) || !al16(s_gu) || !al16(w_d) ||
+      !al16(s_d) || !al16(y_bf16) || !al16(workspace))
+    return CONVROT_ERR_MISALIGNED;
+  convrot_moe_layout_t lay;
+  moe_workspace_layout(T, d, f, E, C, &lay);
+  if (ws_bytes < lay.total) return CONVROT_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  int rc = device_setup(&sms);
+  if (rc != CONVROT_OK) return rc;
+  if (T == 0) return CONVROT_OK;
+  cudaStream_t st = as_stream(stream);
+  char* ws = reinterpret_cast<char*>(workspace);
+  int8_t* x_q = reinterpret_cast<int8_t*>(ws + lay.x_q);
+  float* s_x = reinterpret_cast<float*>(ws + lay.s_x);
+  float* s_t = reinterpret_cast<float*>(ws + lay.s_t);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + lay.idx);
+  float* w = reinterpret_cast<float*>(ws + lay.w);
+  int8_t* x_g = reinterpret_cast<int8_t*>(ws + lay.x_g);
+  float* s_g = reinterpret_cast<float*>(ws + lay.s_g);
+  float* h = reinterpret_cast<float*>(ws + lay.h);
+  int8_t* h_q = reinterpret_cast<int8_t*>(ws + lay.h_q);
+  float* s_h = reinterpret_cast<float*>(ws + lay.s_h);
+  float* out32 = reinterpret_cast<float*>(ws + lay.out32);
+
+  // 1. router softmax (also clears the combine accumulator)
+  if ((rc = softmax_impl(logits_bf16, T, E, s_t, out32, d, st)) != CONVROT_OK) return rc;
+  // 2. rotate + quantise the tokens once (the gate/up rotation is expert-independent)
+  if ((rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, T, d, g_gu, x_q, s_x, st)) != CONVROT_OK)
+    return rc;
+  if (C > 0) {
+    // 3. expert-choice top-C, 4. gather each expert's token codes
+    if ((rc = topc_impl(s_t, T, E, C, idx, w, st)) != CONVROT_OK) return rc;
+    if ((rc = gather_impl(x_q, s_x, T, idx, (int64_t)E * C, d, x_g, s_g, st)) != CONVROT_OK)
+      return rc;
+    // 5. gate/up GEMM with dequant + SwiGLU
+    GemmArgs a1{};
+    a1.s_a = s_g;
+    a1.s_b = s_gu;
+    a1.out = h;
+    if ((rc = launch_gemm<kEpiSwiglu>(x_g, w_gu, E, C, 2 * f, d, f, a1, st)) != CONVROT_OK)
+      return rc;
+    // 6. rotate (g_d) + requantise h per row
+    if ((rc = rotquant_impl(h, CONVROT_DTYPE_F32, (int64_t)E * C, f, g_d, h_q, s_h, st)) !=
+        CONVROT_OK)
+      return rc;
+    // 7. down GEMM with dequant and the router-weighted scatter-add
+    GemmArgs a2{};
+    a2.s_a = s_h;
+    a2.s_b = s_d;
+    a2.out = out32;
+    a2.idx = idx;
+    a2.w = w;
+    a2.out_rows = (int)T;
+    if ((rc = launch_gemm<kEpiScatter>(h_q, w_d, E, C, d, f, d, a2, st)) != CONVROT_OK) return rc;
+  }
+  // 8. one bf16 rounding of the fp32 combine
+  return convert_impl(out32, T * d, y_bf16, sms, st);
+}
+
+}  // extern "C"
