@@ -201,7 +201,7 @@ def test_gemm_swiglu(g, m, f, k):
         ulps = _fp32_ulps(h[gi], ref)
         # CUDA expf is within 2 ulp of exp: silu(g)*u within a few ulp
         assert ulps.max() <= 4
-        assert (ulps == 0).mean() > 0.9
+        assert (ulps == 0).mean() > 0.8  # expf differs from exp in ~1 of 10 elements
 
 
 def test_gemm_scatter():

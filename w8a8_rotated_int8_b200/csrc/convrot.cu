@@ -125,8 +125,9 @@ void launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, cudaStre
   } else {
     tpr = (nch + 31) / 32 * 32;
   }
-  const int threads = std::max(kRqThreads, tpr);
-  const int rpc = threads / tpr;
+  // whole rows per CTA: a CTA never holds threads beyond rpc * tpr
+  const int rpc = std::max(1, kRqThreads / tpr);
+  const int threads = rpc * tpr;
   const size_t smem = 128 + (G >= 64 ? (size_t)rpc * K * 9 : 0);
   const int64_t grid = (rows + rpc - 1) / rpc;
   rotquant_kernel<InT, G><<<(unsigned)grid, threads, smem, st>>>(

@@ -129,7 +129,7 @@ __device__ __forceinline__ double rq_row_max(double m, int tpr, double* red) {
 }
 
 // x: [rows, K] (bf16 or fp32), q: [rows, K] int8, scales: [rows] fp32.
-// blockDim.x = max(kRqThreads, tpr); each CTA handles blockDim.x / tpr rows.
+// blockDim.x = rows_per_cta * tpr exactly (rows_per_cta = max(1, 256 / tpr)).
 template <typename InT, int G>
 __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x, int64_t rows,
                                                       int K, int tpr, int8_t* __restrict__ q,
