@@ -21,9 +21,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -72,52 +70,67 @@ def algorithmic_work(cfg, t):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+    """SM clock and clock-event reasons sampled (read-only, NVML) by a thread
+    every ~2 ms while the timed region runs; nvidia-smi if NVML is missing."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.tmp = None
+    def __init__(self, torch_device):
+        import threading
+        self.dev = torch_device
+        self.samples = []
+        self.stop_evt = threading.Event()
+        self.thread = None
+        self.nvml = None
+        self.handle = None
+        self.max_mhz = None
+
+    def _open(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        self.nvml = pynvml
+
+    def _loop(self):
+        nv = self.nvml
+        while not self.stop_evt.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((mhz, rs))
+            except Exception:  # noqa: BLE001 - sampling is best effort
+                pass
+            self.stop_evt.wait(0.002)
 
     def start(self):
+        import threading
         try:
-            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.tmp, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            self._open()
+        except Exception:  # noqa: BLE001
+            self.nvml = None
+            return
+        self.thread = threading.Thread(target=self._loop, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.tmp.flush()
-        rows = []
-        with open(self.tmp.name) as fh:
-            for line in fh:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 8:
-                    rows.append(parts)
-        os.unlink(self.tmp.name)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+        if self.nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        self.stop_evt.set()
+        self.thread.join(timeout=5)
+        nv = self.nvml
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"]}
+        reasons = sorted({name for _, rs in self.samples for name, const in self.REASONS
+                          if rs & getattr(nv, const)})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
 
 
 def dist_setup():
@@ -149,53 +162,77 @@ def max_over_ranks(value, world):
 
 
 # ------------------------------------------------------------ CPU oracle ----
-def oracle_sample(cfg, inp, n_experts):
-    """Time the oracle on all routing + the first n_experts experts' FFN and
-    extrapolate the block time to all experts. Returns (seconds per block, info)."""
-    import threadpoolctl
-
+def oracle_weights(cfg, inp, n_experts):
+    """Offline oracle quantisation of the first n_experts experts (untimed)."""
     import oracle as O
-    x = inp["x"].float().numpy()
-    logits = inp["logits"].float().numpy()
     wgu_q = np.zeros((cfg.n_exp, 2 * cfg.f, cfg.d), np.int8)
     s_gu = np.zeros((cfg.n_exp, 2 * cfg.f), np.float32)
     wd_q = np.zeros((cfg.n_exp, cfg.d, cfg.f), np.int8)
     s_d = np.zeros((cfg.n_exp, cfg.d), np.float32)
-    for e in range(n_experts):  # offline weight quantisation: not timed
+    for e in range(n_experts):
         wgu_q[e], s_gu[e] = O.rotquant(inp["wgu"][e].float().numpy(), cfg.g_gu)
         wd_q[e], s_d[e] = O.rotquant(inp["wd"][e].float().numpy(), cfg.g_d)
+    return wgu_q, s_gu, wd_q, s_d
+
+
+def oracle_cores():
+    import threadpoolctl
+    threads = max((i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()), default=1)
+    return min(threads, len(os.sched_getaffinity(0)))
+
+
+def oracle_block_time(cfg, inp, weights, n_experts):
+    """Seconds for one oracle block call restricted to the first n_experts
+    experts' FFN (all routing included), extrapolated per expert to all."""
+    import oracle as O
+    x = inp["x"].float().numpy()
+    logits = inp["logits"].float().numpy()
     t0 = time.perf_counter()
-    O.moe_block(x, logits, wgu_q, s_gu, wd_q, s_d, cfg.c, cfg.g_gu, cfg.g_d, experts=[])
+    O.moe_block(x, logits, *weights, cfg.c, cfg.g_gu, cfg.g_d, experts=[])
     t_route = time.perf_counter() - t0
     t0 = time.perf_counter()
-    O.moe_block(x, logits, wgu_q, s_gu, wd_q, s_d, cfg.c, cfg.g_gu, cfg.g_d,
-                experts=list(range(n_experts)))
+    O.moe_block(x, logits, *weights, cfg.c, cfg.g_gu, cfg.g_d, experts=list(range(n_experts)))
     t_sample = time.perf_counter() - t0
     per_expert = max(t_sample - t_route, 0.0) / n_experts
-    block_s = t_route + per_expert * cfg.n_exp
-    threads = max((i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()), default=1)
-    cores = min(threads, len(os.sched_getaffinity(0)))
-    info = {"kind": "oracle", "cores": cores,
-            "sample": (f"oracle block on {cfg.name} inputs: all routing + FFN of experts "
-                       f"0..{n_experts - 1} of {cfg.n_exp} timed ({t_sample:.1f} s), "
-                       f"extrapolated per expert to the full block")}
-    return block_s, info
+    return t_route + per_expert * cfg.n_exp, t_route + t_sample
+
+
+def cpu_baseline(cfg, inp, target_s=12.0):
+    """The oracle as it stands, full blocks (all experts) repeated until about
+    target_s of CPU work; tokens/s over those blocks."""
+    import oracle as O
+    weights = oracle_weights(cfg, inp, cfg.n_exp)
+    x = inp["x"].float().numpy()
+    logits = inp["logits"].float().numpy()
+    reps, spent = 0, 0.0
+    while spent < target_s and reps < 16:
+        t0 = time.perf_counter()
+        O.moe_block(x, logits, *weights, cfg.c, cfg.g_gu, cfg.g_d)
+        spent += time.perf_counter() - t0
+        reps += 1
+    return {"kind": "oracle", "cores": oracle_cores(), "value": reps * cfg.t / spent, "unit": UNIT,
+            "sample": f"{reps} full oracle block(s) on {cfg.name} inputs ({spent:.1f} s of CPU work)"}
 
 
 def run_reference(args, cfg, world, rank):
+    """The oracle timed on the host cores; one step = routing + a quarter of
+    the experts' FFN, extrapolated per expert to the whole block."""
     if rank != 0:
         return
     inp = moe_inputs(cfg)
-    times = []
-    info = None
+    n_exp = max(1, cfg.n_exp // 4)
+    weights = oracle_weights(cfg, inp, n_exp)
+    times, spent = [], 0.0
     for _ in range(args.warmup + args.steps):
-        block_s, info = oracle_sample(cfg, inp, n_experts=1)
+        block_s, cpu_s = oracle_block_time(cfg, inp, weights, n_exp)
         times.append(block_s)
-    timed = times[args.warmup:]
-    block_s = statistics.mean(timed)
+        spent += cpu_s
+    block_s = statistics.mean(times[args.warmup:])
     value = cfg.t / block_s
-    info["value"] = value
-    info["unit"] = UNIT
+    info = {"kind": "oracle", "cores": oracle_cores(), "value": value, "unit": UNIT,
+            "sample": (f"per step: routing of all {cfg.t} tokens + FFN of experts 0..{n_exp - 1} "
+                       f"of {cfg.n_exp} on {cfg.name} inputs, extrapolated per expert to the full "
+                       f"block ({spent:.1f} s of CPU work in total)")}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": block_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64/int64",
@@ -291,8 +328,7 @@ def run_ours(args, cfg, world, rank, local):
     if W.convrot_check_device_error() != 0:
         raise RuntimeError("device-side wait timed out during warm-up")
 
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                          else local)
+    clocks = ClockSampler(dev)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
@@ -392,10 +428,7 @@ def run_ours(args, cfg, world, rank, local):
         "wall_s": wall,
     }
     if args.cpu_baseline and world == 1:
-        block_s, info = oracle_sample(cfg, inp, n_experts=1)
-        info["value"] = cfg.t / block_s
-        info["unit"] = UNIT
-        line["cpu_baseline"] = info
+        line["cpu_baseline"] = cpu_baseline(cfg, inp)
     print(json.dumps(line), flush=True)
 
 
