@@ -173,6 +173,34 @@ int w8a8_convrot_linear(const void* x_bf16, int64_t M, int64_t K, const int8_t* 
                         size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * W8A8 ConvRot linear that allocates nothing and takes no workspace.
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot hand the library device memory for scratch: a host program that owns
+ * only its input and output buffers and no device allocator, a serving loop
+ * where cudaMalloc/cudaFree would synchronise the device and stall the other
+ * streams, or a process whose device-memory budget is fixed at start-up.
+ * Same arguments and result as w8a8_convrot_linear minus the workspace. The
+ * activation codes and token scales go to one static device array of this
+ * library (CONVROT_NOALLOC_MAX_CODES code bytes + CONVROT_NOALLOC_MAX_ROWS
+ * fp32 scales, about 8.1 MiB), which every GPU that loads the library keeps
+ * until the process exits.
+ *  - M * K > CONVROT_NOALLOC_MAX_CODES or M > CONVROT_NOALLOC_MAX_ROWS:
+ *    returns CONVROT_ERR_WORKSPACE_TOO_SMALL and launches nothing.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, no allocation) with that device current; make
+ *    that first call before any stream capture.
+ *  - All calls share the one array: calls that can overlap on the GPU
+ *    (different streams, or host threads without ordering) race on it; order
+ *    them on one stream. Nothing in the array needs to start at zero (every
+ *    code and scale the GEMM reads is written by the same call first).
+ * ------------------------------------------------------------------------- */
+#define CONVROT_NOALLOC_MAX_CODES 8388608
+#define CONVROT_NOALLOC_MAX_ROWS 16384
+int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const int8_t* w_q,
+                                const float* w_scale, int64_t N, int group, void* y_bf16,
+                                void* stream);
+
+/* ---------------------------------------------------------------------------
  * Expert-choice W8A8 ConvRot MoE block (one call = the whole hot path).
  * "MLX Nucleus-Image", opening paragraph and table "Conversion notes";
  * "Nucleus-Image INT8 Convrot Experts + FP8 Text Encoder", "Quantization".

@@ -28,4 +28,5 @@ from .binding import (  # noqa: F401
     moe_workspace_layout,
     moe_workspace_size,
     w8a8_convrot_linear,
+    w8a8_convrot_linear_noalloc,
 )

@@ -66,6 +66,7 @@ _SIGNATURES = {
     "convrot_f32_to_bf16": (_I, [_P, _I64, _P, _P]),
     "convrot_linear_workspace_size": (_SZ, [_I64, _I64]),
     "w8a8_convrot_linear": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _P, _P, _SZ, _P]),
+    "w8a8_convrot_linear_noalloc": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _P, _P]),
     "moe_workspace_layout": (_I, [_I64, _I64, _I64, _I, _I64, ctypes.POINTER(MoeLayout)]),
     "moe_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I64]),
     "moe_expert_choice_forward": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I64, _I, _I,
@@ -288,6 +289,23 @@ def w8a8_convrot_linear(x, w_q, w_scale, group, y=None, workspace=None, stream=N
     _check(lib().w8a8_convrot_linear(_p(x), m, k, _p(w_q), _p(w_scale), n, group, _p(y),
                                      _p(workspace), workspace.numel(), _stream(stream)),
            "w8a8_convrot_linear")
+    return y
+
+
+def w8a8_convrot_linear_noalloc(x, w_q, w_scale, group, y=None, stream=None):
+    """The W8A8 ConvRot linear with the library's static scratch instead of a
+    workspace, for callers that cannot give the library device memory.
+    M * K <= 8,388,608 and M <= 16,384; calls sharing the scratch must be
+    ordered on one stream."""
+    _need(x, torch.bfloat16, "x")
+    _need(w_q, torch.int8, "w_q")
+    _need(w_scale, torch.float32, "w_scale")
+    m, k = x.shape
+    n = w_q.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    _check(lib().w8a8_convrot_linear_noalloc(_p(x), m, k, _p(w_q), _p(w_scale), n, group, _p(y),
+                                             _stream(stream)), "w8a8_convrot_linear_noalloc")
     return y
 
 

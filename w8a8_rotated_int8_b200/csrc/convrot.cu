@@ -552,3 +552,70 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
 }
 
 }  // extern "C"
+
+// ======================================================= no-allocation ==
+// Scratch of w8a8_convrot_linear_noalloc: activation codes then token scales,
+// one file-scope device array reserved on every GPU that loads the library.
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[CONVROT_NOALLOC_MAX_CODES + CONVROT_NOALLOC_MAX_ROWS * sizeof(float)];
+
+namespace {
+
+struct NoAllocSlot {
+  bool ready = false;
+  void* ptr = nullptr;
+};
+NoAllocSlot g_noalloc_slot[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array for the current device, looked up once
+// per device (host code cannot use the array's name as a device pointer).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return CONVROT_ERR_UNSUPPORTED_DEVICE;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocSlot& slot = g_noalloc_slot[dev];
+  if (!slot.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return CONVROT_ERR_CUDA;
+    }
+    slot.ptr = p;
+    slot.ready = true;
+  }
+  *out = slot.ptr;
+  return CONVROT_OK;
+}
+
+}  // namespace
+
+extern "C" int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_t K,
+                                           const int8_t* w_q, const float* w_scale, int64_t N,
+                                           int group, void* y_bf16, void* stream) {
+  if (M < 0 || K < 0) return CONVROT_ERR_INVALID_ARG;
+  if (M > CONVROT_NOALLOC_MAX_ROWS || M * K > (int64_t)CONVROT_NOALLOC_MAX_CODES)
+    return CONVROT_ERR_WORKSPACE_TOO_SMALL;
+  int rc = check_rq_args(x_bf16, CONVROT_DTYPE_BF16, M, K, group, w_q, w_scale);
+  if (rc != CONVROT_OK) return rc;
+  if ((rc = check_gemm_shape(w_q, w_q, 1, M, N, K)) != CONVROT_OK) return rc;
+  if (M > 0 && N > 0 && (!w_scale || !y_bf16)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(w_scale) || !al16(y_bf16)) return CONVROT_ERR_MISALIGNED;
+  if ((rc = device_setup(nullptr)) != CONVROT_OK) return rc;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch)) != CONVROT_OK) return rc;
+  if (M == 0 || N == 0) return CONVROT_OK;
+  cudaStream_t st = as_stream(stream);
+  int8_t* x_q = reinterpret_cast<int8_t*>(scratch);
+  float* s_x = reinterpret_cast<float*>(reinterpret_cast<char*>(scratch) + CONVROT_NOALLOC_MAX_CODES);
+  if ((rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, M, K, group, x_q, s_x, st)) != CONVROT_OK)
+    return rc;
+  GemmArgs args{};
+  args.s_a = s_x;
+  args.s_b = w_scale;
+  args.out = y_bf16;
+  return launch_gemm<kEpiBf16>(x_q, w_q, 1, M, N, K, N, args, st);
+}
