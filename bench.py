@@ -249,7 +249,9 @@ def stage_times(W, ws_views, inp_dev, wq, cfg, t, reps, flush_buf):
     """Device time of every stage, launched through its own C-ABI entry with
     the block's real intermediates, CUDA events on the launching stream."""
     v = ws_views
-    wgu_q, s_gu, wd_q, s_d = wq
+    gu, dn = wq
+    wgu_q, s_gu, wd_q, s_d = gu.data, gu.scale, dn.data, dn.scale
+    tiles = W.binding.LAYOUT_TILES
     stream = torch.cuda.current_stream()
     stages = {
         "router_softmax": lambda: W.binding.lib().convrot_router_softmax(
@@ -265,13 +267,13 @@ def stage_times(W, ws_views, inp_dev, wq, cfg, t, reps, flush_buf):
             W.binding._stream()),
         "gemm_gateup_swiglu": lambda: W.binding.lib().convrot_i8_gemm_swiglu(
             W.binding._p(v["x_g"]), W.binding._p(v["s_g"]), W.binding._p(wgu_q),
-            W.binding._p(s_gu), cfg.n_exp, cfg.c, cfg.f, cfg.d, W.binding._p(v["h"]),
+            W.binding._p(s_gu), tiles, cfg.n_exp, cfg.c, cfg.f, cfg.d, W.binding._p(v["h"]),
             W.binding._stream()),
         "rotquant_h": lambda: W.convrot_rotquant(v["h"].view(-1, cfg.f), cfg.g_d,
                                                  q=v["h_q"].view(-1, cfg.f), scale=v["s_h"].view(-1)),
         "gemm_down_scatter": lambda: W.binding.lib().convrot_i8_gemm_scatter(
             W.binding._p(v["h_q"]), W.binding._p(v["s_h"]), W.binding._p(wd_q),
-            W.binding._p(s_d), W.binding._p(v["idx"]), W.binding._p(v["w"]), cfg.n_exp, cfg.c,
+            W.binding._p(s_d), tiles, W.binding._p(v["idx"]), W.binding._p(v["w"]), cfg.n_exp, cfg.c,
             cfg.d, cfg.f, W.binding._p(v["out32"]), t, W.binding._stream()),
         "f32_to_bf16": lambda: W.binding.lib().convrot_f32_to_bf16(
             W.binding._p(v["out32"]), t * cfg.d, W.binding._p(inp_dev["y"]), W.binding._stream()),
@@ -306,9 +308,8 @@ def run_ours(args, cfg, world, rank, local):
         gen = torch.Generator().manual_seed(cfg.seed * 1000 + rank)
         inp["x"] = (torch.randn(t, cfg.d, generator=gen) * inp["x"].float().std()).to(torch.bfloat16)
         inp["logits"] = torch.randn(t, cfg.n_exp, generator=gen).to(torch.bfloat16)
-    wgu_q, s_gu = W.convrot_quantize_weights(inp["wgu"].to(dev), cfg.g_gu)
-    wd_q, s_d = W.convrot_quantize_weights(inp["wd"].to(dev), cfg.g_d)
-    wq = (wgu_q, s_gu, wd_q, s_d)
+    gu, dn = W.quantize_moe_weights(inp["wgu"].to(dev), inp["wd"].to(dev), cfg.g_gu, cfg.g_d)
+    wq = (gu, dn)
     x = inp["x"].to(dev)
     logits = inp["logits"].to(dev)
     y = torch.empty((t, cfg.d), dtype=torch.bfloat16, device=dev)
@@ -318,8 +319,7 @@ def run_ours(args, cfg, world, rank, local):
     stream = torch.cuda.current_stream()
 
     def step(xx, ll, yy):
-        W.moe_expert_choice_forward(xx, ll, wgu_q, s_gu, wd_q, s_d, cfg.c, cfg.g_gu, cfg.g_d,
-                                    y=yy, workspace=ws)
+        W.moe_expert_choice_forward(xx, ll, gu, dn, cfg.c, cfg.g_gu, cfg.g_d, y=yy, workspace=ws)
 
     for _ in range(args.warmup):
         flush_buf.zero_()

@@ -60,6 +60,18 @@ enum {
 
 enum { CONVROT_DTYPE_BF16 = 0, CONVROT_DTYPE_F32 = 1 };
 
+/* Storage of an int8 weight operand B:
+ *  CONVROT_LAYOUT_ROWS   row-major [G, N, K] (K-contiguous);
+ *  CONVROT_LAYOUT_TILES  the tiled weight format written by
+ *      convrot_quantize_weights_tiled: every matrix is cut into 128-row blocks
+ *      (the last one zero-padded), every block into 128-byte K tiles (the last
+ *      one zero-padded); tile (block rb, k-tile kb) is 16 KB at byte offset
+ *      (rb * ceil(K/128) + kb) * 16384 and holds 128 rows of 128 bytes. Blocks
+ *      of consecutive matrices follow each other. Each GEMM K-step then reads
+ *      whole 16 KB runs of DRAM. For a SwiGLU operand each group holds two
+ *      matrices of F rows (gate, then up). */
+enum { CONVROT_LAYOUT_ROWS = 0, CONVROT_LAYOUT_TILES = 1 };
+
 /* Version of this ABI (incremented on incompatible changes). */
 int convrot_abi_version(void);
 
@@ -102,6 +114,19 @@ int convrot_rotquant(const void* x, int x_dtype, int64_t rows, int64_t K, int gr
 int convrot_quantize_weights(const void* w_bf16, int64_t rows, int64_t K, int group,
                              int8_t* w_q, float* row_scale, void* stream);
 
+/* Offline weight quantisation into the tiled weight format (see
+ * CONVROT_LAYOUT_TILES): n_mats matrices of `rows` x K bf16 rows, stored
+ * back to back in w_bf16 ([n_mats * rows, K]). The codes and per-row scales
+ * equal those of convrot_quantize_weights; only their placement differs.
+ *   w_tiled    device, convrot_tiled_weight_bytes(n_mats, rows, K) bytes
+ *              (padding is written as zero codes)
+ *   row_scale  device, [n_mats * rows] fp32
+ * A MoE gate/up stack [E, 2f, d] is n_mats = 2E matrices of f rows; a down
+ * stack [E, d, f] is n_mats = E matrices of d rows. */
+int64_t convrot_tiled_weight_bytes(int64_t n_mats, int64_t rows, int64_t K);
+int convrot_quantize_weights_tiled(const void* w_bf16, int64_t n_mats, int64_t rows, int64_t K,
+                                   int group, int8_t* w_tiled, float* row_scale, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Router softmax. "MLX Nucleus-Image", opening paragraph (expert-choice).
  *   logits  device, [T, E] bf16;  1 <= E <= 256
@@ -129,31 +154,36 @@ int convrot_gather_rows(const int8_t* src, const float* s_src, int64_t n_src, co
 /* ---------------------------------------------------------------------------
  * Grouped INT8 GEMMs on the tcgen05 tensor cores (exact int32 accumulation).
  * For every group g: acc[g, m, n] = sum_k a[g, m, k] * b[g, n, k].
- *   a  device, [G, M, K] int8;  b device, [G, N, K] int8 (K-contiguous)
+ *   a         device, [G, M, K] int8 (K-contiguous)
+ *   b         device, int8 weights of G matrices of N rows, stored as
+ *             b_layout says (CONVROT_LAYOUT_ROWS: [G, N, K]; TILES: the tiled
+ *             weight format, G matrices, or 2G for the SwiGLU call)
  *   K % 16 == 0, 16 <= K;  N % 16 == 0;  G, M, N < 2^31
  * ------------------------------------------------------------------------- */
 
 /* acc stored as int32 d [G, M, N]. */
-int convrot_i8_gemm_i32(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t N,
-                        int64_t K, int32_t* d, void* stream);
+int convrot_i8_gemm_i32(const int8_t* a, const int8_t* b, int b_layout, int64_t G, int64_t M,
+                        int64_t N, int64_t K, int32_t* d, void* stream);
 
 /* y[g, m, n] = bf16(fp32(acc) * (s_b[g, n] * s_a[g, m])); s_a [G, M], s_b [G, N]. */
 int convrot_i8_gemm_bf16(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
-                         int64_t G, int64_t M, int64_t N, int64_t K, void* y_bf16, void* stream);
+                         int b_layout, int64_t G, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                         void* stream);
 
 /* SwiGLU epilogue: b = [G, 2F, K] with gate rows 0..F-1 and up rows F..2F-1,
  * s_b [G, 2F]. h[g, m, f] = silu(y[g, m, f]) * y[g, m, F + f] in fp32 with
  * y = fp32(acc) * (s_b * s_a); h device [G, M, F] fp32; F % 16 == 0. */
 int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
-                           int64_t G, int64_t M, int64_t F, int64_t K, float* h, void* stream);
+                           int b_layout, int64_t G, int64_t M, int64_t F, int64_t K, float* h,
+                           void* stream);
 
 /* Router-weighted scatter epilogue:
  * out32[idx[g, m], n] += w[g, m] * (fp32(acc) * (s_b[g, n] * s_a[g, m])).
  * out32 device [T, N] fp32 (accumulated with fp32 atomics, order not fixed);
  * idx [G, M] int32 in [0, T); w [G, M] fp32. */
 int convrot_i8_gemm_scatter(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
-                            const int32_t* idx, const float* w, int64_t G, int64_t M, int64_t N,
-                            int64_t K, float* out32, int64_t T, void* stream);
+                            int b_layout, const int32_t* idx, const float* w, int64_t G, int64_t M,
+                            int64_t N, int64_t K, float* out32, int64_t T, void* stream);
 
 /* y = bf16(x) (nearest even), n elements, n % 4 == 0. */
 int convrot_f32_to_bf16(const float* x, int64_t n, void* y_bf16, void* stream);
@@ -205,9 +235,12 @@ int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const 
  * "MLX Nucleus-Image", opening paragraph and table "Conversion notes";
  * "Nucleus-Image INT8 Convrot Experts + FP8 Text Encoder", "Quantization".
  *   x       device, [T, d] bf16;  logits device, [T, E] bf16
- *   w_gu    device, [E, 2f, d] int8 (rows 0..f-1 gate, f..2f-1 up), rotated g_gu
- *   s_gu    device, [E, 2f] fp32
- *   w_d     device, [E, d, f] int8, rotated g_d;  s_d device, [E, d] fp32
+ *   w_gu    device, gate/up codes rotated with g_gu in the tiled weight format:
+ *           2E matrices of f rows x d (expert e: gate = matrix 2e, up = 2e+1),
+ *           convrot_tiled_weight_bytes(2E, f, d) bytes
+ *   s_gu    device, [E, 2f] fp32 (gate rows then up rows per expert)
+ *   w_d     device, down codes rotated with g_d in the tiled weight format:
+ *           E matrices of d rows x f;  s_d device, [E, d] fp32
  *   C       tokens per expert, 0 <= C <= T
  *   y       device, [T, d] bf16 = bf16(sum over experts that chose t of
  *           w[e, c] * down_e(requant(silu(gate_e) * up_e)))

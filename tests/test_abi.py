@@ -61,9 +61,13 @@ def test_argument_checks_need_no_gpu(lib):
     # top-C capacity beyond T
     assert lib.convrot_topc(al, 10, 4, 11, al, al, None) == INVALID
     # GEMM: K not a multiple of 16, N not a multiple of 16, int32 overflow bound
-    assert lib.convrot_i8_gemm_i32(al, al, 1, 8, 16, 40, al, None) == INVALID
-    assert lib.convrot_i8_gemm_i32(al, al, 1, 8, 24, 64, al, None) == INVALID
-    assert lib.convrot_i8_gemm_i32(al, al, 1, 8, 16, 1 << 20, al, None) == INVALID
+    assert lib.convrot_i8_gemm_i32(al, al, 0, 1, 8, 16, 40, al, None) == INVALID
+    assert lib.convrot_i8_gemm_i32(al, al, 0, 1, 8, 24, 64, al, None) == INVALID
+    assert lib.convrot_i8_gemm_i32(al, al, 0, 1, 8, 16, 1 << 20, al, None) == INVALID
+    assert lib.convrot_i8_gemm_i32(al, al, 2, 1, 8, 16, 64, al, None) == INVALID  # bad layout
+    # tiled weight sizes: 128-row blocks x 128-byte K tiles of 16 KB
+    assert lib.convrot_tiled_weight_bytes(2, 300, 200) == 2 * 3 * 2 * 16384
+    assert lib.convrot_tiled_weight_bytes(128, 1536, 2048) == 128 * 12 * 16 * 16384
     # MoE: C > T, bad group, d not a multiple of g_gu, workspace too small
     args = [al] * 6
     assert lib.moe_expert_choice_forward(*args, 8, 256, 64, 4, 9, 256, 64, al, al, 1 << 30, None) == INVALID

@@ -153,13 +153,38 @@ def _codes(shape, seed):
     return torch.randint(-127, 128, shape, generator=g, dtype=torch.int8)
 
 
+def _tiled_codes(b):
+    """Place row-major codes [G, N, K] in the tiled weight format (test-side,
+    plain tensor reshapes) and wrap them like convrot_quantize_weights_tiled."""
+    g, n, k = b.shape
+    rb, kb = -(-n // 128), -(-k // 128)
+    pad = torch.zeros((g, rb * 128, kb * 128), dtype=torch.int8)
+    pad[:, :n, :k] = b
+    data = pad.view(g, rb, 128, kb, 128).permute(0, 1, 3, 2, 4).contiguous().view(-1)
+    return W.TiledWeights(data.cuda(), None, g, n, k)
+
+
+@pytest.mark.parametrize("layout", ["rows", "tiles"])
 @pytest.mark.parametrize("g,m,n,k", GEMM_SHAPES)
-def test_gemm_int32_bit_exact(g, m, n, k):
+def test_gemm_int32_bit_exact(g, m, n, k, layout):
     a = _codes((g, m, k), 1 + m)
     b = _codes((g, n, k), 2 + n)
-    d = W.convrot_i8_gemm_i32(a.cuda(), b.cuda()).cpu().numpy()
+    bb = b.cuda() if layout == "rows" else _tiled_codes(b)
+    d = W.convrot_i8_gemm_i32(a.cuda(), bb).cpu().numpy()
     for gi in range(g):
         assert np.array_equal(d[gi], O.int_gemm(a[gi].numpy(), b[gi].numpy()))
+
+
+def test_tiled_weight_quantisation_matches_row_major():
+    w = bf16_activations(3 * 200, 320, seed=5)
+    rows_q, rows_s = W.convrot_quantize_weights(w.cuda(), 64)
+    tw = W.convrot_quantize_weights_tiled(w.cuda(), 64, n_mats=3)
+    assert torch.equal(W.untile(tw), rows_q)
+    assert torch.equal(tw.scale, rows_s)
+    # padding rows (200..255 of each matrix) and columns (320..383) are zero
+    full = tw.data.view(3, 2, 3, 128, 128)
+    assert int(full[:, 1, :, 72:, :].abs().sum()) == 0
+    assert int(full[:, :, 2, :, 64:].abs().sum()) == 0
 
 
 def test_gemm_int32_extremes():
@@ -188,13 +213,15 @@ def _fp32_ulps(x, ref):
     return np.abs(x.astype(np.float64) - ref) / np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
 
 
+@pytest.mark.parametrize("layout", ["rows", "tiles"])
 @pytest.mark.parametrize("g,m,f,k", [(2, 160, 320, 768), (1, 64, 1536, 2048), (3, 40, 192, 512)])
-def test_gemm_swiglu(g, m, f, k):
+def test_gemm_swiglu(g, m, f, k, layout):
     a = _codes((g, m, k), 5)
     b = _codes((g, 2 * f, k), 6)
     s_a = torch.rand(g, m) * 0.05 + 1e-3
     s_b = torch.rand(g, 2 * f) * 1e-4 + 1e-6
-    h = W.convrot_i8_gemm_swiglu(a.cuda(), s_a.cuda(), b.cuda(), s_b.cuda()).cpu().numpy()
+    bb = b.cuda() if layout == "rows" else _tiled_codes(b.view(2 * g, f, k))
+    h = W.convrot_i8_gemm_swiglu(a.cuda(), s_a.cuda(), bb, s_b.cuda()).cpu().numpy()
     for gi in range(g):
         y = O.dequant(O.int_gemm(a[gi].numpy(), b[gi].numpy()), s_b[gi].numpy(), s_a[gi].numpy())
         ref = (O.silu_f32(y[:, :f]) * y[:, f:]).astype(np.float32)
@@ -204,7 +231,8 @@ def test_gemm_swiglu(g, m, f, k):
         assert (ulps == 0).mean() > 0.8  # expf differs from exp in ~1 of 10 elements
 
 
-def test_gemm_scatter():
+@pytest.mark.parametrize("layout", ["rows", "tiles"])
+def test_gemm_scatter(layout):
     g, m, n, k, t = 4, 100, 320, 512, 150
     a = _codes((g, m, k), 7)
     b = _codes((g, n, k), 8)
@@ -219,7 +247,8 @@ def test_gemm_scatter():
     for gi in range(g):
         z = O.dequant(O.int_gemm(a[gi].numpy(), b[gi].numpy()), s_b[gi].numpy(), s_a[gi].numpy())
         ref[idx[gi].numpy()] += w[gi].numpy()[:, None] * z
-    out_gpu = W.convrot_i8_gemm_scatter(a.cuda(), s_a.cuda(), b.cuda(), s_b.cuda(), idx.cuda(),
+    bb = b.cuda() if layout == "rows" else _tiled_codes(b)
+    out_gpu = W.convrot_i8_gemm_scatter(a.cuda(), s_a.cuda(), bb, s_b.cuda(), idx.cuda(),
                                         w.cuda(), out.cuda()).cpu().numpy()
     # fp32 sums of <= 4 terms in another order: within 4 ulps of the largest term
     assert np.max(np.abs(out_gpu - ref)) <= 4 * np.spacing(np.float32(np.abs(ref).max()))
@@ -248,9 +277,11 @@ def test_linear_empty_batch():
 
 # -------------------------------------------------------------- MoE block --
 def _quantise_moe_on_gpu(inp, cfg):
-    wgu_q, s_gu = W.convrot_quantize_weights(inp["wgu"].cuda(), cfg.g_gu)
-    wd_q, s_d = W.convrot_quantize_weights(inp["wd"].cuda(), cfg.g_d)
-    return wgu_q, s_gu, wd_q, s_d
+    """Tiled weights for the block, plus row-major views of the same codes."""
+    gu, dn = W.quantize_moe_weights(inp["wgu"].cuda(), inp["wd"].cuda(), cfg.g_gu, cfg.g_d)
+    views = (W.untile(gu).view(cfg.n_exp, 2 * cfg.f, cfg.d), gu.scale.view(cfg.n_exp, 2 * cfg.f),
+             W.untile(dn).view(cfg.n_exp, cfg.d, cfg.f), dn.scale.view(cfg.n_exp, cfg.d))
+    return (gu, dn), views
 
 
 def _oracle_weights(inp, cfg, experts):
@@ -267,14 +298,14 @@ def _oracle_weights(inp, cfg, experts):
 
 def _run_moe(inp, cfg, t=None):
     t = cfg.t if t is None else t
-    wgu_q, s_gu, wd_q, s_d = _quantise_moe_on_gpu(inp, cfg)
+    (gu, dn), wq = _quantise_moe_on_gpu(inp, cfg)
     ws = torch.empty(W.moe_workspace_size(t, cfg.d, cfg.f, cfg.n_exp, cfg.c), dtype=torch.uint8,
                      device="cuda")
-    y = W.moe_expert_choice_forward(inp["x"].cuda(), inp["logits"].cuda(), wgu_q, s_gu, wd_q, s_d,
-                                    cfg.c, cfg.g_gu, cfg.g_d, workspace=ws)
+    y = W.moe_expert_choice_forward(inp["x"].cuda(), inp["logits"].cuda(), gu, dn, cfg.c,
+                                    cfg.g_gu, cfg.g_d, workspace=ws)
     torch.cuda.synchronize()
     views = W.moe_stage_views(ws, t, cfg.d, cfg.f, cfg.n_exp, cfg.c)
-    return y, views, (wgu_q, s_gu, wd_q, s_d)
+    return y, views, wq
 
 
 def _max_rel(y, ref):

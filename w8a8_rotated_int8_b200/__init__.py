@@ -7,6 +7,7 @@ the library; the first call does, and raises if it is missing.
 
 from .binding import (  # noqa: F401
     ConvrotError,
+    TiledWeights,
     LIB_PATH,
     convrot_check_device_error,
     convrot_device_check,
@@ -18,6 +19,7 @@ from .binding import (  # noqa: F401
     convrot_i8_gemm_swiglu,
     convrot_linear_workspace_size,
     convrot_quantize_weights,
+    convrot_quantize_weights_tiled,
     convrot_rotquant,
     convrot_router_softmax,
     convrot_topc,
@@ -27,6 +29,9 @@ from .binding import (  # noqa: F401
     moe_stage_views,
     moe_workspace_layout,
     moe_workspace_size,
+    quantize_moe_weights,
+    tiled_weight_bytes,
+    untile,
     w8a8_convrot_linear,
     w8a8_convrot_linear_noalloc,
 )

@@ -27,6 +27,8 @@ CONVROT_ERR_CUDA = 5
 CONVROT_ERR_TIMEOUT = 6
 DTYPE_BF16 = 0
 DTYPE_F32 = 1
+LAYOUT_ROWS = 0
+LAYOUT_TILES = 1
 
 
 class ConvrotError(RuntimeError):
@@ -56,13 +58,16 @@ _SIGNATURES = {
     "convrot_wait_selftest": (_I, [ctypes.c_ulonglong, _P, _P]),
     "convrot_rotquant": (_I, [_P, _I, _I64, _I64, _I, _P, _P, _P]),
     "convrot_quantize_weights": (_I, [_P, _I64, _I64, _I, _P, _P, _P]),
+    "convrot_tiled_weight_bytes": (_I64, [_I64, _I64, _I64]),
+    "convrot_quantize_weights_tiled": (_I, [_P, _I64, _I64, _I64, _I, _P, _P, _P]),
     "convrot_router_softmax": (_I, [_P, _I64, _I, _P, _P]),
     "convrot_topc": (_I, [_P, _I64, _I, _I64, _P, _P, _P]),
     "convrot_gather_rows": (_I, [_P, _P, _I64, _P, _I64, _I64, _P, _P, _P]),
-    "convrot_i8_gemm_i32": (_I, [_P, _P, _I64, _I64, _I64, _I64, _P, _P]),
-    "convrot_i8_gemm_bf16": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P]),
-    "convrot_i8_gemm_swiglu": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P]),
-    "convrot_i8_gemm_scatter": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _I64, _P]),
+    "convrot_i8_gemm_i32": (_I, [_P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
+    "convrot_i8_gemm_bf16": (_I, [_P, _P, _P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
+    "convrot_i8_gemm_swiglu": (_I, [_P, _P, _P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
+    "convrot_i8_gemm_scatter": (_I, [_P, _P, _P, _P, _I, _P, _P, _I64, _I64, _I64, _I64, _P, _I64,
+                                     _P]),
     "convrot_f32_to_bf16": (_I, [_P, _I64, _P, _P]),
     "convrot_linear_workspace_size": (_SZ, [_I64, _I64]),
     "w8a8_convrot_linear": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _P, _P, _SZ, _P]),
@@ -173,6 +178,42 @@ def convrot_quantize_weights(w, group, stream=None):
     return q, s
 
 
+def tiled_weight_bytes(n_mats, rows, k) -> int:
+    return int(lib().convrot_tiled_weight_bytes(n_mats, rows, k))
+
+
+class TiledWeights:
+    """Codes in the tiled weight format plus their per-row scales."""
+
+    def __init__(self, data, scale, n_mats, rows, k):
+        self.data, self.scale, self.n_mats, self.rows, self.k = data, scale, n_mats, rows, k
+
+
+def convrot_quantize_weights_tiled(w, group, n_mats, stream=None):
+    """Quantise bf16 rows (n_mats matrices stacked along rows) into the tiled
+    weight format. Returns TiledWeights(data uint8-bytes as int8, scale)."""
+    _need(w, torch.bfloat16, "w")
+    k = w.shape[-1]
+    total = w.numel() // k
+    if total % n_mats:
+        raise ValueError("rows must split evenly into n_mats matrices")
+    rows = total // n_mats
+    data = torch.empty((tiled_weight_bytes(n_mats, rows, k),), dtype=torch.int8, device=w.device)
+    scale = torch.empty((total,), dtype=torch.float32, device=w.device)
+    _check(lib().convrot_quantize_weights_tiled(_p(w), n_mats, rows, k, group, _p(data), _p(scale),
+                                                _stream(stream)), "convrot_quantize_weights_tiled")
+    return TiledWeights(data, scale, n_mats, rows, k)
+
+
+def untile(tw: TiledWeights):
+    """Row-major [n_mats * rows, K] view of tiled codes (a copy; for checks)."""
+    kb = -(-tw.k // 128)
+    rb = -(-tw.rows // 128)
+    t = tw.data.view(tw.n_mats, rb, kb, 128, 128).permute(0, 1, 3, 2, 4)
+    t = t.reshape(tw.n_mats, rb * 128, kb * 128)[:, :tw.rows, :tw.k]
+    return t.reshape(tw.n_mats * tw.rows, tw.k)
+
+
 def convrot_router_softmax(logits, stream=None):
     """[T, E] bf16 logits -> transposed scores [E, T] fp32."""
     _need(logits, torch.bfloat16, "logits")
@@ -206,57 +247,67 @@ def convrot_gather_rows(src, s_src, idx, stream=None):
     return dst, s_dst
 
 
-def _gemm_dims(a, b):
+def _gemm_dims(a, b, swiglu=False):
+    """(G, M, N, K, b pointer tensor, layout). b is a row-major [G, N, K]
+    (or [N, K]) int8 tensor or TiledWeights."""
     _need(a, torch.int8, "a")
-    _need(b, torch.int8, "b")
     if a.dim() == 2:
-        a, b = a[None], b[None]
+        a = a[None]
     g, m, k = a.shape
+    if isinstance(b, TiledWeights):
+        per = 2 if swiglu else 1
+        if b.n_mats != g * per or b.k != k:
+            raise ValueError("tiled weights do not match a [G,M,K]")
+        return g, m, b.rows * per, k, b.data, LAYOUT_TILES
+    _need(b, torch.int8, "b")
+    if b.dim() == 2:
+        b = b[None]
     gb, n, kb = b.shape
     if gb != g or kb != k:
         raise ValueError("a [G,M,K] and b [G,N,K] disagree")
-    return g, m, n, k
+    return g, m, n, k, b, LAYOUT_ROWS
 
 
 def convrot_i8_gemm_i32(a, b, stream=None):
     """Exact int32 acc[g, m, n] = sum_k a[g, m, k] b[g, n, k]."""
-    g, m, n, k = _gemm_dims(a, b)
+    g, m, n, k, bt, lay = _gemm_dims(a, b)
     d = torch.empty((g, m, n), dtype=torch.int32, device=a.device)
-    _check(lib().convrot_i8_gemm_i32(_p(a), _p(b), g, m, n, k, _p(d), _stream(stream)),
+    _check(lib().convrot_i8_gemm_i32(_p(a), _p(bt), lay, g, m, n, k, _p(d), _stream(stream)),
            "convrot_i8_gemm_i32")
     return d if a.dim() == 3 else d[0]
 
 
 def convrot_i8_gemm_bf16(a, s_a, b, s_b, stream=None):
-    g, m, n, k = _gemm_dims(a, b)
+    g, m, n, k, bt, lay = _gemm_dims(a, b)
     _need(s_a, torch.float32, "s_a")
     _need(s_b, torch.float32, "s_b")
     y = torch.empty((g, m, n), dtype=torch.bfloat16, device=a.device)
-    _check(lib().convrot_i8_gemm_bf16(_p(a), _p(s_a), _p(b), _p(s_b), g, m, n, k, _p(y),
+    _check(lib().convrot_i8_gemm_bf16(_p(a), _p(s_a), _p(bt), _p(s_b), lay, g, m, n, k, _p(y),
                                       _stream(stream)), "convrot_i8_gemm_bf16")
     return y if a.dim() == 3 else y[0]
 
 
 def convrot_i8_gemm_swiglu(a, s_a, b, s_b, stream=None):
-    """b = [G, 2F, K] (gate rows then up rows) -> h [G, M, F] fp32."""
-    g, m, n2, k = _gemm_dims(a, b)
+    """b = [G, 2F, K] (gate rows then up rows) or tiled (2G matrices of F
+    rows) -> h [G, M, F] fp32."""
+    g, m, n2, k, bt, lay = _gemm_dims(a, b, swiglu=True)
     _need(s_a, torch.float32, "s_a")
     _need(s_b, torch.float32, "s_b")
     f = n2 // 2
     h = torch.empty((g, m, f), dtype=torch.float32, device=a.device)
-    _check(lib().convrot_i8_gemm_swiglu(_p(a), _p(s_a), _p(b), _p(s_b), g, m, f, k, _p(h),
+    _check(lib().convrot_i8_gemm_swiglu(_p(a), _p(s_a), _p(bt), _p(s_b), lay, g, m, f, k, _p(h),
                                         _stream(stream)), "convrot_i8_gemm_swiglu")
     return h if a.dim() == 3 else h[0]
 
 
 def convrot_i8_gemm_scatter(a, s_a, b, s_b, idx, w, out32, stream=None):
     """out32[idx[g, m], n] += w[g, m] * dequant(acc)[g, m, n] (in place)."""
-    g, m, n, k = _gemm_dims(a, b)
+    g, m, n, k, bt, lay = _gemm_dims(a, b)
     for t, nm in ((s_a, "s_a"), (s_b, "s_b"), (w, "w"), (out32, "out32")):
         _need(t, torch.float32, nm)
     _need(idx, torch.int32, "idx")
-    _check(lib().convrot_i8_gemm_scatter(_p(a), _p(s_a), _p(b), _p(s_b), _p(idx), _p(w), g, m, n,
-                                         k, _p(out32), out32.shape[0], _stream(stream)),
+    _check(lib().convrot_i8_gemm_scatter(_p(a), _p(s_a), _p(bt), _p(s_b), lay, _p(idx), _p(w), g, m,
+                                         n, k, _p(out32), out32.shape[0], _stream(stream)),
            "convrot_i8_gemm_scatter")
     return out32
 
@@ -320,19 +371,27 @@ def moe_workspace_size(t, d, f, e, c) -> int:
     return int(lib().moe_workspace_size(t, d, f, e, c))
 
 
-def moe_expert_choice_forward(x, logits, w_gu, s_gu, w_d, s_d, c, g_gu=256, g_d=64, y=None,
+def quantize_moe_weights(wgu, wd, g_gu=256, g_d=64, stream=None):
+    """Offline: bf16 wgu [E, 2f, d] and wd [E, d, f] -> tiled codes + scales."""
+    e, two_f, d = wgu.shape
+    gu = convrot_quantize_weights_tiled(wgu.reshape(e * two_f, d), g_gu, 2 * e, stream=stream)
+    dn = convrot_quantize_weights_tiled(wd.reshape(-1, wd.shape[-1]), g_d, e, stream=stream)
+    return gu, dn
+
+
+def moe_expert_choice_forward(x, logits, w_gu, w_d, c, g_gu=256, g_d=64, y=None,
                               workspace=None, stream=None):
     """Expert-choice W8A8 ConvRot MoE block. x [T, d] bf16, logits [T, E] bf16,
-    w_gu [E, 2f, d] int8, s_gu [E, 2f], w_d [E, d, f] int8, s_d [E, d] -> y [T, d] bf16."""
+    w_gu / w_d = TiledWeights from quantize_moe_weights -> y [T, d] bf16."""
     _need(x, torch.bfloat16, "x")
     _need(logits, torch.bfloat16, "logits")
-    _need(w_gu, torch.int8, "w_gu")
-    _need(w_d, torch.int8, "w_d")
-    _need(s_gu, torch.float32, "s_gu")
-    _need(s_d, torch.float32, "s_d")
     t, d = x.shape
-    e, two_f, _ = w_gu.shape
-    f = two_f // 2
+    e = logits.shape[1]
+    f = w_gu.rows
+    if w_gu.n_mats != 2 * e or w_gu.k != d or w_d.n_mats != e or w_d.rows != d or w_d.k != f:
+        raise ValueError("weights do not match x / logits")
+    s_gu, s_d = w_gu.scale, w_d.scale
+    w_gu, w_d = w_gu.data, w_d.data
     size = moe_workspace_size(t, d, f, e, c)
     if workspace is None:
         workspace = torch.empty((max(size, 16),), dtype=torch.uint8, device=x.device)

@@ -10,7 +10,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/convrot.h"
+#include "convrot.h"
 #include "common.cuh"
 #include "gemm_tcgen05.cuh"
 #include "rotquant.cuh"
@@ -65,6 +65,18 @@ void set_rq_attrs() {
   set_rq_attr<InT, 256>();
 }
 
+template <bool BT>
+void set_gemm_attrs() {
+  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiI32, BT>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiBf16, BT>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiSwiglu, BT>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiScatter, BT>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+}
+
 // Per-device one-time setup: capability check, SM count, kernel attributes.
 int device_setup(int* sm_count) {
   int dev = 0;
@@ -86,14 +98,8 @@ int device_setup(int* sm_count) {
     d.supported = (major == 10 && minor == 0);
     d.sm_count = sms;
     if (d.supported) {
-      cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiI32>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
-      cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiBf16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
-      cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiSwiglu>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
-      cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiScatter>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+      set_gemm_attrs<false>();
+      set_gemm_attrs<true>();
       set_rq_attrs<__nv_bfloat16>();
       set_rq_attrs<float>();
       if (cudaGetLastError() != cudaSuccess) return CONVROT_ERR_CUDA;
@@ -116,7 +122,8 @@ int launch_status() {
 
 // --------------------------------------------------------------- rotquant --
 template <typename InT, int G>
-void launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, cudaStream_t st) {
+void launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
+               cudaStream_t st) {
   const int nch = K / 16;
   int tpr;
   if (nch <= 32) {
@@ -131,18 +138,18 @@ void launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, cudaStre
   const size_t smem = 128 + (G >= 64 ? (size_t)rpc * K * 9 : 0);
   const int64_t grid = (rows + rpc - 1) / rpc;
   rotquant_kernel<InT, G><<<(unsigned)grid, threads, smem, st>>>(
-      reinterpret_cast<const InT*>(x), rows, K, tpr, q, s);
+      reinterpret_cast<const InT*>(x), rows, K, tpr, q, s, out);
 }
 
 template <typename InT>
-void dispatch_rq(int group, const void* x, int64_t rows, int K, int8_t* q, float* s,
+void dispatch_rq(int group, const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
                  cudaStream_t st) {
   switch (group) {
-    case 1: launch_rq<InT, 1>(x, rows, K, q, s, st); break;
-    case 4: launch_rq<InT, 4>(x, rows, K, q, s, st); break;
-    case 16: launch_rq<InT, 16>(x, rows, K, q, s, st); break;
-    case 64: launch_rq<InT, 64>(x, rows, K, q, s, st); break;
-    default: launch_rq<InT, 256>(x, rows, K, q, s, st); break;
+    case 1: launch_rq<InT, 1>(x, rows, K, q, s, out, st); break;
+    case 4: launch_rq<InT, 4>(x, rows, K, q, s, out, st); break;
+    case 16: launch_rq<InT, 16>(x, rows, K, q, s, out, st); break;
+    case 64: launch_rq<InT, 64>(x, rows, K, q, s, out, st); break;
+    default: launch_rq<InT, 256>(x, rows, K, q, s, out, st); break;
   }
 }
 
@@ -158,13 +165,20 @@ int check_rq_args(const void* x, int x_dtype, int64_t rows, int64_t K, int group
 }
 
 int rotquant_impl(const void* x, int x_dtype, int64_t rows, int64_t K, int group, int8_t* q,
-                  float* s, cudaStream_t st) {
+                  float* s, cudaStream_t st, RqOut out = RqOut{0, 1, 1, 1}) {
   if (rows == 0) return CONVROT_OK;
   if (x_dtype == CONVROT_DTYPE_BF16)
-    dispatch_rq<__nv_bfloat16>(group, x, rows, (int)K, q, s, st);
+    dispatch_rq<__nv_bfloat16>(group, x, rows, (int)K, q, s, out, st);
   else
-    dispatch_rq<float>(group, x, rows, (int)K, q, s, st);
+    dispatch_rq<float>(group, x, rows, (int)K, q, s, out, st);
   return launch_status();
+}
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Bytes of the tiled weight format for n_mats matrices of `rows` x K.
+int64_t tiled_bytes(int64_t n_mats, int64_t rows, int64_t K) {
+  return n_mats * cdiv(rows, 128) * cdiv(K, 128) * 16384;
 }
 
 // ------------------------------------------------------------------ GEMM --
@@ -195,7 +209,24 @@ int check_gemm_shape(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int
   return CONVROT_OK;
 }
 
-template <int EPI>
+int encode_tiled_b(CUtensorMap* map, const void* base, uint64_t kb_count, uint64_t row_blocks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return CONVROT_ERR_CUDA;
+  const cuuint64_t dims[4] = {128, 128, kb_count, row_blocks};
+  const cuuint64_t strides[3] = {128, 16384, 16384 * kb_count};
+  const cuuint32_t box[4] = {128, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+// NB = rows of one B matrix per group (2F for SwiGLU). With BT the B operand
+// is in the tiled weight format: for SwiGLU each group holds a gate matrix and
+// an up matrix of F rows, each padded to 128-row blocks.
+template <int EPI, bool BT>
 int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t NB, int64_t K,
                 int64_t n_out, GemmArgs args, cudaStream_t st) {
   int sms = 0;
@@ -204,27 +235,46 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
   if (G == 0 || M == 0 || n_out == 0) return CONVROT_OK;
   CUtensorMap ta, tb;
   const uint32_t box_a = (uint32_t)std::min<int64_t>(gemm::BM, M);
-  const uint32_t box_b = (uint32_t)std::min<int64_t>(gemm::BN / 2, NB);
+  uint32_t box_b;
   if ((rc = encode_3d_i8(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)G, box_a)) != CONVROT_OK)
     return rc;
-  if ((rc = encode_3d_i8(&tb, b, (uint64_t)K, (uint64_t)NB, (uint64_t)G, box_b)) != CONVROT_OK)
-    return rc;
+  if (BT) {
+    const int64_t blocks = (EPI == kEpiSwiglu) ? cdiv(n_out, 128) : cdiv(NB, 128);
+    const int64_t per_group = (EPI == kEpiSwiglu) ? 2 * blocks : blocks;
+    args.b_blocks = (int)blocks;
+    box_b = 128;
+    if ((rc = encode_tiled_b(&tb, b, (uint64_t)cdiv(K, 128), (uint64_t)(G * per_group))) !=
+        CONVROT_OK)
+      return rc;
+  } else {
+    box_b = (uint32_t)std::min<int64_t>(gemm::BN / 2, NB);
+    if ((rc = encode_3d_i8(&tb, b, (uint64_t)K, (uint64_t)NB, (uint64_t)G, box_b)) != CONVROT_OK)
+      return rc;
+  }
   args.G = (int)G;
   args.M = (int)M;
   args.NB = (int)NB;
   args.K = (int)K;
   args.n_out = (int)n_out;
-  args.m_blocks = (int)((M + gemm::BM - 1) / gemm::BM);
+  args.m_blocks = (int)cdiv(M, gemm::BM);
   const int64_t n_tile = (EPI == kEpiSwiglu) ? gemm::BN / 2 : gemm::BN;
-  args.n_blocks = (int)((n_out + n_tile - 1) / n_tile);
-  args.k_blocks = (int)((K + gemm::BK - 1) / gemm::BK);
+  args.n_blocks = (int)cdiv(n_out, n_tile);
+  args.k_blocks = (int)cdiv(K, gemm::BK);
   const int64_t tiles = G * args.m_blocks * args.n_blocks;
   if (tiles >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
   args.num_tiles = (int)tiles;
   args.box_bytes = (int)((box_a + 2 * box_b) * gemm::BK);
   const int grid = (int)std::min<int64_t>(tiles, sms);
-  gemm_s8_tcgen05_kernel<EPI><<<grid, gemm::THREADS, gemm::SMEM_BYTES, st>>>(ta, tb, args);
+  gemm_s8_tcgen05_kernel<EPI, BT><<<grid, gemm::THREADS, gemm::SMEM_BYTES, st>>>(ta, tb, args);
   return launch_status();
+}
+
+template <int EPI>
+int launch_gemm_layout(int b_layout, const int8_t* a, const int8_t* b, int64_t G, int64_t M,
+                       int64_t NB, int64_t K, int64_t n_out, GemmArgs args, cudaStream_t st) {
+  if (b_layout == CONVROT_LAYOUT_TILES)
+    return launch_gemm<EPI, true>(a, b, G, M, NB, K, n_out, args, st);
+  return launch_gemm<EPI, false>(a, b, G, M, NB, K, n_out, args, st);
 }
 
 int topc_impl(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float* w,
@@ -318,6 +368,27 @@ int convrot_quantize_weights(const void* w_bf16, int64_t rows, int64_t K, int gr
   return convrot_rotquant(w_bf16, CONVROT_DTYPE_BF16, rows, K, group, w_q, row_scale, stream);
 }
 
+int64_t convrot_tiled_weight_bytes(int64_t n_mats, int64_t rows, int64_t K) {
+  if (n_mats < 0 || rows < 0 || K < 0) return -1;
+  return tiled_bytes(n_mats, rows, K);
+}
+
+int convrot_quantize_weights_tiled(const void* w_bf16, int64_t n_mats, int64_t rows, int64_t K,
+                                   int group, int8_t* w_tiled, float* row_scale, void* stream) {
+  if (n_mats < 0 || rows < 0 || n_mats * rows >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
+  int rc = check_rq_args(w_bf16, CONVROT_DTYPE_BF16, n_mats * rows, K, group, w_tiled, row_scale);
+  if (rc != CONVROT_OK) return rc;
+  if ((rc = device_setup(nullptr)) != CONVROT_OK) return rc;
+  if (n_mats * rows == 0) return CONVROT_OK;
+  cudaStream_t st = as_stream(stream);
+  // padding rows and K columns of the last tiles read as zero codes
+  if (cudaMemsetAsync(w_tiled, 0, (size_t)tiled_bytes(n_mats, rows, K), st) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  const RqOut out{1, rows, (int)cdiv(rows, 128), (int)cdiv(K, 128)};
+  return rotquant_impl(w_bf16, CONVROT_DTYPE_BF16, n_mats * rows, K, group, w_tiled, row_scale, st,
+                       out);
+}
+
 int convrot_router_softmax(const void* logits_bf16, int64_t T, int E, float* s_t, void* stream) {
   if (T < 0 || T >= ((int64_t)1 << 31) || E < 1 || E > 256) return CONVROT_ERR_INVALID_ARG;
   if (T > 0 && (!logits_bf16 || !s_t)) return CONVROT_ERR_INVALID_ARG;
@@ -350,19 +421,24 @@ int convrot_gather_rows(const int8_t* src, const float* s_src, int64_t n_src, co
   return gather_impl(src, s_src, n_src, idx, n_rows, K, dst, s_dst, as_stream(stream));
 }
 
-int convrot_i8_gemm_i32(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t N,
-                        int64_t K, int32_t* d, void* stream) {
+int convrot_i8_gemm_i32(const int8_t* a, const int8_t* b, int b_layout, int64_t G, int64_t M,
+                        int64_t N, int64_t K, int32_t* d, void* stream) {
+  if (b_layout != CONVROT_LAYOUT_ROWS && b_layout != CONVROT_LAYOUT_TILES)
+    return CONVROT_ERR_INVALID_ARG;
   int rc = check_gemm_shape(a, b, G, M, N, K);
   if (rc != CONVROT_OK) return rc;
   if (G * M * N > 0 && !d) return CONVROT_ERR_INVALID_ARG;
   if (!al16(d)) return CONVROT_ERR_MISALIGNED;
   GemmArgs args{};
   args.out = d;
-  return launch_gemm<kEpiI32>(a, b, G, M, N, K, N, args, as_stream(stream));
+  return launch_gemm_layout<kEpiI32>(b_layout, a, b, G, M, N, K, N, args, as_stream(stream));
 }
 
 int convrot_i8_gemm_bf16(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
-                         int64_t G, int64_t M, int64_t N, int64_t K, void* y_bf16, void* stream) {
+                         int b_layout, int64_t G, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                         void* stream) {
+  if (b_layout != CONVROT_LAYOUT_ROWS && b_layout != CONVROT_LAYOUT_TILES)
+    return CONVROT_ERR_INVALID_ARG;
   int rc = check_gemm_shape(a, b, G, M, N, K);
   if (rc != CONVROT_OK) return rc;
   if (G * M * N > 0 && (!s_a || !s_b || !y_bf16)) return CONVROT_ERR_INVALID_ARG;
@@ -371,11 +447,14 @@ int convrot_i8_gemm_bf16(const int8_t* a, const float* s_a, const int8_t* b, con
   args.s_a = s_a;
   args.s_b = s_b;
   args.out = y_bf16;
-  return launch_gemm<kEpiBf16>(a, b, G, M, N, K, N, args, as_stream(stream));
+  return launch_gemm_layout<kEpiBf16>(b_layout, a, b, G, M, N, K, N, args, as_stream(stream));
 }
 
 int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
-                           int64_t G, int64_t M, int64_t F, int64_t K, float* h, void* stream) {
+                           int b_layout, int64_t G, int64_t M, int64_t F, int64_t K, float* h,
+                           void* stream) {
+  if (b_layout != CONVROT_LAYOUT_ROWS && b_layout != CONVROT_LAYOUT_TILES)
+    return CONVROT_ERR_INVALID_ARG;
   if (F < 0 || F % 16 != 0) return CONVROT_ERR_INVALID_ARG;
   int rc = check_gemm_shape(a, b, G, M, 2 * F, K);
   if (rc != CONVROT_OK) return rc;
@@ -385,12 +464,15 @@ int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, c
   args.s_a = s_a;
   args.s_b = s_b;
   args.out = h;
-  return launch_gemm<kEpiSwiglu>(a, b, G, M, 2 * F, K, F, args, as_stream(stream));
+  return launch_gemm_layout<kEpiSwiglu>(b_layout, a, b, G, M, 2 * F, K, F, args,
+                                        as_stream(stream));
 }
 
 int convrot_i8_gemm_scatter(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
-                            const int32_t* idx, const float* w, int64_t G, int64_t M, int64_t N,
-                            int64_t K, float* out32, int64_t T, void* stream) {
+                            int b_layout, const int32_t* idx, const float* w, int64_t G, int64_t M,
+                            int64_t N, int64_t K, float* out32, int64_t T, void* stream) {
+  if (b_layout != CONVROT_LAYOUT_ROWS && b_layout != CONVROT_LAYOUT_TILES)
+    return CONVROT_ERR_INVALID_ARG;
   int rc = check_gemm_shape(a, b, G, M, N, K);
   if (rc != CONVROT_OK) return rc;
   if (T < 0) return CONVROT_ERR_INVALID_ARG;
@@ -405,7 +487,7 @@ int convrot_i8_gemm_scatter(const int8_t* a, const float* s_a, const int8_t* b, 
   args.w = w;
   if (T >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
   args.out_rows = (int)T;
-  return launch_gemm<kEpiScatter>(a, b, G, M, N, K, N, args, as_stream(stream));
+  return launch_gemm_layout<kEpiScatter>(b_layout, a, b, G, M, N, K, N, args, as_stream(stream));
 }
 
 int convrot_f32_to_bf16(const float* x, int64_t n, void* y_bf16, void* stream) {
@@ -445,7 +527,7 @@ int w8a8_convrot_linear(const void* x_bf16, int64_t M, int64_t K, const int8_t* 
   args.s_a = s_x;
   args.s_b = w_scale;
   args.out = y_bf16;
-  return launch_gemm<kEpiBf16>(x_q, w_q, 1, M, N, K, N, args, st);
+  return launch_gemm<kEpiBf16, false>(x_q, w_q, 1, M, N, K, N, args, st);
 }
 
 int moe_workspace_layout(int64_t T, int64_t d, int64_t f, int E, int64_t C,
@@ -531,7 +613,7 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
     a1.s_a = s_g;
     a1.s_b = s_gu;
     a1.out = h;
-    if ((rc = launch_gemm<kEpiSwiglu>(x_g, w_gu, E, C, 2 * f, d, f, a1, st)) != CONVROT_OK)
+    if ((rc = launch_gemm<kEpiSwiglu, true>(x_g, w_gu, E, C, 2 * f, d, f, a1, st)) != CONVROT_OK)
       return rc;
     // 6. rotate (g_d) + requantise h per row
     if ((rc = rotquant_impl(h, CONVROT_DTYPE_F32, (int64_t)E * C, f, g_d, h_q, s_h, st)) !=
@@ -545,7 +627,8 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
     a2.idx = idx;
     a2.w = w;
     a2.out_rows = (int)T;
-    if ((rc = launch_gemm<kEpiScatter>(h_q, w_d, E, C, d, f, d, a2, st)) != CONVROT_OK) return rc;
+    if ((rc = launch_gemm<kEpiScatter, true>(h_q, w_d, E, C, d, f, d, a2, st)) != CONVROT_OK)
+      return rc;
   }
   // 8. one bf16 rounding of the fp32 combine
   return convert_impl(out32, T * d, y_bf16, sms, st);
@@ -617,5 +700,5 @@ extern "C" int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_
   args.s_a = s_x;
   args.s_b = w_scale;
   args.out = y_bf16;
-  return launch_gemm<kEpiBf16>(x_q, w_q, 1, M, N, K, N, args, st);
+  return launch_gemm<kEpiBf16, false>(x_q, w_q, 1, M, N, K, N, args, st);
 }

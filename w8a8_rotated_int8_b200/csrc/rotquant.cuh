@@ -128,12 +128,32 @@ __device__ __forceinline__ double rq_row_max(double m, int tpr, double* red) {
   return r;
 }
 
-// x: [rows, K] (bf16 or fp32), q: [rows, K] int8, scales: [rows] fp32.
+// Where the codes of a row go. Row-major: q[row * K + k]. Tiled (the
+// weight format of the grouped GEMM): the rows are split into matrices of
+// `mat_rows` rows; each matrix into 128-row blocks, each block into 128-byte
+// K tiles; tile (block rb, k-tile kb) is 16 KB at ((rb * kb_count + kb) *
+// 16384) holding 128 rows of 128 bytes. rb = mat * rb_per_mat + row_in_mat/128.
+struct RqOut {
+  int tiled;
+  int64_t mat_rows;
+  int rb_per_mat;
+  int kb_count;
+};
+
+__device__ __forceinline__ int64_t rq_dst(const RqOut& o, int64_t row, int K, int k0) {
+  if (!o.tiled) return row * K + k0;
+  const int64_t mat = row / o.mat_rows;
+  const int64_t r = row - mat * o.mat_rows;
+  const int64_t rb = mat * o.rb_per_mat + (r >> 7);
+  return ((rb * o.kb_count + (k0 >> 7)) * 128 + (r & 127)) * 128 + (k0 & 127);
+}
+
+// x: [rows, K] (bf16 or fp32), q: codes (layout `out`), scales: [rows] fp32.
 // blockDim.x = rows_per_cta * tpr exactly (rows_per_cta = max(1, 256 / tpr)).
 template <typename InT, int G>
 __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x, int64_t rows,
                                                       int K, int tpr, int8_t* __restrict__ q,
-                                                      float* __restrict__ scales) {
+                                                      float* __restrict__ scales, RqOut out) {
   using Tr = RqTraits<G>;
   extern __shared__ __align__(16) unsigned char rq_smem[];
   double* red = reinterpret_cast<double*>(rq_smem);  // 16 warps max
@@ -208,7 +228,7 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x
     __syncthreads();
     if (active) {
       const uint4 c = *reinterpret_cast<const uint4*>(codes + i * 16);
-      *reinterpret_cast<uint4*>(q + row * K + (int64_t)i * 16) = c;
+      *reinterpret_cast<uint4*>(q + rq_dst(out, row, K, i * 16)) = c;
     }
   } else {
     if (active) {
@@ -220,7 +240,7 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x
       c.y = pack4(k[4], k[5], k[6], k[7]);
       c.z = pack4(k[8], k[9], k[10], k[11]);
       c.w = pack4(k[12], k[13], k[14], k[15]);
-      *reinterpret_cast<uint4*>(q + row * K + (int64_t)i * 16) = c;
+      *reinterpret_cast<uint4*>(q + rq_dst(out, row, K, i * 16)) = c;
     }
   }
   if (active && i == 0) scales[row] = nonzero ? s : 0.0f;
