@@ -288,7 +288,7 @@ int softmax_impl(const void* logits, int64_t T, int E, float* s_t, float* clear,
                  int64_t clear_cols, cudaStream_t st) {
   if (T == 0) return CONVROT_OK;
   const int64_t grid = (T + kSmTokens - 1) / kSmTokens;
-  router_softmax_kernel<<<(unsigned)grid, 256, (size_t)E * kSmTokens * sizeof(float), st>>>(
+  router_softmax_kernel<<<(unsigned)grid, 32 * kSmTokens, (size_t)E * kSmTokens * sizeof(float), st>>>(
       reinterpret_cast<const __nv_bfloat16*>(logits), (int)T, E, s_t, clear, clear_cols);
   return launch_status();
 }
@@ -305,7 +305,7 @@ int gather_impl(const int8_t* src, const float* s_src, int64_t n_src, const int3
 int convert_impl(const float* x, int64_t n, void* y, int sms, cudaStream_t st) {
   if (n == 0) return CONVROT_OK;
   const int64_t n4 = n / 4;
-  const int64_t grid = std::min<int64_t>((n4 + 255) / 256, (int64_t)sms * 16);
+  const int64_t grid = std::min<int64_t>((n4 + 255) / 256, (int64_t)sms * 8);
   f32_to_bf16_kernel<<<(unsigned)grid, 256, 0, st>>>(x, n4,
                                                      reinterpret_cast<__nv_bfloat16*>(y));
   return launch_status();

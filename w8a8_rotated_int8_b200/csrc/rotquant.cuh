@@ -20,8 +20,8 @@
 // Layout: each thread owns 16 consecutive elements of a row (one 32-byte bf16
 // or 64-byte fp32 load, one 16-byte code store). Groups up to 16 are finished
 // in registers; for g = 64 / 256 the remaining butterfly stages run after one
-// transpose of the row through shared memory (XOR-swizzled to avoid bank
-// conflicts), then the codes go back through shared memory so the global
+// transpose of the row through shared memory (XOR-swizzled, free of bank
+// conflicts for both group sizes), then the codes go back through shared memory so the global
 // store stays contiguous.
 #pragma once
 
@@ -101,6 +101,14 @@ __device__ __forceinline__ int rq_code(double u, double r_scaled, double inv_sqr
     k = __double2int_rn(__ddiv_rn(__dmul_rn(u, inv_sqrt), s64));
   }
   return max(-127, min(127, k));
+}
+
+// Position of (16-chunk ci, column c) in the transpose buffer: columns are
+// XOR-permuted by the chunk index with its 2-bit halves swapped, which keeps
+// both the row-wise writes and the column-wise reads of g = 64 and g = 256
+// free of 64-bit bank conflicts.
+__device__ __forceinline__ int rq_swz(int ci, int c) {
+  return ci * 16 + (c ^ (((ci & 3) << 2) | ((ci >> 2) & 3)));
 }
 
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
@@ -183,7 +191,7 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x
   if constexpr (G >= 64) {
     if (active) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) buf[i * 16 + (j ^ (i & 15))] = v[j];
+      for (int j = 0; j < 16; ++j) buf[rq_swz(i, j)] = v[j];
     }
     __syncthreads();
     if (active) {
@@ -193,7 +201,7 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x
         for (int jj = 0; jj < CH; ++jj) {
           const int ci = grp * CH + jj;
           const int col = p * CPT + cc;
-          v[cc * CH + jj] = buf[ci * 16 + (col ^ (ci & 15))];
+          v[cc * CH + jj] = buf[rq_swz(ci, col)];
         }
       }
     }

@@ -12,30 +12,28 @@ namespace convrot {
 // ---------------------------------------------------------------- softmax --
 // Per-token softmax of the router logits over E experts, evaluated in fp64 and
 // rounded once to fp32, written transposed (S_t[e, t]) so each expert's
-// scores are contiguous for the top-C selection. 32 tokens per CTA (4 per
+// scores are contiguous for the top-C selection. 32 tokens per CTA (one per
 // warp); the [E, 32] tile goes through shared memory so the transposed store
 // writes 128-byte rows. Optionally zeroes the same 32 rows of an fp32 buffer
 // (the combine accumulator) to save a separate pass.
 constexpr int kSmTokens = 32;
 
-__global__ void __launch_bounds__(256) router_softmax_kernel(
+__global__ void __launch_bounds__(1024) router_softmax_kernel(
     const __nv_bfloat16* __restrict__ logits, int T, int E, float* __restrict__ S_t,
     float* __restrict__ clear, int64_t clear_cols) {
   extern __shared__ float sm_tile[];  // [E][32]
   const int t0 = blockIdx.x * kSmTokens;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned short* lg = reinterpret_cast<const unsigned short*>(logits);
-#pragma unroll 1
-  for (int k = 0; k < 4; ++k) {
-    const int tl = warp * 4 + k;
-    const int t = t0 + tl;
-    if (t >= T) break;
+  const int t = t0 + warp;  // one token per warp
+  if (t < T) {
     double l[8];
     double m = -INFINITY;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = lane + 32 * j;
-      l[j] = (e < E) ? (double)__uint_as_float((uint32_t)lg[(int64_t)t * E + e] << 16) : -INFINITY;
+      l[j] = (e < E) ? (double)__uint_as_float((uint32_t)__ldg(lg + (int64_t)t * E + e) << 16)
+                     : -INFINITY;
       m = fmax(m, l[j]);
     }
 #pragma unroll
@@ -53,7 +51,7 @@ __global__ void __launch_bounds__(256) router_softmax_kernel(
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = lane + 32 * j;
-      if (e < E) sm_tile[e * kSmTokens + tl] = __double2float_rn(__ddiv_rn(ex[j], sum));
+      if (e < E) sm_tile[e * kSmTokens + warp] = __double2float_rn(__ddiv_rn(ex[j], sum));
     }
   }
   __syncthreads();
@@ -125,7 +123,7 @@ __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const float* __restr
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0u;
     __syncthreads();
     for (int t = threadIdx.x; t < T; t += blockDim.x) {
-      const uint32_t key = score_key(u[t]);
+      const uint32_t key = score_key(__ldg(u + t));
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
@@ -226,26 +224,49 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const int8_t* __restri
   }
   const uint4* s = reinterpret_cast<const uint4*>(src + (int64_t)t * K);
   uint4* d = reinterpret_cast<uint4*>(dst + r * K);
-  for (int c = lane; c < (K >> 4); c += 32) d[c] = __ldg(s + c);
+  const int n16 = K >> 4;
+  for (int c0 = 0; c0 < n16; c0 += 128) {
+    uint4 buf[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = c0 + lane + 32 * k;
+      if (c < n16) buf[k] = __ldg(s + c);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = c0 + lane + 32 * k;
+      if (c < n16) d[c] = buf[k];
+    }
+  }
   if (lane == 0) s_dst[r] = __ldg(s_src + t);
 }
 
 // ---------------------------------------------------------------- convert --
 // y = bf16_rne(x), four elements per thread iteration.
+__device__ __forceinline__ uint2 bf16x4(float4 f) {
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(f.x, f.y);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(f.z, f.w);
+  uint2 o;
+  o.x = *reinterpret_cast<const uint32_t*>(&lo);
+  o.y = *reinterpret_cast<const uint32_t*>(&hi);
+  return o;
+}
+
 __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restrict__ x, int64_t n4,
                                                           __nv_bfloat16* __restrict__ y) {
   const float4* x4 = reinterpret_cast<const float4*>(x);
   uint2* y2 = reinterpret_cast<uint2*>(y);
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const float4 f = x4[i];
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(f.x, f.y);
-    const __nv_bfloat162 hi = __floats2bfloat162_rn(f.z, f.w);
-    uint2 o;
-    o.x = *reinterpret_cast<const uint32_t*>(&lo);
-    o.y = *reinterpret_cast<const uint32_t*>(&hi);
-    y2[i] = o;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n4; i += 4 * stride) {
+    const float4 a = __ldcs(x4 + i), b = __ldcs(x4 + i + stride);
+    const float4 c = __ldcs(x4 + i + 2 * stride), d = __ldcs(x4 + i + 3 * stride);
+    y2[i] = bf16x4(a);
+    y2[i + stride] = bf16x4(b);
+    y2[i + 2 * stride] = bf16x4(c);
+    y2[i + 3 * stride] = bf16x4(d);
   }
+  for (; i < n4; i += stride) y2[i] = bf16x4(__ldcs(x4 + i));
 }
 
 // --------------------------------------------------------- wait self-test --
