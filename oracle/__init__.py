@@ -6,9 +6,10 @@ This package is TEST INFRASTRUCTURE. Only the test suite, the smoke check in
 binding) never imports, links or executes anything in here, and nothing in
 here imports the product package.
 
-Everything is plain NumPy: fp64 for the rotation, exact integer GEMMs, and
-fp32 only where the method's definition is fp32 (the scales, the dequantised
-outputs, SwiGLU, the router-weighted combine).
+Everything is plain NumPy: the rotation and rounding in fp32 (with an exact
+fp64 matrix form of the rotation kept for the pins), exact integer GEMMs,
+fp64 for the router softmax, fp32 for the scales, dequantised outputs,
+SwiGLU and the router-weighted combine.
 """
 
 from .convrot_oracle import (  # noqa: F401
@@ -16,6 +17,7 @@ from .convrot_oracle import (  # noqa: F401
     block_rotate,
     dequant,
     expert_choice_topc,
+    fwht_f32,
     hadamard,
     int_gemm,
     moe_block,

@@ -23,11 +23,17 @@ Readings of what the pages leave open (each is fixed here once):
 * Hadamard: Sylvester construction in natural order, no sign flips,
   normalised by 1/sqrt(g); applied block-diagonally along K (contiguous
   groups of g). Only g in {1, 4, 16, 64, 256} (powers of four) are accepted,
-  so 1/sqrt(g) is a power of two and the normalised rotation of bf16 data is
-  exact in fp64.
-* Symmetric INT8: s = fp32(absmax / 127) (the fp64 quotient rounded to fp32),
-  q = clamp(rint(v / s), -127, 127) with ties to even; if s is 0 the row's
-  codes are all 0.
+  so 1/sqrt(g) is a power of two.
+* Precision of rotation and rounding: fp32, as the NitroFusion2 page states
+  for its conversions ("How they were made": the rotation and rounding in
+  fp32). The rotation is the fast Walsh-Hadamard butterfly (a+b, a-b) in
+  fp32 with the stage spans in increasing order 1, 2, ..., g/2, then the
+  exact scaling by 1/sqrt(g); block_rotate (fp64 matrix product) is its
+  exact mathematical counterpart.
+* Symmetric INT8 of a rotated fp32 row v: a = max|v|, s = fp32(a / 127),
+  r = fp32(127 / a), q = clamp(rint(fp32(v * r)), -127, 127) with ties to
+  even. A row with a < 2^-120 (zero, or too small for r to be finite) gets
+  s = 0 and q = 0.
 * Activations: per-token dynamic scales, the same rotation and quantiser as
   the weights.
 * Router score: per-token softmax over the experts, evaluated in fp64 and
@@ -87,31 +93,55 @@ def block_rotate(v: np.ndarray, g: int) -> np.ndarray:
     return (grouped @ r).reshape(v.shape)
 
 
+def fwht_f32(v: np.ndarray, g: int) -> np.ndarray:
+    """The fp32 rotation: per contiguous group of g along the last axis,
+    butterflies (a + b, a - b) in fp32 with spans 1, 2, ..., g/2 in that
+    order, then multiplication by 1/sqrt(g) (a power of two)."""
+    if g not in ALLOWED_GROUPS:
+        raise ValueError(f"group must be one of {ALLOWED_GROUPS}, got {g}")
+    x = np.array(v, dtype=np.float32)
+    k = x.shape[-1]
+    if k % g != 0:
+        raise ValueError(f"K={k} is not a multiple of the group size {g}")
+    lead = x.shape[:-1]
+    span = 1
+    while span < g:
+        y = x.reshape(lead + (k // (2 * span), 2, span))
+        a = y[..., 0, :].copy()
+        b = y[..., 1, :].copy()
+        y[..., 0, :] = a + b
+        y[..., 1, :] = a - b
+        x = y.reshape(lead + (k,))
+        span *= 2
+    return (x * np.float32(1.0 / np.sqrt(g))).astype(np.float32)
+
+
 # ------------------------------------------------------------ quantisation --
+TINY = np.float32(2.0 ** -120)
+
+
 def quantize_rows(v: np.ndarray):
-    """Symmetric per-row INT8 of an fp64 matrix [rows, K].
+    """Symmetric per-row INT8 of an fp32 matrix [rows, K] (see the header).
 
     Returns (q int8 [rows, K], s float32 [rows]).
     """
-    v = np.asarray(v, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float32)
     a = np.max(np.abs(v), axis=-1)
-    s = (a / np.float64(QMAX)).astype(np.float32)
-    q = np.zeros(v.shape, dtype=np.int8)
-    nz = s != 0
-    if np.any(nz):
-        quot = v[nz] / s[nz].astype(np.float64)[:, None]
-        q[nz] = np.clip(np.rint(quot), -QMAX, QMAX).astype(np.int8)
-    s = np.where(nz, s, np.float32(0))
+    ok = a >= TINY
+    a_safe = np.where(ok, a, np.float32(1))
+    s = np.where(ok, a_safe / np.float32(QMAX), np.float32(0)).astype(np.float32)
+    r = (np.float32(QMAX) / a_safe).astype(np.float32)
+    prod = (v * r[..., None]).astype(np.float32)
+    q = np.clip(np.rint(prod), -QMAX, QMAX).astype(np.int8)
+    q[~ok] = 0
     return q, s
 
 
 def rotquant(x: np.ndarray, g: int):
-    """Rotate each row by blockdiag(R_g) (fp64) and quantise it per row.
-
-    Serves the weights (offline, per output row), the activations (per
-    token) and the SwiGLU output h before the down projection (g = 64).
-    """
-    return quantize_rows(block_rotate(x, g))
+    """Rotate each row in groups of g (fp32 butterflies) and quantise it per
+    row. Serves the weights (offline, per output row), the activations (per
+    token) and the SwiGLU output h before the down projection (g = 64)."""
+    return quantize_rows(fwht_f32(x, g))
 
 
 # --------------------------------------------------------- integer GEMM -----

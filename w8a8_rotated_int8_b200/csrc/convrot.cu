@@ -50,21 +50,6 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <typename InT, int G>
-void set_rq_attr() {
-  cudaFuncSetAttribute(rotquant_kernel<InT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       96 * 1024);
-}
-
-template <typename InT>
-void set_rq_attrs() {
-  set_rq_attr<InT, 1>();
-  set_rq_attr<InT, 4>();
-  set_rq_attr<InT, 16>();
-  set_rq_attr<InT, 64>();
-  set_rq_attr<InT, 256>();
-}
-
 template <bool BT>
 void set_gemm_attrs() {
   cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiI32, BT>,
@@ -100,8 +85,6 @@ int device_setup(int* sm_count) {
     if (d.supported) {
       set_gemm_attrs<false>();
       set_gemm_attrs<true>();
-      set_rq_attrs<__nv_bfloat16>();
-      set_rq_attrs<float>();
       if (cudaGetLastError() != cudaSuccess) return CONVROT_ERR_CUDA;
     }
     d.ready = true;
@@ -135,9 +118,8 @@ void launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut ou
   // whole rows per CTA: a CTA never holds threads beyond rpc * tpr
   const int rpc = std::max(1, kRqThreads / tpr);
   const int threads = rpc * tpr;
-  const size_t smem = 128 + (G >= 64 ? (size_t)rpc * K * 9 : 0);
   const int64_t grid = (rows + rpc - 1) / rpc;
-  rotquant_kernel<InT, G><<<(unsigned)grid, threads, smem, st>>>(
+  rotquant_kernel<InT, G><<<(unsigned)grid, threads, 0, st>>>(
       reinterpret_cast<const InT*>(x), rows, K, tpr, q, s, out);
 }
 

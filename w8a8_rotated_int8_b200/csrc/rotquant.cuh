@@ -5,24 +5,24 @@
 // (ConvRot) and quantised to symmetric INT8 with nearest rounding and one
 // FP32 scale per row. "NitroFusion2 for ComfyUI: int8, W6A8, W4A8", section
 // "How they were made": block Hadamard rotation, one scale per row, 8-bit
-// activations. The same operation serves the weights (offline, per output
-// row), the activations (per token) and the SwiGLU output before the down
-// projection.
+// activations, with the rotation and rounding done in fp32. The same
+// operation serves the weights (offline, per output row), the activations
+// (per token) and the SwiGLU output before the down projection.
 //
-// Arithmetic: the rotation runs in fp64 butterflies. Inputs are bf16 or fp32
-// and g is a power of four, so every partial sum and the 1/sqrt(g) scaling
-// are exact for ordinary data and the rotated value equals the exact one.
-// Scale s = fp32(absmax / 127); code q = clamp(rint(v / s), -127, 127), ties
-// to even. The division is replaced by a multiply with the reciprocal plus a
-// distance check: only values that land within 1e-9 of a rounding boundary
-// take the true fp64 division, so the codes equal those of the definition.
+// Arithmetic (fp32, IEEE, no contraction):
+//   rotation  fast Walsh-Hadamard butterflies (a + b, a - b) with spans
+//             1, 2, ..., g/2 in that order, then v' = v * (1/sqrt(g)) (a
+//             power of two for g a power of four);
+//   scale     a = max|v'|, s = a / 127, r = 127 / a (one IEEE division each);
+//   codes     q = rint(v' * r), ties to even (|v' * r| <= 127 (1 + 2^-24), so
+//             the code never leaves [-127, 127]);
+//   a row with a < 2^-120 gets s = 0 and all-zero codes.
 //
 // Layout: each thread owns 16 consecutive elements of a row (one 32-byte bf16
-// or 64-byte fp32 load, one 16-byte code store). Groups up to 16 are finished
-// in registers; for g = 64 / 256 the remaining butterfly stages run after one
-// transpose of the row through shared memory (XOR-swizzled, free of bank
-// conflicts for both group sizes), then the codes go back through shared memory so the global
-// store stays contiguous.
+// or 64-byte fp32 load, one 16-byte code store). Spans 1..8 are butterflies
+// in registers; the larger spans pair 16-element chunks held by lanes whose
+// indices differ in one bit, exchanged with warp shuffles (a row's chunks sit
+// in consecutive lanes, so chunk i and chunk i ^ d are lane and lane ^ d).
 #pragma once
 
 #include "common.cuh"
@@ -32,84 +32,41 @@ namespace convrot {
 constexpr int kRqThreads = 256;
 
 template <typename InT>
-__device__ __forceinline__ void rq_load16(const InT* p, double (&v)[16]);
+__device__ __forceinline__ void rq_load16(const InT* p, float (&v)[16]);
 
 template <>
-__device__ __forceinline__ void rq_load16<__nv_bfloat16>(const __nv_bfloat16* p, double (&v)[16]) {
+__device__ __forceinline__ void rq_load16<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[16]) {
   const uint4* q = reinterpret_cast<const uint4*>(p);
   const uint4 a = __ldg(q);
   const uint4 b = __ldg(q + 1);
   const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    v[2 * k] = (double)__uint_as_float(w[k] << 16);
-    v[2 * k + 1] = (double)__uint_as_float(w[k] & 0xFFFF0000u);
+    v[2 * k] = __uint_as_float(w[k] << 16);
+    v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
   }
 }
 
 template <>
-__device__ __forceinline__ void rq_load16<float>(const float* p, double (&v)[16]) {
+__device__ __forceinline__ void rq_load16<float>(const float* p, float (&v)[16]) {
   const float4* q = reinterpret_cast<const float4*>(p);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const float4 f = __ldg(q + k);
-    v[4 * k] = (double)f.x;
-    v[4 * k + 1] = (double)f.y;
-    v[4 * k + 2] = (double)f.z;
-    v[4 * k + 3] = (double)f.w;
-  }
-}
-
-// Butterflies (a+b, a-b) for spans 1 .. 2^(STAGES-1) over N consecutive values.
-template <int STAGES, int N>
-__device__ __forceinline__ void fwht_inreg(double* v) {
-#pragma unroll
-  for (int s = 0; s < STAGES; ++s) {
-    const int span = 1 << s;
-#pragma unroll
-    for (int j = 0; j < N; ++j) {
-      if ((j & span) == 0) {
-        const double a = v[j];
-        const double b = v[j + span];
-        v[j] = __dadd_rn(a, b);
-        v[j + span] = __dsub_rn(a, b);
-      }
-    }
+    v[4 * k] = f.x;
+    v[4 * k + 1] = f.y;
+    v[4 * k + 2] = f.z;
+    v[4 * k + 3] = f.w;
   }
 }
 
 template <int G>
 struct RqTraits {
   static_assert(G == 1 || G == 4 || G == 16 || G == 64 || G == 256, "group must be a power of four <= 256");
-  static constexpr int kLog2 = G == 1 ? 0 : G == 4 ? 2 : G == 16 ? 4 : G == 64 ? 6 : 8;
-  static constexpr int kInReg = kLog2 < 4 ? kLog2 : 4;       // stages inside a 16-chunk
-  static constexpr int kChunks = G >= 16 ? G / 16 : 1;       // 16-chunks per group
-  static constexpr int kCross = kLog2 - kInReg;              // stages across chunks
-  static constexpr double kInvSqrt = G == 1 ? 1.0 : G == 4 ? 0.5 : G == 16 ? 0.25 : G == 64 ? 0.125 : 0.0625;
+  static constexpr int kInRegSpanEnd = G < 16 ? G : 16;  // spans 1 .. kInRegSpanEnd/2 in registers
+  static constexpr int kLaneSpanEnd = G >= 16 ? G / 16 : 1;  // lane distances 1 .. kLaneSpanEnd/2
+  static constexpr float kInvSqrt = G == 1 ? 1.0f : G == 4 ? 0.5f : G == 16 ? 0.25f : G == 64 ? 0.125f : 0.0625f;
 };
-
-// One code from an unnormalised rotated value u (v' = u * inv_sqrt exactly).
-__device__ __forceinline__ int rq_code(double u, double r_scaled, double inv_sqrt, double s64) {
-  const double magic = 6755399441055744.0;  // 1.5 * 2^52: adding it rounds to an integer
-  const double y = __dmul_rn(u, r_scaled);  // v' / s up to a few fp64 ulps
-  const double t = __dadd_rn(y, magic);
-  const double ry = __dsub_rn(t, magic);     // rint(y), ties to even
-  int k;
-  if (fabs(__dsub_rn(y, ry)) < 0.4999999990) {
-    k = __double2loint(t);                   // two's complement integer in the low word
-  } else {
-    k = __double2int_rn(__ddiv_rn(__dmul_rn(u, inv_sqrt), s64));
-  }
-  return max(-127, min(127, k));
-}
-
-// Position of (16-chunk ci, column c) in the transpose buffer: columns are
-// XOR-permuted by the chunk index with its 2-bit halves swapped, which keeps
-// both the row-wise writes and the column-wise reads of g = 64 and g = 256
-// free of 64-bit bank conflicts.
-__device__ __forceinline__ int rq_swz(int ci, int c) {
-  return ci * 16 + (c ^ (((ci & 3) << 2) | ((ci >> 2) & 3)));
-}
 
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
   return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
@@ -118,21 +75,21 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
 
 // Row-wise max over the `tpr` threads of a row. tpr is a power of two <= 32
 // (rows live in aligned lane segments) or a multiple of 32.
-__device__ __forceinline__ double rq_row_max(double m, int tpr, double* red) {
+__device__ __forceinline__ float rq_row_max(float m, int tpr, float* red) {
   const int lane = threadIdx.x & 31;
   if (tpr <= 32) {
-    for (int off = tpr >> 1; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+    for (int off = tpr >> 1; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     return m;
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
   const int warp = threadIdx.x >> 5;
   if (lane == 0) red[warp] = m;
   __syncthreads();
   const int wpr = tpr >> 5;
   const int w0 = (threadIdx.x / tpr) * wpr;
-  double r = 0.0;
-  for (int w = 0; w < wpr; ++w) r = fmax(r, red[w0 + w]);
+  float r = 0.0f;
+  for (int w = 0; w < wpr; ++w) r = fmaxf(r, red[w0 + w]);
   return r;
 }
 
@@ -163,8 +120,8 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x
                                                       int K, int tpr, int8_t* __restrict__ q,
                                                       float* __restrict__ scales, RqOut out) {
   using Tr = RqTraits<G>;
-  extern __shared__ __align__(16) unsigned char rq_smem[];
-  double* red = reinterpret_cast<double*>(rq_smem);  // 16 warps max
+  __shared__ float red[16];  // per-warp maxima (512 threads at most)
+  const int lane = threadIdx.x & 31;
   const int rows_per_cta = blockDim.x / tpr;
   const int r_local = threadIdx.x / tpr;
   const int i = threadIdx.x - r_local * tpr;  // 16-chunk index in the row
@@ -172,86 +129,62 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x
   const int nchunks = K >> 4;
   const bool active = (row < rows) && (i < nchunks);
 
-  double v[16];
+  float v[16];
   if (active) {
     rq_load16<InT>(x + row * K + (int64_t)i * 16, v);
   } else {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = 0.0;
+    for (int j = 0; j < 16; ++j) v[j] = 0.0f;
   }
-  fwht_inreg<Tr::kInReg, 16>(v);
-
-  double* buf = reinterpret_cast<double*>(rq_smem + 128) + (int64_t)r_local * K;
-  unsigned char* codes =
-      rq_smem + 128 + (size_t)rows_per_cta * K * sizeof(double) + (size_t)r_local * K;
-  constexpr int CH = Tr::kChunks;
-  constexpr int CPT = 16 / CH;  // columns held per thread after the transpose
-  const int grp = i / CH;
-  const int p = i - grp * CH;
-  if constexpr (G >= 64) {
-    if (active) {
+  // spans 1, 2, 4, 8 inside the thread's 16 elements
 #pragma unroll
-      for (int j = 0; j < 16; ++j) buf[rq_swz(i, j)] = v[j];
-    }
-    __syncthreads();
-    if (active) {
+  for (int span = 1; span < Tr::kInRegSpanEnd; span <<= 1) {
 #pragma unroll
-      for (int cc = 0; cc < CPT; ++cc) {
-#pragma unroll
-        for (int jj = 0; jj < CH; ++jj) {
-          const int ci = grp * CH + jj;
-          const int col = p * CPT + cc;
-          v[cc * CH + jj] = buf[rq_swz(ci, col)];
-        }
+    for (int j = 0; j < 16; ++j) {
+      if ((j & span) == 0) {
+        const float a = v[j];
+        const float b = v[j + span];
+        v[j] = __fadd_rn(a, b);
+        v[j + span] = __fsub_rn(a, b);
       }
     }
-#pragma unroll
-    for (int cc = 0; cc < CPT; ++cc) fwht_inreg<Tr::kCross, CH>(v + cc * CH);
   }
-
-  double m = 0.0;
+  // spans 16, 32, ... between chunks: the lower chunk of a pair keeps a + b,
+  // the upper one a - b, as one rounding each: fma(+-1, own, partner)
 #pragma unroll
-  for (int j = 0; j < 16; ++j) m = fmax(m, fabs(v[j]));
+  for (int d = 1; d < Tr::kLaneSpanEnd; d <<= 1) {
+    const float sgn = (lane & d) ? -1.0f : 1.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float p = __shfl_xor_sync(0xffffffffu, v[j], d);
+      v[j] = __fmaf_rn(sgn, v[j], p);
+    }
+  }
+  float m = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    v[j] = __fmul_rn(v[j], Tr::kInvSqrt);
+    m = fmaxf(m, fabsf(v[j]));
+  }
   m = rq_row_max(m, tpr, red);
 
-  const double a = __dmul_rn(m, Tr::kInvSqrt);
-  const float s = __double2float_rn(__ddiv_rn(a, 127.0));
-  const double s64 = (double)s;
-  const bool nonzero = s != 0.0f;
-  const double r_scaled = nonzero ? __dmul_rn(__drcp_rn(s64), Tr::kInvSqrt) : 0.0;
-
-  if constexpr (G >= 64) {
-    if (active) {
+  const bool nonzero = m >= 7.52316384526264e-37f;  // 2^-120
+  const float s = nonzero ? __fdiv_rn(m, 127.0f) : 0.0f;
+  const float r = nonzero ? __fdiv_rn(127.0f, m) : 0.0f;
+  if (active) {
+    // rint by adding 1.5 * 2^23 (the fp32 add rounds to nearest even)
+    int k[16];
 #pragma unroll
-      for (int cc = 0; cc < CPT; ++cc) {
-#pragma unroll
-        for (int jj = 0; jj < CH; ++jj) {
-          const int ci = grp * CH + jj;
-          const int col = p * CPT + cc;
-          const int k = nonzero ? rq_code(v[cc * CH + jj], r_scaled, Tr::kInvSqrt, s64) : 0;
-          codes[ci * 16 + col] = (unsigned char)(k & 0xFF);
-        }
-      }
-    }
-    __syncthreads();
-    if (active) {
-      const uint4 c = *reinterpret_cast<const uint4*>(codes + i * 16);
-      *reinterpret_cast<uint4*>(q + rq_dst(out, row, K, i * 16)) = c;
-    }
-  } else {
-    if (active) {
-      int k[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) k[j] = nonzero ? rq_code(v[j], r_scaled, Tr::kInvSqrt, s64) : 0;
-      uint4 c;
-      c.x = pack4(k[0], k[1], k[2], k[3]);
-      c.y = pack4(k[4], k[5], k[6], k[7]);
-      c.z = pack4(k[8], k[9], k[10], k[11]);
-      c.w = pack4(k[12], k[13], k[14], k[15]);
-      *reinterpret_cast<uint4*>(q + rq_dst(out, row, K, i * 16)) = c;
-    }
+    for (int j = 0; j < 16; ++j)
+      k[j] = __float_as_int(__fadd_rn(__fmul_rn(v[j], r), 12582912.0f)) - 0x4B400000;
+    uint4 c;
+    c.x = pack4(k[0], k[1], k[2], k[3]);
+    c.y = pack4(k[4], k[5], k[6], k[7]);
+    c.z = pack4(k[8], k[9], k[10], k[11]);
+    c.w = pack4(k[12], k[13], k[14], k[15]);
+    *reinterpret_cast<uint4*>(q + rq_dst(out, row, K, i * 16)) = c;
+    if (i == 0) scales[row] = s;
   }
-  if (active && i == 0) scales[row] = nonzero ? s : 0.0f;
 }
 
 }  // namespace convrot
