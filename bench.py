@@ -63,8 +63,8 @@ def algorithmic_work(cfg, t):
     }
     down = {
         "ops": 2 * e * c * f * d,
-        # weights + scales + h codes and scales in + fp32 red-add of the combine
-        "bytes": e * d * f + e * d * 4 + e * c * (f + 4) + e * c * d * 4,
+        # weights + scales + h codes, scales and router weights in + fp32 rows out
+        "bytes": e * d * f + e * d * 4 + e * c * (f + 8) + e * c * d * 4,
     }
     return {"ops": ops, "block_bytes": block_bytes, "gateup": gateup, "down": down}
 
@@ -260,7 +260,7 @@ def stage_times(W, ws_views, inp_dev, wq, cfg, t, reps, flush_buf):
         "rotquant_x": lambda: W.convrot_rotquant(inp_dev["x"], cfg.g_gu, q=v["x_q"], scale=v["s_x"]),
         "topc": lambda: W.binding.lib().convrot_topc(
             W.binding._p(v["s_t"]), t, cfg.n_exp, cfg.c, W.binding._p(v["idx"]),
-            W.binding._p(v["w"]), W.binding._stream()),
+            W.binding._p(v["w"]), W.binding._p(v["slot"]), W.binding._stream()),
         "gather": lambda: W.binding.lib().convrot_gather_rows(
             W.binding._p(v["x_q"]), W.binding._p(v["s_x"]), t, W.binding._p(v["idx"]),
             cfg.n_exp * cfg.c, cfg.d, W.binding._p(v["x_g"]), W.binding._p(v["s_g"]),
@@ -271,12 +271,13 @@ def stage_times(W, ws_views, inp_dev, wq, cfg, t, reps, flush_buf):
             W.binding._stream()),
         "rotquant_h": lambda: W.convrot_rotquant(v["h"].view(-1, cfg.f), cfg.g_d,
                                                  q=v["h_q"].view(-1, cfg.f), scale=v["s_h"].view(-1)),
-        "gemm_down_scatter": lambda: W.binding.lib().convrot_i8_gemm_scatter(
+        "gemm_down_weighted": lambda: W.binding.lib().convrot_i8_gemm_weighted(
             W.binding._p(v["h_q"]), W.binding._p(v["s_h"]), W.binding._p(wd_q),
-            W.binding._p(s_d), tiles, W.binding._p(v["idx"]), W.binding._p(v["w"]), cfg.n_exp, cfg.c,
-            cfg.d, cfg.f, W.binding._p(v["out32"]), t, W.binding._stream()),
-        "f32_to_bf16": lambda: W.binding.lib().convrot_f32_to_bf16(
-            W.binding._p(v["out32"]), t * cfg.d, W.binding._p(inp_dev["y"]), W.binding._stream()),
+            W.binding._p(s_d), tiles, W.binding._p(v["w"]), cfg.n_exp, cfg.c, cfg.d, cfg.f,
+            W.binding._p(v["zw"]), W.binding._stream()),
+        "combine": lambda: W.binding.lib().convrot_combine_rows(
+            W.binding._p(v["zw"]), W.binding._p(v["slot"]), cfg.n_exp, t, cfg.c, cfg.d,
+            W.binding._p(inp_dev["y"]), W.binding._stream()),
     }
     out = {}
     for name, fn in stages.items():
@@ -384,7 +385,7 @@ def run_ours(args, cfg, world, rank, local):
         return
     peaks = load_peaks()
     work = algorithmic_work(cfg, t)
-    dom = max(("gemm_gateup_swiglu", "gemm_down_scatter"), key=lambda k: st[k])
+    dom = max(("gemm_gateup_swiglu", "gemm_down_weighted"), key=lambda k: st[k])
     dk = work["gateup"] if dom == "gemm_gateup_swiglu" else work["down"]
     int8_peak_tops = 2.0 * peaks["bf16_tflops"]  # int8 dense = 2x bf16 dense (nominal ratio)
     t_hbm = dk["bytes"] / (peaks["hbm_gbs"] * 1e9)

@@ -59,7 +59,7 @@ def test_argument_checks_need_no_gpu(lib):
     assert lib.convrot_rotquant(al, 7, 4, 256, 256, al, al, None) == INVALID
     assert lib.convrot_rotquant(mis, 0, 4, 256, 256, al, al, None) == MISALIGNED
     # top-C capacity beyond T
-    assert lib.convrot_topc(al, 10, 4, 11, al, al, None) == INVALID
+    assert lib.convrot_topc(al, 10, 4, 11, al, al, None, None) == INVALID
     # GEMM: K not a multiple of 16, N not a multiple of 16, int32 overflow bound
     assert lib.convrot_i8_gemm_i32(al, al, 0, 1, 8, 16, 40, al, None) == INVALID
     assert lib.convrot_i8_gemm_i32(al, al, 0, 1, 8, 24, 64, al, None) == INVALID
@@ -90,4 +90,4 @@ def test_workspace_layout_is_disjoint_and_aligned(lib):
     offs = sorted(lay[n] for n in names)
     assert all(o % 256 == 0 for o in offs)
     assert len(set(offs)) == len(offs)
-    assert lay["total"] >= lay["out32"] + 8192 * 2048 * 4
+    assert lay["total"] >= lay["zw"] + 64 * 256 * 2048 * 4

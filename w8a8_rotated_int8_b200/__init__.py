@@ -10,6 +10,7 @@ from .binding import (  # noqa: F401
     TiledWeights,
     LIB_PATH,
     convrot_check_device_error,
+    convrot_combine_rows,
     convrot_device_check,
     convrot_f32_to_bf16,
     convrot_gather_rows,
@@ -17,6 +18,7 @@ from .binding import (  # noqa: F401
     convrot_i8_gemm_i32,
     convrot_i8_gemm_scatter,
     convrot_i8_gemm_swiglu,
+    convrot_i8_gemm_weighted,
     convrot_linear_workspace_size,
     convrot_quantize_weights,
     convrot_quantize_weights_tiled,

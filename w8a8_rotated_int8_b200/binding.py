@@ -39,7 +39,8 @@ class ConvrotError(RuntimeError):
 
 class MoeLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
-                ("x_q", "s_x", "s_t", "idx", "w", "x_g", "s_g", "h", "h_q", "s_h", "out32", "total")]
+                ("x_q", "s_x", "s_t", "idx", "w", "x_g", "s_g", "h", "h_q", "s_h", "slot", "zw",
+                 "total")]
 
 
 _lib = None
@@ -61,7 +62,9 @@ _SIGNATURES = {
     "convrot_tiled_weight_bytes": (_I64, [_I64, _I64, _I64]),
     "convrot_quantize_weights_tiled": (_I, [_P, _I64, _I64, _I64, _I, _P, _P, _P]),
     "convrot_router_softmax": (_I, [_P, _I64, _I, _P, _P]),
-    "convrot_topc": (_I, [_P, _I64, _I, _I64, _P, _P, _P]),
+    "convrot_topc": (_I, [_P, _I64, _I, _I64, _P, _P, _P, _P]),
+    "convrot_combine_rows": (_I, [_P, _P, _I, _I64, _I64, _I64, _P, _P]),
+    "convrot_i8_gemm_weighted": (_I, [_P, _P, _P, _P, _I, _P, _I64, _I64, _I64, _I64, _P, _P]),
     "convrot_gather_rows": (_I, [_P, _P, _I64, _P, _I64, _I64, _P, _P, _P]),
     "convrot_i8_gemm_i32": (_I, [_P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
     "convrot_i8_gemm_bf16": (_I, [_P, _P, _P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
@@ -224,14 +227,30 @@ def convrot_router_softmax(logits, stream=None):
     return s_t
 
 
-def convrot_topc(s_t, c, stream=None):
-    """[E, T] fp32 scores -> (idx int32 [E, C], w fp32 [E, C])."""
+def convrot_topc(s_t, c, with_slot=False, stream=None):
+    """[E, T] fp32 scores -> (idx int32 [E, C], w fp32 [E, C]) and, with
+    with_slot, slot int32 [E, T] (position of each token per expert or -1)."""
     _need(s_t, torch.float32, "s_t")
     e, t = s_t.shape
     idx = torch.empty((e, c), dtype=torch.int32, device=s_t.device)
     w = torch.empty((e, c), dtype=torch.float32, device=s_t.device)
-    _check(lib().convrot_topc(_p(s_t), t, e, c, _p(idx), _p(w), _stream(stream)), "convrot_topc")
-    return idx, w
+    slot = torch.empty((e, t), dtype=torch.int32, device=s_t.device) if with_slot else None
+    _check(lib().convrot_topc(_p(s_t), t, e, c, _p(idx), _p(w), _p(slot), _stream(stream)),
+           "convrot_topc")
+    return (idx, w, slot) if with_slot else (idx, w)
+
+
+def convrot_combine_rows(zw, slot, c, stream=None):
+    """zw [E*C, d] fp32 + slot [E, T] -> y [T, d] bf16 (per-token fp32 sum in
+    ascending expert order)."""
+    _need(zw, torch.float32, "zw")
+    _need(slot, torch.int32, "slot")
+    e, t = slot.shape
+    d = zw.shape[-1]
+    y = torch.empty((t, d), dtype=torch.bfloat16, device=zw.device)
+    _check(lib().convrot_combine_rows(_p(zw), _p(slot), e, t, c, d, _p(y), _stream(stream)),
+           "convrot_combine_rows")
+    return y
 
 
 def convrot_gather_rows(src, s_src, idx, stream=None):
@@ -310,6 +329,17 @@ def convrot_i8_gemm_scatter(a, s_a, b, s_b, idx, w, out32, stream=None):
                                          n, k, _p(out32), out32.shape[0], _stream(stream)),
            "convrot_i8_gemm_scatter")
     return out32
+
+
+def convrot_i8_gemm_weighted(a, s_a, b, s_b, w, stream=None):
+    """zw[g*M + m, n] = w[g, m] * dequant(acc)[g, m, n] -> zw [G*M, N] fp32."""
+    g, m, n, k, bt, lay = _gemm_dims(a, b)
+    for t, nm in ((s_a, "s_a"), (s_b, "s_b"), (w, "w")):
+        _need(t, torch.float32, nm)
+    zw = torch.empty((g * m, n), dtype=torch.float32, device=a.device)
+    _check(lib().convrot_i8_gemm_weighted(_p(a), _p(s_a), _p(bt), _p(s_b), lay, _p(w), g, m, n, k,
+                                          _p(zw), _stream(stream)), "convrot_i8_gemm_weighted")
+    return zw
 
 
 def convrot_f32_to_bf16(x, stream=None):
@@ -426,5 +456,6 @@ def moe_stage_views(workspace, t, d, f, e, c) -> dict:
         "h": view("h", torch.float32, (e, c, f)),
         "h_q": view("h_q", torch.int8, (e, c, f)),
         "s_h": view("s_h", torch.float32, (e, c)),
-        "out32": view("out32", torch.float32, (t, d)),
+        "slot": view("slot", torch.int32, (e, t)),
+        "zw": view("zw", torch.float32, (e, c, d)),
     }

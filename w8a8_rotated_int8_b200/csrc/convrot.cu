@@ -60,6 +60,8 @@ void set_gemm_attrs() {
                        cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
   cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiScatter, BT>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiWeighted, BT>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
 }
 
 // Per-device one-time setup: capability check, SM count, kernel attributes.
@@ -260,9 +262,17 @@ int launch_gemm_layout(int b_layout, const int8_t* a, const int8_t* b, int64_t G
 }
 
 int topc_impl(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float* w,
-              cudaStream_t st) {
-  if (C == 0 || E == 0) return CONVROT_OK;
-  topc_kernel<<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w);
+              int32_t* slot, cudaStream_t st) {
+  if (E == 0 || (C == 0 && slot == nullptr)) return CONVROT_OK;
+  topc_kernel<<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+  return launch_status();
+}
+
+int combine_impl(const float* zw, const int32_t* slot, int E, int64_t T, int64_t C, int64_t d,
+                 void* y, cudaStream_t st) {
+  if (T == 0) return CONVROT_OK;
+  combine_rows_kernel<<<(unsigned)T, kCombineThreads, 0, st>>>(
+      zw, slot, E, (int)T, (int)C, (int)d, reinterpret_cast<__nv_bfloat16*>(y));
   return launch_status();
 }
 
@@ -381,14 +391,43 @@ int convrot_router_softmax(const void* logits_bf16, int64_t T, int E, float* s_t
 }
 
 int convrot_topc(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float* w,
-                 void* stream) {
+                 int32_t* slot, void* stream) {
   if (T < 0 || T >= ((int64_t)1 << 31) || E < 0 || E > 65535 || C < 0 || C > T)
     return CONVROT_ERR_INVALID_ARG;
   if (C > 0 && E > 0 && (!s_t || !idx || !w)) return CONVROT_ERR_INVALID_ARG;
-  if (!al16(s_t) || !al16(idx) || !al16(w)) return CONVROT_ERR_MISALIGNED;
+  if (!al16(s_t) || !al16(idx) || !al16(w) || !al16(slot)) return CONVROT_ERR_MISALIGNED;
   int rc = device_setup(nullptr);
   if (rc != CONVROT_OK) return rc;
-  return topc_impl(s_t, T, E, C, idx, w, as_stream(stream));
+  return topc_impl(s_t, T, E, C, idx, w, slot, as_stream(stream));
+}
+
+int convrot_combine_rows(const float* zw, const int32_t* slot, int E, int64_t T, int64_t C,
+                         int64_t d, void* y_bf16, void* stream) {
+  if (E < 1 || E > 256 || T < 0 || T >= ((int64_t)1 << 31) || C < 0 || C > T || d < 4 ||
+      d % 4 != 0 || (int64_t)E * C * d >= ((int64_t)1 << 40))
+    return CONVROT_ERR_INVALID_ARG;
+  if (T > 0 && (!slot || !y_bf16 || (C > 0 && !zw))) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(zw) || !al16(slot) || !al16(y_bf16)) return CONVROT_ERR_MISALIGNED;
+  int rc = device_setup(nullptr);
+  if (rc != CONVROT_OK) return rc;
+  return combine_impl(zw, slot, E, T, C, d, y_bf16, as_stream(stream));
+}
+
+int convrot_i8_gemm_weighted(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
+                             int b_layout, const float* w, int64_t G, int64_t M, int64_t N,
+                             int64_t K, float* zw, void* stream) {
+  if (b_layout != CONVROT_LAYOUT_ROWS && b_layout != CONVROT_LAYOUT_TILES)
+    return CONVROT_ERR_INVALID_ARG;
+  int rc = check_gemm_shape(a, b, G, M, N, K);
+  if (rc != CONVROT_OK) return rc;
+  if (G * M * N > 0 && (!s_a || !s_b || !w || !zw)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(s_a) || !al16(s_b) || !al16(zw)) return CONVROT_ERR_MISALIGNED;
+  GemmArgs args{};
+  args.s_a = s_a;
+  args.s_b = s_b;
+  args.out = zw;
+  args.w = w;
+  return launch_gemm_layout<kEpiWeighted>(b_layout, a, b, G, M, N, K, N, args, as_stream(stream));
 }
 
 int convrot_gather_rows(const int8_t* src, const float* s_src, int64_t n_src, const int32_t* idx,
@@ -532,7 +571,8 @@ int moe_workspace_layout(int64_t T, int64_t d, int64_t f, int E, int64_t C,
   lay->h = take(ec * f * 4);
   lay->h_q = take(ec * f);
   lay->s_h = take(ec * 4);
-  lay->out32 = take((size_t)T * d * 4);
+  lay->slot = take((size_t)E * T * 4);
+  lay->zw = take(ec * d * 4);
   lay->total = off;
   return CONVROT_OK;
 }
@@ -578,16 +618,18 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
   float* h = reinterpret_cast<float*>(ws + lay.h);
   int8_t* h_q = reinterpret_cast<int8_t*>(ws + lay.h_q);
   float* s_h = reinterpret_cast<float*>(ws + lay.s_h);
-  float* out32 = reinterpret_cast<float*>(ws + lay.out32);
+  int32_t* slot = reinterpret_cast<int32_t*>(ws + lay.slot);
+  float* zw = reinterpret_cast<float*>(ws + lay.zw);
 
-  // 1. router softmax (also clears the combine accumulator)
-  if ((rc = softmax_impl(logits_bf16, T, E, s_t, out32, d, st)) != CONVROT_OK) return rc;
+  // 1. router softmax
+  if ((rc = softmax_impl(logits_bf16, T, E, s_t, nullptr, 0, st)) != CONVROT_OK) return rc;
   // 2. rotate + quantise the tokens once (the gate/up rotation is expert-independent)
   if ((rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, T, d, g_gu, x_q, s_x, st)) != CONVROT_OK)
     return rc;
+  // 3. expert-choice top-C (+ each token's slot per expert)
+  if ((rc = topc_impl(s_t, T, E, C, idx, w, slot, st)) != CONVROT_OK) return rc;
   if (C > 0) {
-    // 3. expert-choice top-C, 4. gather each expert's token codes
-    if ((rc = topc_impl(s_t, T, E, C, idx, w, st)) != CONVROT_OK) return rc;
+    // 4. gather each expert's token codes
     if ((rc = gather_impl(x_q, s_x, T, idx, (int64_t)E * C, d, x_g, s_g, st)) != CONVROT_OK)
       return rc;
     // 5. gate/up GEMM with dequant + SwiGLU
@@ -601,19 +643,17 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
     if ((rc = rotquant_impl(h, CONVROT_DTYPE_F32, (int64_t)E * C, f, g_d, h_q, s_h, st)) !=
         CONVROT_OK)
       return rc;
-    // 7. down GEMM with dequant and the router-weighted scatter-add
+    // 7. down GEMM with dequant, times the router weight of each row
     GemmArgs a2{};
     a2.s_a = s_h;
     a2.s_b = s_d;
-    a2.out = out32;
-    a2.idx = idx;
+    a2.out = zw;
     a2.w = w;
-    a2.out_rows = (int)T;
-    if ((rc = launch_gemm<kEpiScatter, true>(h_q, w_d, E, C, d, f, d, a2, st)) != CONVROT_OK)
+    if ((rc = launch_gemm<kEpiWeighted, true>(h_q, w_d, E, C, d, f, d, a2, st)) != CONVROT_OK)
       return rc;
   }
-  // 8. one bf16 rounding of the fp32 combine
-  return convert_impl(out32, T * d, y_bf16, sms, st);
+  // 8. per token: fp32 sum over its experts in ascending order, one bf16 rounding
+  return combine_impl(zw, slot, E, T, C, d, y_bf16, st);
 }
 
 }  // extern "C"

@@ -109,15 +109,22 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_t
 // takes every key above the threshold and the first k keys equal to it in
 // token order. Result: the C largest scores with ties to the lower token
 // index, listed in ascending token order.
+// When `slot` is given it also receives, for every token t, the position c of
+// t in this expert's list (slot[e, t] = c) or -1 if the expert did not pick t.
 __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const float* __restrict__ S_t, int T,
                                                             int C, int32_t* __restrict__ idx,
-                                                            float* __restrict__ w) {
+                                                            float* __restrict__ w,
+                                                            int32_t* __restrict__ slot) {
   const int e = blockIdx.x;
   const uint32_t* u = reinterpret_cast<const uint32_t*>(S_t) + (int64_t)e * T;
   __shared__ uint32_t hist[256];
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t s_digit, s_k;
-  if (C <= 0) return;
+  if (C <= 0) {
+    if (slot != nullptr)
+      for (int t = threadIdx.x; t < T; t += blockDim.x) slot[(int64_t)e * T + t] = -1;
+    return;
+  }
   uint32_t prefix = 0u, mask = 0u, k = (uint32_t)C;
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0u;
@@ -192,15 +199,18 @@ __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const float* __restr
         take = seen < k;
         ++seen;
       }
+      int32_t my_slot = -1;
       if (take) {
         if (pos < (uint32_t)C) {
           idx[(int64_t)e * C + pos] = t;
           w[(int64_t)e * C + pos] = __uint_as_float(bits);
+          my_slot = (int32_t)pos;
         } else {
           atomicOr(&g_device_error, kErrBadIndex);
         }
         ++pos;
       }
+      if (slot != nullptr) slot[(int64_t)e * T + t] = my_slot;
     }
   }
 }
@@ -239,6 +249,95 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const int8_t* __restri
     }
   }
   if (lane == 0) s_dst[r] = __ldg(s_src + t);
+}
+
+// ---------------------------------------------------------------- combine --
+// y[t, :] = bf16(sum over experts e = 0, 1, ..., E-1 that picked t of
+// zw[e * C + slot[e, t], :]) with the sum in fp32 in that order (a token no
+// expert picked gets 0). One CTA of kCombineThreads per token: the first warp
+// lists the token's rows in expert order, then every thread owns up to
+// kCombineQuads float4 columns and loads them for two experts at a time
+// before adding, so many independent reads are in flight.
+constexpr int kCombineMaxE = 256;
+constexpr int kCombineThreads = 128;
+constexpr int kCombineQuads = 4;  // float4 columns per thread per pass
+__global__ void __launch_bounds__(kCombineThreads) combine_rows_kernel(
+    const float* __restrict__ zw, const int32_t* __restrict__ slot, int E, int T, int C, int d,
+    __nv_bfloat16* __restrict__ y) {
+  __shared__ int32_t sel[kCombineMaxE];
+  __shared__ int s_n;
+  const int t = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {
+    int n = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int c = (e < E) ? __ldg(slot + (int64_t)e * T + t) : -1;
+      const bool bad = c >= C;
+      if (bad) atomicOr(&g_device_error, kErrBadIndex);
+      const bool has = c >= 0 && !bad;
+      const unsigned m = __ballot_sync(0xffffffffu, has);
+      if (has) sel[n + __popc(m & ((1u << lane) - 1u))] = e * C + c;
+      n += __popc(m);
+    }
+    if (lane == 0) s_n = n;
+  }
+  __syncthreads();
+  const int n = s_n;
+  const int d4 = d >> 2;
+  uint2* yrow = reinterpret_cast<uint2*>(y + (int64_t)t * d);
+  for (int q0 = threadIdx.x; q0 < d4; q0 += kCombineThreads * kCombineQuads) {
+    float4 acc[kCombineQuads];
+#pragma unroll
+    for (int u = 0; u < kCombineQuads; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    int k = 0;
+    for (; k + 2 <= n; k += 2) {
+      const float4* r0 = reinterpret_cast<const float4*>(zw + (int64_t)sel[k] * d);
+      const float4* r1 = reinterpret_cast<const float4*>(zw + (int64_t)sel[k + 1] * d);
+      float4 a[kCombineQuads], b[kCombineQuads];
+#pragma unroll
+      for (int u = 0; u < kCombineQuads; ++u) {
+        const int q = q0 + u * kCombineThreads;
+        if (q < d4) {
+          a[u] = __ldcs(r0 + q);
+          b[u] = __ldcs(r1 + q);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kCombineQuads; ++u) {
+        acc[u].x = __fadd_rn(__fadd_rn(acc[u].x, a[u].x), b[u].x);
+        acc[u].y = __fadd_rn(__fadd_rn(acc[u].y, a[u].y), b[u].y);
+        acc[u].z = __fadd_rn(__fadd_rn(acc[u].z, a[u].z), b[u].z);
+        acc[u].w = __fadd_rn(__fadd_rn(acc[u].w, a[u].w), b[u].w);
+      }
+    }
+    if (k < n) {
+      const float4* r0 = reinterpret_cast<const float4*>(zw + (int64_t)sel[k] * d);
+#pragma unroll
+      for (int u = 0; u < kCombineQuads; ++u) {
+        const int q = q0 + u * kCombineThreads;
+        if (q < d4) {
+          const float4 a = __ldcs(r0 + q);
+          acc[u].x = __fadd_rn(acc[u].x, a.x);
+          acc[u].y = __fadd_rn(acc[u].y, a.y);
+          acc[u].z = __fadd_rn(acc[u].z, a.z);
+          acc[u].w = __fadd_rn(acc[u].w, a.w);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCombineQuads; ++u) {
+      const int q = q0 + u * kCombineThreads;
+      if (q < d4) {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[u].x, acc[u].y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[u].z, acc[u].w);
+        uint2 o;
+        o.x = *reinterpret_cast<const uint32_t*>(&lo);
+        o.y = *reinterpret_cast<const uint32_t*>(&hi);
+        yrow[q] = o;
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------- convert --
