@@ -133,16 +133,19 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
 
 
-def dist_setup():
+def dist_setup(backend="nccl"):
+    """Process group for N > 1 ranks (one per GPU). Returns (world, rank, local)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
@@ -152,13 +155,30 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(value, world):
+def max_over_ranks(value, world, device="cuda"):
+    """The slowest rank's value (the job is as fast as its slowest replica)."""
     if world == 1:
         return value
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_inputs(cfg, rank):
+    """Inputs of one replica: every rank shares the weights (the model) and gets
+    its own batch of tokens; rank 0's batch is the config's own."""
+    inp = moe_inputs(cfg)
+    if rank > 0:
+        gen = torch.Generator().manual_seed(cfg.seed * 1000 + rank)
+        inp["x"] = (torch.randn(cfg.t, cfg.d, generator=gen) * inp["x"].float().std()).to(torch.bfloat16)
+        inp["logits"] = torch.randn(cfg.t, cfg.n_exp, generator=gen).to(torch.bfloat16)
+    return inp
+
+
+def job_throughput(tokens_per_rank, world, step_s_max):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return world * tokens_per_rank / step_s_max
 
 
 # ------------------------------------------------------------ CPU oracle ----
@@ -304,11 +324,7 @@ def run_ours(args, cfg, world, rank, local):
     W.convrot_device_check()
     dev = torch.device("cuda", local)
     t = cfg.t
-    inp = moe_inputs(cfg)
-    if rank > 0:  # every rank gets its own batch of tokens; weights are shared
-        gen = torch.Generator().manual_seed(cfg.seed * 1000 + rank)
-        inp["x"] = (torch.randn(t, cfg.d, generator=gen) * inp["x"].float().std()).to(torch.bfloat16)
-        inp["logits"] = torch.randn(t, cfg.n_exp, generator=gen).to(torch.bfloat16)
+    inp = rank_inputs(cfg, rank)
     gu, dn = W.quantize_moe_weights(inp["wgu"].to(dev), inp["wd"].to(dev), cfg.g_gu, cfg.g_d)
     wq = (gu, dn)
     x = inp["x"].to(dev)
@@ -405,7 +421,7 @@ def run_ours(args, cfg, world, rank, local):
     block_roof_t = max(work["block_bytes"] / (peaks["hbm_gbs"] * 1e9),
                        work["ops"] / (int8_peak_tops * 1e12))
 
-    value = world * t / mean_step
+    value = job_throughput(t, world, mean_step)
     launches_per_step = 8 if cfg.c > 0 else 3
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -417,7 +433,7 @@ def run_ours(args, cfg, world, rank, local):
                    "parallelism": f"replicas x{world} (independent batches)",
                    "l2": "flushed before every step (256 MiB write outside the timed events)"},
         "gpu_launches": launches_per_step * args.steps,
-        "e2e": {"value": world * t / e2e_step, "unit": UNIT,
+        "e2e": {"value": job_throughput(t, world, e2e_step), "unit": UNIT,
                 "h2d_bytes_per_step": int(x_h.numel() * 2 + l_h.numel() * 2),
                 "d2h_bytes_per_step": int(y_h.numel() * 2)},
         "roofline": roof,
