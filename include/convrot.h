@@ -268,6 +268,10 @@ int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const 
  *   f % g_d == 0, 16 <= f <= 8192; 1 <= E <= 256.
  * The workspace holds every intermediate; its layout is reported by
  * moe_workspace_layout so a caller can inspect each stage after the call.
+ * Inside the call the routing (softmax, top-C) runs on a second stream the
+ * library keeps per device, forked from and joined back to `stream` with
+ * events, so it overlaps the activation rotation; the call as a whole is
+ * still ordered on `stream` (and can be captured on it).
  * ------------------------------------------------------------------------- */
 typedef struct {
   size_t x_q;      /* [T, d] int8     rotated activation codes      */

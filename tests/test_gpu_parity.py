@@ -396,6 +396,36 @@ def test_moe_block_small_end_to_end(name):
     assert np.array_equal(y_np[clean], y_ref[clean])
 
 
+def test_moe_block_graph_capture_matches_eager():
+    """The whole call (with its side-stream routing fork) captured in a CUDA
+    graph and replayed on fresh inputs gives the eager result."""
+    cfg = MOE_CONFIGS["moe_small"]
+    inp = moe_inputs(cfg)
+    gu, dn = W.quantize_moe_weights(inp["wgu"].cuda(), inp["wd"].cuda(), cfg.g_gu, cfg.g_d)
+    x = inp["x"].cuda()
+    logits = inp["logits"].cuda()
+    ws = torch.empty(W.moe_workspace_size(cfg.t, cfg.d, cfg.f, cfg.n_exp, cfg.c), dtype=torch.uint8,
+                     device="cuda")
+    y = torch.empty(cfg.t, cfg.d, dtype=torch.bfloat16, device="cuda")
+    W.moe_expert_choice_forward(x, logits, gu, dn, cfg.c, cfg.g_gu, cfg.g_d, y=y, workspace=ws)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        W.moe_expert_choice_forward(x, logits, gu, dn, cfg.c, cfg.g_gu, cfg.g_d, y=y, workspace=ws)
+    gen = torch.Generator().manual_seed(77)
+    x2 = torch.randn(cfg.t, cfg.d, generator=gen).to(torch.bfloat16)
+    l2 = torch.randn(cfg.t, cfg.n_exp, generator=gen).to(torch.bfloat16)
+    x.copy_(x2.cuda())
+    logits.copy_(l2.cuda())
+    graph.replay()
+    torch.cuda.synchronize()
+    y_graph = y.clone()
+    y_eager = W.moe_expert_choice_forward(x2.cuda(), l2.cuda(), gu, dn, cfg.c, cfg.g_gu, cfg.g_d)
+    torch.cuda.synchronize()
+    assert torch.equal(y_graph, y_eager)
+    del graph
+
+
 def test_moe_block_capacity_extremes():
     base = MOE_CONFIGS["moe_small_c40"]
     for c in (0, 1, base.t):

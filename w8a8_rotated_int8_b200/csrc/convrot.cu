@@ -31,6 +31,43 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
+// Second stream of a device for work of one call that can run beside the
+// caller's stream (joined back with events before its results are used).
+// Created once per device; `mu` serialises the fork/join of concurrent calls.
+struct SideStream {
+  bool ready = false;
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join = nullptr;
+  std::mutex mu;
+};
+SideStream g_side[kMaxDevices];
+
+int side_stream(SideStream** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return CONVROT_ERR_UNSUPPORTED_DEVICE;
+  }
+  SideStream& ss = g_side[dev];
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  if (!ss.ready) {
+    // highest priority: the routing chain is the longer branch of the fork,
+    // so its CTAs should take SMs first as they free up
+    int least = 0, greatest = 0;
+    cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      return CONVROT_ERR_CUDA;
+    }
+    ss.ready = true;
+  }
+  *out = &ss;
+  return CONVROT_OK;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -621,13 +658,26 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
   int32_t* slot = reinterpret_cast<int32_t*>(ws + lay.slot);
   float* zw = reinterpret_cast<float*>(ws + lay.zw);
 
+  // Routing (1, 3) runs on the side stream while the caller's stream rotates
+  // and quantises the tokens (2); the streams join before the gather.
+  SideStream* ss = nullptr;
+  if ((rc = side_stream(&ss)) != CONVROT_OK) return rc;
+  std::lock_guard<std::mutex> side_lock(ss->mu);
+  if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
   // 1. router softmax
-  if ((rc = softmax_impl(logits_bf16, T, E, s_t, nullptr, 0, st)) != CONVROT_OK) return rc;
-  // 2. rotate + quantise the tokens once (the gate/up rotation is expert-independent)
-  if ((rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, T, d, g_gu, x_q, s_x, st)) != CONVROT_OK)
-    return rc;
+  int rc_side = softmax_impl(logits_bf16, T, E, s_t, nullptr, 0, ss->stream);
   // 3. expert-choice top-C (+ each token's slot per expert)
-  if ((rc = topc_impl(s_t, T, E, C, idx, w, slot, st)) != CONVROT_OK) return rc;
+  if (rc_side == CONVROT_OK) rc_side = topc_impl(s_t, T, E, C, idx, w, slot, ss->stream);
+  // 2. rotate + quantise the tokens once (the gate/up rotation is expert-independent)
+  rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, T, d, g_gu, x_q, s_x, st);
+  // the join is recorded even after a failed launch so the side stream never dangles
+  if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess ||
+      cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  if (rc_side != CONVROT_OK) return rc_side;
+  if (rc != CONVROT_OK) return rc;
   if (C > 0) {
     // 4. gather each expert's token codes
     if ((rc = gather_impl(x_q, s_x, T, idx, (int64_t)E * C, d, x_g, s_g, st)) != CONVROT_OK)
