@@ -36,7 +36,7 @@ METRIC = "W8A8 ConvRot MoE block tokens/s"
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
 # kernel, from the ncu capture summarised in profiles/ (per config); to be set
 # to None whenever that kernel changes
-DOMINANT_TRAFFIC_BYTES = {"moe_T8192": 486.5e6}
+DOMINANT_TRAFFIC_BYTES = {}
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 

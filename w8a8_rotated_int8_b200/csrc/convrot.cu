@@ -99,6 +99,16 @@ void set_gemm_attrs() {
                        cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
   cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiWeighted, BT>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
+  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiI32, BT>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
+  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiBf16, BT>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
+  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiSwiglu, BT>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
+  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiScatter, BT>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
+  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiWeighted, BT>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
 }
 
 // Per-device one-time setup: capability check, SM count, kernel attributes.
@@ -277,6 +287,37 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
   args.NB = (int)NB;
   args.K = (int)K;
   args.n_out = (int)n_out;
+  // CTA pairs (M = 256 tiles) once a group has more than 128 rows and the
+  // weight boxes are whole 128-row blocks
+  const bool pairs = M > gemm::BM && box_b == 128 && sms >= 2;
+  if (pairs) {
+    args.m_blocks = (int)cdiv(M, gemm2::BM);
+    const int64_t n_tile = (EPI == kEpiSwiglu) ? gemm::BN / 2 : gemm::BN;
+    args.n_blocks = (int)cdiv(n_out, n_tile);
+    args.k_blocks = (int)cdiv(K, gemm::BK);
+    const int64_t tiles = G * args.m_blocks * args.n_blocks;
+    if (tiles >= ((int64_t)1 << 30)) return CONVROT_ERR_INVALID_ARG;
+    args.num_tiles = (int)tiles;
+    args.box_bytes = 2 * (128 + 128) * gemm::BK;  // both CTAs' A and B boxes
+    const int grid = 2 * (int)std::min<int64_t>(tiles, sms / 2);
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(grid);
+    lc.blockDim = dim3(gemm::THREADS);
+    lc.dynamicSmemBytes = gemm2::SMEM_BYTES;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&lc, gemm_s8_tcgen05_pair_kernel<EPI, BT>, ta, tb, args) != cudaSuccess) {
+      cudaGetLastError();
+      return CONVROT_ERR_CUDA;
+    }
+    return launch_status();
+  }
   args.m_blocks = (int)cdiv(M, gemm::BM);
   const int64_t n_tile = (EPI == kEpiSwiglu) ? gemm::BN / 2 : gemm::BN;
   args.n_blocks = (int)cdiv(n_out, n_tile);
