@@ -24,8 +24,9 @@
  *  - router score: per-token softmax over the experts (fp64, rounded to
  *    fp32); top-C ties go to the lower token index; each expert's tokens are
  *    listed in ascending order;
- *  - dequant y = fp32(acc) * (s_w * s_x); h = silu(g) * u in fp32; combine
- *    out32[t] += w * z in fp32, one bf16 rounding at the end.
+ *  - dequant y = fp32(acc) * (s_w * s_x); h = silu(g) * u in fp32; the down
+ *    projection's output z is bf16 (a W8A8 linear with BF16 outputs); combine
+ *    out32[t] += fp32(w * z) in fp32, one bf16 rounding at the end.
  *
  * Conventions for every call:
  *  - All buffers are owned by the caller; the library allocates nothing.
@@ -147,16 +148,19 @@ int convrot_router_softmax(const void* logits_bf16, int64_t T, int E, float* s_t
 int convrot_topc(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float* w,
                  int32_t* slot, void* stream);
 
-/* Combine. "MLX Nucleus-Image", table "Conversion notes" (the experts'
- * outputs are scattered back to their tokens):
- *   y[t, :] = bf16(sum over e = 0, 1, ..., E-1 with slot[e, t] >= 0 of
- *             zw[e * C + slot[e, t], :]), summed in fp32 in that order;
- *   a token no expert picked gets 0.
- *   zw    device, [E * C, d] fp32 router-weighted expert outputs
+/* Router-weighted combine. "MLX Nucleus-Image", table "Conversion notes" (the
+ * experts' outputs are scattered back to their tokens), weighted by the
+ * router scores of the choices:
+ *   y[t, :] = bf16(sum over e = 0, 1, ..., E-1 with c = slot[e, t] >= 0 of
+ *             fp32(w[e * C + c] * z[e * C + c, :])), every product rounded to
+ *             fp32 and added in fp32 in that order; a token no expert picked
+ *             gets 0.
+ *   z     device, [E * C, d] bf16 expert outputs (down projection)
+ *   w     device, [E * C] fp32 router weights (convrot_topc)
  *   slot  device, [E, T] int32 from convrot_topc;  y device, [T, d] bf16
- *   1 <= E <= 256, d % 4 == 0. */
-int convrot_combine_rows(const float* zw, const int32_t* slot, int E, int64_t T, int64_t C,
-                         int64_t d, void* y_bf16, void* stream);
+ *   1 <= E <= 256, d % 8 == 0. */
+int convrot_combine_rows(const void* z_bf16, const float* w, const int32_t* slot, int E,
+                         int64_t T, int64_t C, int64_t d, void* y_bf16, void* stream);
 
 /* Gather rows: dst[r, :] = src[idx[r], :], s_dst[r] = s_src[idx[r]].
  *   src [n_src, K] int8, s_src [n_src] fp32, idx [n_rows] int32 (each in
@@ -197,12 +201,6 @@ int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, c
 int convrot_i8_gemm_scatter(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
                             int b_layout, const int32_t* idx, const float* w, int64_t G, int64_t M,
                             int64_t N, int64_t K, float* out32, int64_t T, void* stream);
-
-/* Router-weighted epilogue: zw[g * M + m, n] = w[g, m] * (fp32(acc) *
- * (s_b[g, n] * s_a[g, m])); zw device [G * M, N] fp32, w [G, M] fp32. */
-int convrot_i8_gemm_weighted(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
-                             int b_layout, const float* w, int64_t G, int64_t M, int64_t N,
-                             int64_t K, float* zw, void* stream);
 
 /* y = bf16(x) (nearest even), n elements, n % 4 == 0. */
 int convrot_f32_to_bf16(const float* x, int64_t n, void* y_bf16, void* stream);
@@ -262,8 +260,9 @@ int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const 
  *           E matrices of d rows x f;  s_d device, [E, d] fp32
  *   C       tokens per expert, 0 <= C <= T
  *   y       device, [T, d] bf16 = bf16(sum over the experts that chose t, in
- *           ascending expert order, of w[e, c] * down_e(requant(silu(gate_e) *
- *           up_e))), the sum in fp32
+ *           ascending expert order, of w[e, c] * z_e), the sum in fp32, where
+ *           z_e = bf16(down_e(requant(silu(gate_e) * up_e))) is the expert's
+ *           BF16 output
  *   Sizes: d % 16 == 0, d % g_gu == 0, 16 <= d <= 8192; f % 16 == 0,
  *   f % g_d == 0, 16 <= f <= 8192; 1 <= E <= 256.
  * The workspace holds every intermediate; its layout is reported by
@@ -285,7 +284,7 @@ typedef struct {
   size_t h_q;      /* [E, C, f] int8  rotated, requantised h        */
   size_t s_h;      /* [E, C] fp32     scales of h                   */
   size_t slot;     /* [E, T] int32    slot of each token per expert */
-  size_t zw;       /* [E, C, d] fp32  router-weighted expert outputs */
+  size_t z;        /* [E, C, d] bf16  expert outputs (down projection) */
   size_t total;    /* bytes required                                */
 } convrot_moe_layout_t;
 

@@ -42,8 +42,12 @@ Readings of what the pages leave open (each is fixed here once):
 * Dequant: fp32(acc) * (s_w * s_x), the scale product first, IEEE fp32.
 * SwiGLU: h = (g / (1 + e)) * u in fp32 with e = fp32(exp(-g)) (the
   exponential correctly rounded to fp32, computed here through fp64).
-* Combine: out32[t] += w * z in fp32 over experts in ascending order, one
-  bf16 round-to-nearest-even at the end; tokens no expert picked give 0.
+* Down projection output: z = bf16(fp32(acc) * (s_d * s_h)), since each
+  expert linear is a W8A8 ConvRot linear with BF16 outputs (Nucleus-Image,
+  "Quantization"). The gate/up output is not rounded: it feeds SwiGLU inside
+  the same fused step, in fp32.
+* Combine: out32[t] += fp32(w * z) in fp32 over experts in ascending order,
+  one bf16 round-to-nearest-even at the end; tokens no expert picked give 0.
 
 Numeric inputs are NumPy arrays. bf16 tensors are passed as float32 arrays
 holding bf16-representable values (NumPy has no bf16 type).
@@ -258,7 +262,7 @@ def moe_block(x, logits, wgu_q, s_gu, wd_q, s_d, c, g_gu=256, g_d=64,
     idx, w = expert_choice_topc(scores, c)
     out32 = np.zeros((t, d), dtype=np.float32)
     inter = {"x_q": x_q, "s_x": s_x, "scores": scores, "idx": idx, "w": w,
-             "h": {}, "h_q": {}, "s_h": {}}
+             "h": {}, "h_q": {}, "s_h": {}, "z": {}}
     for e in (range(n_exp) if experts is None else experts):
         rows = idx[e]
         if out_tokens is not None:
@@ -270,11 +274,14 @@ def moe_block(x, logits, wgu_q, s_gu, wd_q, s_d, c, g_gu=256, g_d=64,
         gate, up = y[:, :f], y[:, f:]
         h = (silu_f32(gate) * up).astype(np.float32)
         h_q, s_h = rotquant(h, g_d)
-        z = dequant(int_gemm(h_q, wd_q[e]), s_d[e], s_h)
-        # rows are distinct within an expert, so fancy-index += is exact
+        # the down projection is a W8A8 linear with BF16 output
+        z = bf16_round(dequant(int_gemm(h_q, wd_q[e]), s_d[e], s_h))
+        # rows are distinct within an expert, so fancy-index += is exact;
+        # the product w*z is rounded to fp32, then added in fp32
         out32[rows] = out32[rows] + (w[e][sel][:, None] * z).astype(np.float32)
         if keep:
             inter["h"][e], inter["h_q"][e], inter["s_h"][e] = h, h_q, s_h
+            inter["z"][e] = z
     y_out = bf16_round(out32)
     if keep:
         inter["out32"] = out32

@@ -90,4 +90,4 @@ def test_workspace_layout_is_disjoint_and_aligned(lib):
     offs = sorted(lay[n] for n in names)
     assert all(o % 256 == 0 for o in offs)
     assert len(set(offs)) == len(offs)
-    assert lay["total"] >= lay["zw"] + 64 * 256 * 2048 * 4
+    assert lay["total"] >= lay["z"] + 64 * 256 * 2048 * 2

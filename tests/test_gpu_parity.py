@@ -1,9 +1,10 @@
 """GPU parity: every stage of the CUDA path through the C ABI against the oracle.
 
 Bar: bit-exact codes, scales, int32 accumulators, top-C index sets and
-dequantised outputs; the SwiGLU output and the fp32 combine within the bounds
-their arithmetic allows (CUDA expf vs a correctly rounded exp; atomic
-accumulation order); the block output within the 1e-2 max-relative budget.
+dequantised outputs and the router-weighted combine; the SwiGLU output and the
+atomic scatter epilogue within the bounds their arithmetic allows (CUDA expf vs
+a correctly rounded exp; atomic accumulation order); the block output within
+the 1e-2 max-relative budget.
 """
 
 import numpy as np
@@ -55,6 +56,7 @@ def bf16_activations(rows, k, seed, outliers=True):
 @pytest.mark.parametrize("rows,k,g", [
     (64, 256, 256), (300, 768, 256), (257, 2048, 256), (5, 8192, 256), (33, 320, 64),
     (100, 1536, 64), (77, 512, 16), (50, 256, 4), (40, 64, 1), (3, 16, 16), (1, 4096, 64),
+    (20000, 2048, 256),  # many more row groups than resident CTAs (persistent loop)
 ])
 def test_rotquant_bf16_bit_exact(rows, k, g):
     x = bf16_activations(rows, k, seed=rows * 7 + k)
@@ -64,7 +66,8 @@ def test_rotquant_bf16_bit_exact(rows, k, g):
     assert np.array_equal(q.cpu().numpy(), q_ref)
 
 
-@pytest.mark.parametrize("rows,k,g", [(160, 320, 64), (513, 1536, 64), (64, 2048, 256)])
+@pytest.mark.parametrize("rows,k,g", [(160, 320, 64), (513, 1536, 64), (64, 2048, 256),
+                                      (9001, 1536, 64)])
 def test_rotquant_f32_bit_exact(rows, k, g):
     gen = torch.Generator().manual_seed(k)
     a = torch.randn(rows, k, generator=gen)
@@ -110,7 +113,8 @@ def _ulp_diff(a, b):
     return np.abs(ai - bi)
 
 
-@pytest.mark.parametrize("t,e", [(8192, 64), (1000, 8), (33, 256), (1, 1)])
+@pytest.mark.parametrize("t,e", [(8192, 64), (1000, 8), (33, 256), (1, 1), (500, 100),
+                                 (77, 200)])
 def test_router_softmax(t, e):
     gen = torch.Generator().manual_seed(t + e)
     logits = torch.randn(t, e, generator=gen).to(torch.bfloat16)
@@ -121,12 +125,17 @@ def test_router_softmax(t, e):
     assert (d != 0).mean() <= 1e-4
 
 
+# T <= 1024, 2048, 4096, 8192, 16384 scores per expert use the register-resident
+# kernel with 1, 2, 4, 8, 16 tokens per thread (vector loads when T % 4 == 0);
+# larger T the general one
 @pytest.mark.parametrize("t,e,c", [(8192, 64, 256), (2048, 64, 64), (1000, 8, 100),
-                                   (300, 5, 300), (50, 3, 1), (1, 2, 1), (64, 4, 0)])
+                                   (300, 5, 300), (50, 3, 1), (1, 2, 1), (64, 4, 0),
+                                   (16384, 2, 512), (8190, 3, 255), (5000, 4, 700),
+                                   (20000, 3, 600), (4097, 2, 4097)])
 def test_topc_exact_given_scores(t, e, c):
     gen = torch.Generator().manual_seed(t * 3 + c)
     s = torch.softmax(torch.randn(t, e, generator=gen), dim=1).numpy().astype(np.float32)
-    if t == 1000:
+    if t in (1000, 5000, 20000):
         s = (np.floor(s * 16) / 16).astype(np.float32)  # heavy ties
     idx, w = W.convrot_topc(torch.from_numpy(np.ascontiguousarray(s.T)).cuda(), c)
     idx_ref, w_ref = O.expert_choice_topc(s, c)
@@ -134,15 +143,16 @@ def test_topc_exact_given_scores(t, e, c):
     assert np.array_equal(w.cpu().numpy(), w_ref)
 
 
-def test_topc_slot_table_inverts_idx():
-    gen = torch.Generator().manual_seed(5)
-    s = torch.softmax(torch.randn(700, 6, generator=gen), dim=1).numpy().astype(np.float32)
-    idx, w, slot = W.convrot_topc(torch.from_numpy(np.ascontiguousarray(s.T)).cuda(), 90,
+@pytest.mark.parametrize("t,c", [(700, 90), (8192, 256), (3001, 77), (17000, 300)])
+def test_topc_slot_table_inverts_idx(t, c):
+    gen = torch.Generator().manual_seed(5 + t)
+    s = torch.softmax(torch.randn(t, 6, generator=gen), dim=1).numpy().astype(np.float32)
+    idx, w, slot = W.convrot_topc(torch.from_numpy(np.ascontiguousarray(s.T)).cuda(), c,
                                   with_slot=True)
     idx, slot = idx.cpu().numpy(), slot.cpu().numpy()
-    expect = np.full((6, 700), -1, np.int32)
+    expect = np.full((6, t), -1, np.int32)
     for e in range(6):
-        expect[e, idx[e]] = np.arange(90)
+        expect[e, idx[e]] = np.arange(c)
     assert np.array_equal(slot, expect)
 
 
@@ -267,34 +277,44 @@ def test_gemm_scatter(layout):
 
 
 @pytest.mark.parametrize("layout", ["rows", "tiles"])
-def test_gemm_weighted_bit_exact(layout):
-    g, m, n, k = 3, 100, 320, 512
+@pytest.mark.parametrize("g,m", [(3, 100), (2, 300)])
+def test_gemm_bf16_grouped_rows_bit_exact(g, m, layout):
+    """The experts' down projection: grouped bf16 output rows in (group, row)
+    order, through the 1-CTA (M <= 128) and the CTA-pair (M > 128) kernels."""
+    n, k = 320, 512
     a = _codes((g, m, k), 10)
     b = _codes((g, n, k), 11)
     s_a = torch.rand(g, m) * 0.05 + 1e-3
     s_b = torch.rand(g, n) * 1e-4 + 1e-6
-    w = torch.rand(g, m)
     bb = b.cuda() if layout == "rows" else _tiled_codes(b)
-    zw = W.convrot_i8_gemm_weighted(a.cuda(), s_a.cuda(), bb, s_b.cuda(), w.cuda()).cpu().numpy()
+    z = W.convrot_i8_gemm_bf16(a.cuda(), s_a.cuda(), bb, s_b.cuda()).cpu()
     for gi in range(g):
-        z = O.dequant(O.int_gemm(a[gi].numpy(), b[gi].numpy()), s_b[gi].numpy(), s_a[gi].numpy())
-        assert np.array_equal(zw[gi * m:(gi + 1) * m], (w[gi].numpy()[:, None] * z).astype(np.float32))
+        ref = O.bf16_round(O.dequant(O.int_gemm(a[gi].numpy(), b[gi].numpy()),
+                                     s_b[gi].numpy(), s_a[gi].numpy()))
+        assert np.array_equal(np32(z[gi]), ref)
 
 
-def test_combine_sums_in_expert_order():
-    e_n, t, c, d = 5, 300, 40, 256
-    gen = torch.Generator().manual_seed(3)
-    zw = (torch.randn(e_n * c, d, generator=gen) * 10.0 ** torch.randint(-3, 3, (e_n * c, 1),
-                                                                        generator=gen)).float()
+@pytest.mark.parametrize("e_n,t,c,d", [(5, 300, 40, 256), (7, 64, 64, 2056), (3, 50, 0, 64),
+                                       (70, 1000, 30, 128), (64, 5000, 160, 2048)])
+def test_combine_sums_in_expert_order(e_n, t, c, d):
+    """y[t] = bf16(sum_e fp32(w * z)) in ascending expert order; d = 2056
+    leaves a ragged tail of 8-column vectors past two full passes of 2048."""
+    gen = torch.Generator().manual_seed(3 + d)
+    z = (torch.randn(e_n * c, d, generator=gen) * 10.0 ** torch.randint(-3, 3, (e_n * c, 1),
+                                                                       generator=gen))
+    z = z.to(torch.bfloat16)
+    w = torch.rand(e_n * c, generator=gen)
     slot = torch.full((e_n, t), -1, dtype=torch.int32)
     for e in range(e_n):
         toks = torch.randperm(t, generator=gen)[:c].sort().values
         slot[e, toks] = torch.arange(c, dtype=torch.int32)
-    y = W.convrot_combine_rows(zw.cuda(), slot.cuda(), c).cpu()
+    y = W.convrot_combine_rows(z.cuda(), w.cuda(), slot.cuda(), c).cpu()
     ref = np.zeros((t, d), np.float32)
-    for e in range(e_n):       # fp32, ascending expert order
+    zf, wf = np32(z), w.numpy()
+    for e in range(e_n):       # fp32 products, fp32 sums, ascending expert order
         toks = np.nonzero(slot[e].numpy() >= 0)[0]
-        ref[toks] = ref[toks] + zw.numpy()[e * c + slot[e].numpy()[toks]]
+        rows = e * c + slot[e].numpy()[toks]
+        ref[toks] = ref[toks] + (wf[rows][:, None] * zf[rows]).astype(np.float32)
     assert np.array_equal(np32(y), O.bf16_round(ref))
 
 
@@ -392,6 +412,8 @@ def test_moe_block_small_end_to_end(name):
         bad = (np.any(v["h_q"][e].cpu().numpy() != it["h_q"][e], axis=1)
                | (v["s_h"][e].cpu().numpy() != it["s_h"][e]))
         touched.update(it["idx"][e][bad].tolist())
+        # the experts' bf16 outputs of the rows whose codes agree are bit-exact
+        assert np.array_equal(np32(v["z"][e])[~bad], it["z"][e][~bad])
     clean = np.setdiff1d(np.arange(cfg.t), np.array(sorted(touched), dtype=np.int64))
     assert np.array_equal(y_np[clean], y_ref[clean])
 

@@ -18,7 +18,6 @@ from .binding import (  # noqa: F401
     convrot_i8_gemm_i32,
     convrot_i8_gemm_scatter,
     convrot_i8_gemm_swiglu,
-    convrot_i8_gemm_weighted,
     convrot_linear_workspace_size,
     convrot_quantize_weights,
     convrot_quantize_weights_tiled,

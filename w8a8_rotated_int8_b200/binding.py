@@ -39,7 +39,7 @@ class ConvrotError(RuntimeError):
 
 class MoeLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
-                ("x_q", "s_x", "s_t", "idx", "w", "x_g", "s_g", "h", "h_q", "s_h", "slot", "zw",
+                ("x_q", "s_x", "s_t", "idx", "w", "x_g", "s_g", "h", "h_q", "s_h", "slot", "z",
                  "total")]
 
 
@@ -63,8 +63,7 @@ _SIGNATURES = {
     "convrot_quantize_weights_tiled": (_I, [_P, _I64, _I64, _I64, _I, _P, _P, _P]),
     "convrot_router_softmax": (_I, [_P, _I64, _I, _P, _P]),
     "convrot_topc": (_I, [_P, _I64, _I, _I64, _P, _P, _P, _P]),
-    "convrot_combine_rows": (_I, [_P, _P, _I, _I64, _I64, _I64, _P, _P]),
-    "convrot_i8_gemm_weighted": (_I, [_P, _P, _P, _P, _I, _P, _I64, _I64, _I64, _I64, _P, _P]),
+    "convrot_combine_rows": (_I, [_P, _P, _P, _I, _I64, _I64, _I64, _P, _P]),
     "convrot_gather_rows": (_I, [_P, _P, _I64, _P, _I64, _I64, _P, _P, _P]),
     "convrot_i8_gemm_i32": (_I, [_P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
     "convrot_i8_gemm_bf16": (_I, [_P, _P, _P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
@@ -240,16 +239,18 @@ def convrot_topc(s_t, c, with_slot=False, stream=None):
     return (idx, w, slot) if with_slot else (idx, w)
 
 
-def convrot_combine_rows(zw, slot, c, stream=None):
-    """zw [E*C, d] fp32 + slot [E, T] -> y [T, d] bf16 (per-token fp32 sum in
-    ascending expert order)."""
-    _need(zw, torch.float32, "zw")
+def convrot_combine_rows(z, w, slot, c, stream=None):
+    """z [E*C, d] bf16 expert outputs, w [E*C] fp32 router weights, slot
+    [E, T] -> y [T, d] bf16 (per token, the fp32 sum of w*z over its experts
+    in ascending expert order)."""
+    _need(z, torch.bfloat16, "z")
+    _need(w, torch.float32, "w")
     _need(slot, torch.int32, "slot")
     e, t = slot.shape
-    d = zw.shape[-1]
-    y = torch.empty((t, d), dtype=torch.bfloat16, device=zw.device)
-    _check(lib().convrot_combine_rows(_p(zw), _p(slot), e, t, c, d, _p(y), _stream(stream)),
-           "convrot_combine_rows")
+    d = z.shape[-1]
+    y = torch.empty((t, d), dtype=torch.bfloat16, device=z.device)
+    _check(lib().convrot_combine_rows(_p(z), _p(w), _p(slot), e, t, c, d, _p(y),
+                                      _stream(stream)), "convrot_combine_rows")
     return y
 
 
@@ -329,17 +330,6 @@ def convrot_i8_gemm_scatter(a, s_a, b, s_b, idx, w, out32, stream=None):
                                          n, k, _p(out32), out32.shape[0], _stream(stream)),
            "convrot_i8_gemm_scatter")
     return out32
-
-
-def convrot_i8_gemm_weighted(a, s_a, b, s_b, w, stream=None):
-    """zw[g*M + m, n] = w[g, m] * dequant(acc)[g, m, n] -> zw [G*M, N] fp32."""
-    g, m, n, k, bt, lay = _gemm_dims(a, b)
-    for t, nm in ((s_a, "s_a"), (s_b, "s_b"), (w, "w")):
-        _need(t, torch.float32, nm)
-    zw = torch.empty((g * m, n), dtype=torch.float32, device=a.device)
-    _check(lib().convrot_i8_gemm_weighted(_p(a), _p(s_a), _p(bt), _p(s_b), lay, _p(w), g, m, n, k,
-                                          _p(zw), _stream(stream)), "convrot_i8_gemm_weighted")
-    return zw
 
 
 def convrot_f32_to_bf16(x, stream=None):
@@ -457,5 +447,5 @@ def moe_stage_views(workspace, t, d, f, e, c) -> dict:
         "h_q": view("h_q", torch.int8, (e, c, f)),
         "s_h": view("s_h", torch.float32, (e, c)),
         "slot": view("slot", torch.int32, (e, t)),
-        "zw": view("zw", torch.float32, (e, c, d)),
+        "z": view("z", torch.bfloat16, (e, c, d)),
     }

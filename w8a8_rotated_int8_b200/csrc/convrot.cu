@@ -97,8 +97,6 @@ void set_gemm_attrs() {
                        cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
   cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiScatter, BT>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
-  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiWeighted, BT>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
   cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiI32, BT>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
   cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiBf16, BT>,
@@ -106,8 +104,6 @@ void set_gemm_attrs() {
   cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiSwiglu, BT>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
   cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiScatter, BT>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
-  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiWeighted, BT>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
 }
 
@@ -153,9 +149,39 @@ int launch_status() {
 }
 
 // --------------------------------------------------------------- rotquant --
+constexpr int kRqWarpThreads = 128;
+
+template <typename InT, int G, int SEG>
+void launch_rq_warp(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
+                    cudaStream_t st) {
+  const int64_t units = (rows + (32 / SEG) - 1) / (32 / SEG);  // warp-rows
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotquant_warp_kernel<InT, G, SEG>,
+                                                    kRqWarpThreads, 0) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  int sms = 0;
+  device_setup(&sms);
+  const int64_t ctas = (units + kRqWarpThreads / 32 - 1) / (kRqWarpThreads / 32);
+  const int64_t grid = std::min<int64_t>(ctas, (int64_t)per_sm * std::max(sms, 1));
+  rotquant_warp_kernel<InT, G, SEG><<<(unsigned)grid, kRqWarpThreads, 0, st>>>(
+      reinterpret_cast<const InT*>(x), rows, K, q, s, out);
+}
+
 template <typename InT, int G>
 void launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
                cudaStream_t st) {
+  // K % 64 == 0, K <= 2048: one warp segment of SEG lanes per row, 64
+  // elements per lane (G = 256 needs at least the four lanes of one group)
+  if (K % 64 == 0 && K <= 2048) {
+    const int lanes = K / 64;
+    if (lanes <= 1 && G < 256) return launch_rq_warp<InT, G, (G < 256 ? 1 : 4)>(x, rows, K, q, s, out, st);
+    if (lanes <= 2 && G < 256) return launch_rq_warp<InT, G, (G < 256 ? 2 : 4)>(x, rows, K, q, s, out, st);
+    if (lanes <= 4) return launch_rq_warp<InT, G, 4>(x, rows, K, q, s, out, st);
+    if (lanes <= 8) return launch_rq_warp<InT, G, 8>(x, rows, K, q, s, out, st);
+    if (lanes <= 16) return launch_rq_warp<InT, G, 16>(x, rows, K, q, s, out, st);
+    return launch_rq_warp<InT, G, 32>(x, rows, K, q, s, out, st);
+  }
   const int nch = K / 16;
   int tpr;
   if (nch <= 32) {
@@ -167,7 +193,16 @@ void launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut ou
   // whole rows per CTA: a CTA never holds threads beyond rpc * tpr
   const int rpc = std::max(1, kRqThreads / tpr);
   const int threads = rpc * tpr;
-  const int64_t grid = (rows + rpc - 1) / rpc;
+  const int64_t groups = (rows + rpc - 1) / rpc;
+  // persistent: as many CTAs as fit on the device at once
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotquant_kernel<InT, G>, threads, 0) !=
+          cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  int sms = 0;
+  device_setup(&sms);
+  const int64_t grid = std::min<int64_t>(groups, (int64_t)per_sm * std::max(sms, 1));
   rotquant_kernel<InT, G><<<(unsigned)grid, threads, 0, st>>>(
       reinterpret_cast<const InT*>(x), rows, K, tpr, q, s, out);
 }
@@ -342,24 +377,71 @@ int launch_gemm_layout(int b_layout, const int8_t* a, const int8_t* b, int64_t G
 int topc_impl(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float* w,
               int32_t* slot, cudaStream_t st) {
   if (E == 0 || (C == 0 && slot == nullptr)) return CONVROT_OK;
-  topc_kernel<<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+  // scores held in registers when T <= 16 per thread; the general kernel
+  // re-reads them from memory on every pass
+  const int per_thread = (int)((T + kTopcThreads - 1) / kTopcThreads);
+  if (per_thread <= 1)
+    topc_reg_kernel<1><<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+  else if (per_thread <= 2)
+    topc_reg_kernel<2><<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+  else if (per_thread <= 4)
+    topc_reg_kernel<4><<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+  else if (per_thread <= 8)
+    topc_reg_kernel<8><<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+  else if (per_thread <= 16)
+    topc_reg_kernel<16><<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+  else
+    topc_kernel<<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
   return launch_status();
 }
 
-int combine_impl(const float* zw, const int32_t* slot, int E, int64_t T, int64_t C, int64_t d,
-                 void* y, cudaStream_t st) {
+template <int NJ>
+void launch_combine(const void* z, const float* w, const int32_t* slot, int E, int64_t T,
+                    int64_t C, int64_t d, void* y, int sms, cudaStream_t st) {
+  // persistent: resident CTAs only (two per SM at <= 128 registers), one warp
+  // per token at a time
+  const int64_t grid = std::min<int64_t>((T + kCombineWarps - 1) / kCombineWarps, 2 * sms);
+  combine_rows_kernel<NJ><<<(unsigned)grid, kCombineThreads, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(z), w, slot, E, (int)T, (int)C, (int)d,
+      reinterpret_cast<__nv_bfloat16*>(y));
+}
+
+// E <= 256 (checked by the entry points)
+int combine_impl(const void* z, const float* w, const int32_t* slot, int E, int64_t T, int64_t C,
+                 int64_t d, void* y, int sms, cudaStream_t st) {
   if (T == 0) return CONVROT_OK;
-  combine_rows_kernel<<<(unsigned)T, kCombineThreads, 0, st>>>(
-      zw, slot, E, (int)T, (int)C, (int)d, reinterpret_cast<__nv_bfloat16*>(y));
+  if (E <= 32)
+    launch_combine<1>(z, w, slot, E, T, C, d, y, sms, st);
+  else if (E <= 64)
+    launch_combine<2>(z, w, slot, E, T, C, d, y, sms, st);
+  else if (E <= 128)
+    launch_combine<4>(z, w, slot, E, T, C, d, y, sms, st);
+  else
+    launch_combine<8>(z, w, slot, E, T, C, d, y, sms, st);
   return launch_status();
 }
 
-int softmax_impl(const void* logits, int64_t T, int E, float* s_t, float* clear,
-                 int64_t clear_cols, cudaStream_t st) {
-  if (T == 0) return CONVROT_OK;
+template <int NJ>
+void launch_softmax(const void* logits, int64_t T, int E, float* s_t, cudaStream_t st) {
   const int64_t grid = (T + kSmTokens - 1) / kSmTokens;
-  router_softmax_kernel<<<(unsigned)grid, 32 * kSmTokens, (size_t)E * kSmTokens * sizeof(float), st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(logits), (int)T, E, s_t, clear, clear_cols);
+  router_softmax_kernel<NJ><<<(unsigned)grid, 32 * kSmTokens,
+                              (size_t)E * kSmTokens * sizeof(float), st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(logits), (int)T, E, s_t);
+}
+
+// E <= 256 (checked by the entry points): NJ = ceil(E / 32) experts per lane
+int softmax_impl(const void* logits, int64_t T, int E, float* s_t, cudaStream_t st) {
+  if (T == 0) return CONVROT_OK;
+  switch ((E + 31) / 32) {
+    case 1: launch_softmax<1>(logits, T, E, s_t, st); break;
+    case 2: launch_softmax<2>(logits, T, E, s_t, st); break;
+    case 3: launch_softmax<3>(logits, T, E, s_t, st); break;
+    case 4: launch_softmax<4>(logits, T, E, s_t, st); break;
+    case 5: launch_softmax<5>(logits, T, E, s_t, st); break;
+    case 6: launch_softmax<6>(logits, T, E, s_t, st); break;
+    case 7: launch_softmax<7>(logits, T, E, s_t, st); break;
+    default: launch_softmax<8>(logits, T, E, s_t, st); break;
+  }
   return launch_status();
 }
 
@@ -465,7 +547,7 @@ int convrot_router_softmax(const void* logits_bf16, int64_t T, int E, float* s_t
   if (!al16(logits_bf16) || !al16(s_t)) return CONVROT_ERR_MISALIGNED;
   int rc = device_setup(nullptr);
   if (rc != CONVROT_OK) return rc;
-  return softmax_impl(logits_bf16, T, E, s_t, nullptr, 0, as_stream(stream));
+  return softmax_impl(logits_bf16, T, E, s_t, as_stream(stream));
 }
 
 int convrot_topc(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float* w,
@@ -479,33 +561,17 @@ int convrot_topc(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, fl
   return topc_impl(s_t, T, E, C, idx, w, slot, as_stream(stream));
 }
 
-int convrot_combine_rows(const float* zw, const int32_t* slot, int E, int64_t T, int64_t C,
-                         int64_t d, void* y_bf16, void* stream) {
-  if (E < 1 || E > 256 || T < 0 || T >= ((int64_t)1 << 31) || C < 0 || C > T || d < 4 ||
-      d % 4 != 0 || (int64_t)E * C * d >= ((int64_t)1 << 40))
+int convrot_combine_rows(const void* z_bf16, const float* w, const int32_t* slot, int E,
+                         int64_t T, int64_t C, int64_t d, void* y_bf16, void* stream) {
+  if (E < 1 || E > 256 || T < 0 || T >= ((int64_t)1 << 31) || C < 0 || C > T || d < 8 ||
+      d % 8 != 0 || (int64_t)E * C >= ((int64_t)1 << 31) || (int64_t)E * C * d >= ((int64_t)1 << 40))
     return CONVROT_ERR_INVALID_ARG;
-  if (T > 0 && (!slot || !y_bf16 || (C > 0 && !zw))) return CONVROT_ERR_INVALID_ARG;
-  if (!al16(zw) || !al16(slot) || !al16(y_bf16)) return CONVROT_ERR_MISALIGNED;
-  int rc = device_setup(nullptr);
+  if (T > 0 && (!slot || !y_bf16 || (C > 0 && (!z_bf16 || !w)))) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(z_bf16) || !al16(w) || !al16(slot) || !al16(y_bf16)) return CONVROT_ERR_MISALIGNED;
+  int sms = 0;
+  int rc = device_setup(&sms);
   if (rc != CONVROT_OK) return rc;
-  return combine_impl(zw, slot, E, T, C, d, y_bf16, as_stream(stream));
-}
-
-int convrot_i8_gemm_weighted(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
-                             int b_layout, const float* w, int64_t G, int64_t M, int64_t N,
-                             int64_t K, float* zw, void* stream) {
-  if (b_layout != CONVROT_LAYOUT_ROWS && b_layout != CONVROT_LAYOUT_TILES)
-    return CONVROT_ERR_INVALID_ARG;
-  int rc = check_gemm_shape(a, b, G, M, N, K);
-  if (rc != CONVROT_OK) return rc;
-  if (G * M * N > 0 && (!s_a || !s_b || !w || !zw)) return CONVROT_ERR_INVALID_ARG;
-  if (!al16(s_a) || !al16(s_b) || !al16(zw)) return CONVROT_ERR_MISALIGNED;
-  GemmArgs args{};
-  args.s_a = s_a;
-  args.s_b = s_b;
-  args.out = zw;
-  args.w = w;
-  return launch_gemm_layout<kEpiWeighted>(b_layout, a, b, G, M, N, K, N, args, as_stream(stream));
+  return combine_impl(z_bf16, w, slot, E, T, C, d, y_bf16, sms, as_stream(stream));
 }
 
 int convrot_gather_rows(const int8_t* src, const float* s_src, int64_t n_src, const int32_t* idx,
@@ -650,7 +716,7 @@ int moe_workspace_layout(int64_t T, int64_t d, int64_t f, int E, int64_t C,
   lay->h_q = take(ec * f);
   lay->s_h = take(ec * 4);
   lay->slot = take((size_t)E * T * 4);
-  lay->zw = take(ec * d * 4);
+  lay->z = take(ec * d * 2);
   lay->total = off;
   return CONVROT_OK;
 }
@@ -697,7 +763,7 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
   int8_t* h_q = reinterpret_cast<int8_t*>(ws + lay.h_q);
   float* s_h = reinterpret_cast<float*>(ws + lay.s_h);
   int32_t* slot = reinterpret_cast<int32_t*>(ws + lay.slot);
-  float* zw = reinterpret_cast<float*>(ws + lay.zw);
+  void* z = ws + lay.z;
 
   // Routing (1, 3) runs on the side stream while the caller's stream rotates
   // and quantises the tokens (2); the streams join before the gather.
@@ -708,7 +774,7 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
       cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
     return CONVROT_ERR_CUDA;
   // 1. router softmax
-  int rc_side = softmax_impl(logits_bf16, T, E, s_t, nullptr, 0, ss->stream);
+  int rc_side = softmax_impl(logits_bf16, T, E, s_t, ss->stream);
   // 3. expert-choice top-C (+ each token's slot per expert)
   if (rc_side == CONVROT_OK) rc_side = topc_impl(s_t, T, E, C, idx, w, slot, ss->stream);
   // 2. rotate + quantise the tokens once (the gate/up rotation is expert-independent)
@@ -734,17 +800,17 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
     if ((rc = rotquant_impl(h, CONVROT_DTYPE_F32, (int64_t)E * C, f, g_d, h_q, s_h, st)) !=
         CONVROT_OK)
       return rc;
-    // 7. down GEMM with dequant, times the router weight of each row
+    // 7. down GEMM with dequant to the experts' BF16 outputs
     GemmArgs a2{};
     a2.s_a = s_h;
     a2.s_b = s_d;
-    a2.out = zw;
-    a2.w = w;
-    if ((rc = launch_gemm<kEpiWeighted, true>(h_q, w_d, E, C, d, f, d, a2, st)) != CONVROT_OK)
+    a2.out = z;
+    if ((rc = launch_gemm<kEpiBf16, true>(h_q, w_d, E, C, d, f, d, a2, st)) != CONVROT_OK)
       return rc;
   }
-  // 8. per token: fp32 sum over its experts in ascending order, one bf16 rounding
-  return combine_impl(zw, slot, E, T, C, d, y_bf16, st);
+  // 8. per token: router-weighted fp32 sum over its experts in ascending
+  // order, one bf16 rounding
+  return combine_impl(z, w, slot, E, T, C, d, y_bf16, sms, st);
 }
 
 }  // extern "C"

@@ -31,15 +31,25 @@ namespace convrot {
 
 constexpr int kRqThreads = 256;
 
+// The raw 16 elements of one thread's chunk, as loaded (2 x 16 bytes of bf16
+// or 4 x 16 bytes of fp32), so the next row's load can be in flight while
+// this row is computed.
 template <typename InT>
-__device__ __forceinline__ void rq_load16(const InT* p, float (&v)[16]);
+struct RqRaw {
+  static constexpr int kVecs = (int)(16 * sizeof(InT) / 16);
+  uint4 u[kVecs];
+};
 
-template <>
-__device__ __forceinline__ void rq_load16<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[16]) {
+template <typename InT>
+__device__ __forceinline__ void rq_load_raw(const InT* p, RqRaw<InT>& r) {
   const uint4* q = reinterpret_cast<const uint4*>(p);
-  const uint4 a = __ldg(q);
-  const uint4 b = __ldg(q + 1);
-  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int k = 0; k < RqRaw<InT>::kVecs; ++k) r.u[k] = __ldg(q + k);
+}
+
+__device__ __forceinline__ void rq_unpack(const RqRaw<__nv_bfloat16>& r, float (&v)[16]) {
+  const uint32_t w[8] = {r.u[0].x, r.u[0].y, r.u[0].z, r.u[0].w,
+                         r.u[1].x, r.u[1].y, r.u[1].z, r.u[1].w};
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     v[2 * k] = __uint_as_float(w[k] << 16);
@@ -47,16 +57,13 @@ __device__ __forceinline__ void rq_load16<__nv_bfloat16>(const __nv_bfloat16* p,
   }
 }
 
-template <>
-__device__ __forceinline__ void rq_load16<float>(const float* p, float (&v)[16]) {
-  const float4* q = reinterpret_cast<const float4*>(p);
+__device__ __forceinline__ void rq_unpack(const RqRaw<float>& r, float (&v)[16]) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const float4 f = __ldg(q + k);
-    v[4 * k] = f.x;
-    v[4 * k + 1] = f.y;
-    v[4 * k + 2] = f.z;
-    v[4 * k + 3] = f.w;
+    v[4 * k] = __uint_as_float(r.u[k].x);
+    v[4 * k + 1] = __uint_as_float(r.u[k].y);
+    v[4 * k + 2] = __uint_as_float(r.u[k].z);
+    v[4 * k + 3] = __uint_as_float(r.u[k].w);
   }
 }
 
@@ -74,7 +81,8 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
 }
 
 // Row-wise max over the `tpr` threads of a row. tpr is a power of two <= 32
-// (rows live in aligned lane segments) or a multiple of 32.
+// (rows live in aligned lane segments) or a multiple of 32 (then every thread
+// of the CTA must call it: it synchronises the CTA once).
 __device__ __forceinline__ float rq_row_max(float m, int tpr, float* red) {
   const int lane = threadIdx.x & 31;
   if (tpr <= 32) {
@@ -115,75 +123,280 @@ __device__ __forceinline__ int64_t rq_dst(const RqOut& o, int64_t row, int K, in
 
 // x: [rows, K] (bf16 or fp32), q: codes (layout `out`), scales: [rows] fp32.
 // blockDim.x = rows_per_cta * tpr exactly (rows_per_cta = max(1, 256 / tpr)).
+// Persistent: CTA b handles the row groups b, b + gridDim.x, ... (a group is
+// rows_per_cta consecutive rows) and loads its next group's chunk before
+// computing the current one.
 template <typename InT, int G>
 __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x, int64_t rows,
                                                       int K, int tpr, int8_t* __restrict__ q,
                                                       float* __restrict__ scales, RqOut out) {
   using Tr = RqTraits<G>;
-  __shared__ float red[16];  // per-warp maxima (512 threads at most)
+  __shared__ float red[2][16];  // per-warp maxima (512 threads at most), by iteration parity
   const int lane = threadIdx.x & 31;
   const int rows_per_cta = blockDim.x / tpr;
   const int r_local = threadIdx.x / tpr;
   const int i = threadIdx.x - r_local * tpr;  // 16-chunk index in the row
-  const int64_t row = (int64_t)blockIdx.x * rows_per_cta + r_local;
   const int nchunks = K >> 4;
-  const bool active = (row < rows) && (i < nchunks);
+  const int64_t groups = (rows + rows_per_cta - 1) / rows_per_cta;
 
-  float v[16];
-  if (active) {
-    rq_load16<InT>(x + row * K + (int64_t)i * 16, v);
-  } else {
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+  RqRaw<InT> raw;
+  int64_t grp = blockIdx.x;
+  {
+    const int64_t row = grp * rows_per_cta + r_local;
+    if (grp < groups && row < rows && i < nchunks) rq_load_raw<InT>(x + row * K + (int64_t)i * 16, raw);
   }
-  // spans 1, 2, 4, 8 inside the thread's 16 elements
+  for (int it = 0; grp < groups; grp += gridDim.x, ++it) {
+    const int64_t row = grp * rows_per_cta + r_local;
+    const bool active = (row < rows) && (i < nchunks);
+    float v[16];
+    if (active) {
+      rq_unpack(raw, v);
+    } else {
 #pragma unroll
-  for (int span = 1; span < Tr::kInRegSpanEnd; span <<= 1) {
+      for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+    }
+    {
+      const int64_t row_n = (grp + gridDim.x) * rows_per_cta + r_local;
+      if (grp + gridDim.x < groups && row_n < rows && i < nchunks)
+        rq_load_raw<InT>(x + row_n * K + (int64_t)i * 16, raw);
+    }
+    // spans 1, 2, 4, 8 inside the thread's 16 elements
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if ((j & span) == 0) {
-        const float a = v[j];
-        const float b = v[j + span];
-        v[j] = __fadd_rn(a, b);
-        v[j + span] = __fsub_rn(a, b);
+    for (int span = 1; span < Tr::kInRegSpanEnd; span <<= 1) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if ((j & span) == 0) {
+          const float a = v[j];
+          const float b = v[j + span];
+          v[j] = __fadd_rn(a, b);
+          v[j + span] = __fsub_rn(a, b);
+        }
       }
     }
-  }
-  // spans 16, 32, ... between chunks: the lower chunk of a pair keeps a + b,
-  // the upper one a - b, as one rounding each: fma(+-1, own, partner)
+    // spans 16, 32, ... between chunks: the lower chunk of a pair keeps a + b,
+    // the upper one a - b, as one rounding each: fma(+-1, own, partner)
 #pragma unroll
-  for (int d = 1; d < Tr::kLaneSpanEnd; d <<= 1) {
-    const float sgn = (lane & d) ? -1.0f : 1.0f;
+    for (int d = 1; d < Tr::kLaneSpanEnd; d <<= 1) {
+      const float sgn = (lane & d) ? -1.0f : 1.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float p = __shfl_xor_sync(0xffffffffu, v[j], d);
+        v[j] = __fmaf_rn(sgn, v[j], p);
+      }
+    }
+    float m = 0.0f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const float p = __shfl_xor_sync(0xffffffffu, v[j], d);
-      v[j] = __fmaf_rn(sgn, v[j], p);
+      v[j] = __fmul_rn(v[j], Tr::kInvSqrt);
+      m = fmaxf(m, fabsf(v[j]));
+    }
+    m = rq_row_max(m, tpr, red[it & 1]);
+
+    const bool nonzero = m >= 7.52316384526264e-37f;  // 2^-120
+    const float s = nonzero ? __fdiv_rn(m, 127.0f) : 0.0f;
+    const float r = nonzero ? __fdiv_rn(127.0f, m) : 0.0f;
+    if (active) {
+      // rint by adding 1.5 * 2^23 (the fp32 add rounds to nearest even)
+      int k[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        k[j] = __float_as_int(__fadd_rn(__fmul_rn(v[j], r), 12582912.0f)) - 0x4B400000;
+      uint4 c;
+      c.x = pack4(k[0], k[1], k[2], k[3]);
+      c.y = pack4(k[4], k[5], k[6], k[7]);
+      c.z = pack4(k[8], k[9], k[10], k[11]);
+      c.w = pack4(k[12], k[13], k[14], k[15]);
+      *reinterpret_cast<uint4*>(q + rq_dst(out, row, K, i * 16)) = c;
+      if (i == 0) scales[row] = s;
     }
   }
-  float m = 0.0f;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    v[j] = __fmul_rn(v[j], Tr::kInvSqrt);
-    m = fmaxf(m, fabsf(v[j]));
-  }
-  m = rq_row_max(m, tpr, red);
+}
 
-  const bool nonzero = m >= 7.52316384526264e-37f;  // 2^-120
-  const float s = nonzero ? __fdiv_rn(m, 127.0f) : 0.0f;
-  const float r = nonzero ? __fdiv_rn(127.0f, m) : 0.0f;
-  if (active) {
-    // rint by adding 1.5 * 2^23 (the fp32 add rounds to nearest even)
-    int k[16];
+// ------------------------------------------------------- warp-per-row form --
+// The same operation for K % 64 == 0 and K <= 2048, with fewer instructions
+// per element: lane l of a row segment (SEG lanes, a power of two) owns the 64
+// consecutive elements [64 l, 64 l + 64) of the row, held as 32 pairs
+// p[m] = (v[2m], v[2m+1]). Span 1 pairs the two halves of each register
+// (scalar ops); spans 2 .. 32 pair whole registers and use the packed
+// add/sub.rn.f32x2 (two IEEE fp32 operations each); for G = 256 the spans 64
+// and 128 pair lanes l ^ 1 and l ^ 2 (warp shuffles, one packed fma each).
+// The row maximum is a shuffle reduction over the segment. SEG * 64 >= K; a
+// warp holds 32 / SEG rows. bf16 inputs prefetch the warp's next rows while
+// the current ones are computed.
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ float2 f2_unpack(unsigned long long p) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_sub(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+template <typename InT>
+struct RqRaw64 {
+  static constexpr int kVecs = (int)(64 * sizeof(InT) / 16);
+  uint4 u[kVecs];
+};
+
+template <typename InT>
+__device__ __forceinline__ void rq_load64(const InT* p, RqRaw64<InT>& r) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      k[j] = __float_as_int(__fadd_rn(__fmul_rn(v[j], r), 12582912.0f)) - 0x4B400000;
-    uint4 c;
-    c.x = pack4(k[0], k[1], k[2], k[3]);
-    c.y = pack4(k[4], k[5], k[6], k[7]);
-    c.z = pack4(k[8], k[9], k[10], k[11]);
-    c.w = pack4(k[12], k[13], k[14], k[15]);
-    *reinterpret_cast<uint4*>(q + rq_dst(out, row, K, i * 16)) = c;
-    if (i == 0) scales[row] = s;
+  for (int k = 0; k < RqRaw64<InT>::kVecs; ++k) r.u[k] = __ldg(q + k);
+}
+
+__device__ __forceinline__ void rq_unpack64(const RqRaw64<__nv_bfloat16>& r,
+                                            unsigned long long (&p)[32]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t w[4] = {r.u[k].x, r.u[k].y, r.u[k].z, r.u[k].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      p[4 * k + j] = f2_pack(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
+  }
+}
+
+__device__ __forceinline__ void rq_unpack64(const RqRaw64<float>& r, unsigned long long (&p)[32]) {
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    p[2 * k] = f2_pack(__uint_as_float(r.u[k].x), __uint_as_float(r.u[k].y));
+    p[2 * k + 1] = f2_pack(__uint_as_float(r.u[k].z), __uint_as_float(r.u[k].w));
+  }
+}
+
+template <typename InT, int G, int SEG>
+__global__ void __launch_bounds__(256) rotquant_warp_kernel(const InT* __restrict__ x,
+                                                           int64_t rows, int K,
+                                                           int8_t* __restrict__ q,
+                                                           float* __restrict__ scales, RqOut out) {
+  static_assert(SEG >= 1 && SEG <= 32 && (SEG & (SEG - 1)) == 0, "segment of 2^k lanes");
+  static_assert(G != 256 || SEG >= 4, "a 256-group spans four lanes");
+  constexpr int kRowsPerWarp = 32 / SEG;
+  constexpr bool kPrefetch = sizeof(InT) == 2;
+  using Tr = RqTraits<G>;
+  const int lane = threadIdx.x & 31;
+  const int li = lane & (SEG - 1);
+  const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t units = (rows + kRowsPerWarp - 1) / kRowsPerWarp;
+  const bool lane_on = li * 64 < K;
+
+  RqRaw64<InT> raw;
+  int64_t u = warp0;
+  if (kPrefetch) {
+    const int64_t row = u * kRowsPerWarp + lane / SEG;
+    if (u < units && row < rows && lane_on) rq_load64<InT>(x + row * K + li * 64, raw);
+  }
+  for (; u < units; u += nwarps) {
+    const int64_t row = u * kRowsPerWarp + lane / SEG;
+    const bool active = row < rows && lane_on;
+    unsigned long long p[32];
+    if (active) {
+      if (!kPrefetch) rq_load64<InT>(x + row * K + li * 64, raw);
+      rq_unpack64(raw, p);
+    } else {
+#pragma unroll
+      for (int m = 0; m < 32; ++m) p[m] = 0ull;
+    }
+    if (kPrefetch) {
+      const int64_t row_n = (u + nwarps) * kRowsPerWarp + lane / SEG;
+      if (u + nwarps < units && row_n < rows && lane_on)
+        rq_load64<InT>(x + row_n * K + li * 64, raw);
+    }
+    // span 1: the two halves of each pair
+    if (G >= 2) {
+#pragma unroll
+      for (int m = 0; m < 32; ++m) {
+        const float2 ab = f2_unpack(p[m]);
+        p[m] = f2_pack(__fadd_rn(ab.x, ab.y), __fsub_rn(ab.x, ab.y));
+      }
+    }
+    // spans 2 .. min(G, 64) / 2: pairs of registers m, m + span / 2
+#pragma unroll
+    for (int hs = 1; 2 * hs < (G < 64 ? G : 64); hs <<= 1) {
+#pragma unroll
+      for (int m = 0; m < 32; ++m) {
+        if ((m & hs) == 0) {
+          const unsigned long long a = p[m], b = p[m + hs];
+          p[m] = f2_add(a, b);
+          p[m + hs] = f2_sub(a, b);
+        }
+      }
+    }
+    // spans 64, 128 (G = 256): lanes l ^ 1, l ^ 2 of the segment
+    if (G == 256) {
+#pragma unroll
+      for (int d = 1; d <= 2; d <<= 1) {
+        const float sg = (li & d) ? -1.0f : 1.0f;
+        const unsigned long long sg2 = f2_pack(sg, sg);
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {
+          const float2 own = f2_unpack(p[m]);
+          const float px = __shfl_xor_sync(0xffffffffu, own.x, d);
+          const float py = __shfl_xor_sync(0xffffffffu, own.y, d);
+          p[m] = f2_fma(sg2, p[m], f2_pack(px, py));
+        }
+      }
+    }
+    const unsigned long long inv2 = f2_pack(Tr::kInvSqrt, Tr::kInvSqrt);
+    float mx = 0.0f;
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+      p[m] = f2_mul(p[m], inv2);
+      const float2 t = f2_unpack(p[m]);
+      mx = fmaxf(mx, fmaxf(fabsf(t.x), fabsf(t.y)));
+    }
+#pragma unroll
+    for (int off = SEG >> 1; off > 0; off >>= 1)
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    const bool nonzero = mx >= 7.52316384526264e-37f;  // 2^-120
+    const float sc = nonzero ? __fdiv_rn(mx, 127.0f) : 0.0f;
+    const float r = nonzero ? __fdiv_rn(127.0f, mx) : 0.0f;
+    if (active) {
+      // rint by adding 1.5 * 2^23: the code is the low byte of the sum's bits.
+      // Scalar intrinsics on purpose: a packed mul.rn.f32x2 followed by a
+      // packed add.rn.f32x2 was contracted into one fma (the product then is
+      // not rounded to fp32 before the rint).
+      uint32_t cw[16];
+#pragma unroll
+      for (int m = 0; m < 32; m += 2) {
+        const float2 a = f2_unpack(p[m]);
+        const float2 b = f2_unpack(p[m + 1]);
+        const uint32_t c0 = __float_as_uint(__fadd_rn(__fmul_rn(a.x, r), 12582912.0f));
+        const uint32_t c1 = __float_as_uint(__fadd_rn(__fmul_rn(a.y, r), 12582912.0f));
+        const uint32_t c2 = __float_as_uint(__fadd_rn(__fmul_rn(b.x, r), 12582912.0f));
+        const uint32_t c3 = __float_as_uint(__fadd_rn(__fmul_rn(b.y, r), 12582912.0f));
+        cw[m >> 1] = __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(q + rq_dst(out, row, K, li * 64 + 16 * c)) =
+            make_uint4(cw[4 * c], cw[4 * c + 1], cw[4 * c + 2], cw[4 * c + 3]);
+      if (li == 0) scales[row] = sc;
+    }
   }
 }
 

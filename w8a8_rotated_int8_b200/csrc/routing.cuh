@@ -13,24 +13,24 @@ namespace convrot {
 // Per-token softmax of the router logits over E experts, evaluated in fp64 and
 // rounded once to fp32, written transposed (S_t[e, t]) so each expert's
 // scores are contiguous for the top-C selection. 32 tokens per CTA (one per
-// warp); the [E, 32] tile goes through shared memory so the transposed store
-// writes 128-byte rows. Optionally zeroes the same 32 rows of an fp32 buffer
-// (the combine accumulator) to save a separate pass.
+// warp, NJ = ceil(E / 32) experts per lane, so no lane evaluates an exp for
+// an expert that does not exist); the [E, 32] tile goes through shared memory
+// so the transposed store writes 128-byte rows.
 constexpr int kSmTokens = 32;
 
+template <int NJ>
 __global__ void __launch_bounds__(1024) router_softmax_kernel(
-    const __nv_bfloat16* __restrict__ logits, int T, int E, float* __restrict__ S_t,
-    float* __restrict__ clear, int64_t clear_cols) {
+    const __nv_bfloat16* __restrict__ logits, int T, int E, float* __restrict__ S_t) {
   extern __shared__ float sm_tile[];  // [E][32]
   const int t0 = blockIdx.x * kSmTokens;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned short* lg = reinterpret_cast<const unsigned short*>(logits);
   const int t = t0 + warp;  // one token per warp
   if (t < T) {
-    double l[8];
+    double l[NJ];
     double m = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < NJ; ++j) {
       const int e = lane + 32 * j;
       l[j] = (e < E) ? (double)__uint_as_float((uint32_t)__ldg(lg + (int64_t)t * E + e) << 16)
                      : -INFINITY;
@@ -38,18 +38,19 @@ __global__ void __launch_bounds__(1024) router_softmax_kernel(
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
-    double ex[8];
+    double ex[NJ];
     double sum = 0.0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < NJ; ++j) {
       const int e = lane + 32 * j;
-      ex[j] = (e < E) ? exp(__dsub_rn(l[j], m)) : 0.0;
+      ex[j] = 0.0;
+      if (e < E) ex[j] = exp(__dsub_rn(l[j], m));
       sum = __dadd_rn(sum, ex[j]);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum = __dadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, off));
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < NJ; ++j) {
       const int e = lane + 32 * j;
       if (e < E) sm_tile[e * kSmTokens + warp] = __double2float_rn(__ddiv_rn(ex[j], sum));
     }
@@ -59,13 +60,6 @@ __global__ void __launch_bounds__(1024) router_softmax_kernel(
     const int e = idx / kSmTokens, tl = idx - e * kSmTokens;
     if (t0 + tl < T) S_t[(int64_t)e * T + t0 + tl] = sm_tile[idx];
   }
-  if (clear != nullptr) {
-    const int nrows = min(kSmTokens, T - t0);
-    float4* base = reinterpret_cast<float4*>(clear + (int64_t)t0 * clear_cols);
-    const int64_t n4 = (int64_t)nrows * clear_cols / 4;
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int64_t j = threadIdx.x; j < n4; j += blockDim.x) base[j] = z;
-  }
 }
 
 // ------------------------------------------------------------------ top-C --
@@ -73,6 +67,11 @@ __global__ void __launch_bounds__(1024) router_softmax_kernel(
 __device__ __forceinline__ uint32_t score_key(uint32_t bits) {
   if (bits == 0x80000000u) bits = 0u;
   return (bits & 0x80000000u) ? ~bits : (bits | 0x80000000u);
+}
+
+// Inverse of score_key (a -0 score comes back as +0; softmax scores are >= +0).
+__device__ __forceinline__ float key_score(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
 constexpr int kTopcThreads = 1024;
@@ -215,6 +214,146 @@ __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const float* __restr
   }
 }
 
+// Register-resident top-C for T <= kTopcThreads * KPT: the same selection as
+// topc_kernel (radix select of the C-th largest key, four 8-bit digits, then
+// an ordered compaction), with every score read once into registers. Thread
+// i owns the KPT consecutive tokens [i * KPT, i * KPT + KPT). The digit
+// histograms are replicated per lane ([bin][lane] words), so the 32 lanes of
+// a warp always hit 32 different banks even when they all count the same
+// digit (softmax scores share their leading bits). One scan of packed
+// (greater, equal) counts places every pick: a token's list position is
+// (keys above the threshold before it) + min(equal keys before it, k).
+template <int KPT>
+__global__ void __launch_bounds__(kTopcThreads) topc_reg_kernel(const float* __restrict__ S_t,
+                                                                int T, int C,
+                                                                int32_t* __restrict__ idx,
+                                                                float* __restrict__ w,
+                                                                int32_t* __restrict__ slot) {
+  const int e = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float* row = S_t + (int64_t)e * T;
+  __shared__ uint32_t hist[256 * 32];
+  __shared__ uint32_t tot[256];
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t s_digit, s_k;
+  const int t0 = threadIdx.x * KPT;
+  if (C <= 0) {
+    if (slot != nullptr)
+      for (int t = threadIdx.x; t < T; t += blockDim.x) slot[(int64_t)e * T + t] = -1;
+    return;
+  }
+  uint32_t key[KPT];
+  if (KPT >= 4 && (T & 3) == 0 && t0 + KPT <= T) {
+#pragma unroll
+    for (int j = 0; j < KPT; j += 4) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + t0 + j));
+      key[j] = score_key(v.x);
+      key[j + 1] = score_key(v.y);
+      key[j + 2] = score_key(v.z);
+      key[j + 3] = score_key(v.w);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      key[j] = (t0 + j < T) ? score_key(__float_as_uint(__ldg(row + t0 + j))) : 0u;
+  }
+  const int n_valid = max(0, min(KPT, T - t0));
+
+  uint32_t prefix = 0u, mask = 0u, k = (uint32_t)C;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    uint4* h4 = reinterpret_cast<uint4*>(hist);
+    for (int i = threadIdx.x; i < 256 * 32 / 4; i += blockDim.x) h4[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if (j < n_valid && (key[j] & mask) == prefix)
+        atomicAdd(&hist[((key[j] >> shift) & 255u) * 32 + lane], 1u);
+    __syncthreads();
+    // bin totals: warp w sums bins 8w .. 8w+7 over the 32 lane copies
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const int bin = warp * 8 + b;
+      const uint32_t v = __reduce_add_sync(0xffffffffu, hist[bin * 32 + lane]);
+      if (lane == 0) tot[bin] = v;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t c[8];
+      uint32_t local = 0u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = tot[8 * lane + j];
+        local += c[j];
+      }
+      uint32_t incl = local;  // sum over lanes >= lane
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_down_sync(0xffffffffu, incl, off);
+        if (lane + off < 32) incl += o;
+      }
+      uint32_t run = incl - local;  // keys in higher digits
+#pragma unroll
+      for (int j = 7; j >= 0; --j) {
+        const uint32_t above = run;
+        run += c[j];
+        if (above < k && run >= k) {
+          s_digit = (uint32_t)(8 * lane + j);
+          s_k = k - above;
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= s_digit << shift;
+    mask |= 255u << shift;
+    k = s_k;
+  }
+  const uint32_t thr = prefix;
+  uint32_t n_gt = 0u, n_eq = 0u;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    if (j < n_valid) {
+      n_gt += key[j] > thr ? 1u : 0u;
+      n_eq += key[j] == thr ? 1u : 0u;
+    }
+  }
+  // counts stay below 2^16 (T <= 16384): one scan of both
+  const uint32_t before = block_excl_scan((n_gt << 16) | n_eq, warp_tot);
+  uint32_t gt_seen = before >> 16, eq_seen = before & 0xffffu;
+  int32_t my_slot[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    my_slot[j] = -1;
+    if (j < n_valid) {
+      const bool gt = key[j] > thr, eq = key[j] == thr;
+      if (gt || (eq && eq_seen < k)) {
+        const uint32_t pos = gt_seen + min(eq_seen, k);
+        if (pos < (uint32_t)C) {
+          idx[(int64_t)e * C + pos] = t0 + j;
+          w[(int64_t)e * C + pos] = key_score(key[j]);
+          my_slot[j] = (int32_t)pos;
+        } else {
+          atomicOr(&g_device_error, kErrBadIndex);
+        }
+      }
+      gt_seen += gt ? 1u : 0u;
+      eq_seen += eq ? 1u : 0u;
+    }
+  }
+  if (slot != nullptr) {
+    int32_t* srow = slot + (int64_t)e * T;
+    if (KPT >= 4 && (T & 3) == 0 && t0 + KPT <= T) {
+#pragma unroll
+      for (int j = 0; j < KPT; j += 4)
+        *reinterpret_cast<int4*>(srow + t0 + j) =
+            make_int4(my_slot[j], my_slot[j + 1], my_slot[j + 2], my_slot[j + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < KPT; ++j)
+        if (j < n_valid) srow[t0 + j] = my_slot[j];
+    }
+  }
+}
+
 // ----------------------------------------------------------------- gather --
 // dst[r, :] = src[idx[r], :], s_dst[r] = s_src[idx[r]]; one warp per row.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const int8_t* __restrict__ src,
@@ -252,90 +391,161 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const int8_t* __restri
 }
 
 // ---------------------------------------------------------------- combine --
-// y[t, :] = bf16(sum over experts e = 0, 1, ..., E-1 that picked t of
-// zw[e * C + slot[e, t], :]) with the sum in fp32 in that order (a token no
-// expert picked gets 0). One CTA of kCombineThreads per token: the first warp
-// lists the token's rows in expert order, then every thread owns up to
-// kCombineQuads float4 columns and loads them for two experts at a time
-// before adding, so many independent reads are in flight.
-constexpr int kCombineMaxE = 256;
-constexpr int kCombineThreads = 128;
-constexpr int kCombineQuads = 4;  // float4 columns per thread per pass
-__global__ void __launch_bounds__(kCombineThreads) combine_rows_kernel(
-    const float* __restrict__ zw, const int32_t* __restrict__ slot, int E, int T, int C, int d,
-    __nv_bfloat16* __restrict__ y) {
-  __shared__ int32_t sel[kCombineMaxE];
-  __shared__ int s_n;
-  const int t = blockIdx.x;
-  const int lane = threadIdx.x & 31;
-  if (threadIdx.x < 32) {
+// y[t, :] = bf16(sum over experts e = 0, 1, ..., E-1 that picked t, with
+// c = slot[e, t], of fp32(w[e*C + c] * z[e*C + c, :])): every product rounded
+// to fp32, the sum in fp32 in that order (a token no expert picked gets 0).
+// z holds the experts' BF16 outputs.
+//
+// One warp per token, persistent over the tokens t = warp, warp + #warps, ...
+// Lane l looks at experts l, l + 32, ... (NJ of them). The slot entries of
+// the next token are loaded while this token's rows stream in, and the router
+// weights of the next token's picks once its slots have arrived, so the index
+// look-ups stay off the critical path. A token's list (rows and weights in
+// ascending expert order) goes to the warp's shared-memory slice; the row is
+// then summed in chunks of 32 * kCombineVecs 8-column (16-byte) vectors, two
+// experts' loads in flight at a time.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineWarps = kCombineThreads / 32;
+constexpr int kCombineVecs = 4;  // 8-column vectors per lane per chunk
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&f)[8]) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(u[i] << 16);
+    f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+  }
+}
+
+template <int NJ>
+__device__ __forceinline__ void comb_load_slots(const int32_t* __restrict__ slot, int E, int T,
+                                                int t, int lane, int32_t (&sv)[NJ]) {
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int e = lane + 32 * j;
+    sv[j] = (t < T && e < E) ? __ldg(slot + (int64_t)e * T + t) : -1;
+  }
+}
+
+template <int NJ>
+__device__ __forceinline__ void comb_load_weights(const float* __restrict__ w, int C, int lane,
+                                                  const int32_t (&sv)[NJ], float (&wv)[NJ]) {
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int e = lane + 32 * j;
+    wv[j] = (sv[j] >= 0 && sv[j] < C) ? __ldg(w + (int64_t)e * C + sv[j]) : 0.0f;
+  }
+}
+
+template <int NJ>
+__global__ void __launch_bounds__(kCombineThreads, 2) combine_rows_kernel(
+    const __nv_bfloat16* __restrict__ z, const float* __restrict__ w,
+    const int32_t* __restrict__ slot, int E, int T, int C, int d, __nv_bfloat16* __restrict__ y) {
+  __shared__ int32_t sel_all[kCombineWarps][32 * NJ];
+  __shared__ float sw_all[kCombineWarps][32 * NJ];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int32_t* sel = sel_all[warp];
+  float* sw = sw_all[warp];
+  const int stride = gridDim.x * kCombineWarps;
+  const int d8 = d >> 3;
+  int t = blockIdx.x * kCombineWarps + warp;
+  int32_t sc[NJ];
+  float wc[NJ];
+  comb_load_slots<NJ>(slot, E, T, t, lane, sc);
+  comb_load_weights<NJ>(w, C, lane, sc, wc);
+  for (; t < T; t += stride) {
+    int32_t sn[NJ];
+    comb_load_slots<NJ>(slot, E, T, t + stride, lane, sn);
+    // this token's list, ascending expert order
     int n = 0;
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + lane;
-      const int c = (e < E) ? __ldg(slot + (int64_t)e * T + t) : -1;
-      const bool bad = c >= C;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const bool bad = sc[j] >= C;
       if (bad) atomicOr(&g_device_error, kErrBadIndex);
-      const bool has = c >= 0 && !bad;
+      const bool has = sc[j] >= 0 && !bad;
       const unsigned m = __ballot_sync(0xffffffffu, has);
-      if (has) sel[n + __popc(m & ((1u << lane) - 1u))] = e * C + c;
+      if (has) {
+        const int pos = n + __popc(m & ((1u << lane) - 1u));
+        sel[pos] = (lane + 32 * j) * C + sc[j];
+        sw[pos] = wc[j];
+      }
       n += __popc(m);
     }
-    if (lane == 0) s_n = n;
-  }
-  __syncthreads();
-  const int n = s_n;
-  const int d4 = d >> 2;
-  uint2* yrow = reinterpret_cast<uint2*>(y + (int64_t)t * d);
-  for (int q0 = threadIdx.x; q0 < d4; q0 += kCombineThreads * kCombineQuads) {
-    float4 acc[kCombineQuads];
+    __syncwarp();
+    float wn[NJ];
+    bool next_weights = false;
+    uint4* yrow = reinterpret_cast<uint4*>(y + (int64_t)t * d);
+    for (int q0 = lane; q0 < d8; q0 += 32 * kCombineVecs) {
+      float acc[kCombineVecs][8];
 #pragma unroll
-    for (int u = 0; u < kCombineQuads; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-    int k = 0;
-    for (; k + 2 <= n; k += 2) {
-      const float4* r0 = reinterpret_cast<const float4*>(zw + (int64_t)sel[k] * d);
-      const float4* r1 = reinterpret_cast<const float4*>(zw + (int64_t)sel[k + 1] * d);
-      float4 a[kCombineQuads], b[kCombineQuads];
+      for (int u = 0; u < kCombineVecs; ++u)
 #pragma unroll
-      for (int u = 0; u < kCombineQuads; ++u) {
-        const int q = q0 + u * kCombineThreads;
-        if (q < d4) {
-          a[u] = __ldcs(r0 + q);
-          b[u] = __ldcs(r1 + q);
+        for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+      int k = 0;
+      for (; k + 2 <= n; k += 2) {
+        const uint4* r0 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k] * d);
+        const uint4* r1 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k + 1] * d);
+        const float w0 = sw[k], w1 = sw[k + 1];
+        uint4 a[kCombineVecs], b[kCombineVecs];
+#pragma unroll
+        for (int u = 0; u < kCombineVecs; ++u) {
+          const int q = q0 + 32 * u;
+          if (q < d8) {
+            a[u] = __ldcs(r0 + q);
+            b[u] = __ldcs(r1 + q);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kCombineVecs; ++u) {
+          if (q0 + 32 * u < d8) {
+            float fa[8], fb[8];
+            bf16x8_to_f32(a[u], fa);
+            bf16x8_to_f32(b[u], fb);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              acc[u][i] = __fadd_rn(__fadd_rn(acc[u][i], __fmul_rn(w0, fa[i])), __fmul_rn(w1, fb[i]));
+          }
         }
       }
+      if (k < n) {
+        const uint4* r0 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k] * d);
+        const float w0 = sw[k];
 #pragma unroll
-      for (int u = 0; u < kCombineQuads; ++u) {
-        acc[u].x = __fadd_rn(__fadd_rn(acc[u].x, a[u].x), b[u].x);
-        acc[u].y = __fadd_rn(__fadd_rn(acc[u].y, a[u].y), b[u].y);
-        acc[u].z = __fadd_rn(__fadd_rn(acc[u].z, a[u].z), b[u].z);
-        acc[u].w = __fadd_rn(__fadd_rn(acc[u].w, a[u].w), b[u].w);
+        for (int u = 0; u < kCombineVecs; ++u) {
+          const int q = q0 + 32 * u;
+          if (q < d8) {
+            float fa[8];
+            bf16x8_to_f32(__ldcs(r0 + q), fa);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[u][i] = __fadd_rn(acc[u][i], __fmul_rn(w0, fa[i]));
+          }
+        }
       }
-    }
-    if (k < n) {
-      const float4* r0 = reinterpret_cast<const float4*>(zw + (int64_t)sel[k] * d);
+      // the next token's slots have had one chunk of loads to arrive
+      if (!next_weights) {
+        comb_load_weights<NJ>(w, C, lane, sn, wn);
+        next_weights = true;
+      }
 #pragma unroll
-      for (int u = 0; u < kCombineQuads; ++u) {
-        const int q = q0 + u * kCombineThreads;
-        if (q < d4) {
-          const float4 a = __ldcs(r0 + q);
-          acc[u].x = __fadd_rn(acc[u].x, a.x);
-          acc[u].y = __fadd_rn(acc[u].y, a.y);
-          acc[u].z = __fadd_rn(acc[u].z, a.z);
-          acc[u].w = __fadd_rn(acc[u].w, a.w);
+      for (int u = 0; u < kCombineVecs; ++u) {
+        const int q = q0 + 32 * u;
+        if (q < d8) {
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 p = __floats2bfloat162_rn(acc[u][2 * i], acc[u][2 * i + 1]);
+            o[i] = *reinterpret_cast<const uint32_t*>(&p);
+          }
+          yrow[q] = make_uint4(o[0], o[1], o[2], o[3]);
         }
       }
     }
+    if (!next_weights) comb_load_weights<NJ>(w, C, lane, sn, wn);
+    __syncwarp();  // the list slice is rewritten for the next token
 #pragma unroll
-    for (int u = 0; u < kCombineQuads; ++u) {
-      const int q = q0 + u * kCombineThreads;
-      if (q < d4) {
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[u].x, acc[u].y);
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[u].z, acc[u].w);
-        uint2 o;
-        o.x = *reinterpret_cast<const uint32_t*>(&lo);
-        o.y = *reinterpret_cast<const uint32_t*>(&hi);
-        yrow[q] = o;
-      }
+    for (int j = 0; j < NJ; ++j) {
+      sc[j] = sn[j];
+      wc[j] = wn[j];
     }
   }
 }
