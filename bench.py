@@ -315,7 +315,7 @@ def stage_times(W, ws_views, inp_dev, wq, cfg, t, reps, flush_buf):
             W.binding._p(s_d), tiles, cfg.n_exp, cfg.c, cfg.d, cfg.f,
             W.binding._p(v["z"]), W.binding._stream()),
         "combine": lambda: W.binding.lib().convrot_combine_rows(
-            W.binding._p(v["z"]), W.binding._p(v["w"]), W.binding._p(v["slot"]), cfg.n_exp, t,
+            W.binding._p(v["z"]), W.binding._p(v["s_t"]), W.binding._p(v["slot"]), cfg.n_exp, t,
             cfg.c, cfg.d, W.binding._p(inp_dev["y"]), W.binding._stream()),
     }
     out = {}

@@ -152,14 +152,15 @@ int convrot_topc(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, fl
  * experts' outputs are scattered back to their tokens), weighted by the
  * router scores of the choices:
  *   y[t, :] = bf16(sum over e = 0, 1, ..., E-1 with c = slot[e, t] >= 0 of
- *             fp32(w[e * C + c] * z[e * C + c, :])), every product rounded to
+ *             fp32(s_t[e, t] * z[e * C + c, :])), every product rounded to
  *             fp32 and added in fp32 in that order; a token no expert picked
  *             gets 0.
  *   z     device, [E * C, d] bf16 expert outputs (down projection)
- *   w     device, [E * C] fp32 router weights (convrot_topc)
+ *   s_t   device, [E, T] fp32 router scores, transposed (the weight of a pick
+ *         is its score: convrot_router_softmax)
  *   slot  device, [E, T] int32 from convrot_topc;  y device, [T, d] bf16
- *   1 <= E <= 256, d % 8 == 0. */
-int convrot_combine_rows(const void* z_bf16, const float* w, const int32_t* slot, int E,
+ *   1 <= E <= 256, d % 8 == 0, d <= 8192. */
+int convrot_combine_rows(const void* z_bf16, const float* s_t, const int32_t* slot, int E,
                          int64_t T, int64_t C, int64_t d, void* y_bf16, void* stream);
 
 /* Gather rows: dst[r, :] = src[idx[r], :], s_dst[r] = s_src[idx[r]].

@@ -295,26 +295,29 @@ def test_gemm_bf16_grouped_rows_bit_exact(g, m, layout):
 
 
 @pytest.mark.parametrize("e_n,t,c,d", [(5, 300, 40, 256), (7, 64, 64, 2056), (3, 50, 0, 64),
-                                       (70, 1000, 30, 128), (64, 5000, 160, 2048)])
+                                       (70, 1000, 30, 128), (64, 5000, 160, 2048),
+                                       (9, 40, 40, 8192), (200, 300, 250, 64)])
 def test_combine_sums_in_expert_order(e_n, t, c, d):
-    """y[t] = bf16(sum_e fp32(w * z)) in ascending expert order; d = 2056
-    leaves a ragged tail of 8-column vectors past two full passes of 2048."""
+    """y[t] = bf16(sum_e fp32(s_t[e, t] * z[e, slot])) in ascending expert order.
+    d = 2056 leaves a ragged tail of 16-byte pieces; d = 8192 stages one row
+    per slot (the rest from global memory); E = 200 with C = 250 of T = 300
+    gives tokens far more expert rows than a slot holds."""
     gen = torch.Generator().manual_seed(3 + d)
     z = (torch.randn(e_n * c, d, generator=gen) * 10.0 ** torch.randint(-3, 3, (e_n * c, 1),
                                                                        generator=gen))
     z = z.to(torch.bfloat16)
-    w = torch.rand(e_n * c, generator=gen)
+    s_t = torch.rand(e_n, t, generator=gen)
     slot = torch.full((e_n, t), -1, dtype=torch.int32)
     for e in range(e_n):
         toks = torch.randperm(t, generator=gen)[:c].sort().values
         slot[e, toks] = torch.arange(c, dtype=torch.int32)
-    y = W.convrot_combine_rows(z.cuda(), w.cuda(), slot.cuda(), c).cpu()
+    y = W.convrot_combine_rows(z.cuda(), s_t.cuda(), slot.cuda(), c).cpu()
     ref = np.zeros((t, d), np.float32)
-    zf, wf = np32(z), w.numpy()
+    zf, sf = np32(z), s_t.numpy()
     for e in range(e_n):       # fp32 products, fp32 sums, ascending expert order
         toks = np.nonzero(slot[e].numpy() >= 0)[0]
         rows = e * c + slot[e].numpy()[toks]
-        ref[toks] = ref[toks] + (wf[rows][:, None] * zf[rows]).astype(np.float32)
+        ref[toks] = ref[toks] + (sf[e, toks][:, None] * zf[rows]).astype(np.float32)
     assert np.array_equal(np32(y), O.bf16_round(ref))
 
 

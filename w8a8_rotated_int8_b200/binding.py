@@ -239,17 +239,17 @@ def convrot_topc(s_t, c, with_slot=False, stream=None):
     return (idx, w, slot) if with_slot else (idx, w)
 
 
-def convrot_combine_rows(z, w, slot, c, stream=None):
-    """z [E*C, d] bf16 expert outputs, w [E*C] fp32 router weights, slot
-    [E, T] -> y [T, d] bf16 (per token, the fp32 sum of w*z over its experts
-    in ascending expert order)."""
+def convrot_combine_rows(z, s_t, slot, c, stream=None):
+    """z [E*C, d] bf16 expert outputs, s_t [E, T] fp32 router scores, slot
+    [E, T] -> y [T, d] bf16 (per token, the fp32 sum of s_t * z over its
+    experts in ascending expert order)."""
     _need(z, torch.bfloat16, "z")
-    _need(w, torch.float32, "w")
+    _need(s_t, torch.float32, "s_t")
     _need(slot, torch.int32, "slot")
     e, t = slot.shape
     d = z.shape[-1]
-    y = torch.empty((t, d), dtype=torch.bfloat16, device=z.device)
-    _check(lib().convrot_combine_rows(_p(z), _p(w), _p(slot), e, t, c, d, _p(y),
+    y = torch.empty((t, d), dtype=torch.bfloat16, device=slot.device)
+    _check(lib().convrot_combine_rows(_p(z), _p(s_t), _p(slot), e, t, c, d, _p(y),
                                       _stream(stream)), "convrot_combine_rows")
     return y
 

@@ -24,6 +24,7 @@ enum DeviceErrorBits : unsigned {
   kErrTimeoutTeardown = 1u << 4,  // in-flight work did not drain at exit
   kErrSelfTest = 1u << 5,         // the wait self-test ran out (expected)
   kErrBadIndex = 1u << 6,         // a row index was out of range; the access was skipped
+  kErrTimeoutStream = 1u << 7,    // a streaming kernel waited too long for a TMA copy
 };
 
 __device__ unsigned int g_device_error = 0;
@@ -99,6 +100,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_limit(bar, parity, abort_flag, err_bit, g_wait_limit_ns);
 }
 
+// Waits (bounded, ignoring any abort flag) for a phase to complete: used on
+// the way out of a kernel that gave up, so that no copy is still writing into
+// its shared memory when the CTA ends. Returns false on timeout.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) {
+      atomicOr(&g_device_error, kErrTimeoutTeardown);
+      return false;
+    }
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------- TMA --
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
@@ -124,6 +139,18 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+
+// 1-D bulk copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) from global memory into this CTA's shared memory, no multicast;
+// completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes,
+                                             uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
 

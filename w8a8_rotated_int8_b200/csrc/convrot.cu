@@ -149,38 +149,64 @@ int launch_status() {
 }
 
 // --------------------------------------------------------------- rotquant --
-constexpr int kRqWarpThreads = 128;
+// 3-D byte view {128, K * esize / 128, rows} of a row-major [rows, K] matrix,
+// box = `box_rows` whole rows, 128-byte swizzle (see rotquant_tma_kernel).
+int encode_rows_sw128(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
+                      uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return CONVROT_ERR_CUDA;
+  const cuuint64_t dims[3] = {128, row_bytes / 128, rows};
+  const cuuint64_t strides[2] = {128, row_bytes};
+  const cuuint32_t box[3] = {128, (cuuint32_t)(row_bytes / 128), box_rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
 
 template <typename InT, int G, int SEG>
-void launch_rq_warp(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
-                    cudaStream_t st) {
-  const int64_t units = (rows + (32 / SEG) - 1) / (32 / SEG);  // warp-rows
+int launch_rq_tma(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
+                   cudaStream_t st) {
+  constexpr int kRowsPerWarp = 32 / SEG;
+  const uint64_t row_bytes = (uint64_t)K * sizeof(InT);
+  CUtensorMap tm;
+  if (encode_rows_sw128(&tm, x, row_bytes, (uint64_t)rows, kRowsPerWarp) != CONVROT_OK)
+    return CONVROT_ERR_CUDA;
+  const int slot_bytes = (int)((kRowsPerWarp * row_bytes + 1023) / 1024 * 1024);
+  int slots = (int)((110 * 1024) / ((int64_t)kRqTmaWarps * slot_bytes));
+  slots = std::max(2, std::min(kRqMaxSlots, slots));
+  const size_t smem = 1024 + (size_t)kRqTmaWarps * slots * (slot_bytes + 8) + kRqTmaWarps * 4;
+  auto kern = rotquant_tma_kernel<InT, G, SEG>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotquant_warp_kernel<InT, G, SEG>,
-                                                    kRqWarpThreads, 0) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRqTmaWarps * 32, smem) !=
+          cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
   int sms = 0;
   device_setup(&sms);
-  const int64_t ctas = (units + kRqWarpThreads / 32 - 1) / (kRqWarpThreads / 32);
+  const int64_t units = (rows + kRowsPerWarp - 1) / kRowsPerWarp;
+  const int64_t ctas = (units + kRqTmaWarps - 1) / kRqTmaWarps;
   const int64_t grid = std::min<int64_t>(ctas, (int64_t)per_sm * std::max(sms, 1));
-  rotquant_warp_kernel<InT, G, SEG><<<(unsigned)grid, kRqWarpThreads, 0, st>>>(
-      reinterpret_cast<const InT*>(x), rows, K, q, s, out);
+  kern<<<(unsigned)grid, kRqTmaWarps * 32, smem, st>>>(tm, rows, K, slots, slot_bytes, q, s, out);
+  return CONVROT_OK;
 }
 
 template <typename InT, int G>
-void launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
+int launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
                cudaStream_t st) {
   // K % 64 == 0, K <= 2048: one warp segment of SEG lanes per row, 64
   // elements per lane (G = 256 needs at least the four lanes of one group)
   if (K % 64 == 0 && K <= 2048) {
     const int lanes = K / 64;
-    if (lanes <= 1 && G < 256) return launch_rq_warp<InT, G, (G < 256 ? 1 : 4)>(x, rows, K, q, s, out, st);
-    if (lanes <= 2 && G < 256) return launch_rq_warp<InT, G, (G < 256 ? 2 : 4)>(x, rows, K, q, s, out, st);
-    if (lanes <= 4) return launch_rq_warp<InT, G, 4>(x, rows, K, q, s, out, st);
-    if (lanes <= 8) return launch_rq_warp<InT, G, 8>(x, rows, K, q, s, out, st);
-    if (lanes <= 16) return launch_rq_warp<InT, G, 16>(x, rows, K, q, s, out, st);
-    return launch_rq_warp<InT, G, 32>(x, rows, K, q, s, out, st);
+    if (lanes <= 1 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 1 : 4)>(x, rows, K, q, s, out, st);
+    if (lanes <= 2 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 2 : 4)>(x, rows, K, q, s, out, st);
+    if (lanes <= 4) return launch_rq_tma<InT, G, 4>(x, rows, K, q, s, out, st);
+    if (lanes <= 8) return launch_rq_tma<InT, G, 8>(x, rows, K, q, s, out, st);
+    if (lanes <= 16) return launch_rq_tma<InT, G, 16>(x, rows, K, q, s, out, st);
+    return launch_rq_tma<InT, G, 32>(x, rows, K, q, s, out, st);
   }
   const int nch = K / 16;
   int tpr;
@@ -205,17 +231,18 @@ void launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut ou
   const int64_t grid = std::min<int64_t>(groups, (int64_t)per_sm * std::max(sms, 1));
   rotquant_kernel<InT, G><<<(unsigned)grid, threads, 0, st>>>(
       reinterpret_cast<const InT*>(x), rows, K, tpr, q, s, out);
+  return CONVROT_OK;
 }
 
 template <typename InT>
-void dispatch_rq(int group, const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
-                 cudaStream_t st) {
+int dispatch_rq(int group, const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
+                cudaStream_t st) {
   switch (group) {
-    case 1: launch_rq<InT, 1>(x, rows, K, q, s, out, st); break;
-    case 4: launch_rq<InT, 4>(x, rows, K, q, s, out, st); break;
-    case 16: launch_rq<InT, 16>(x, rows, K, q, s, out, st); break;
-    case 64: launch_rq<InT, 64>(x, rows, K, q, s, out, st); break;
-    default: launch_rq<InT, 256>(x, rows, K, q, s, out, st); break;
+    case 1: return launch_rq<InT, 1>(x, rows, K, q, s, out, st);
+    case 4: return launch_rq<InT, 4>(x, rows, K, q, s, out, st);
+    case 16: return launch_rq<InT, 16>(x, rows, K, q, s, out, st);
+    case 64: return launch_rq<InT, 64>(x, rows, K, q, s, out, st);
+    default: return launch_rq<InT, 256>(x, rows, K, q, s, out, st);
   }
 }
 
@@ -233,10 +260,10 @@ int check_rq_args(const void* x, int x_dtype, int64_t rows, int64_t K, int group
 int rotquant_impl(const void* x, int x_dtype, int64_t rows, int64_t K, int group, int8_t* q,
                   float* s, cudaStream_t st, RqOut out = RqOut{0, 1, 1, 1}) {
   if (rows == 0) return CONVROT_OK;
-  if (x_dtype == CONVROT_DTYPE_BF16)
-    dispatch_rq<__nv_bfloat16>(group, x, rows, (int)K, q, s, out, st);
-  else
-    dispatch_rq<float>(group, x, rows, (int)K, q, s, out, st);
+  const int rc = (x_dtype == CONVROT_DTYPE_BF16)
+                     ? dispatch_rq<__nv_bfloat16>(group, x, rows, (int)K, q, s, out, st)
+                     : dispatch_rq<float>(group, x, rows, (int)K, q, s, out, st);
+  if (rc != CONVROT_OK) return rc;
   return launch_status();
 }
 
@@ -396,28 +423,29 @@ int topc_impl(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float
 }
 
 template <int NJ>
-void launch_combine(const void* z, const float* w, const int32_t* slot, int E, int64_t T,
-                    int64_t C, int64_t d, void* y, int sms, cudaStream_t st) {
-  // persistent: resident CTAs only (two per SM at <= 128 registers), one warp
-  // per token at a time
-  const int64_t grid = std::min<int64_t>((T + kCombineWarps - 1) / kCombineWarps, 2 * sms);
-  combine_rows_kernel<NJ><<<(unsigned)grid, kCombineThreads, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(z), w, slot, E, (int)T, (int)C, (int)d,
+int launch_combine(const void* z, const float* s_t, const int32_t* slot, int E, int64_t T,
+                   int64_t C, int64_t d, void* y, int sms, cudaStream_t st) {
+  (void)sms;
+  combine_rows_kernel<NJ><<<(unsigned)T, kCombineThreads, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(z), s_t, slot, E, (int)T, (int)C, (int)d,
       reinterpret_cast<__nv_bfloat16*>(y));
+  return CONVROT_OK;
 }
 
 // E <= 256 (checked by the entry points)
-int combine_impl(const void* z, const float* w, const int32_t* slot, int E, int64_t T, int64_t C,
+int combine_impl(const void* z, const float* s_t, const int32_t* slot, int E, int64_t T, int64_t C,
                  int64_t d, void* y, int sms, cudaStream_t st) {
   if (T == 0) return CONVROT_OK;
+  int rc;
   if (E <= 32)
-    launch_combine<1>(z, w, slot, E, T, C, d, y, sms, st);
+    rc = launch_combine<1>(z, s_t, slot, E, T, C, d, y, sms, st);
   else if (E <= 64)
-    launch_combine<2>(z, w, slot, E, T, C, d, y, sms, st);
+    rc = launch_combine<2>(z, s_t, slot, E, T, C, d, y, sms, st);
   else if (E <= 128)
-    launch_combine<4>(z, w, slot, E, T, C, d, y, sms, st);
+    rc = launch_combine<4>(z, s_t, slot, E, T, C, d, y, sms, st);
   else
-    launch_combine<8>(z, w, slot, E, T, C, d, y, sms, st);
+    rc = launch_combine<8>(z, s_t, slot, E, T, C, d, y, sms, st);
+  if (rc != CONVROT_OK) return rc;
   return launch_status();
 }
 
@@ -561,17 +589,17 @@ int convrot_topc(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, fl
   return topc_impl(s_t, T, E, C, idx, w, slot, as_stream(stream));
 }
 
-int convrot_combine_rows(const void* z_bf16, const float* w, const int32_t* slot, int E,
+int convrot_combine_rows(const void* z_bf16, const float* s_t, const int32_t* slot, int E,
                          int64_t T, int64_t C, int64_t d, void* y_bf16, void* stream) {
   if (E < 1 || E > 256 || T < 0 || T >= ((int64_t)1 << 31) || C < 0 || C > T || d < 8 ||
-      d % 8 != 0 || (int64_t)E * C >= ((int64_t)1 << 31) || (int64_t)E * C * d >= ((int64_t)1 << 40))
+      d > 8192 || d % 8 != 0 || (int64_t)E * C >= ((int64_t)1 << 31))
     return CONVROT_ERR_INVALID_ARG;
-  if (T > 0 && (!slot || !y_bf16 || (C > 0 && (!z_bf16 || !w)))) return CONVROT_ERR_INVALID_ARG;
-  if (!al16(z_bf16) || !al16(w) || !al16(slot) || !al16(y_bf16)) return CONVROT_ERR_MISALIGNED;
+  if (T > 0 && (!slot || !s_t || !y_bf16 || (C > 0 && !z_bf16))) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(z_bf16) || !al16(s_t) || !al16(slot) || !al16(y_bf16)) return CONVROT_ERR_MISALIGNED;
   int sms = 0;
   int rc = device_setup(&sms);
   if (rc != CONVROT_OK) return rc;
-  return combine_impl(z_bf16, w, slot, E, T, C, d, y_bf16, sms, as_stream(stream));
+  return combine_impl(z_bf16, s_t, slot, E, T, C, d, y_bf16, sms, as_stream(stream));
 }
 
 int convrot_gather_rows(const int8_t* src, const float* s_src, int64_t n_src, const int32_t* idx,
@@ -810,7 +838,7 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
   }
   // 8. per token: router-weighted fp32 sum over its experts in ascending
   // order, one bf16 rounding
-  return combine_impl(z, w, slot, E, T, C, d, y_bf16, sms, st);
+  return combine_impl(z, s_t, slot, E, T, C, d, y_bf16, sms, st);
 }
 
 }  // extern "C"

@@ -221,8 +221,7 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x
 // add/sub.rn.f32x2 (two IEEE fp32 operations each); for G = 256 the spans 64
 // and 128 pair lanes l ^ 1 and l ^ 2 (warp shuffles, one packed fma each).
 // The row maximum is a shuffle reduction over the segment. SEG * 64 >= K; a
-// warp holds 32 / SEG rows. bf16 inputs prefetch the warp's next rows while
-// the current ones are computed.
+// warp holds 32 / SEG rows. The rows reach shared memory by TMA (below).
 __device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
   unsigned long long d;
   asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
@@ -255,148 +254,214 @@ __device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsig
   return d;
 }
 
+// 16 bytes of a lane's 64 elements (piece j: elements 8j.. of bf16, 4j.. of
+// fp32) into their pairs of p.
 template <typename InT>
-struct RqRaw64 {
-  static constexpr int kVecs = (int)(64 * sizeof(InT) / 16);
-  uint4 u[kVecs];
-};
+__device__ __forceinline__ void rq_unpack_piece(const uint4 v, int j, unsigned long long (&p)[32]);
 
-template <typename InT>
-__device__ __forceinline__ void rq_load64(const InT* p, RqRaw64<InT>& r) {
-  const uint4* q = reinterpret_cast<const uint4*>(p);
+template <>
+__device__ __forceinline__ void rq_unpack_piece<__nv_bfloat16>(const uint4 v, int j,
+                                                               unsigned long long (&p)[32]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int k = 0; k < RqRaw64<InT>::kVecs; ++k) r.u[k] = __ldg(q + k);
+  for (int i = 0; i < 4; ++i)
+    p[4 * j + i] = f2_pack(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
 }
 
-__device__ __forceinline__ void rq_unpack64(const RqRaw64<__nv_bfloat16>& r,
-                                            unsigned long long (&p)[32]) {
+template <>
+__device__ __forceinline__ void rq_unpack_piece<float>(const uint4 v, int j,
+                                                       unsigned long long (&p)[32]) {
+  p[2 * j] = f2_pack(__uint_as_float(v.x), __uint_as_float(v.y));
+  p[2 * j + 1] = f2_pack(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+
+// Rotation, scale and codes of the 64 elements (32 pairs) a lane holds;
+// every lane of the warp calls it (shuffles).
+template <int G, int SEG>
+__device__ __forceinline__ void rq_lane64(unsigned long long (&p)[32], bool active, int li,
+                                          int64_t row, int K, int8_t* __restrict__ q,
+                                          float* __restrict__ scales, const RqOut& out) {
+  using Tr = RqTraits<G>;
+  // span 1: the two halves of each pair
+  if (G >= 2) {
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t w[4] = {r.u[k].x, r.u[k].y, r.u[k].z, r.u[k].w};
+    for (int m = 0; m < 32; ++m) {
+      const float2 ab = f2_unpack(p[m]);
+      p[m] = f2_pack(__fadd_rn(ab.x, ab.y), __fsub_rn(ab.x, ab.y));
+    }
+  }
+  // spans 2 .. min(G, 64) / 2: pairs of registers m, m + span / 2
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      p[4 * k + j] = f2_pack(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
+  for (int hs = 1; 2 * hs < (G < 64 ? G : 64); hs <<= 1) {
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+      if ((m & hs) == 0) {
+        const unsigned long long a = p[m], b = p[m + hs];
+        p[m] = f2_add(a, b);
+        p[m + hs] = f2_sub(a, b);
+      }
+    }
+  }
+  // spans 64, 128 (G = 256): lanes l ^ 1, l ^ 2 of the segment
+  if (G == 256) {
+#pragma unroll
+    for (int d = 1; d <= 2; d <<= 1) {
+      const float sg = (li & d) ? -1.0f : 1.0f;
+      const unsigned long long sg2 = f2_pack(sg, sg);
+#pragma unroll
+      for (int m = 0; m < 32; ++m) {
+        const float2 own = f2_unpack(p[m]);
+        const float px = __shfl_xor_sync(0xffffffffu, own.x, d);
+        const float py = __shfl_xor_sync(0xffffffffu, own.y, d);
+        p[m] = f2_fma(sg2, p[m], f2_pack(px, py));
+      }
+    }
+  }
+  const unsigned long long inv2 = f2_pack(Tr::kInvSqrt, Tr::kInvSqrt);
+  float mx = 0.0f;
+#pragma unroll
+  for (int m = 0; m < 32; ++m) {
+    p[m] = f2_mul(p[m], inv2);
+    const float2 t = f2_unpack(p[m]);
+    mx = fmaxf(mx, fmaxf(fabsf(t.x), fabsf(t.y)));
+  }
+#pragma unroll
+  for (int off = SEG >> 1; off > 0; off >>= 1)
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  const bool nonzero = mx >= 7.52316384526264e-37f;  // 2^-120
+  const float sc = nonzero ? __fdiv_rn(mx, 127.0f) : 0.0f;
+  const float r = nonzero ? __fdiv_rn(127.0f, mx) : 0.0f;
+  if (active) {
+    // rint by adding 1.5 * 2^23: the code is the low byte of the sum's bits.
+    // Scalar intrinsics on purpose: a packed mul.rn.f32x2 followed by a
+    // packed add.rn.f32x2 was contracted into one fma (the product then is
+    // not rounded to fp32 before the rint).
+    uint32_t cw[16];
+#pragma unroll
+    for (int m = 0; m < 32; m += 2) {
+      const float2 a = f2_unpack(p[m]);
+      const float2 b = f2_unpack(p[m + 1]);
+      const uint32_t c0 = __float_as_uint(__fadd_rn(__fmul_rn(a.x, r), 12582912.0f));
+      const uint32_t c1 = __float_as_uint(__fadd_rn(__fmul_rn(a.y, r), 12582912.0f));
+      const uint32_t c2 = __float_as_uint(__fadd_rn(__fmul_rn(b.x, r), 12582912.0f));
+      const uint32_t c3 = __float_as_uint(__fadd_rn(__fmul_rn(b.y, r), 12582912.0f));
+      cw[m >> 1] = __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      *reinterpret_cast<uint4*>(q + rq_dst(out, row, K, li * 64 + 16 * c)) =
+          make_uint4(cw[4 * c], cw[4 * c + 1], cw[4 * c + 2], cw[4 * c + 3]);
+    if (li == 0) scales[row] = sc;
   }
 }
 
-__device__ __forceinline__ void rq_unpack64(const RqRaw64<float>& r, unsigned long long (&p)[32]) {
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    p[2 * k] = f2_pack(__uint_as_float(r.u[k].x), __uint_as_float(r.u[k].y));
-    p[2 * k + 1] = f2_pack(__uint_as_float(r.u[k].z), __uint_as_float(r.u[k].w));
-  }
-}
+// TMA-fed form: every warp keeps a ring of kRqSlots shared-memory slots, each
+// holding one unit (32 / SEG rows) as loaded by a 3-D tiled TMA copy
+// {128 bytes, K * sizeof(InT) / 128 chunks, rows} with the 128-byte swizzle;
+// lane 0 refills a slot as soon as the warp has read it, so kRqSlots - 1
+// units stream in while one is computed. A lane reads its 16-byte pieces k at
+// position k ^ (smem row & 7): the swizzle makes those reads conflict-free
+// for the 8 lanes of each phase while the piece index stays static.
+constexpr int kRqTmaWarps = 8;
+constexpr int kRqMaxSlots = 4;  // ring depth per warp
 
 template <typename InT, int G, int SEG>
-__global__ void __launch_bounds__(256) rotquant_warp_kernel(const InT* __restrict__ x,
-                                                           int64_t rows, int K,
-                                                           int8_t* __restrict__ q,
-                                                           float* __restrict__ scales, RqOut out) {
+__global__ void __launch_bounds__(kRqTmaWarps * 32, 2) rotquant_tma_kernel(
+    const __grid_constant__ CUtensorMap tm, int64_t rows, int K, int slots, int slot_bytes,
+    int8_t* __restrict__ q, float* __restrict__ scales, RqOut out) {
   static_assert(SEG >= 1 && SEG <= 32 && (SEG & (SEG - 1)) == 0, "segment of 2^k lanes");
   static_assert(G != 256 || SEG >= 4, "a 256-group spans four lanes");
   constexpr int kRowsPerWarp = 32 / SEG;
-  constexpr bool kPrefetch = sizeof(InT) == 2;
-  using Tr = RqTraits<G>;
-  const int lane = threadIdx.x & 31;
+  constexpr int kChunksPerLane = (int)(64 * sizeof(InT) / 128);  // 128-byte smem rows
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int li = lane & (SEG - 1);
-  const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  uint8_t* ring = smem + (size_t)warp * slots * slot_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kRqTmaWarps * slots * slot_bytes) +
+                   warp * slots;
+  volatile int* abort_flag =
+      reinterpret_cast<volatile int*>(smem + (size_t)kRqTmaWarps * slots * (slot_bytes + 8)) +
+      warp;
+  const int kb = K * (int)sizeof(InT) / 128;
+  const uint32_t tx_bytes = (uint32_t)(kRowsPerWarp * kb * 128);
   const int64_t units = (rows + kRowsPerWarp - 1) / kRowsPerWarp;
+  const int64_t u0 = (int64_t)blockIdx.x * kRqTmaWarps + warp;
+  const int64_t nw = (int64_t)gridDim.x * kRqTmaWarps;
   const bool lane_on = li * 64 < K;
+  const uint64_t policy = l2_policy_evict_first();
 
-  RqRaw64<InT> raw;
-  int64_t u = warp0;
-  if (kPrefetch) {
-    const int64_t row = u * kRowsPerWarp + lane / SEG;
-    if (u < units && row < rows && lane_on) rq_load64<InT>(x + row * K + li * 64, raw);
+  if (lane == 0) {
+    for (int k = 0; k < slots; ++k) mbar_init(&bars[k], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm);
+    for (int k = 0; k < slots; ++k) {
+      const int64_t u = u0 + k * nw;
+      if (u >= units) break;
+      mbar_arrive_expect_tx(&bars[k], tx_bytes);
+      tma_load_3d(ring + (size_t)k * slot_bytes, &tm, &bars[k], 0, 0, (int)(u * kRowsPerWarp),
+                  policy);
+    }
   }
-  for (; u < units; u += nwarps) {
+  __syncwarp();
+  // iteration `it` consumes unit u0 + it * nw from slot it % slots (phase
+  // parity (it / slots) & 1); its load was issued `slots` iterations earlier
+  int64_t it = 0;
+  for (int64_t u = u0; u < units; u += nw, ++it) {
+    const int k = (int)(it % slots);
+    const uint32_t parity = (uint32_t)((it / slots) & 1);
+    const bool ok = mbar_wait(&bars[k], parity, abort_flag, kErrTimeoutStream);
+    if (__any_sync(0xffffffffu, !ok)) {  // the whole warp leaves together
+      *abort_flag = 1;
+      break;
+    }
+
     const int64_t row = u * kRowsPerWarp + lane / SEG;
     const bool active = row < rows && lane_on;
     unsigned long long p[32];
     if (active) {
-      if (!kPrefetch) rq_load64<InT>(x + row * K + li * 64, raw);
-      rq_unpack64(raw, p);
+      const int srow0 = (lane / SEG) * kb + li * kChunksPerLane;
+#pragma unroll
+      for (int h = 0; h < kChunksPerLane; ++h) {
+        const int srow = srow0 + h;
+        const uint8_t* base = ring + (size_t)k * slot_bytes + (size_t)srow * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          rq_unpack_piece<InT>(*reinterpret_cast<const uint4*>(base + ((c ^ (srow & 7)) << 4)),
+                               h * 8 + c, p);
+      }
     } else {
 #pragma unroll
       for (int m = 0; m < 32; ++m) p[m] = 0ull;
     }
-    if (kPrefetch) {
-      const int64_t row_n = (u + nwarps) * kRowsPerWarp + lane / SEG;
-      if (u + nwarps < units && row_n < rows && lane_on)
-        rq_load64<InT>(x + row_n * K + li * 64, raw);
-    }
-    // span 1: the two halves of each pair
-    if (G >= 2) {
-#pragma unroll
-      for (int m = 0; m < 32; ++m) {
-        const float2 ab = f2_unpack(p[m]);
-        p[m] = f2_pack(__fadd_rn(ab.x, ab.y), __fsub_rn(ab.x, ab.y));
+    __syncwarp();
+    // the generic-proxy reads of this slot are ordered before the next TMA write
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (lane == 0) {
+      const int64_t un = u + (int64_t)slots * nw;
+      if (un < units) {
+        mbar_arrive_expect_tx(&bars[k], tx_bytes);
+        tma_load_3d(ring + (size_t)k * slot_bytes, &tm, &bars[k], 0, 0, (int)(un * kRowsPerWarp),
+                    policy);
       }
     }
-    // spans 2 .. min(G, 64) / 2: pairs of registers m, m + span / 2
-#pragma unroll
-    for (int hs = 1; 2 * hs < (G < 64 ? G : 64); hs <<= 1) {
-#pragma unroll
-      for (int m = 0; m < 32; ++m) {
-        if ((m & hs) == 0) {
-          const unsigned long long a = p[m], b = p[m + hs];
-          p[m] = f2_add(a, b);
-          p[m + hs] = f2_sub(a, b);
-        }
+
+    rq_lane64<G, SEG>(p, active, li, row, K, q, scales, out);
+  }
+  if (*abort_flag) {
+    // a wait ran out: let every copy this warp still has in flight land
+    // (bounded) before the CTA's shared memory is released
+    // (the loads of iterations it .. it + slots - 1 were issued, not consumed)
+    if (lane == 0) {
+      for (int j = 0; j < slots; ++j) {
+        const int64_t itj = it + j;
+        if (u0 + itj * nw < units)
+          mbar_drain(&bars[itj % slots], (uint32_t)((itj / slots) & 1), g_wait_limit_ns);
       }
     }
-    // spans 64, 128 (G = 256): lanes l ^ 1, l ^ 2 of the segment
-    if (G == 256) {
-#pragma unroll
-      for (int d = 1; d <= 2; d <<= 1) {
-        const float sg = (li & d) ? -1.0f : 1.0f;
-        const unsigned long long sg2 = f2_pack(sg, sg);
-#pragma unroll
-        for (int m = 0; m < 32; ++m) {
-          const float2 own = f2_unpack(p[m]);
-          const float px = __shfl_xor_sync(0xffffffffu, own.x, d);
-          const float py = __shfl_xor_sync(0xffffffffu, own.y, d);
-          p[m] = f2_fma(sg2, p[m], f2_pack(px, py));
-        }
-      }
-    }
-    const unsigned long long inv2 = f2_pack(Tr::kInvSqrt, Tr::kInvSqrt);
-    float mx = 0.0f;
-#pragma unroll
-    for (int m = 0; m < 32; ++m) {
-      p[m] = f2_mul(p[m], inv2);
-      const float2 t = f2_unpack(p[m]);
-      mx = fmaxf(mx, fmaxf(fabsf(t.x), fabsf(t.y)));
-    }
-#pragma unroll
-    for (int off = SEG >> 1; off > 0; off >>= 1)
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    const bool nonzero = mx >= 7.52316384526264e-37f;  // 2^-120
-    const float sc = nonzero ? __fdiv_rn(mx, 127.0f) : 0.0f;
-    const float r = nonzero ? __fdiv_rn(127.0f, mx) : 0.0f;
-    if (active) {
-      // rint by adding 1.5 * 2^23: the code is the low byte of the sum's bits.
-      // Scalar intrinsics on purpose: a packed mul.rn.f32x2 followed by a
-      // packed add.rn.f32x2 was contracted into one fma (the product then is
-      // not rounded to fp32 before the rint).
-      uint32_t cw[16];
-#pragma unroll
-      for (int m = 0; m < 32; m += 2) {
-        const float2 a = f2_unpack(p[m]);
-        const float2 b = f2_unpack(p[m + 1]);
-        const uint32_t c0 = __float_as_uint(__fadd_rn(__fmul_rn(a.x, r), 12582912.0f));
-        const uint32_t c1 = __float_as_uint(__fadd_rn(__fmul_rn(a.y, r), 12582912.0f));
-        const uint32_t c2 = __float_as_uint(__fadd_rn(__fmul_rn(b.x, r), 12582912.0f));
-        const uint32_t c3 = __float_as_uint(__fadd_rn(__fmul_rn(b.y, r), 12582912.0f));
-        cw[m >> 1] = __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
-      }
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        *reinterpret_cast<uint4*>(q + rq_dst(out, row, K, li * 64 + 16 * c)) =
-            make_uint4(cw[4 * c], cw[4 * c + 1], cw[4 * c + 2], cw[4 * c + 3]);
-      if (li == 0) scales[row] = sc;
-    }
+    __syncwarp();
   }
 }
 

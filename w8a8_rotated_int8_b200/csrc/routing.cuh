@@ -392,21 +392,20 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const int8_t* __restri
 
 // ---------------------------------------------------------------- combine --
 // y[t, :] = bf16(sum over experts e = 0, 1, ..., E-1 that picked t, with
-// c = slot[e, t], of fp32(w[e*C + c] * z[e*C + c, :])): every product rounded
+// c = slot[e, t], of fp32(s_t[e, t] * z[e*C + c, :])): every product rounded
 // to fp32, the sum in fp32 in that order (a token no expert picked gets 0).
-// z holds the experts' BF16 outputs.
+// z holds the experts' BF16 outputs; s_t[e, t] is the router score of token t
+// for expert e, i.e. the weight top-C stored for the pick, so the slot and
+// weight look-ups are independent loads.
 //
-// One warp per token, persistent over the tokens t = warp, warp + #warps, ...
-// Lane l looks at experts l, l + 32, ... (NJ of them). The slot entries of
-// the next token are loaded while this token's rows stream in, and the router
-// weights of the next token's picks once its slots have arrived, so the index
-// look-ups stay off the critical path. A token's list (rows and weights in
-// ascending expert order) goes to the warp's shared-memory slice; the row is
-// then summed in chunks of 32 * kCombineVecs 8-column (16-byte) vectors, two
-// experts' loads in flight at a time.
-constexpr int kCombineThreads = 256;
+// One CTA of kCombineThreads per token. Every warp builds the token's list
+// (rows and weights in ascending expert order) itself from one round of
+// loads, so no CTA-wide barrier is needed; then each thread sums its
+// 8-column (16-byte) vectors over the rows, two rows' loads in flight at a
+// time.
+constexpr int kCombineThreads = 128;
 constexpr int kCombineWarps = kCombineThreads / 32;
-constexpr int kCombineVecs = 4;  // 8-column vectors per lane per chunk
+constexpr int kCombineVecs = 2;  // 8-column vectors per thread per pass
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&f)[8]) {
   const uint32_t u[4] = {v.x, v.y, v.z, v.w};
@@ -418,134 +417,98 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&f)[8]) {
 }
 
 template <int NJ>
-__device__ __forceinline__ void comb_load_slots(const int32_t* __restrict__ slot, int E, int T,
-                                                int t, int lane, int32_t (&sv)[NJ]) {
-#pragma unroll
-  for (int j = 0; j < NJ; ++j) {
-    const int e = lane + 32 * j;
-    sv[j] = (t < T && e < E) ? __ldg(slot + (int64_t)e * T + t) : -1;
-  }
-}
-
-template <int NJ>
-__device__ __forceinline__ void comb_load_weights(const float* __restrict__ w, int C, int lane,
-                                                  const int32_t (&sv)[NJ], float (&wv)[NJ]) {
-#pragma unroll
-  for (int j = 0; j < NJ; ++j) {
-    const int e = lane + 32 * j;
-    wv[j] = (sv[j] >= 0 && sv[j] < C) ? __ldg(w + (int64_t)e * C + sv[j]) : 0.0f;
-  }
-}
-
-template <int NJ>
-__global__ void __launch_bounds__(kCombineThreads, 2) combine_rows_kernel(
-    const __nv_bfloat16* __restrict__ z, const float* __restrict__ w,
+__global__ void __launch_bounds__(kCombineThreads) combine_rows_kernel(
+    const __nv_bfloat16* __restrict__ z, const float* __restrict__ s_t,
     const int32_t* __restrict__ slot, int E, int T, int C, int d, __nv_bfloat16* __restrict__ y) {
   __shared__ int32_t sel_all[kCombineWarps][32 * NJ];
   __shared__ float sw_all[kCombineWarps][32 * NJ];
+  const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int32_t* sel = sel_all[warp];
   float* sw = sw_all[warp];
-  const int stride = gridDim.x * kCombineWarps;
-  const int d8 = d >> 3;
-  int t = blockIdx.x * kCombineWarps + warp;
-  int32_t sc[NJ];
-  float wc[NJ];
-  comb_load_slots<NJ>(slot, E, T, t, lane, sc);
-  comb_load_weights<NJ>(w, C, lane, sc, wc);
-  for (; t < T; t += stride) {
-    int32_t sn[NJ];
-    comb_load_slots<NJ>(slot, E, T, t + stride, lane, sn);
-    // this token's list, ascending expert order
-    int n = 0;
+  int32_t sv[NJ];
+  float wv[NJ];
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      const bool bad = sc[j] >= C;
-      if (bad) atomicOr(&g_device_error, kErrBadIndex);
-      const bool has = sc[j] >= 0 && !bad;
-      const unsigned m = __ballot_sync(0xffffffffu, has);
-      if (has) {
-        const int pos = n + __popc(m & ((1u << lane) - 1u));
-        sel[pos] = (lane + 32 * j) * C + sc[j];
-        sw[pos] = wc[j];
-      }
-      n += __popc(m);
+  for (int j = 0; j < NJ; ++j) {
+    const int e = lane + 32 * j;
+    sv[j] = e < E ? __ldg(slot + (int64_t)e * T + t) : -1;
+    wv[j] = e < E ? __ldg(s_t + (int64_t)e * T + t) : 0.0f;
+  }
+  int n = 0;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const bool bad = sv[j] >= C;
+    if (bad && warp == 0) atomicOr(&g_device_error, kErrBadIndex);
+    const bool has = sv[j] >= 0 && !bad;
+    const unsigned m = __ballot_sync(0xffffffffu, has);
+    if (has) {
+      const int pos = n + __popc(m & ((1u << lane) - 1u));
+      sel[pos] = (lane + 32 * j) * C + sv[j];
+      sw[pos] = wv[j];
     }
-    __syncwarp();
-    float wn[NJ];
-    bool next_weights = false;
-    uint4* yrow = reinterpret_cast<uint4*>(y + (int64_t)t * d);
-    for (int q0 = lane; q0 < d8; q0 += 32 * kCombineVecs) {
-      float acc[kCombineVecs][8];
+    n += __popc(m);
+  }
+  __syncwarp();
+  const int d8 = d >> 3;
+  uint4* yrow = reinterpret_cast<uint4*>(y + (int64_t)t * d);
+  for (int q0 = threadIdx.x; q0 < d8; q0 += kCombineThreads * kCombineVecs) {
+    float acc[kCombineVecs][8];
 #pragma unroll
-      for (int u = 0; u < kCombineVecs; ++u)
+    for (int u = 0; u < kCombineVecs; ++u)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
-      int k = 0;
-      for (; k + 2 <= n; k += 2) {
-        const uint4* r0 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k] * d);
-        const uint4* r1 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k + 1] * d);
-        const float w0 = sw[k], w1 = sw[k + 1];
-        uint4 a[kCombineVecs], b[kCombineVecs];
+      for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+    int k = 0;
+    for (; k + 2 <= n; k += 2) {
+      const uint4* r0 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k] * d);
+      const uint4* r1 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k + 1] * d);
+      const float w0 = sw[k], w1 = sw[k + 1];
+      uint4 a[kCombineVecs], b[kCombineVecs];
 #pragma unroll
-        for (int u = 0; u < kCombineVecs; ++u) {
-          const int q = q0 + 32 * u;
-          if (q < d8) {
-            a[u] = __ldcs(r0 + q);
-            b[u] = __ldcs(r1 + q);
-          }
+      for (int u = 0; u < kCombineVecs; ++u) {
+        const int q = q0 + u * kCombineThreads;
+        if (q < d8) {
+          a[u] = __ldcs(r0 + q);
+          b[u] = __ldcs(r1 + q);
         }
-#pragma unroll
-        for (int u = 0; u < kCombineVecs; ++u) {
-          if (q0 + 32 * u < d8) {
-            float fa[8], fb[8];
-            bf16x8_to_f32(a[u], fa);
-            bf16x8_to_f32(b[u], fb);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              acc[u][i] = __fadd_rn(__fadd_rn(acc[u][i], __fmul_rn(w0, fa[i])), __fmul_rn(w1, fb[i]));
-          }
-        }
-      }
-      if (k < n) {
-        const uint4* r0 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k] * d);
-        const float w0 = sw[k];
-#pragma unroll
-        for (int u = 0; u < kCombineVecs; ++u) {
-          const int q = q0 + 32 * u;
-          if (q < d8) {
-            float fa[8];
-            bf16x8_to_f32(__ldcs(r0 + q), fa);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[u][i] = __fadd_rn(acc[u][i], __fmul_rn(w0, fa[i]));
-          }
-        }
-      }
-      // the next token's slots have had one chunk of loads to arrive
-      if (!next_weights) {
-        comb_load_weights<NJ>(w, C, lane, sn, wn);
-        next_weights = true;
       }
 #pragma unroll
       for (int u = 0; u < kCombineVecs; ++u) {
-        const int q = q0 + 32 * u;
-        if (q < d8) {
-          uint32_t o[4];
+        if (q0 + u * kCombineThreads < d8) {
+          float fa[8], fb[8];
+          bf16x8_to_f32(a[u], fa);
+          bf16x8_to_f32(b[u], fb);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const __nv_bfloat162 p = __floats2bfloat162_rn(acc[u][2 * i], acc[u][2 * i + 1]);
-            o[i] = *reinterpret_cast<const uint32_t*>(&p);
-          }
-          yrow[q] = make_uint4(o[0], o[1], o[2], o[3]);
+          for (int i = 0; i < 8; ++i)
+            acc[u][i] = __fadd_rn(__fadd_rn(acc[u][i], __fmul_rn(w0, fa[i])), __fmul_rn(w1, fb[i]));
         }
       }
     }
-    if (!next_weights) comb_load_weights<NJ>(w, C, lane, sn, wn);
-    __syncwarp();  // the list slice is rewritten for the next token
+    if (k < n) {
+      const uint4* r0 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k] * d);
+      const float w0 = sw[k];
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      sc[j] = sn[j];
-      wc[j] = wn[j];
+      for (int u = 0; u < kCombineVecs; ++u) {
+        const int q = q0 + u * kCombineThreads;
+        if (q < d8) {
+          float fa[8];
+          bf16x8_to_f32(__ldcs(r0 + q), fa);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[u][i] = __fadd_rn(acc[u][i], __fmul_rn(w0, fa[i]));
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCombineVecs; ++u) {
+      const int q = q0 + u * kCombineThreads;
+      if (q < d8) {
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(acc[u][2 * i], acc[u][2 * i + 1]);
+          o[i] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        yrow[q] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
   }
 }
