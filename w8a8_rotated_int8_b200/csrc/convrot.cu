@@ -87,24 +87,23 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+template <int EPI, bool BT, bool GA>
+void set_gemm_attr() {
+  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<EPI, BT, GA>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<EPI>::kSmem1);
+  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<EPI, BT, GA>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<EPI>::kSmem2);
+}
+
+// every GEMM instantiation the entry points launch
 template <bool BT>
 void set_gemm_attrs() {
-  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiI32, BT>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
-  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiBf16, BT>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
-  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiSwiglu, BT>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
-  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<kEpiScatter, BT>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES);
-  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiI32, BT>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
-  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiBf16, BT>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
-  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiSwiglu, BT>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
-  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<kEpiScatter, BT>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
+  set_gemm_attr<kEpiI32, BT, false>();
+  set_gemm_attr<kEpiI32, BT, true>();
+  set_gemm_attr<kEpiBf16, BT, false>();
+  set_gemm_attr<kEpiSwiglu, BT, false>();
+  set_gemm_attr<kEpiSwiglu, BT, true>();
+  set_gemm_attr<kEpiScatter, BT, false>();
 }
 
 // Per-device one-time setup: capability check, SM count, kernel attributes.
@@ -316,10 +315,28 @@ int encode_tiled_b(CUtensorMap* map, const void* base, uint64_t kb_count, uint64
   return r == CUDA_SUCCESS ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
+// 2-D map over a [rows, K] code matrix with a {128-byte, 1-row} box and the
+// 128-byte swizzle, for tile::gather4 loads of single rows.
+int encode_gather_rows(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return CONVROT_ERR_CUDA;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K};
+  const cuuint32_t box[2] = {(cuuint32_t)gemm::BK, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
 // NB = rows of one B matrix per group (2F for SwiGLU). With BT the B operand
 // is in the tiled weight format: for SwiGLU each group holds a gate matrix and
-// an up matrix of F rows, each padded to 128-row blocks.
-template <int EPI, bool BT>
+// an up matrix of F rows, each padded to 128-row blocks. With GA the rows of A
+// are gathered: `a` is the [args.a_src_rows, K] source and args.a_idx [G*M]
+// names the source row of every A row.
+template <int EPI, bool BT, bool GA = false>
 int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t NB, int64_t K,
                 int64_t n_out, GemmArgs args, cudaStream_t st) {
   int sms = 0;
@@ -329,8 +346,14 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
   CUtensorMap ta, tb;
   const uint32_t box_a = (uint32_t)std::min<int64_t>(gemm::BM, M);
   uint32_t box_b;
-  if ((rc = encode_3d_i8(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)G, box_a)) != CONVROT_OK)
+  if (GA) {
+    if (args.a_idx == nullptr || args.a_src_rows < 1) return CONVROT_ERR_INVALID_ARG;
+    if ((rc = encode_gather_rows(&ta, a, (uint64_t)K, (uint64_t)args.a_src_rows)) != CONVROT_OK)
+      return rc;
+  } else if ((rc = encode_3d_i8(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)G, box_a)) !=
+             CONVROT_OK) {
     return rc;
+  }
   if (BT) {
     const int64_t blocks = (EPI == kEpiSwiglu) ? cdiv(n_out, 128) : cdiv(NB, 128);
     const int64_t per_group = (EPI == kEpiSwiglu) ? 2 * blocks : blocks;
@@ -360,12 +383,13 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
     const int64_t tiles = G * args.m_blocks * args.n_blocks;
     if (tiles >= ((int64_t)1 << 30)) return CONVROT_ERR_INVALID_ARG;
     args.num_tiles = (int)tiles;
-    args.box_bytes = 2 * (128 + 128) * gemm::BK;  // both CTAs' A and B boxes
+    // both CTAs' A and B boxes (gathered A rows are counted in the kernel)
+    args.box_bytes = GA ? 2 * 128 * gemm::BK : 2 * (128 + 128) * gemm::BK;
     const int grid = 2 * (int)std::min<int64_t>(tiles, sms / 2);
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(grid);
-    lc.blockDim = dim3(gemm::THREADS);
-    lc.dynamicSmemBytes = gemm2::SMEM_BYTES;
+    lc.blockDim = dim3(EpiCfg<EPI>::kThreads);
+    lc.dynamicSmemBytes = EpiCfg<EPI>::kSmem2;
     lc.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -374,7 +398,8 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
     attr[0].val.clusterDim.z = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&lc, gemm_s8_tcgen05_pair_kernel<EPI, BT>, ta, tb, args) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&lc, gemm_s8_tcgen05_pair_kernel<EPI, BT, GA>, ta, tb, args) !=
+        cudaSuccess) {
       cudaGetLastError();
       return CONVROT_ERR_CUDA;
     }
@@ -387,18 +412,20 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
   const int64_t tiles = G * args.m_blocks * args.n_blocks;
   if (tiles >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
   args.num_tiles = (int)tiles;
-  args.box_bytes = (int)((box_a + 2 * box_b) * gemm::BK);
+  // A and B boxes of one stage (gathered A rows are counted in the kernel)
+  args.box_bytes = (int)(((GA ? 0 : box_a) + 2 * box_b) * gemm::BK);
   const int grid = (int)std::min<int64_t>(tiles, sms);
-  gemm_s8_tcgen05_kernel<EPI, BT><<<grid, gemm::THREADS, gemm::SMEM_BYTES, st>>>(ta, tb, args);
+  gemm_s8_tcgen05_kernel<EPI, BT, GA><<<grid, EpiCfg<EPI>::kThreads, EpiCfg<EPI>::kSmem1, st>>>(
+      ta, tb, args);
   return launch_status();
 }
 
-template <int EPI>
+template <int EPI, bool GA = false>
 int launch_gemm_layout(int b_layout, const int8_t* a, const int8_t* b, int64_t G, int64_t M,
                        int64_t NB, int64_t K, int64_t n_out, GemmArgs args, cudaStream_t st) {
   if (b_layout == CONVROT_LAYOUT_TILES)
-    return launch_gemm<EPI, true>(a, b, G, M, NB, K, n_out, args, st);
-  return launch_gemm<EPI, false>(a, b, G, M, NB, K, n_out, args, st);
+    return launch_gemm<EPI, true, GA>(a, b, G, M, NB, K, n_out, args, st);
+  return launch_gemm<EPI, false, GA>(a, b, G, M, NB, K, n_out, args, st);
 }
 
 int topc_impl(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float* w,
@@ -425,10 +452,20 @@ int topc_impl(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float
 template <int NJ>
 int launch_combine(const void* z, const float* s_t, const int32_t* slot, int E, int64_t T,
                    int64_t C, int64_t d, void* y, int sms, cudaStream_t st) {
-  (void)sms;
-  combine_rows_kernel<NJ><<<(unsigned)T, kCombineThreads, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(z), s_t, slot, E, (int)T, (int)C, (int)d,
-      reinterpret_cast<__nv_bfloat16*>(y));
+  // tokens per CTA: a power of two in [1, 32] that leaves about four CTAs per
+  // SM, so every SM streams rows while each CTA's slot tiles stay coalesced
+  int tpc = 32;
+  while (tpc > 1 && T < (int64_t)tpc * 4 * std::max(sms, 1)) tpc >>= 1;
+  const size_t smem = combine_tokens_smem(E, tpc);
+  auto kern = combine_tokens_kernel<NJ>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  const int64_t grid = (T + tpc - 1) / tpc;
+  kern<<<(unsigned)grid, kCombThreads, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(z), s_t,
+                                                   slot, E, (int)T, (int)C, (int)d, tpc,
+                                                   reinterpret_cast<__nv_bfloat16*>(y));
   return CONVROT_OK;
 }
 
@@ -659,6 +696,47 @@ int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, c
   args.out = h;
   return launch_gemm_layout<kEpiSwiglu>(b_layout, a, b, G, M, 2 * F, K, F, args,
                                         as_stream(stream));
+}
+
+int convrot_i8_gemm_i32_gather(const int8_t* a_src, int64_t n_src, const int32_t* a_idx,
+                               const int8_t* b, int b_layout, int64_t G, int64_t M, int64_t N,
+                               int64_t K, int32_t* d, void* stream) {
+  if (b_layout != CONVROT_LAYOUT_ROWS && b_layout != CONVROT_LAYOUT_TILES)
+    return CONVROT_ERR_INVALID_ARG;
+  int rc = check_gemm_shape(a_src, b, G, M, N, K);
+  if (rc != CONVROT_OK) return rc;
+  if (n_src < 0 || n_src >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
+  if (G * M * N > 0 && (!d || !a_idx || n_src == 0)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(d)) return CONVROT_ERR_MISALIGNED;
+  GemmArgs args{};
+  args.out = d;
+  args.a_idx = a_idx;
+  args.a_src_rows = (int)n_src;
+  return launch_gemm_layout<kEpiI32, true>(b_layout, a_src, b, G, M, N, K, N, args,
+                                           as_stream(stream));
+}
+
+int convrot_i8_gemm_swiglu_gather(const int8_t* a_src, const float* s_src, int64_t n_src,
+                                  const int32_t* a_idx, const int8_t* b, const float* s_b,
+                                  int b_layout, int64_t G, int64_t M, int64_t F, int64_t K,
+                                  float* h, void* stream) {
+  if (b_layout != CONVROT_LAYOUT_ROWS && b_layout != CONVROT_LAYOUT_TILES)
+    return CONVROT_ERR_INVALID_ARG;
+  if (F < 0 || F % 16 != 0) return CONVROT_ERR_INVALID_ARG;
+  int rc = check_gemm_shape(a_src, b, G, M, 2 * F, K);
+  if (rc != CONVROT_OK) return rc;
+  if (n_src < 0 || n_src >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
+  if (G * M * F > 0 && (!s_src || !s_b || !h || !a_idx || n_src == 0))
+    return CONVROT_ERR_INVALID_ARG;
+  if (!al16(s_src) || !al16(s_b) || !al16(h)) return CONVROT_ERR_MISALIGNED;
+  GemmArgs args{};
+  args.s_a = s_src;
+  args.s_b = s_b;
+  args.out = h;
+  args.a_idx = a_idx;
+  args.a_src_rows = (int)n_src;
+  return launch_gemm_layout<kEpiSwiglu, true>(b_layout, a_src, b, G, M, 2 * F, K, F, args,
+                                              as_stream(stream));
 }
 
 int convrot_i8_gemm_scatter(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,

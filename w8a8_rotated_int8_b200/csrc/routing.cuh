@@ -397,16 +397,6 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const int8_t* __restri
 // z holds the experts' BF16 outputs; s_t[e, t] is the router score of token t
 // for expert e, i.e. the weight top-C stored for the pick, so the slot and
 // weight look-ups are independent loads.
-//
-// One CTA of kCombineThreads per token. Every warp builds the token's list
-// (rows and weights in ascending expert order) itself from one round of
-// loads, so no CTA-wide barrier is needed; then each thread sums its
-// 8-column (16-byte) vectors over the rows, two rows' loads in flight at a
-// time.
-constexpr int kCombineThreads = 128;
-constexpr int kCombineWarps = kCombineThreads / 32;
-constexpr int kCombineVecs = 2;  // 8-column vectors per thread per pass
-
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&f)[8]) {
   const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -416,99 +406,141 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&f)[8]) {
   }
 }
 
+// One CTA per run of `tpc` consecutive tokens. The [E, tpc] tiles of slots and
+// router scores are read with coalesced loads (tpc consecutive tokens of one
+// expert are contiguous), the picks of all tpc tokens are laid out as one
+// flat list in shared memory (token by token, each in ascending expert
+// order), and every thread streams its 16-byte column vector of the listed
+// rows, eight loads in flight, closing a token's bf16 output when the list
+// moves on to the next token. Tokens without picks get 0.
+constexpr int kCombThreads = 256;
+constexpr int kCombBatch = 8;
+
+__device__ __forceinline__ uint4 f32x8_to_bf16x8(const float (&a)[8]) {
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 pr = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+    o[i] = *reinterpret_cast<const uint32_t*>(&pr);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// shared memory: E * (tpc + 1) int32 slots and as many fp32 scores (stride
+// tpc + 1 so a warp reading one token's column hits distinct banks), then the
+// flat list: E * tpc rows (int32), weights (fp32) and token indices (uint8),
+// then tpc + 1 list starts.
+__host__ __device__ inline size_t combine_tokens_smem(int E, int tpc) {
+  return (size_t)E * (tpc + 1) * 8 + (size_t)E * tpc * 9 + (size_t)(tpc + 1) * 4 + 64;
+}
+
 template <int NJ>
-__global__ void __launch_bounds__(kCombineThreads) combine_rows_kernel(
+__global__ void __launch_bounds__(kCombThreads) combine_tokens_kernel(
     const __nv_bfloat16* __restrict__ z, const float* __restrict__ s_t,
-    const int32_t* __restrict__ slot, int E, int T, int C, int d, __nv_bfloat16* __restrict__ y) {
-  __shared__ int32_t sel_all[kCombineWarps][32 * NJ];
-  __shared__ float sw_all[kCombineWarps][32 * NJ];
-  const int t = blockIdx.x;
+    const int32_t* __restrict__ slot, int E, int T, int C, int d, int tpc,
+    __nv_bfloat16* __restrict__ y) {
+  extern __shared__ __align__(16) uint8_t cm_smem[];
+  const int ld = tpc + 1;
+  int32_t* sl = reinterpret_cast<int32_t*>(cm_smem);
+  float* sw = reinterpret_cast<float*>(sl + (size_t)E * ld);
+  int32_t* fr = reinterpret_cast<int32_t*>(sw + (size_t)E * ld);
+  float* fw = reinterpret_cast<float*>(fr + (size_t)E * tpc);
+  int32_t* start = reinterpret_cast<int32_t*>(fw + (size_t)E * tpc);
+  uint8_t* ftok = reinterpret_cast<uint8_t*>(start + tpc + 1);
+  const int t0 = blockIdx.x * tpc;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int32_t* sel = sel_all[warp];
-  float* sw = sw_all[warp];
-  int32_t sv[NJ];
-  float wv[NJ];
-#pragma unroll
-  for (int j = 0; j < NJ; ++j) {
-    const int e = lane + 32 * j;
-    sv[j] = e < E ? __ldg(slot + (int64_t)e * T + t) : -1;
-    wv[j] = e < E ? __ldg(s_t + (int64_t)e * T + t) : 0.0f;
-  }
-  int n = 0;
-#pragma unroll
-  for (int j = 0; j < NJ; ++j) {
-    const bool bad = sv[j] >= C;
-    if (bad && warp == 0) atomicOr(&g_device_error, kErrBadIndex);
-    const bool has = sv[j] >= 0 && !bad;
-    const unsigned m = __ballot_sync(0xffffffffu, has);
-    if (has) {
-      const int pos = n + __popc(m & ((1u << lane) - 1u));
-      sel[pos] = (lane + 32 * j) * C + sv[j];
-      sw[pos] = wv[j];
+  const int nwarps = kCombThreads / 32;
+
+  // 1. the [E, tpc] slot and score tiles (coalesced along the tokens)
+  for (int i = threadIdx.x; i < E * tpc; i += kCombThreads) {
+    const int e = i / tpc, j = i - e * tpc;
+    const int t = t0 + j;
+    int32_t sv = -1;
+    float wv = 0.0f;
+    if (t < T) {
+      sv = __ldg(slot + (int64_t)e * T + t);
+      wv = __ldg(s_t + (int64_t)e * T + t);
+      if (sv >= C) {
+        atomicOr(&g_device_error, kErrBadIndex);
+        sv = -1;
+      }
     }
-    n += __popc(m);
+    sl[e * ld + j] = sv;
+    sw[e * ld + j] = wv;
   }
-  __syncwarp();
+  __syncthreads();
+  // 2. picks per token (warp w counts tokens w, w + 8, ...)
+  for (int j = warp; j < tpc; j += nwarps) {
+    int n = 0;
+#pragma unroll
+    for (int k = 0; k < NJ; ++k) {
+      const int e = lane + 32 * k;
+      n += __popc(__ballot_sync(0xffffffffu, e < E && sl[e * ld + j] >= 0));
+    }
+    if (lane == 0) start[j + 1] = n;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    start[0] = 0;
+    for (int j = 0; j < tpc; ++j) start[j + 1] += start[j];
+  }
+  __syncthreads();
+  // 3. the flat list, each token's picks in ascending expert order
+  for (int j = warp; j < tpc; j += nwarps) {
+    int pos = start[j];
+#pragma unroll
+    for (int k = 0; k < NJ; ++k) {
+      const int e = lane + 32 * k;
+      const int32_t sv = e < E ? sl[e * ld + j] : -1;
+      const unsigned m = __ballot_sync(0xffffffffu, sv >= 0);
+      if (sv >= 0) {
+        const int p = pos + __popc(m & ((1u << lane) - 1u));
+        fr[p] = e * C + sv;
+        fw[p] = sw[e * ld + j];
+        ftok[p] = (uint8_t)j;
+      }
+      pos += __popc(m);
+    }
+  }
+  __syncthreads();
+  // 4. stream the rows
+  const int n_total = start[tpc];
+  const int n_tok = min(tpc, T - t0);
   const int d8 = d >> 3;
-  uint4* yrow = reinterpret_cast<uint4*>(y + (int64_t)t * d);
-  for (int q0 = threadIdx.x; q0 < d8; q0 += kCombineThreads * kCombineVecs) {
-    float acc[kCombineVecs][8];
+  for (int q = threadIdx.x; q < d8; q += kCombThreads) {
+    float acc[8];
 #pragma unroll
-    for (int u = 0; u < kCombineVecs; ++u)
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    int cur = 0;  // token whose sum is being accumulated
+    for (int p0 = 0; p0 < n_total; p0 += kCombBatch) {
+      uint4 v[kCombBatch];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
-    int k = 0;
-    for (; k + 2 <= n; k += 2) {
-      const uint4* r0 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k] * d);
-      const uint4* r1 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k + 1] * d);
-      const float w0 = sw[k], w1 = sw[k + 1];
-      uint4 a[kCombineVecs], b[kCombineVecs];
+      for (int u = 0; u < kCombBatch; ++u)
+        if (p0 + u < n_total)
+          v[u] = __ldcs(reinterpret_cast<const uint4*>(z + (int64_t)fr[p0 + u] * d) + q);
 #pragma unroll
-      for (int u = 0; u < kCombineVecs; ++u) {
-        const int q = q0 + u * kCombineThreads;
-        if (q < d8) {
-          a[u] = __ldcs(r0 + q);
-          b[u] = __ldcs(r1 + q);
-        }
-      }
+      for (int u = 0; u < kCombBatch; ++u) {
+        if (p0 + u < n_total) {
+          const int tok = ftok[p0 + u];
+          while (cur < tok) {  // close the tokens before this pick
+            reinterpret_cast<uint4*>(y + (int64_t)(t0 + cur) * d)[q] = f32x8_to_bf16x8(acc);
 #pragma unroll
-      for (int u = 0; u < kCombineVecs; ++u) {
-        if (q0 + u * kCombineThreads < d8) {
-          float fa[8], fb[8];
-          bf16x8_to_f32(a[u], fa);
-          bf16x8_to_f32(b[u], fb);
+            for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+            ++cur;
+          }
+          float f[8];
+          bf16x8_to_f32(v[u], f);
+          const float w = fw[p0 + u];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            acc[u][i] = __fadd_rn(__fadd_rn(acc[u][i], __fmul_rn(w0, fa[i])), __fmul_rn(w1, fb[i]));
+          for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(w, f[i]));
         }
       }
     }
-    if (k < n) {
-      const uint4* r0 = reinterpret_cast<const uint4*>(z + (int64_t)sel[k] * d);
-      const float w0 = sw[k];
+    while (cur < n_tok) {
+      reinterpret_cast<uint4*>(y + (int64_t)(t0 + cur) * d)[q] = f32x8_to_bf16x8(acc);
 #pragma unroll
-      for (int u = 0; u < kCombineVecs; ++u) {
-        const int q = q0 + u * kCombineThreads;
-        if (q < d8) {
-          float fa[8];
-          bf16x8_to_f32(__ldcs(r0 + q), fa);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[u][i] = __fadd_rn(acc[u][i], __fmul_rn(w0, fa[i]));
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kCombineVecs; ++u) {
-      const int q = q0 + u * kCombineThreads;
-      if (q < d8) {
-        uint32_t o[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(acc[u][2 * i], acc[u][2 * i + 1]);
-          o[i] = *reinterpret_cast<const uint32_t*>(&pr);
-        }
-        yrow[q] = make_uint4(o[0], o[1], o[2], o[3]);
-      }
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+      ++cur;
     }
   }
 }
