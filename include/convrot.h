@@ -195,23 +195,6 @@ int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, c
                            int b_layout, int64_t G, int64_t M, int64_t F, int64_t K, float* h,
                            void* stream);
 
-/* Gathered forms (the expert-choice gather inside the GEMM): row m of group g
- * of A is row a_idx[g * M + m] of the code matrix a_src [n_src, K], loaded by
- * TMA tile::gather4; every a_idx entry must lie in [0, n_src) (an entry
- * outside is recorded in the device error word as a bad index and replaced
- * by row 0). Otherwise as the calls above.
- *   a_src  device, [n_src, K] int8;  a_idx device, [G, M] int32 */
-int convrot_i8_gemm_i32_gather(const int8_t* a_src, int64_t n_src, const int32_t* a_idx,
-                               const int8_t* b, int b_layout, int64_t G, int64_t M, int64_t N,
-                               int64_t K, int32_t* d, void* stream);
-
-/* Gathered SwiGLU: as convrot_i8_gemm_swiglu with A row (g, m) = a_src row
- * a_idx[g * M + m] and its token scale s_src[a_idx[g * M + m]]. */
-int convrot_i8_gemm_swiglu_gather(const int8_t* a_src, const float* s_src, int64_t n_src,
-                                  const int32_t* a_idx, const int8_t* b, const float* s_b,
-                                  int b_layout, int64_t G, int64_t M, int64_t F, int64_t K,
-                                  float* h, void* stream);
-
 /* Router-weighted scatter epilogue:
  * out32[idx[g, m], n] += w[g, m] * (fp32(acc) * (s_b[g, n] * s_a[g, m])).
  * out32 device [T, N] fp32 (accumulated with fp32 atomics, order not fixed);

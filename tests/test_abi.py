@@ -65,12 +65,6 @@ def test_argument_checks_need_no_gpu(lib):
     assert lib.convrot_i8_gemm_i32(al, al, 0, 1, 8, 24, 64, al, None) == INVALID
     assert lib.convrot_i8_gemm_i32(al, al, 0, 1, 8, 16, 1 << 20, al, None) == INVALID
     assert lib.convrot_i8_gemm_i32(al, al, 2, 1, 8, 16, 64, al, None) == INVALID  # bad layout
-    # gathered GEMMs: no source rows; misaligned output
-    assert lib.convrot_i8_gemm_i32_gather(al, 0, al, al, 0, 1, 8, 16, 64, al, None) == INVALID
-    assert lib.convrot_i8_gemm_swiglu_gather(al, al, 0, al, al, al, 0, 1, 8, 16, 64, al,
-                                             None) == INVALID
-    assert lib.convrot_i8_gemm_swiglu_gather(al, al, 10, al, al, al, 0, 1, 8, 16, 64, mis,
-                                             None) == MISALIGNED
     # tiled weight sizes: 128-row blocks x 128-byte K tiles of 16 KB
     assert lib.convrot_tiled_weight_bytes(2, 300, 200) == 2 * 3 * 2 * 16384
     assert lib.convrot_tiled_weight_bytes(128, 1536, 2048) == 128 * 12 * 16 * 16384

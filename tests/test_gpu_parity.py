@@ -253,48 +253,6 @@ def test_gemm_swiglu(g, m, f, k, layout):
         assert (ulps == 0).mean() > 0.8  # expf differs from exp in ~1 of 10 elements
 
 
-GATHER_SHAPES = [(1, 64, 256, 256, 100), (3, 160, 320, 768, 200), (2, 37, 48, 2048, 50),
-                 (1, 300, 272, 1536, 333), (2, 129, 512, 64, 1000), (1, 1, 16, 16, 1),
-                 (4, 256, 3072, 2048, 700)]
-
-
-@pytest.mark.parametrize("layout", ["rows", "tiles"])
-@pytest.mark.parametrize("g,m,n,k,n_src", GATHER_SHAPES)
-def test_gemm_gather_int32_bit_exact(g, m, n, k, n_src, layout):
-    """The expert-choice gather inside the GEMM (TMA gather4, both the
-    single-CTA and the CTA-pair kernels, ragged row counts): exact int32
-    accumulators of a_src[idx[g]] @ b[g]^T, repeated indices included."""
-    a_src = _codes((n_src, k), 11 + m)
-    gen = torch.Generator().manual_seed(12 + n)
-    idx = torch.randint(0, n_src, (g, m), generator=gen, dtype=torch.int32)
-    b = _codes((g, n, k), 13 + k)
-    bb = b.cuda() if layout == "rows" else _tiled_codes(b)
-    d = W.convrot_i8_gemm_i32_gather(a_src.cuda(), idx.cuda(), bb).cpu().numpy()
-    for gi in range(g):
-        ref = O.int_gemm(a_src[idx[gi].long()].numpy(), b[gi].numpy())
-        assert np.array_equal(d[gi], ref)
-
-
-@pytest.mark.parametrize("layout", ["rows", "tiles"])
-@pytest.mark.parametrize("g,m,f,k,n_src", [(2, 160, 320, 768, 300), (1, 64, 1536, 2048, 90),
-                                           (3, 40, 192, 512, 41), (2, 300, 256, 256, 500)])
-def test_gemm_swiglu_gather_exact(g, m, f, k, n_src, layout):
-    """The gathered SwiGLU GEMM equals the SwiGLU GEMM on rows gathered on the
-    host, bit for bit (same epilogue arithmetic on the same accumulators)."""
-    a_src = _codes((n_src, k), 21 + m)
-    s_src = torch.rand(n_src) * 0.05 + 1e-3
-    gen = torch.Generator().manual_seed(22 + f)
-    idx = torch.randint(0, n_src, (g, m), generator=gen, dtype=torch.int32)
-    b = _codes((g, 2 * f, k), 23)
-    s_b = torch.rand(g, 2 * f) * 1e-4 + 1e-6
-    bb = b.cuda() if layout == "rows" else _tiled_codes(b.view(2 * g, f, k))
-    h = W.convrot_i8_gemm_swiglu_gather(a_src.cuda(), s_src.cuda(), idx.cuda(), bb, s_b.cuda())
-    a_g = a_src[idx.long()]
-    s_g = s_src[idx.long()]
-    h_plain = W.convrot_i8_gemm_swiglu(a_g.cuda(), s_g.cuda(), bb, s_b.cuda())
-    assert torch.equal(h.cpu(), h_plain.cpu())
-
-
 @pytest.mark.parametrize("layout", ["rows", "tiles"])
 def test_gemm_scatter(layout):
     g, m, n, k, t = 4, 100, 320, 512, 150

@@ -16,10 +16,8 @@ from .binding import (  # noqa: F401
     convrot_gather_rows,
     convrot_i8_gemm_bf16,
     convrot_i8_gemm_i32,
-    convrot_i8_gemm_i32_gather,
     convrot_i8_gemm_scatter,
     convrot_i8_gemm_swiglu,
-    convrot_i8_gemm_swiglu_gather,
     convrot_linear_workspace_size,
     convrot_quantize_weights,
     convrot_quantize_weights_tiled,

@@ -68,9 +68,6 @@ _SIGNATURES = {
     "convrot_i8_gemm_i32": (_I, [_P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
     "convrot_i8_gemm_bf16": (_I, [_P, _P, _P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
     "convrot_i8_gemm_swiglu": (_I, [_P, _P, _P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
-    "convrot_i8_gemm_i32_gather": (_I, [_P, _I64, _P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
-    "convrot_i8_gemm_swiglu_gather": (_I, [_P, _P, _I64, _P, _P, _P, _I, _I64, _I64, _I64, _I64, _P,
-                                           _P]),
     "convrot_i8_gemm_scatter": (_I, [_P, _P, _P, _P, _I, _P, _P, _I64, _I64, _I64, _I64, _P, _I64,
                                      _P]),
     "convrot_f32_to_bf16": (_I, [_P, _I64, _P, _P]),
@@ -321,58 +318,6 @@ def convrot_i8_gemm_swiglu(a, s_a, b, s_b, stream=None):
     _check(lib().convrot_i8_gemm_swiglu(_p(a), _p(s_a), _p(bt), _p(s_b), lay, g, m, f, k, _p(h),
                                         _stream(stream)), "convrot_i8_gemm_swiglu")
     return h if a.dim() == 3 else h[0]
-
-
-def _gather_dims(a_src, a_idx, b, swiglu=False):
-    """(G, M, N, K, b pointer tensor, layout) of a gathered GEMM: a_idx is
-    [G, M] int32 rows of a_src [n_src, K]."""
-    _need(a_src, torch.int8, "a_src")
-    _need(a_idx, torch.int32, "a_idx")
-    if a_idx.dim() == 1:
-        a_idx = a_idx[None]
-    g, m = a_idx.shape
-    return _gemm_dims_shape((g, m, a_src.shape[1]), b, swiglu)
-
-
-def _gemm_dims_shape(shape, b, swiglu):
-    g, m, k = shape
-    if isinstance(b, TiledWeights):
-        per = 2 if swiglu else 1
-        if b.n_mats != g * per or b.k != k:
-            raise ValueError("tiled weights do not match a [G,M,K]")
-        return g, m, b.rows * per, k, b.data, LAYOUT_TILES
-    _need(b, torch.int8, "b")
-    if b.dim() == 2:
-        b = b[None]
-    gb, n, kb = b.shape
-    if gb != g or kb != k:
-        raise ValueError("a [G,M,K] and b [G,N,K] disagree")
-    return g, m, n, k, b, LAYOUT_ROWS
-
-
-def convrot_i8_gemm_i32_gather(a_src, a_idx, b, stream=None):
-    """Exact int32 acc[g, m, n] = sum_k a_src[a_idx[g, m], k] b[g, n, k]
-    (the gather happens inside the GEMM)."""
-    g, m, n, k, bt, lay = _gather_dims(a_src, a_idx, b)
-    d = torch.empty((g, m, n), dtype=torch.int32, device=a_src.device)
-    _check(lib().convrot_i8_gemm_i32_gather(_p(a_src), a_src.shape[0], _p(a_idx), _p(bt), lay, g, m,
-                                            n, k, _p(d), _stream(stream)),
-           "convrot_i8_gemm_i32_gather")
-    return d
-
-
-def convrot_i8_gemm_swiglu_gather(a_src, s_src, a_idx, b, s_b, stream=None):
-    """Gathered SwiGLU GEMM: A row (g, m) = a_src[a_idx[g, m]] -> h [G, M, F] fp32."""
-    g, m, n2, k, bt, lay = _gather_dims(a_src, a_idx, b, swiglu=True)
-    _need(s_src, torch.float32, "s_src")
-    _need(s_b, torch.float32, "s_b")
-    f = n2 // 2
-    h = torch.empty((g, m, f), dtype=torch.float32, device=a_src.device)
-    _check(lib().convrot_i8_gemm_swiglu_gather(_p(a_src), _p(s_src), a_src.shape[0], _p(a_idx),
-                                               _p(bt), _p(s_b), lay, g, m, f, k, _p(h),
-                                               _stream(stream)),
-           "convrot_i8_gemm_swiglu_gather")
-    return h
 
 
 def convrot_i8_gemm_scatter(a, s_a, b, s_b, idx, w, out32, stream=None):

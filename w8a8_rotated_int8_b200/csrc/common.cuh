@@ -114,6 +114,20 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint6
   return true;
 }
 
+// ------------------------------------------- programmatic dependent launch --
+// A kernel of the block's chain lets its successor on the stream launch early
+// (its CTAs are scheduled once every CTA of this grid has executed the
+// trigger or exited, so they can only take resources this grid no longer
+// waits for), and waits for its predecessor's completion and memory before
+// touching what the predecessor wrote. Both are no-ops for a kernel launched
+// without the programmatic-serialization attribute.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------------- TMA --
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
@@ -161,21 +175,6 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
-      : "memory");
-}
-
-// Gathered load (no multicast): four rows r0..r3 of a 2-D tensor map whose box
-// is {128 bytes, 1 row}, starting at inner coordinate c0, land in four
-// consecutive 128-byte rows of shared memory at dst (512 bytes). With the
-// 128-byte swizzle the placement depends only on the shared-memory address,
-// so 32 such loads at dst = base + 512 j (base 1024-aligned) give the same
-// layout as one 128-row tiled box.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int c0,
-                                            int r0, int r1, int r2, int r3, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "l"(policy)
       : "memory");
 }
 
@@ -333,19 +332,6 @@ __device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* m
       "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(dst)),
       "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
-      : "memory");
-}
-
-// Gathered load of a CTA pair: as tma_gather4, the byte count completing on
-// the mbarrier at `bar_cluster` (the leader CTA's barrier). No multicast.
-__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* map,
-                                                 uint32_t bar_cluster, int c0, int r0, int r1,
-                                                 int r2, int r3, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
-      ".mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(
-          smem_u32(dst)),
-      "l"(map), "r"(bar_cluster), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "l"(policy)
       : "memory");
 }
 

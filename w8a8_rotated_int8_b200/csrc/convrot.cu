@@ -87,23 +87,21 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <int EPI, bool BT, bool GA>
+template <int EPI, bool BT>
 void set_gemm_attr() {
-  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<EPI, BT, GA>,
+  cudaFuncSetAttribute(gemm_s8_tcgen05_kernel<EPI, BT>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<EPI>::kSmem1);
-  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<EPI, BT, GA>,
+  cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<EPI, BT>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<EPI>::kSmem2);
 }
 
 // every GEMM instantiation the entry points launch
 template <bool BT>
 void set_gemm_attrs() {
-  set_gemm_attr<kEpiI32, BT, false>();
-  set_gemm_attr<kEpiI32, BT, true>();
-  set_gemm_attr<kEpiBf16, BT, false>();
-  set_gemm_attr<kEpiSwiglu, BT, false>();
-  set_gemm_attr<kEpiSwiglu, BT, true>();
-  set_gemm_attr<kEpiScatter, BT, false>();
+  set_gemm_attr<kEpiI32, BT>();
+  set_gemm_attr<kEpiBf16, BT>();
+  set_gemm_attr<kEpiSwiglu, BT>();
+  set_gemm_attr<kEpiScatter, BT>();
 }
 
 // Per-device one-time setup: capability check, SM count, kernel attributes.
@@ -147,6 +145,40 @@ int launch_status() {
   return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
+// Launches `kern` on `st`; `pdl` adds programmatic stream serialization (the
+// kernel may start while its predecessor on the stream finishes; it waits for
+// it with griddepcontrol.wait), `cluster_x` > 1 a cluster dimension.
+template <typename... KArgs, typename... Args>
+int launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                  bool pdl, int cluster_x, Args... args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  lc.attrs = attr;
+  lc.numAttrs = n;
+  if (cudaLaunchKernelEx(&lc, kern, args...) != cudaSuccess) {
+    cudaGetLastError();
+    return CONVROT_ERR_CUDA;
+  }
+  return CONVROT_OK;
+}
+
 // --------------------------------------------------------------- rotquant --
 // 3-D byte view {128, K * esize / 128, rows} of a row-major [rows, K] matrix,
 // box = `box_rows` whole rows, 128-byte swizzle (see rotquant_tma_kernel).
@@ -167,7 +199,7 @@ int encode_rows_sw128(CUtensorMap* map, const void* base, uint64_t row_bytes, ui
 
 template <typename InT, int G, int SEG>
 int launch_rq_tma(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
-                   cudaStream_t st) {
+                   cudaStream_t st, bool pdl) {
   constexpr int kRowsPerWarp = 32 / SEG;
   const uint64_t row_bytes = (uint64_t)K * sizeof(InT);
   CUtensorMap tm;
@@ -189,23 +221,23 @@ int launch_rq_tma(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut
   const int64_t units = (rows + kRowsPerWarp - 1) / kRowsPerWarp;
   const int64_t ctas = (units + kRqTmaWarps - 1) / kRqTmaWarps;
   const int64_t grid = std::min<int64_t>(ctas, (int64_t)per_sm * std::max(sms, 1));
-  kern<<<(unsigned)grid, kRqTmaWarps * 32, smem, st>>>(tm, rows, K, slots, slot_bytes, q, s, out);
-  return CONVROT_OK;
+  return launch_kernel(kern, dim3((unsigned)grid), dim3(kRqTmaWarps * 32), smem, st, pdl, 1, tm,
+                       rows, K, slots, slot_bytes, q, s, out);
 }
 
 template <typename InT, int G>
 int launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
-               cudaStream_t st) {
+               cudaStream_t st, bool pdl) {
   // K % 64 == 0, K <= 2048: one warp segment of SEG lanes per row, 64
   // elements per lane (G = 256 needs at least the four lanes of one group)
   if (K % 64 == 0 && K <= 2048) {
     const int lanes = K / 64;
-    if (lanes <= 1 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 1 : 4)>(x, rows, K, q, s, out, st);
-    if (lanes <= 2 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 2 : 4)>(x, rows, K, q, s, out, st);
-    if (lanes <= 4) return launch_rq_tma<InT, G, 4>(x, rows, K, q, s, out, st);
-    if (lanes <= 8) return launch_rq_tma<InT, G, 8>(x, rows, K, q, s, out, st);
-    if (lanes <= 16) return launch_rq_tma<InT, G, 16>(x, rows, K, q, s, out, st);
-    return launch_rq_tma<InT, G, 32>(x, rows, K, q, s, out, st);
+    if (lanes <= 1 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 1 : 4)>(x, rows, K, q, s, out, st, pdl);
+    if (lanes <= 2 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 2 : 4)>(x, rows, K, q, s, out, st, pdl);
+    if (lanes <= 4) return launch_rq_tma<InT, G, 4>(x, rows, K, q, s, out, st, pdl);
+    if (lanes <= 8) return launch_rq_tma<InT, G, 8>(x, rows, K, q, s, out, st, pdl);
+    if (lanes <= 16) return launch_rq_tma<InT, G, 16>(x, rows, K, q, s, out, st, pdl);
+    return launch_rq_tma<InT, G, 32>(x, rows, K, q, s, out, st, pdl);
   }
   const int nch = K / 16;
   int tpr;
@@ -228,20 +260,19 @@ int launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out
   int sms = 0;
   device_setup(&sms);
   const int64_t grid = std::min<int64_t>(groups, (int64_t)per_sm * std::max(sms, 1));
-  rotquant_kernel<InT, G><<<(unsigned)grid, threads, 0, st>>>(
-      reinterpret_cast<const InT*>(x), rows, K, tpr, q, s, out);
-  return CONVROT_OK;
+  return launch_kernel(rotquant_kernel<InT, G>, dim3((unsigned)grid), dim3(threads), 0, st, pdl, 1,
+                       reinterpret_cast<const InT*>(x), rows, K, tpr, q, s, out);
 }
 
 template <typename InT>
 int dispatch_rq(int group, const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
-                cudaStream_t st) {
+                cudaStream_t st, bool pdl) {
   switch (group) {
-    case 1: return launch_rq<InT, 1>(x, rows, K, q, s, out, st);
-    case 4: return launch_rq<InT, 4>(x, rows, K, q, s, out, st);
-    case 16: return launch_rq<InT, 16>(x, rows, K, q, s, out, st);
-    case 64: return launch_rq<InT, 64>(x, rows, K, q, s, out, st);
-    default: return launch_rq<InT, 256>(x, rows, K, q, s, out, st);
+    case 1: return launch_rq<InT, 1>(x, rows, K, q, s, out, st, pdl);
+    case 4: return launch_rq<InT, 4>(x, rows, K, q, s, out, st, pdl);
+    case 16: return launch_rq<InT, 16>(x, rows, K, q, s, out, st, pdl);
+    case 64: return launch_rq<InT, 64>(x, rows, K, q, s, out, st, pdl);
+    default: return launch_rq<InT, 256>(x, rows, K, q, s, out, st, pdl);
   }
 }
 
@@ -257,11 +288,11 @@ int check_rq_args(const void* x, int x_dtype, int64_t rows, int64_t K, int group
 }
 
 int rotquant_impl(const void* x, int x_dtype, int64_t rows, int64_t K, int group, int8_t* q,
-                  float* s, cudaStream_t st, RqOut out = RqOut{0, 1, 1, 1}) {
+                  float* s, cudaStream_t st, RqOut out = RqOut{0, 1, 1, 1}, bool pdl = false) {
   if (rows == 0) return CONVROT_OK;
   const int rc = (x_dtype == CONVROT_DTYPE_BF16)
-                     ? dispatch_rq<__nv_bfloat16>(group, x, rows, (int)K, q, s, out, st)
-                     : dispatch_rq<float>(group, x, rows, (int)K, q, s, out, st);
+                     ? dispatch_rq<__nv_bfloat16>(group, x, rows, (int)K, q, s, out, st, pdl)
+                     : dispatch_rq<float>(group, x, rows, (int)K, q, s, out, st, pdl);
   if (rc != CONVROT_OK) return rc;
   return launch_status();
 }
@@ -315,30 +346,12 @@ int encode_tiled_b(CUtensorMap* map, const void* base, uint64_t kb_count, uint64
   return r == CUDA_SUCCESS ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
-// 2-D map over a [rows, K] code matrix with a {128-byte, 1-row} box and the
-// 128-byte swizzle, for tile::gather4 loads of single rows.
-int encode_gather_rows(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return CONVROT_ERR_CUDA;
-  const cuuint64_t dims[2] = {K, rows};
-  const cuuint64_t strides[1] = {K};
-  const cuuint32_t box[2] = {(cuuint32_t)gemm::BK, 1};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? CONVROT_OK : CONVROT_ERR_CUDA;
-}
-
 // NB = rows of one B matrix per group (2F for SwiGLU). With BT the B operand
 // is in the tiled weight format: for SwiGLU each group holds a gate matrix and
-// an up matrix of F rows, each padded to 128-row blocks. With GA the rows of A
-// are gathered: `a` is the [args.a_src_rows, K] source and args.a_idx [G*M]
-// names the source row of every A row.
-template <int EPI, bool BT, bool GA = false>
+// an up matrix of F rows, each padded to 128-row blocks.
+template <int EPI, bool BT>
 int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t NB, int64_t K,
-                int64_t n_out, GemmArgs args, cudaStream_t st) {
+                int64_t n_out, GemmArgs args, cudaStream_t st, bool pdl = false) {
   int sms = 0;
   int rc = device_setup(&sms);
   if (rc != CONVROT_OK) return rc;
@@ -346,14 +359,8 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
   CUtensorMap ta, tb;
   const uint32_t box_a = (uint32_t)std::min<int64_t>(gemm::BM, M);
   uint32_t box_b;
-  if (GA) {
-    if (args.a_idx == nullptr || args.a_src_rows < 1) return CONVROT_ERR_INVALID_ARG;
-    if ((rc = encode_gather_rows(&ta, a, (uint64_t)K, (uint64_t)args.a_src_rows)) != CONVROT_OK)
-      return rc;
-  } else if ((rc = encode_3d_i8(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)G, box_a)) !=
-             CONVROT_OK) {
+  if ((rc = encode_3d_i8(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)G, box_a)) != CONVROT_OK)
     return rc;
-  }
   if (BT) {
     const int64_t blocks = (EPI == kEpiSwiglu) ? cdiv(n_out, 128) : cdiv(NB, 128);
     const int64_t per_group = (EPI == kEpiSwiglu) ? 2 * blocks : blocks;
@@ -383,26 +390,12 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
     const int64_t tiles = G * args.m_blocks * args.n_blocks;
     if (tiles >= ((int64_t)1 << 30)) return CONVROT_ERR_INVALID_ARG;
     args.num_tiles = (int)tiles;
-    // both CTAs' A and B boxes (gathered A rows are counted in the kernel)
-    args.box_bytes = GA ? 2 * 128 * gemm::BK : 2 * (128 + 128) * gemm::BK;
+    args.box_bytes = 2 * (128 + 128) * gemm::BK;  // both CTAs' A and B boxes
     const int grid = 2 * (int)std::min<int64_t>(tiles, sms / 2);
-    cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3(grid);
-    lc.blockDim = dim3(EpiCfg<EPI>::kThreads);
-    lc.dynamicSmemBytes = EpiCfg<EPI>::kSmem2;
-    lc.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    lc.attrs = attr;
-    lc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&lc, gemm_s8_tcgen05_pair_kernel<EPI, BT, GA>, ta, tb, args) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      return CONVROT_ERR_CUDA;
-    }
+    if ((rc = launch_kernel(gemm_s8_tcgen05_pair_kernel<EPI, BT>, dim3(grid),
+                            dim3(EpiCfg<EPI>::kThreads), EpiCfg<EPI>::kSmem2, st, pdl, 2, ta, tb,
+                            args)) != CONVROT_OK)
+      return rc;
     return launch_status();
   }
   args.m_blocks = (int)cdiv(M, gemm::BM);
@@ -412,46 +405,48 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
   const int64_t tiles = G * args.m_blocks * args.n_blocks;
   if (tiles >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
   args.num_tiles = (int)tiles;
-  // A and B boxes of one stage (gathered A rows are counted in the kernel)
-  args.box_bytes = (int)(((GA ? 0 : box_a) + 2 * box_b) * gemm::BK);
+  args.box_bytes = (int)((box_a + 2 * box_b) * gemm::BK);  // A and B boxes of one stage
   const int grid = (int)std::min<int64_t>(tiles, sms);
-  gemm_s8_tcgen05_kernel<EPI, BT, GA><<<grid, EpiCfg<EPI>::kThreads, EpiCfg<EPI>::kSmem1, st>>>(
-      ta, tb, args);
+  if ((rc = launch_kernel(gemm_s8_tcgen05_kernel<EPI, BT>, dim3(grid), dim3(EpiCfg<EPI>::kThreads),
+                          EpiCfg<EPI>::kSmem1, st, pdl, 1, ta, tb, args)) != CONVROT_OK)
+    return rc;
   return launch_status();
 }
 
-template <int EPI, bool GA = false>
+template <int EPI>
 int launch_gemm_layout(int b_layout, const int8_t* a, const int8_t* b, int64_t G, int64_t M,
                        int64_t NB, int64_t K, int64_t n_out, GemmArgs args, cudaStream_t st) {
   if (b_layout == CONVROT_LAYOUT_TILES)
-    return launch_gemm<EPI, true, GA>(a, b, G, M, NB, K, n_out, args, st);
-  return launch_gemm<EPI, false, GA>(a, b, G, M, NB, K, n_out, args, st);
+    return launch_gemm<EPI, true>(a, b, G, M, NB, K, n_out, args, st);
+  return launch_gemm<EPI, false>(a, b, G, M, NB, K, n_out, args, st);
 }
 
 int topc_impl(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float* w,
-              int32_t* slot, cudaStream_t st) {
+              int32_t* slot, cudaStream_t st, bool pdl = false) {
   if (E == 0 || (C == 0 && slot == nullptr)) return CONVROT_OK;
   // scores held in registers when T <= 16 per thread; the general kernel
   // re-reads them from memory on every pass
   const int per_thread = (int)((T + kTopcThreads - 1) / kTopcThreads);
+  auto kern = topc_kernel;
   if (per_thread <= 1)
-    topc_reg_kernel<1><<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+    kern = topc_reg_kernel<1>;
   else if (per_thread <= 2)
-    topc_reg_kernel<2><<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+    kern = topc_reg_kernel<2>;
   else if (per_thread <= 4)
-    topc_reg_kernel<4><<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+    kern = topc_reg_kernel<4>;
   else if (per_thread <= 8)
-    topc_reg_kernel<8><<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+    kern = topc_reg_kernel<8>;
   else if (per_thread <= 16)
-    topc_reg_kernel<16><<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
-  else
-    topc_kernel<<<E, kTopcThreads, 0, st>>>(s_t, (int)T, (int)C, idx, w, slot);
+    kern = topc_reg_kernel<16>;
+  const int rc = launch_kernel(kern, dim3(E), dim3(kTopcThreads), 0, st, pdl, 1, s_t, (int)T,
+                               (int)C, idx, w, slot);
+  if (rc != CONVROT_OK) return rc;
   return launch_status();
 }
 
 template <int NJ>
 int launch_combine(const void* z, const float* s_t, const int32_t* slot, int E, int64_t T,
-                   int64_t C, int64_t d, void* y, int sms, cudaStream_t st) {
+                   int64_t C, int64_t d, void* y, int sms, cudaStream_t st, bool pdl) {
   // tokens per CTA: a power of two in [1, 32] that leaves about four CTAs per
   // SM, so every SM streams rows while each CTA's slot tiles stay coalesced
   int tpc = 32;
@@ -463,25 +458,24 @@ int launch_combine(const void* z, const float* s_t, const int32_t* slot, int E, 
           cudaSuccess)
     return CONVROT_ERR_CUDA;
   const int64_t grid = (T + tpc - 1) / tpc;
-  kern<<<(unsigned)grid, kCombThreads, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(z), s_t,
-                                                   slot, E, (int)T, (int)C, (int)d, tpc,
-                                                   reinterpret_cast<__nv_bfloat16*>(y));
-  return CONVROT_OK;
+  return launch_kernel(kern, dim3((unsigned)grid), dim3(kCombThreads), smem, st, pdl, 1,
+                       reinterpret_cast<const __nv_bfloat16*>(z), s_t, slot, E, (int)T, (int)C,
+                       (int)d, tpc, reinterpret_cast<__nv_bfloat16*>(y));
 }
 
 // E <= 256 (checked by the entry points)
 int combine_impl(const void* z, const float* s_t, const int32_t* slot, int E, int64_t T, int64_t C,
-                 int64_t d, void* y, int sms, cudaStream_t st) {
+                 int64_t d, void* y, int sms, cudaStream_t st, bool pdl = false) {
   if (T == 0) return CONVROT_OK;
   int rc;
   if (E <= 32)
-    rc = launch_combine<1>(z, s_t, slot, E, T, C, d, y, sms, st);
+    rc = launch_combine<1>(z, s_t, slot, E, T, C, d, y, sms, st, pdl);
   else if (E <= 64)
-    rc = launch_combine<2>(z, s_t, slot, E, T, C, d, y, sms, st);
+    rc = launch_combine<2>(z, s_t, slot, E, T, C, d, y, sms, st, pdl);
   else if (E <= 128)
-    rc = launch_combine<4>(z, s_t, slot, E, T, C, d, y, sms, st);
+    rc = launch_combine<4>(z, s_t, slot, E, T, C, d, y, sms, st, pdl);
   else
-    rc = launch_combine<8>(z, s_t, slot, E, T, C, d, y, sms, st);
+    rc = launch_combine<8>(z, s_t, slot, E, T, C, d, y, sms, st, pdl);
   if (rc != CONVROT_OK) return rc;
   return launch_status();
 }
@@ -698,47 +692,6 @@ int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, c
                                         as_stream(stream));
 }
 
-int convrot_i8_gemm_i32_gather(const int8_t* a_src, int64_t n_src, const int32_t* a_idx,
-                               const int8_t* b, int b_layout, int64_t G, int64_t M, int64_t N,
-                               int64_t K, int32_t* d, void* stream) {
-  if (b_layout != CONVROT_LAYOUT_ROWS && b_layout != CONVROT_LAYOUT_TILES)
-    return CONVROT_ERR_INVALID_ARG;
-  int rc = check_gemm_shape(a_src, b, G, M, N, K);
-  if (rc != CONVROT_OK) return rc;
-  if (n_src < 0 || n_src >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
-  if (G * M * N > 0 && (!d || !a_idx || n_src == 0)) return CONVROT_ERR_INVALID_ARG;
-  if (!al16(d)) return CONVROT_ERR_MISALIGNED;
-  GemmArgs args{};
-  args.out = d;
-  args.a_idx = a_idx;
-  args.a_src_rows = (int)n_src;
-  return launch_gemm_layout<kEpiI32, true>(b_layout, a_src, b, G, M, N, K, N, args,
-                                           as_stream(stream));
-}
-
-int convrot_i8_gemm_swiglu_gather(const int8_t* a_src, const float* s_src, int64_t n_src,
-                                  const int32_t* a_idx, const int8_t* b, const float* s_b,
-                                  int b_layout, int64_t G, int64_t M, int64_t F, int64_t K,
-                                  float* h, void* stream) {
-  if (b_layout != CONVROT_LAYOUT_ROWS && b_layout != CONVROT_LAYOUT_TILES)
-    return CONVROT_ERR_INVALID_ARG;
-  if (F < 0 || F % 16 != 0) return CONVROT_ERR_INVALID_ARG;
-  int rc = check_gemm_shape(a_src, b, G, M, 2 * F, K);
-  if (rc != CONVROT_OK) return rc;
-  if (n_src < 0 || n_src >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
-  if (G * M * F > 0 && (!s_src || !s_b || !h || !a_idx || n_src == 0))
-    return CONVROT_ERR_INVALID_ARG;
-  if (!al16(s_src) || !al16(s_b) || !al16(h)) return CONVROT_ERR_MISALIGNED;
-  GemmArgs args{};
-  args.s_a = s_src;
-  args.s_b = s_b;
-  args.out = h;
-  args.a_idx = a_idx;
-  args.a_src_rows = (int)n_src;
-  return launch_gemm_layout<kEpiSwiglu, true>(b_layout, a_src, b, G, M, 2 * F, K, F, args,
-                                              as_stream(stream));
-}
-
 int convrot_i8_gemm_scatter(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
                             int b_layout, const int32_t* idx, const float* w, int64_t G, int64_t M,
                             int64_t N, int64_t K, float* out32, int64_t T, void* stream) {
@@ -872,7 +825,10 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
   void* z = ws + lay.z;
 
   // Routing (1, 3) runs on the side stream while the caller's stream rotates
-  // and quantises the tokens (2); the streams join before the gather.
+  // and quantises the tokens (2); the streams join before the gather. The
+  // kernels after the gather (and top-C after the softmax) are launched with
+  // programmatic stream serialization: each starts while its predecessor
+  // finishes and waits for it (griddepcontrol.wait) before reading its output.
   SideStream* ss = nullptr;
   if ((rc = side_stream(&ss)) != CONVROT_OK) return rc;
   std::lock_guard<std::mutex> side_lock(ss->mu);
@@ -882,7 +838,7 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
   // 1. router softmax
   int rc_side = softmax_impl(logits_bf16, T, E, s_t, ss->stream);
   // 3. expert-choice top-C (+ each token's slot per expert)
-  if (rc_side == CONVROT_OK) rc_side = topc_impl(s_t, T, E, C, idx, w, slot, ss->stream);
+  if (rc_side == CONVROT_OK) rc_side = topc_impl(s_t, T, E, C, idx, w, slot, ss->stream, true);
   // 2. rotate + quantise the tokens once (the gate/up rotation is expert-independent)
   rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, T, d, g_gu, x_q, s_x, st);
   // the join is recorded even after a failed launch so the side stream never dangles
@@ -900,23 +856,24 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
     a1.s_a = s_g;
     a1.s_b = s_gu;
     a1.out = h;
-    if ((rc = launch_gemm<kEpiSwiglu, true>(x_g, w_gu, E, C, 2 * f, d, f, a1, st)) != CONVROT_OK)
+    if ((rc = launch_gemm<kEpiSwiglu, true>(x_g, w_gu, E, C, 2 * f, d, f, a1, st, true)) !=
+        CONVROT_OK)
       return rc;
     // 6. rotate (g_d) + requantise h per row
-    if ((rc = rotquant_impl(h, CONVROT_DTYPE_F32, (int64_t)E * C, f, g_d, h_q, s_h, st)) !=
-        CONVROT_OK)
+    if ((rc = rotquant_impl(h, CONVROT_DTYPE_F32, (int64_t)E * C, f, g_d, h_q, s_h, st,
+                            RqOut{0, 1, 1, 1}, true)) != CONVROT_OK)
       return rc;
     // 7. down GEMM with dequant to the experts' BF16 outputs
     GemmArgs a2{};
     a2.s_a = s_h;
     a2.s_b = s_d;
     a2.out = z;
-    if ((rc = launch_gemm<kEpiBf16, true>(h_q, w_d, E, C, d, f, d, a2, st)) != CONVROT_OK)
+    if ((rc = launch_gemm<kEpiBf16, true>(h_q, w_d, E, C, d, f, d, a2, st, true)) != CONVROT_OK)
       return rc;
   }
   // 8. per token: router-weighted fp32 sum over its experts in ascending
   // order, one bf16 rounding
-  return combine_impl(z, s_t, slot, E, T, C, d, y_bf16, sms, st);
+  return combine_impl(z, s_t, slot, E, T, C, d, y_bf16, sms, st, C > 0);
 }
 
 }  // extern "C"

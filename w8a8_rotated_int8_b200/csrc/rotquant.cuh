@@ -130,6 +130,8 @@ template <typename InT, int G>
 __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x, int64_t rows,
                                                       int K, int tpr, int8_t* __restrict__ q,
                                                       float* __restrict__ scales, RqOut out) {
+  griddep_launch_dependents();
+  griddep_wait();
   using Tr = RqTraits<G>;
   __shared__ float red[2][16];  // per-warp maxima (512 threads at most), by iteration parity
   const int lane = threadIdx.x & 31;
@@ -337,6 +339,8 @@ template <typename InT, int G, int SEG>
 __global__ void __launch_bounds__(kRqTmaWarps * 32, 2) rotquant_tma_kernel(
     const __grid_constant__ CUtensorMap tm, int64_t rows, int K, int slots, int slot_bytes,
     int8_t* __restrict__ q, float* __restrict__ scales, RqOut out) {
+  griddep_launch_dependents();
+  griddep_wait();
   static_assert(SEG >= 1 && SEG <= 32 && (SEG & (SEG - 1)) == 0, "segment of 2^k lanes");
   static_assert(G != 256 || SEG >= 4, "a 256-group spans four lanes");
   constexpr int kRowsPerWarp = 32 / SEG;

@@ -21,6 +21,8 @@ constexpr int kSmTokens = 32;
 template <int NJ>
 __global__ void __launch_bounds__(1024) router_softmax_kernel(
     const __nv_bfloat16* __restrict__ logits, int T, int E, float* __restrict__ S_t) {
+  griddep_launch_dependents();
+  griddep_wait();
   extern __shared__ float sm_tile[];  // [E][32]
   const int t0 = blockIdx.x * kSmTokens;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -114,6 +116,8 @@ __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const float* __restr
                                                             int C, int32_t* __restrict__ idx,
                                                             float* __restrict__ w,
                                                             int32_t* __restrict__ slot) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int e = blockIdx.x;
   const uint32_t* u = reinterpret_cast<const uint32_t*>(S_t) + (int64_t)e * T;
   __shared__ uint32_t hist[256];
@@ -229,6 +233,8 @@ __global__ void __launch_bounds__(kTopcThreads) topc_reg_kernel(const float* __r
                                                                 int32_t* __restrict__ idx,
                                                                 float* __restrict__ w,
                                                                 int32_t* __restrict__ slot) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int e = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float* row = S_t + (int64_t)e * T;
@@ -363,6 +369,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const int8_t* __restri
                                                           int64_t n_rows, int K,
                                                           int8_t* __restrict__ dst,
                                                           float* __restrict__ s_dst) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= n_rows) return;
@@ -439,6 +447,8 @@ __global__ void __launch_bounds__(kCombThreads) combine_tokens_kernel(
     const __nv_bfloat16* __restrict__ z, const float* __restrict__ s_t,
     const int32_t* __restrict__ slot, int E, int T, int C, int d, int tpc,
     __nv_bfloat16* __restrict__ y) {
+  griddep_launch_dependents();
+  griddep_wait();
   extern __shared__ __align__(16) uint8_t cm_smem[];
   const int ld = tpc + 1;
   int32_t* sl = reinterpret_cast<int32_t*>(cm_smem);
