@@ -34,9 +34,12 @@ from synthetic import MOE_CONFIGS, moe_inputs  # noqa: E402
 
 METRIC = "W8A8 ConvRot MoE block tokens/s"
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
-# kernel, from the ncu capture summarised in profiles/ (per config); to be set
-# to None whenever that kernel changes
-DOMINANT_TRAFFIC_BYTES = {}
+# kernel (the gate/up GEMM with the SwiGLU epilogue), from the ncu captures
+# summarised in profiles/block_kernels_moe_T8192.md and
+# profiles/gemm_s8_tcgen05_moe_T2048.md; to be dropped whenever that kernel
+# changes
+DOMINANT_TRAFFIC_BYTES = {"moe_T8192": 437.105664e6 + 50.836992e6,
+                          "moe_T2048": 411.88864e6 + 8.630016e6}
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 
