@@ -167,7 +167,9 @@ def test_gather_rows():
 
 # -------------------------------------------------------------------- GEMM --
 GEMM_SHAPES = [(1, 64, 256, 256), (3, 160, 320, 768), (2, 40, 48, 2048), (1, 128, 256, 128),
-               (1, 300, 272, 1536), (4, 256, 3072, 2048), (1, 1, 16, 16), (2, 129, 512, 64)]
+               (1, 300, 272, 1536), (4, 256, 3072, 2048), (1, 1, 16, 16), (2, 129, 512, 64),
+               # groups of <= 128 rows with >= 148 single-CTA tiles run on CTA pairs
+               (40, 64, 1024, 512), (150, 100, 256, 128)]
 
 
 def _codes(shape, seed):
@@ -218,7 +220,8 @@ def test_gemm_int32_extremes():
     assert int(d[0, 0, 0]) == -k * 127 * 127 and int(d[0, 5, 1]) == k * 127 * 127
 
 
-@pytest.mark.parametrize("g,m,n,k", [(1, 64, 256, 256), (2, 200, 320, 512), (1, 513, 528, 1536)])
+@pytest.mark.parametrize("g,m,n,k", [(1, 64, 256, 256), (2, 200, 320, 512), (1, 513, 528, 1536),
+                                     (40, 64, 1024, 512)])
 def test_gemm_bf16_dequant_bit_exact(g, m, n, k):
     a = _codes((g, m, k), 3)
     b = _codes((g, n, k), 4)
@@ -236,7 +239,8 @@ def _fp32_ulps(x, ref):
 
 
 @pytest.mark.parametrize("layout", ["rows", "tiles"])
-@pytest.mark.parametrize("g,m,f,k", [(2, 160, 320, 768), (1, 64, 1536, 2048), (3, 40, 192, 512)])
+@pytest.mark.parametrize("g,m,f,k", [(2, 160, 320, 768), (1, 64, 1536, 2048), (3, 40, 192, 512),
+                                     (40, 64, 512, 256)])
 def test_gemm_swiglu(g, m, f, k, layout):
     a = _codes((g, m, k), 5)
     b = _codes((g, 2 * f, k), 6)
@@ -299,9 +303,9 @@ def test_gemm_bf16_grouped_rows_bit_exact(g, m, layout):
                                        (9, 40, 40, 8192), (200, 300, 250, 64)])
 def test_combine_sums_in_expert_order(e_n, t, c, d):
     """y[t] = bf16(sum_e fp32(s_t[e, t] * z[e, slot])) in ascending expert order.
-    d = 2056 leaves a ragged tail of 16-byte pieces; d = 8192 stages one row
-    per slot (the rest from global memory); E = 200 with C = 250 of T = 300
-    gives tokens far more expert rows than a slot holds."""
+    d = 2056 leaves a ragged tail of 16-byte column vectors; d = 8192 gives
+    every thread four column vectors; E = 200 with C = 250 of T = 300 gives
+    tokens far more expert rows than one batch of loads covers."""
     gen = torch.Generator().manual_seed(3 + d)
     z = (torch.randn(e_n * c, d, generator=gen) * 10.0 ** torch.randint(-3, 3, (e_n * c, 1),
                                                                        generator=gen))

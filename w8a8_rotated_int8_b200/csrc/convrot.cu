@@ -447,10 +447,11 @@ int topc_impl(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float
 template <int NJ>
 int launch_combine(const void* z, const float* s_t, const int32_t* slot, int E, int64_t T,
                    int64_t C, int64_t d, void* y, int sms, cudaStream_t st, bool pdl) {
-  // tokens per CTA: a power of two in [1, 32] that leaves about four CTAs per
-  // SM, so every SM streams rows while each CTA's slot tiles stay coalesced
+  // tokens per CTA: a power of two in [1, 32] that leaves about eight CTAs
+  // per SM, so every SM streams rows while each CTA's slot tiles stay
+  // coalesced
   int tpc = 32;
-  while (tpc > 1 && T < (int64_t)tpc * 4 * std::max(sms, 1)) tpc >>= 1;
+  while (tpc > 1 && T < (int64_t)tpc * 8 * std::max(sms, 1)) tpc >>= 1;
   const size_t smem = combine_tokens_smem(E, tpc);
   auto kern = combine_tokens_kernel<NJ>;
   if (smem > 48 * 1024 &&

@@ -419,10 +419,16 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&f)[8]) {
 // expert are contiguous), the picks of all tpc tokens are laid out as one
 // flat list in shared memory (token by token, each in ascending expert
 // order), and every thread streams its 16-byte column vector of the listed
-// rows, eight loads in flight, closing a token's bf16 output when the list
-// moves on to the next token. Tokens without picks get 0.
+// rows, four loads in flight, closing a token's bf16 output when the list
+// moves on to the next token. Tokens without picks get 0. Launched after the
+// down GEMM with programmatic dependent launch, it builds the lists (from
+// slots and scores completed before that chain began) before waiting for the
+// GEMM, so the list building overlaps the GEMM's tail. (Measured on B200:
+// more loads in flight per thread, larger token runs, or a shared-memory
+// ring fed by bulk copies were all slower; the kernel is bound by the
+// latency of its dependent phases, and small runs keep more CTAs resident.)
 constexpr int kCombThreads = 256;
-constexpr int kCombBatch = 8;
+constexpr int kCombBatch = 4;
 
 __device__ __forceinline__ uint4 f32x8_to_bf16x8(const float (&a)[8]) {
   uint32_t o[4];
@@ -448,7 +454,6 @@ __global__ void __launch_bounds__(kCombThreads) combine_tokens_kernel(
     const int32_t* __restrict__ slot, int E, int T, int C, int d, int tpc,
     __nv_bfloat16* __restrict__ y) {
   griddep_launch_dependents();
-  griddep_wait();
   extern __shared__ __align__(16) uint8_t cm_smem[];
   const int ld = tpc + 1;
   int32_t* sl = reinterpret_cast<int32_t*>(cm_smem);
@@ -513,6 +518,10 @@ __global__ void __launch_bounds__(kCombThreads) combine_tokens_kernel(
     }
   }
   __syncthreads();
+  // the slots and scores were written by the routing kernels, which the
+  // caller's stream joined (fully) before the chain this kernel ends began;
+  // the rows z are the output of its immediate predecessor
+  griddep_wait();
   // 4. stream the rows
   const int n_total = start[tpc];
   const int n_tok = min(tpc, T - t0);
