@@ -67,12 +67,18 @@ def test_rotquant_bf16_bit_exact(rows, k, g):
 
 
 @pytest.mark.parametrize("rows,k,g", [(160, 320, 64), (513, 1536, 64), (64, 2048, 256),
-                                      (9001, 1536, 64)])
+                                      (9001, 1536, 64), (3, 192, 64), (11, 8192 - 64, 64)])
 def test_rotquant_f32_bit_exact(rows, k, g):
+    """fp32 rows (the SwiGLU output); K = 320, 1536, 192, 8128 have group
+    counts that are not powers of two (one thread per group); the first row
+    is zero and the second below the 2^-120 threshold."""
     gen = torch.Generator().manual_seed(k)
     a = torch.randn(rows, k, generator=gen)
     b = torch.randn(rows, k, generator=gen)
     h = (torch.nn.functional.silu(a) * b).float()  # SwiGLU-shaped fp32 rows
+    h[0] = 0.0
+    if rows > 1:
+        h[1] = h[1] * 1e-38
     q, s = W.convrot_rotquant(h.cuda(), g)
     q_ref, s_ref = O.rotquant(h.numpy(), g)
     assert np.array_equal(s.cpu().numpy(), s_ref)
