@@ -6,13 +6,14 @@ rotate+requantise, down GEMM to bf16, router-weighted combine) over one
 batch of synthetic tokens, through the C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config moe_T8192]
-                    [--impl ours|reference] [--no-cpu-baseline]
+                    [--impl ours|reference] [--no-cpu-baseline] [--ablation]
 
 Multi-GPU (launched by torch.distributed.run): every rank runs its own batch
 of T tokens against the same weights (weak scaling, no data-path
 collective); the barrier and the max-over-ranks timing use the process group.
 `--impl reference` times the CPU oracle (the only reference there is) on a
-bounded sample of the same workload.
+bounded sample of the same workload. `--ablation` measures, instead of
+throughput, the block's error with ConvRot and with the rotation off.
 """
 
 from __future__ import annotations
@@ -489,6 +490,60 @@ def run_ours(args, cfg, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_ablation(args, cfg):
+    """Rotation-off ablation on the block (g_gu = g_d = 1: per-token and
+    per-channel INT8 with no Hadamard, the same kernels) against ConvRot
+    (the config's groups): the relative error of each block output against an
+    unquantised fp32 evaluation of the same routed experts (bf16 inputs and
+    weights, torch matmuls), on a sample of tokens. Prints one JSON line."""
+    import w8a8_rotated_int8_b200 as W
+    W.load_library()
+    dev = torch.device("cuda", 0)
+    inp = moe_inputs(cfg)
+    x = inp["x"].to(dev)
+    logits = inp["logits"].to(dev)
+    wgu = inp["wgu"].to(dev)
+    wd = inp["wd"].to(dev)
+    ws = torch.empty(W.moe_workspace_size(cfg.t, cfg.d, cfg.f, cfg.n_exp, cfg.c), dtype=torch.uint8,
+                     device=dev)
+    gen = torch.Generator().manual_seed(7)
+    sample = torch.randperm(cfg.t, generator=gen)[:256].sort().values.to(dev)
+    result = {}
+    ref = None
+    for name, g_gu, g_d in (("convrot", cfg.g_gu, cfg.g_d), ("rotation_off", 1, 1)):
+        gu, dn = W.quantize_moe_weights(wgu, wd, g_gu, g_d)
+        y = W.moe_expert_choice_forward(x, logits, gu, dn, cfg.c, g_gu, g_d, workspace=ws)
+        torch.cuda.synchronize()
+        v = W.moe_stage_views(ws, cfg.t, cfg.d, cfg.f, cfg.n_exp, cfg.c)
+        if ref is None:  # routing does not depend on the groups
+            ref = torch.zeros(cfg.t, cfg.d, dtype=torch.float32, device=dev)
+            idx = v["idx"].long()
+            s_t = v["s_t"]
+            keep = torch.zeros(cfg.t, dtype=torch.bool, device=dev)
+            keep[sample] = True
+            for e in range(cfg.n_exp):
+                rows = idx[e][keep[idx[e]]]
+                if rows.numel() == 0:
+                    continue
+                xe = x[rows].float()
+                gu_out = xe @ wgu[e].float().t()
+                h = torch.nn.functional.silu(gu_out[:, :cfg.f]) * gu_out[:, cfg.f:]
+                ref[rows] += s_t[e, rows][:, None] * (h @ wd[e].float().t())
+        ys, rs = y[sample].float(), ref[sample]
+        result[name] = {
+            "g_gu": g_gu, "g_d": g_d,
+            "max_rel": float((ys - rs).abs().max() / rs.abs().max()),
+            "rel_fro": float(torch.linalg.norm(ys - rs) / torch.linalg.norm(rs)),
+        }
+        del gu, dn
+    line = {"metric": "W8A8 MoE block relative error vs an unquantised fp32 evaluation "
+                      "(rotation-off ablation)",
+            "config": {"workload": cfg.name, "tokens_sampled": int(sample.numel())},
+            "data": "synthetic (seeded; 1% of the activation channels x20 as outliers)",
+            **result}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -497,12 +552,17 @@ def main():
     ap.add_argument("--config", default="moe_T8192", choices=sorted(MOE_CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--ablation", action="store_true",
+                    help="rotation-off ablation: block error with and without ConvRot")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = MOE_CONFIGS[args.config]
+    if args.ablation:
+        run_ablation(args, cfg)
+        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

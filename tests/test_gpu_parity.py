@@ -345,6 +345,39 @@ def test_w8a8_linear_bit_exact(name):
     assert np.array_equal(np32(y), y_ref)
 
 
+@pytest.mark.parametrize("g", [1, 16, 256])
+def test_linear_rotation_off_ablation(g):
+    """The rotation-off ablation (g = 1: per-token / per-channel INT8 with no
+    Hadamard) runs through the same kernels, bit-exact with the oracle; on the
+    outlier-laden gate|up inputs the rotation lowers the error against the
+    exact product (the reason for ConvRot)."""
+    x, w = linear_inputs(LINEAR_CONFIGS["gateup_4096x3072x2048"])
+    x, w = x[:256], w[:512]
+    w_q, s_w = W.convrot_quantize_weights(w.cuda(), g)
+    y = np32(W.w8a8_convrot_linear(x.cuda(), w_q, s_w, g))
+    w_q_ref, s_w_ref = O.rotquant(np32(w), g)
+    assert np.array_equal(y, O.w8a8_linear(np32(x), w_q_ref, s_w_ref, g))
+    exact = np32(x).astype(np.float64) @ np32(w).astype(np.float64).T
+    rel = np.linalg.norm(y - exact) / np.linalg.norm(exact)
+    assert rel < {1: 0.06, 16: 0.02, 256: 0.014}[g]
+    if g == 1:
+        assert rel > 0.03  # without rotation the outlier channels cost accuracy
+
+
+def test_moe_block_rotation_off():
+    """The whole block with g_gu = g_d = 1 (rotation off) against the oracle."""
+    base = MOE_CONFIGS["moe_small"]
+    cfg = base.__class__(**{**base.__dict__, "g_gu": 1, "g_d": 1})
+    inp = moe_inputs(cfg)
+    y, v, _ = _run_moe(inp, cfg)
+    ow = _oracle_weights(inp, cfg, range(cfg.n_exp))
+    y_ref, it = O.moe_block(np32(inp["x"]), np32(inp["logits"]), *ow, c=cfg.c, g_gu=1, g_d=1,
+                            keep=True)
+    assert np.array_equal(v["x_q"].cpu().numpy(), it["x_q"])
+    assert np.array_equal(v["idx"].cpu().numpy(), it["idx"])
+    assert _max_rel(np32(y), y_ref) <= 1e-2
+
+
 def test_linear_empty_batch():
     w = torch.randn(32, 256).to(torch.bfloat16).cuda()
     w_q, s_w = W.convrot_quantize_weights(w, 256)
