@@ -39,8 +39,8 @@ METRIC = "W8A8 ConvRot MoE block tokens/s"
 # summarised in profiles/block_kernels_moe_T8192.md and
 # profiles/gemm_s8_tcgen05_moe_T2048.md; to be dropped whenever that kernel
 # changes
-DOMINANT_TRAFFIC_BYTES = {"moe_T8192": 437.105664e6 + 50.836992e6,
-                          "moe_T2048": 411.88864e6 + 8.630016e6}
+DOMINANT_TRAFFIC_BYTES = {"moe_T8192": 437.1e6 + 50.5e6,
+                          "moe_T2048": 411.9e6 + 6.8e6}
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 
