@@ -12,18 +12,20 @@ namespace convrot {
 // ---------------------------------------------------------------- softmax --
 // Per-token softmax of the router logits over E experts, evaluated in fp64 and
 // rounded once to fp32, written transposed (S_t[e, t]) so each expert's
-// scores are contiguous for the top-C selection. 32 tokens per CTA (one per
-// warp, NJ = ceil(E / 32) experts per lane, so no lane evaluates an exp for
-// an expert that does not exist); the [E, 32] tile goes through shared memory
-// so the transposed store writes 128-byte rows.
-constexpr int kSmTokens = 32;
+// scores are contiguous for the top-C selection. kSmTokens tokens per CTA
+// (one per warp, NJ = ceil(E / 32) experts per lane, so no lane evaluates an
+// exp for an expert that does not exist); the [E, kSmTokens] tile goes
+// through shared memory so the transposed store writes whole 32-byte
+// sectors. Eight tokens per CTA spread even T = 2048 over every SM (measured
+// faster than 32 tokens per CTA at T = 2048 and 8192).
+constexpr int kSmTokens = 8;
 
 template <int NJ>
 __global__ void __launch_bounds__(1024) router_softmax_kernel(
     const __nv_bfloat16* __restrict__ logits, int T, int E, float* __restrict__ S_t) {
   griddep_launch_dependents();
   griddep_wait();
-  extern __shared__ float sm_tile[];  // [E][32]
+  extern __shared__ float sm_tile[];  // [E][kSmTokens]
   const int t0 = blockIdx.x * kSmTokens;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned short* lg = reinterpret_cast<const unsigned short*>(logits);
