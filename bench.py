@@ -1,9 +1,9 @@
 """Benchmark of the W8A8 ConvRot expert-choice MoE block on B200.
 
 One step = one pass of the whole hot path (router softmax, activation
-rotate+quantise, expert-choice top-C, gather, gate/up GEMM + SwiGLU, h
-rotate+requantise, down GEMM to bf16, router-weighted combine) over one
-batch of synthetic tokens, through the C ABI.
+rotate+quantise, expert-choice top-C, gather, gate/up GEMM + SwiGLU with the
+h rotate+requantise in its epilogue, down GEMM to bf16, router-weighted
+combine) over one batch of synthetic tokens, through the C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config moe_T8192]
                     [--impl ours|reference] [--no-cpu-baseline] [--ablation]
@@ -35,12 +35,10 @@ from synthetic import MOE_CONFIGS, moe_inputs  # noqa: E402
 
 METRIC = "W8A8 ConvRot MoE block tokens/s"
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
-# kernel (the gate/up GEMM with the SwiGLU epilogue), from the ncu captures
-# summarised in profiles/block_kernels_moe_T8192.md and
-# profiles/gemm_s8_tcgen05_moe_T2048.md; to be dropped whenever that kernel
+# kernel (the gate/up GEMM with the requantising SwiGLU epilogue), from the
+# ncu captures summarised in profiles/; to be dropped whenever that kernel
 # changes
-DOMINANT_TRAFFIC_BYTES = {"moe_T8192": 437.1e6 + 50.5e6,
-                          "moe_T2048": 411.9e6 + 6.8e6}
+DOMINANT_TRAFFIC_BYTES = {}
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 
@@ -69,12 +67,24 @@ def algorithmic_work(cfg, t):
         # weights + their scales + gathered codes and scales in + h (fp32) out
         "bytes": e * 2 * f * d + e * 2 * f * 4 + e * c * (d + 4) + e * c * f * 4,
     }
+    gateup_rq = {
+        "ops": 2 * e * c * d * 2 * f,
+        # the same inputs; out: h codes and their scales (h stays on chip)
+        "bytes": e * 2 * f * d + e * 2 * f * 4 + e * c * (d + 4) + e * c * (f + 4),
+    }
     down = {
         "ops": 2 * e * c * f * d,
         # weights + scales + h codes and scales in + bf16 rows out
         "bytes": e * d * f + e * d * 4 + e * c * (f + 4) + e * c * d * 2,
     }
-    return {"ops": ops, "block_bytes": block_bytes, "gateup": gateup, "down": down}
+    return {"ops": ops, "block_bytes": block_bytes, "gateup": gateup, "gateup_rq": gateup_rq,
+            "down": down}
+
+
+def fused_h(cfg):
+    """Whether the block requantises h in the gate/up GEMM's epilogue (the
+    library does for g_d <= 64 on a full B200)."""
+    return cfg.g_d <= 64
 
 
 class ClockSampler:
@@ -310,6 +320,8 @@ def stage_times(W, ws_views, inp_dev, wq, cfg, t, reps, flush_buf):
     wgu_q, s_gu, wd_q, s_d = gu.data, gu.scale, dn.data, dn.scale
     tiles = W.binding.LAYOUT_TILES
     stream = torch.cuda.current_stream()
+    sync = torch.empty(W.binding.lib().convrot_swiglu_rq_sync_bytes(cfg.n_exp, cfg.c),
+                       dtype=torch.uint8, device=flush_buf.w.device)
     stages = {
         "router_softmax": lambda: W.binding.lib().convrot_router_softmax(
             W.binding._p(inp_dev["logits"]), t, cfg.n_exp, W.binding._p(v["s_t"]),
@@ -328,6 +340,12 @@ def stage_times(W, ws_views, inp_dev, wq, cfg, t, reps, flush_buf):
             W.binding._stream()),
         "rotquant_h": lambda: W.convrot_rotquant(v["h"].view(-1, cfg.f), cfg.g_d,
                                                  q=v["h_q"].view(-1, cfg.f), scale=v["s_h"].view(-1)),
+        # (the entry clears its 0.1 MB synchronisation scratch first, inside the events)
+        "gemm_gateup_swiglu_rq": lambda: W.binding.lib().convrot_i8_gemm_swiglu_rq(
+            W.binding._p(v["x_g"]), W.binding._p(v["s_g"]), W.binding._p(wgu_q),
+            W.binding._p(s_gu), tiles, cfg.n_exp, cfg.c, cfg.f, cfg.d, cfg.g_d,
+            W.binding._p(v["h_q"]), W.binding._p(v["s_h"]), W.binding._p(sync), sync.numel(),
+            W.binding._stream()),
         "gemm_down_bf16": lambda: W.binding.lib().convrot_i8_gemm_bf16(
             W.binding._p(v["h_q"]), W.binding._p(v["s_h"]), W.binding._p(wd_q),
             W.binding._p(s_d), tiles, cfg.n_exp, cfg.c, cfg.d, cfg.f,
@@ -336,6 +354,10 @@ def stage_times(W, ws_views, inp_dev, wq, cfg, t, reps, flush_buf):
             W.binding._p(v["z"]), W.binding._p(v["s_t"]), W.binding._p(v["slot"]), cfg.n_exp, t,
             cfg.c, cfg.d, W.binding._p(inp_dev["y"]), W.binding._stream()),
     }
+    # the stages one block call runs
+    for name in (("gemm_gateup_swiglu", "rotquant_h") if fused_h(cfg)
+                 else ("gemm_gateup_swiglu_rq",)):
+        del stages[name]
     out = {}
     for name, fn in stages.items():
         ts = []
@@ -440,8 +462,10 @@ def run_ours(args, cfg, world, rank, local):
         return
     peaks = load_peaks()
     work = algorithmic_work(cfg, t)
-    dom = max(("gemm_gateup_swiglu", "gemm_down_bf16"), key=lambda k: st[k])
-    dk = work["gateup"] if dom == "gemm_gateup_swiglu" else work["down"]
+    gateup_stage = "gemm_gateup_swiglu_rq" if fused_h(cfg) else "gemm_gateup_swiglu"
+    dom = max((gateup_stage, "gemm_down_bf16"), key=lambda k: st[k])
+    dk = {"gemm_gateup_swiglu_rq": work["gateup_rq"], "gemm_gateup_swiglu": work["gateup"],
+          "gemm_down_bf16": work["down"]}[dom]
     int8_peak_tops = 2.0 * peaks["bf16_tflops"]  # int8 dense = 2x bf16 dense (nominal ratio)
     t_hbm = dk["bytes"] / (peaks["hbm_gbs"] * 1e9)
     t_tc = dk["ops"] / (int8_peak_tops * 1e12)
@@ -462,8 +486,8 @@ def run_ours(args, cfg, world, rank, local):
                        work["ops"] / (int8_peak_tops * 1e12))
 
     value = job_throughput(t, world, mean_step)
-    # softmax, rotation, top-C, [gather, GEMM, rotation, GEMM], combine
-    launches_per_step = 8 if cfg.c > 0 else 4
+    # softmax, rotation, top-C, [gather, GEMM, (h rotation,) GEMM], combine
+    launches_per_step = (7 if fused_h(cfg) else 8) if cfg.c > 0 else 4
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": mean_step * 1e3, "higher_is_better": True,

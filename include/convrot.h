@@ -195,6 +195,30 @@ int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, c
                            int b_layout, int64_t G, int64_t M, int64_t F, int64_t K, float* h,
                            void* stream);
 
+/* SwiGLU followed by the rotation and requantisation of h, all in the GEMM's
+ * epilogue, so h is never stored ("Nucleus-Image INT8 Convrot Experts + FP8
+ * Text Encoder", section "Quantization": the down projection's input is
+ * rotated in groups of 64 and quantised per row):
+ *   h[g, m, :] as convrot_i8_gemm_swiglu computes it, then per row the same
+ *   rotation (group g_h in {1, 4, 16, 64}, F % g_h == 0) and quantiser as
+ *   convrot_rotquant: h_q device [G, M, F] int8 codes, s_h device [G, M] fp32.
+ *   The results equal convrot_i8_gemm_swiglu followed by convrot_rotquant
+ *   (CONVROT_DTYPE_F32, group g_h) bit for bit.
+ *   sync    device scratch of at least convrot_swiglu_rq_sync_bytes(G, M)
+ *           bytes (the rows' running maxima and the tiles' arrival counters);
+ *           the call clears it on `stream` before the GEMM, so calls sharing
+ *           one scratch must be ordered on one stream.
+ * The tiles of a row wait for one another (bounded; a wait that runs out sets
+ * the device error flag and the call's results are invalid). Returns
+ * CONVROT_ERR_INVALID_ARG when the device cannot keep enough of the GEMM's
+ * CTAs resident at once for that (ceil(F / 128) of them, or CTA pairs for
+ * M > 128); convrot_i8_gemm_swiglu + convrot_rotquant then do the same work. */
+size_t convrot_swiglu_rq_sync_bytes(int64_t G, int64_t M);
+int convrot_i8_gemm_swiglu_rq(const int8_t* a, const float* s_a, const int8_t* b,
+                              const float* s_b, int b_layout, int64_t G, int64_t M, int64_t F,
+                              int64_t K, int g_h, int8_t* h_q, float* s_h, void* sync,
+                              size_t sync_bytes, void* stream);
+
 /* Router-weighted scatter epilogue:
  * out32[idx[g, m], n] += w[g, m] * (fp32(acc) * (s_b[g, n] * s_a[g, m])).
  * out32 device [T, N] fp32 (accumulated with fp32 atomics, order not fixed);
@@ -268,6 +292,10 @@ int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const 
  *   f % g_d == 0, 16 <= f <= 8192; 1 <= E <= 256.
  * The workspace holds every intermediate; its layout is reported by
  * moe_workspace_layout so a caller can inspect each stage after the call.
+ * With g_d <= 64 (and a device that keeps enough of the gate/up GEMM's CTAs
+ * resident, as convrot_i8_gemm_swiglu_rq needs) h is rotated and requantised
+ * in the gate/up GEMM's epilogue and the fp32 h region is left untouched;
+ * with g_d = 256 h is stored in fp32 and rotated by a separate kernel.
  * Inside the call the routing (softmax, top-C) runs on a second stream the
  * library keeps per device, forked from and joined back to `stream` with
  * events, so it overlaps the activation rotation; the call as a whole is
@@ -281,9 +309,11 @@ typedef struct {
   size_t w;        /* [E, C] fp32     router weights of the choices */
   size_t x_g;      /* [E, C, d] int8  gathered codes                */
   size_t s_g;      /* [E, C] fp32     gathered scales               */
-  size_t h;        /* [E, C, f] fp32  silu(gate) * up               */
+  size_t h;        /* [E, C, f] fp32  silu(gate) * up (g_d = 256 only) */
   size_t h_q;      /* [E, C, f] int8  rotated, requantised h        */
   size_t s_h;      /* [E, C] fp32     scales of h                   */
+  size_t hsync;    /* convrot_swiglu_rq_sync_bytes(E, C) bytes: scratch of
+                      the fused requantisation                      */
   size_t slot;     /* [E, T] int32    slot of each token per expert */
   size_t z;        /* [E, C, d] bf16  expert outputs (down projection) */
   size_t total;    /* bytes required                                */

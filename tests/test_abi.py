@@ -42,7 +42,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_strings(lib):
-    assert lib.convrot_abi_version() == 1
+    assert lib.convrot_abi_version() == 2
     for code in range(7):
         assert binding.status_string(code)
     assert binding.status_string(99) == "unknown status"

@@ -263,6 +263,56 @@ def test_gemm_swiglu(g, m, f, k, layout):
         assert (ulps == 0).mean() > 0.8  # expf differs from exp in ~1 of 10 elements
 
 
+# The requantising SwiGLU epilogue: h rotated and quantised per row inside the
+# GEMM. Shapes cover the single-CTA and the CTA-pair kernels, a last tile with
+# one half of its h columns (F % 128 = 64) or a part of one (F % 64 = 16),
+# a pair m-block whose second slab holds no row, more tiles than resident
+# CTAs (row blocks spread over two tiles of one CTA's loop) and every group.
+@pytest.mark.parametrize("layout", ["rows", "tiles"])
+@pytest.mark.parametrize("g,m,f,k,g_h", [
+    (2, 160, 320, 768, 64), (1, 64, 1536, 2048, 64), (3, 40, 192, 512, 16),
+    (2, 300, 256, 256, 4), (5, 100, 208, 256, 16), (40, 64, 512, 256, 64),
+    (3, 130, 64, 128, 1), (24, 256, 1536, 256, 64),
+])
+def test_gemm_swiglu_rq_matches_two_step(g, m, f, k, g_h, layout):
+    """Codes and scales equal the SwiGLU GEMM followed by the rotation kernel
+    bit for bit, and the oracle's rotation + quantiser of that same h."""
+    a = _codes((g, m, k), 7 + m)
+    b = _codes((g, 2 * f, k), 8 + f)
+    s_a = (torch.rand(g, m) * 0.05 + 1e-3).cuda()
+    s_b = (torch.rand(g, 2 * f) * 1e-4 + 1e-6).cuda()
+    bb = b.cuda() if layout == "rows" else _tiled_codes(b.view(2 * g, f, k))
+    s_a[0, 3] = 0.0  # an all-zero row of h: scale 0, codes 0
+    h = W.convrot_i8_gemm_swiglu(a.cuda(), s_a, bb, s_b)
+    q2, s2 = W.convrot_rotquant(h.view(-1, f), g_h)
+    q1, s1 = W.convrot_i8_gemm_swiglu_rq(a.cuda(), s_a, bb, s_b, g_h)
+    assert torch.equal(q1.view(-1, f), q2)
+    assert torch.equal(s1.view(-1), s2)
+    assert float(s1[0, 3]) == 0.0 and int(q1[0, 3].abs().sum()) == 0
+    q_ref, s_ref = O.rotquant(h.view(-1, f).cpu().numpy(), g_h)
+    assert np.array_equal(q1.view(-1, f).cpu().numpy(), q_ref)
+    assert np.array_equal(s1.view(-1).cpu().numpy(), s_ref)
+
+
+def test_gemm_swiglu_rq_repeated_calls_reuse_nothing():
+    """Back-to-back calls on one stream (each clears its own scratch) give the
+    same codes; a different input right after gives its own."""
+    g, m, f, k = 6, 200, 384, 512
+    a = _codes((g, m, k), 21).cuda()
+    b = _codes((g, 2 * f, k), 22)
+    bb = _tiled_codes(b.view(2 * g, f, k))
+    s_a = (torch.rand(g, m) * 0.05 + 1e-3).cuda()
+    s_b = (torch.rand(g, 2 * f) * 1e-4 + 1e-6).cuda()
+    first = W.convrot_i8_gemm_swiglu_rq(a, s_a, bb, s_b, 64)
+    for _ in range(3):
+        again = W.convrot_i8_gemm_swiglu_rq(a, s_a, bb, s_b, 64)
+        assert torch.equal(again[0], first[0]) and torch.equal(again[1], first[1])
+    other = W.convrot_i8_gemm_swiglu_rq(a, s_a * 2, bb, s_b, 64)
+    h = W.convrot_i8_gemm_swiglu(a, s_a * 2, bb, s_b)
+    q2, s2 = W.convrot_rotquant(h.view(-1, f), 64)
+    assert torch.equal(other[0].view(-1, f), q2) and torch.equal(other[1].view(-1), s2)
+
+
 @pytest.mark.parametrize("layout", ["rows", "tiles"])
 def test_gemm_scatter(layout):
     g, m, n, k, t = 4, 100, 320, 512, 150
@@ -422,9 +472,21 @@ def _max_rel(y, ref):
     return float(np.max(np.abs(y - ref)) / max(np.max(np.abs(ref)), 1e-30))
 
 
-@pytest.mark.parametrize("name", ["moe_small", "moe_small_c40"])
+# g_d = 256 takes the fp32 h + rotation-kernel path (a group of 256 spans
+# four epilogue threads); g_d <= 64 rotates and requantises h in the gate/up
+# GEMM's epilogue and stores no fp32 h.
+_MOE_EXTRA = {
+    "moe_small_gd256": MOE_CONFIGS["moe_small_c40"].__class__(
+        "moe_small_gd256", 300, 512, 5, 256, 40, 13, g_gu=256, g_d=256),
+    "moe_small_gd16": MOE_CONFIGS["moe_small"].__class__(
+        "moe_small_gd16", 640, 768, 6, 320, 160, 14, g_gu=64, g_d=16),
+}
+
+
+@pytest.mark.parametrize("name", ["moe_small", "moe_small_c40", "moe_small_gd256",
+                                  "moe_small_gd16"])
 def test_moe_block_small_end_to_end(name):
-    cfg = MOE_CONFIGS[name]
+    cfg = MOE_CONFIGS[name] if name in MOE_CONFIGS else _MOE_EXTRA[name]
     inp = moe_inputs(cfg)
     y, v, wq = _run_moe(inp, cfg)
     ow = _oracle_weights(inp, cfg, range(cfg.n_exp))
@@ -441,7 +503,8 @@ def test_moe_block_small_end_to_end(name):
     h_q_diff = 0
     n_codes = 0
     for e in range(cfg.n_exp):
-        assert _fp32_ulps(v["h"][e].cpu().numpy(), it["h"][e]).max() <= 4
+        if cfg.g_d == 256:
+            assert _fp32_ulps(v["h"][e].cpu().numpy(), it["h"][e]).max() <= 4
         dq = np.abs(v["h_q"][e].cpu().numpy().astype(np.int32) - it["h_q"][e].astype(np.int32))
         assert dq.max() <= 1
         h_q_diff += int((dq != 0).sum())

@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     convrot_i8_gemm_i32,
     convrot_i8_gemm_scatter,
     convrot_i8_gemm_swiglu,
+    convrot_i8_gemm_swiglu_rq,
     convrot_linear_workspace_size,
     convrot_quantize_weights,
     convrot_quantize_weights_tiled,

@@ -39,8 +39,8 @@ class ConvrotError(RuntimeError):
 
 class MoeLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
-                ("x_q", "s_x", "s_t", "idx", "w", "x_g", "s_g", "h", "h_q", "s_h", "slot", "z",
-                 "total")]
+                ("x_q", "s_x", "s_t", "idx", "w", "x_g", "s_g", "h", "h_q", "s_h", "hsync", "slot",
+                 "z", "total")]
 
 
 _lib = None
@@ -68,6 +68,9 @@ _SIGNATURES = {
     "convrot_i8_gemm_i32": (_I, [_P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
     "convrot_i8_gemm_bf16": (_I, [_P, _P, _P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
     "convrot_i8_gemm_swiglu": (_I, [_P, _P, _P, _P, _I, _I64, _I64, _I64, _I64, _P, _P]),
+    "convrot_swiglu_rq_sync_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "convrot_i8_gemm_swiglu_rq": (_I, [_P, _P, _P, _P, _I, _I64, _I64, _I64, _I64, _I, _P, _P,
+                                       _P, ctypes.c_size_t, _P]),
     "convrot_i8_gemm_scatter": (_I, [_P, _P, _P, _P, _I, _P, _P, _I64, _I64, _I64, _I64, _P, _I64,
                                      _P]),
     "convrot_f32_to_bf16": (_I, [_P, _I64, _P, _P]),
@@ -318,6 +321,23 @@ def convrot_i8_gemm_swiglu(a, s_a, b, s_b, stream=None):
     _check(lib().convrot_i8_gemm_swiglu(_p(a), _p(s_a), _p(bt), _p(s_b), lay, g, m, f, k, _p(h),
                                         _stream(stream)), "convrot_i8_gemm_swiglu")
     return h if a.dim() == 3 else h[0]
+
+
+def convrot_i8_gemm_swiglu_rq(a, s_a, b, s_b, g_h=64, stream=None):
+    """SwiGLU, then h rotated in groups of g_h and requantised per row, all in
+    the GEMM epilogue -> (h_q [G, M, F] int8, s_h [G, M] fp32)."""
+    g, m, n2, k, bt, lay = _gemm_dims(a, b, swiglu=True)
+    _need(s_a, torch.float32, "s_a")
+    _need(s_b, torch.float32, "s_b")
+    f = n2 // 2
+    h_q = torch.empty((g, m, f), dtype=torch.int8, device=a.device)
+    s_h = torch.empty((g, m), dtype=torch.float32, device=a.device)
+    nbytes = lib().convrot_swiglu_rq_sync_bytes(g, m)
+    sync = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=a.device)
+    _check(lib().convrot_i8_gemm_swiglu_rq(_p(a), _p(s_a), _p(bt), _p(s_b), lay, g, m, f, k, g_h,
+                                           _p(h_q), _p(s_h), _p(sync), nbytes, _stream(stream)),
+           "convrot_i8_gemm_swiglu_rq")
+    return (h_q, s_h) if a.dim() == 3 else (h_q[0], s_h[0])
 
 
 def convrot_i8_gemm_scatter(a, s_a, b, s_b, idx, w, out32, stream=None):

@@ -25,6 +25,7 @@ enum DeviceErrorBits : unsigned {
   kErrSelfTest = 1u << 5,         // the wait self-test ran out (expected)
   kErrBadIndex = 1u << 6,         // a row index was out of range; the access was skipped
   kErrTimeoutStream = 1u << 7,    // a streaming kernel waited too long for a TMA copy
+  kErrTimeoutRowSync = 1u << 8,   // a GEMM tile waited too long for the other tiles of its rows
 };
 
 __device__ unsigned int g_device_error = 0;
@@ -112,6 +113,36 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint6
     }
   }
   return true;
+}
+
+// Waits until *count >= target (a counter other CTAs of the same grid raise),
+// bounded like mbar_wait. `grid_abort` is a word of the same launch that a
+// CTA which gave up sets, so the others stop waiting for it at once. On
+// giving up the CTA's abort flag is raised too. Returns false then.
+__device__ __forceinline__ bool wait_count_geq(const int* count, int target, int* grid_abort,
+                                               volatile int* abort_flag, unsigned err_bit) {
+  const uint64_t t0 = global_timer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(count) : "memory");
+    if (v >= target) return true;
+    if ((++spins & 15u) == 0) {
+      int ab;
+      asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(ab) : "l"(grid_abort) : "memory");
+      if (ab != 0 || *abort_flag) {
+        *abort_flag = 1;
+        return false;
+      }
+      if (global_timer_ns() - t0 > g_wait_limit_ns) {
+        atomicOr(&g_device_error, err_bit);
+        atomicExch(grid_abort, 1);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+    __nanosleep(64);
+  }
 }
 
 // ------------------------------------------- programmatic dependent launch --

@@ -26,6 +26,11 @@ struct DeviceInfo {
   bool ready = false;
   bool supported = false;
   int sm_count = 0;
+  // how many CTAs (single-CTA kernel) and CTA pairs (pair kernel) of the
+  // requantising SwiGLU GEMM can be resident at once: its grid never exceeds
+  // them, since its tiles wait for one another
+  int rq_ctas = 0;
+  int rq_pairs = 0;
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -102,6 +107,35 @@ void set_gemm_attrs() {
   set_gemm_attr<kEpiBf16, BT>();
   set_gemm_attr<kEpiSwiglu, BT>();
   set_gemm_attr<kEpiScatter, BT>();
+  set_gemm_attr<kEpiSwigluRq, BT>();
+}
+
+// Co-resident CTAs / CTA pairs of the requantising SwiGLU GEMM on this device.
+int swiglu_rq_residency(int sms, int* ctas, int* pairs) {
+  using Cfg = EpiCfg<kEpiSwigluRq>;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+          &per_sm, gemm_s8_tcgen05_kernel<kEpiSwigluRq, true>, Cfg::kThreads, Cfg::kSmem1) !=
+      cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  *ctas = per_sm * sms;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(2 * (unsigned)(sms / 2));
+  lc.blockDim = dim3(Cfg::kThreads);
+  lc.dynamicSmemBytes = Cfg::kSmem2;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  lc.attrs = &attr;
+  lc.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, gemm_s8_tcgen05_pair_kernel<kEpiSwigluRq, true>,
+                                     &lc) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  *pairs = clusters;
+  return CONVROT_OK;
 }
 
 // Per-device one-time setup: capability check, SM count, kernel attributes.
@@ -128,12 +162,25 @@ int device_setup(int* sm_count) {
       set_gemm_attrs<false>();
       set_gemm_attrs<true>();
       if (cudaGetLastError() != cudaSuccess) return CONVROT_ERR_CUDA;
+      if (swiglu_rq_residency(sms, &d.rq_ctas, &d.rq_pairs) != CONVROT_OK) {
+        cudaGetLastError();
+        return CONVROT_ERR_CUDA;
+      }
     }
     d.ready = true;
   }
   if (!d.supported) return CONVROT_ERR_UNSUPPORTED_DEVICE;
   if (sm_count) *sm_count = d.sm_count;
   return CONVROT_OK;
+}
+
+// Co-resident CTAs (pairs = false) or CTA pairs of the requantising SwiGLU
+// GEMM on the current device; 0 before device_setup.
+int swiglu_rq_capacity(bool pairs) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  return pairs ? g_dev[dev].rq_pairs : g_dev[dev].rq_ctas;
 }
 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -346,6 +393,37 @@ int encode_tiled_b(CUtensorMap* map, const void* base, uint64_t kb_count, uint64
   return r == CUDA_SUCCESS ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
+// Units (CTAs, or CTA pairs) the requantising SwiGLU GEMM runs `tiles` tiles
+// on, n_blocks of them per row block; 0 when the device cannot keep enough of
+// them resident for the tiles of a row block to meet.
+int64_t swiglu_rq_units(int64_t tiles, int64_t n_blocks, bool pairs, int sms) {
+  int64_t cap = std::min<int64_t>(pairs ? sms / 2 : sms, swiglu_rq_capacity(pairs));
+  if (tiles <= cap) return tiles;
+  if (cap < n_blocks) return 0;
+  // a whole number of row blocks per wave: the tiles of a row block then run
+  // side by side instead of one wave apart
+  return cap / n_blocks * n_blocks;
+}
+
+// Whether the gate/up GEMM over G groups of M rows (tiled weights, F h
+// columns) can requantise h in its epilogue on this device.
+bool swiglu_rq_fits(int64_t G, int64_t M, int64_t F, int sms) {
+  const bool pairs = M > gemm::BM && sms >= 2;
+  const int64_t n_blocks = cdiv(F, gemm::BN / 2);
+  const int64_t tiles = G * cdiv(M, pairs ? gemm2::BM : gemm::BM) * n_blocks;
+  return swiglu_rq_units(tiles, n_blocks, pairs, sms) > 0;
+}
+
+// Bytes of the fused h requantisation's synchronisation scratch for G groups
+// of M rows: the row maxima [G*M] (fp32 bits), then at a 256-byte boundary
+// the tile arrivals of every 128-row slab [G*(ceil(M/128)+1)] and one abort
+// word. All zero before the GEMM starts.
+size_t swiglu_rq_sync_bytes(int64_t G, int64_t M) {
+  const size_t rows = (size_t)G * (size_t)M;
+  const size_t counters = (size_t)G * (size_t)(cdiv(M, 128) + 1) + 1;
+  return ((rows * 4 + 255) & ~(size_t)255) + counters * 4;
+}
+
 // NB = rows of one B matrix per group (2F for SwiGLU). With BT the B operand
 // is in the tiled weight format: for SwiGLU each group holds a gate matrix and
 // an up matrix of F rows, each padded to 128-row blocks.
@@ -362,8 +440,8 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
   if ((rc = encode_3d_i8(&ta, a, (uint64_t)K, (uint64_t)M, (uint64_t)G, box_a)) != CONVROT_OK)
     return rc;
   if (BT) {
-    const int64_t blocks = (EPI == kEpiSwiglu) ? cdiv(n_out, 128) : cdiv(NB, 128);
-    const int64_t per_group = (EPI == kEpiSwiglu) ? 2 * blocks : blocks;
+    const int64_t blocks = epi_is_swiglu(EPI) ? cdiv(n_out, 128) : cdiv(NB, 128);
+    const int64_t per_group = epi_is_swiglu(EPI) ? 2 * blocks : blocks;
     args.b_blocks = (int)blocks;
     box_b = 128;
     if ((rc = encode_tiled_b(&tb, b, (uint64_t)cdiv(K, 128), (uint64_t)(G * per_group))) !=
@@ -382,16 +460,27 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
   // CTA pairs (M = 256 tiles) once a group has more than 128 rows and the
   // weight boxes are whole 128-row blocks
   const bool pairs = M > gemm::BM && box_b == 128 && sms >= 2;
+  // The requantising SwiGLU epilogue: tiles n-block fastest, the grid within
+  // what can be resident at once and, when it cannot hold every tile, at
+  // least one row block's n_blocks tiles (its tiles wait for one another).
+  args.nb_fast = EPI == kEpiSwigluRq ? 1 : 0;
+  const int64_t n_tile = epi_is_swiglu(EPI) ? gemm::BN / 2 : gemm::BN;
+  args.n_blocks = (int)cdiv(n_out, n_tile);
+  args.k_blocks = (int)cdiv(K, gemm::BK);
+  auto resident_units = [&](int64_t tiles, int64_t units) -> int64_t {
+    if (EPI != kEpiSwigluRq) return std::min<int64_t>(tiles, units);
+    return swiglu_rq_units(tiles, args.n_blocks, pairs, sms);
+  };
   if (pairs) {
     args.m_blocks = (int)cdiv(M, gemm2::BM);
-    const int64_t n_tile = (EPI == kEpiSwiglu) ? gemm::BN / 2 : gemm::BN;
-    args.n_blocks = (int)cdiv(n_out, n_tile);
-    args.k_blocks = (int)cdiv(K, gemm::BK);
+    args.slabs = 2 * args.m_blocks;
     const int64_t tiles = G * args.m_blocks * args.n_blocks;
     if (tiles >= ((int64_t)1 << 30)) return CONVROT_ERR_INVALID_ARG;
     args.num_tiles = (int)tiles;
     args.box_bytes = 2 * (128 + 128) * gemm::BK;  // both CTAs' A and B boxes
-    const int grid = 2 * (int)std::min<int64_t>(tiles, sms / 2);
+    const int64_t n_pairs = resident_units(tiles, sms / 2);
+    if (n_pairs < 1) return CONVROT_ERR_INVALID_ARG;
+    const int grid = 2 * (int)n_pairs;
     if ((rc = launch_kernel(gemm_s8_tcgen05_pair_kernel<EPI, BT>, dim3(grid),
                             dim3(EpiCfg<EPI>::kThreads), EpiCfg<EPI>::kSmem2, st, pdl, 2, ta, tb,
                             args)) != CONVROT_OK)
@@ -399,14 +488,13 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
     return launch_status();
   }
   args.m_blocks = (int)cdiv(M, gemm::BM);
-  const int64_t n_tile = (EPI == kEpiSwiglu) ? gemm::BN / 2 : gemm::BN;
-  args.n_blocks = (int)cdiv(n_out, n_tile);
-  args.k_blocks = (int)cdiv(K, gemm::BK);
+  args.slabs = args.m_blocks;
   const int64_t tiles = G * args.m_blocks * args.n_blocks;
   if (tiles >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
   args.num_tiles = (int)tiles;
   args.box_bytes = (int)((box_a + 2 * box_b) * gemm::BK);  // A and B boxes of one stage
-  const int grid = (int)std::min<int64_t>(tiles, sms);
+  const int grid = (int)resident_units(tiles, sms);
+  if (grid < 1) return CONVROT_ERR_INVALID_ARG;
   if ((rc = launch_kernel(gemm_s8_tcgen05_kernel<EPI, BT>, dim3(grid), dim3(EpiCfg<EPI>::kThreads),
                           EpiCfg<EPI>::kSmem1, st, pdl, 1, ta, tb, args)) != CONVROT_OK)
     return rc;
@@ -506,11 +594,12 @@ int softmax_impl(const void* logits, int64_t T, int E, float* s_t, cudaStream_t 
 }
 
 int gather_impl(const int8_t* src, const float* s_src, int64_t n_src, const int32_t* idx,
-                int64_t n_rows, int64_t K, int8_t* dst, float* s_dst, cudaStream_t st) {
+                int64_t n_rows, int64_t K, int8_t* dst, float* s_dst, cudaStream_t st,
+                uint32_t* zero = nullptr, int64_t n_zero = 0) {
   if (n_rows == 0) return CONVROT_OK;
   const int64_t grid = (n_rows + 7) / 8;
   gather_rows_kernel<<<(unsigned)grid, 256, 0, st>>>(src, s_src, n_src, idx, n_rows, (int)K, dst,
-                                                      s_dst);
+                                                      s_dst, zero, n_zero);
   return launch_status();
 }
 
@@ -530,7 +619,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // ===================================================================== ABI ==
 extern "C" {
 
-int convrot_abi_version(void) { return 1; }
+int convrot_abi_version(void) { return 2; }
 
 const char* convrot_status_string(int status) {
   switch (status) {
@@ -693,6 +782,42 @@ int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, c
                                         as_stream(stream));
 }
 
+size_t convrot_swiglu_rq_sync_bytes(int64_t G, int64_t M) {
+  if (G < 0 || M < 0) return 0;
+  return swiglu_rq_sync_bytes(G, M);
+}
+
+int convrot_i8_gemm_swiglu_rq(const int8_t* a, const float* s_a, const int8_t* b,
+                              const float* s_b, int b_layout, int64_t G, int64_t M, int64_t F,
+                              int64_t K, int g_h, int8_t* h_q, float* s_h, void* sync,
+                              size_t sync_bytes, void* stream) {
+  if (b_layout != CONVROT_LAYOUT_ROWS && b_layout != CONVROT_LAYOUT_TILES)
+    return CONVROT_ERR_INVALID_ARG;
+  if (F < 0 || F % 16 != 0 || F % g_h != 0) return CONVROT_ERR_INVALID_ARG;
+  if (g_h != 1 && g_h != 4 && g_h != 16 && g_h != 64) return CONVROT_ERR_INVALID_ARG;
+  int rc = check_gemm_shape(a, b, G, M, 2 * F, K);
+  if (rc != CONVROT_OK) return rc;
+  if (G * M * F > 0 && (!s_a || !s_b || !h_q || !s_h || !sync)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(s_a) || !al16(s_b) || !al16(h_q) || !al16(s_h) || !al16(sync))
+    return CONVROT_ERR_MISALIGNED;
+  if (G * M * F == 0) return device_setup(nullptr);
+  if (sync_bytes < swiglu_rq_sync_bytes(G, M)) return CONVROT_ERR_WORKSPACE_TOO_SMALL;
+  if ((rc = device_setup(nullptr)) != CONVROT_OK) return rc;
+  cudaStream_t st = as_stream(stream);
+  if (cudaMemsetAsync(sync, 0, swiglu_rq_sync_bytes(G, M), st) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  GemmArgs args{};
+  args.s_a = s_a;
+  args.s_b = s_b;
+  args.out = h_q;
+  args.g_h = g_h;
+  args.s_h = s_h;
+  args.hmax = reinterpret_cast<unsigned*>(sync);
+  args.rsync = reinterpret_cast<int*>(reinterpret_cast<char*>(sync) +
+                                      (((size_t)G * (size_t)M * 4 + 255) & ~(size_t)255));
+  return launch_gemm_layout<kEpiSwigluRq>(b_layout, a, b, G, M, 2 * F, K, F, args, st);
+}
+
 int convrot_i8_gemm_scatter(const int8_t* a, const float* s_a, const int8_t* b, const float* s_b,
                             int b_layout, const int32_t* idx, const float* w, int64_t G, int64_t M,
                             int64_t N, int64_t K, float* out32, int64_t T, void* stream) {
@@ -775,6 +900,7 @@ int moe_workspace_layout(int64_t T, int64_t d, int64_t f, int E, int64_t C,
   lay->h = take(ec * f * 4);
   lay->h_q = take(ec * f);
   lay->s_h = take(ec * 4);
+  lay->hsync = take(swiglu_rq_sync_bytes(E, C));
   lay->slot = take((size_t)E * T * 4);
   lay->z = take(ec * d * 2);
   lay->total = off;
@@ -849,21 +975,42 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
   if (rc_side != CONVROT_OK) return rc_side;
   if (rc != CONVROT_OK) return rc;
   if (C > 0) {
-    // 4. gather each expert's token codes
-    if ((rc = gather_impl(x_q, s_x, T, idx, (int64_t)E * C, d, x_g, s_g, st)) != CONVROT_OK)
+    // h is rotated and requantised inside the gate/up GEMM's epilogue when its
+    // groups fit one thread (g_d <= 64) and the device holds enough of the
+    // GEMM's CTAs at once; otherwise h goes through HBM in fp32 and the
+    // rotation kernel
+    const bool fused_h = g_d <= 64 && swiglu_rq_fits(E, C, f, sms);
+    char* hsync = ws + lay.hsync;
+    // 4. gather each expert's token codes (and clear the fused epilogue's
+    // synchronisation words)
+    if ((rc = gather_impl(x_q, s_x, T, idx, (int64_t)E * C, d, x_g, s_g, st,
+                          fused_h ? reinterpret_cast<uint32_t*>(hsync) : nullptr,
+                          fused_h ? (int64_t)(swiglu_rq_sync_bytes(E, C) / 4) : 0)) != CONVROT_OK)
       return rc;
-    // 5. gate/up GEMM with dequant + SwiGLU
     GemmArgs a1{};
     a1.s_a = s_g;
     a1.s_b = s_gu;
-    a1.out = h;
-    if ((rc = launch_gemm<kEpiSwiglu, true>(x_g, w_gu, E, C, 2 * f, d, f, a1, st, true)) !=
-        CONVROT_OK)
-      return rc;
-    // 6. rotate (g_d) + requantise h per row
-    if ((rc = rotquant_impl(h, CONVROT_DTYPE_F32, (int64_t)E * C, f, g_d, h_q, s_h, st,
-                            RqOut{0, 1, 1, 1}, true)) != CONVROT_OK)
-      return rc;
+    if (fused_h) {
+      // 5 + 6. gate/up GEMM: dequant, SwiGLU, rotation (g_d) and requantisation
+      a1.out = h_q;
+      a1.g_h = g_d;
+      a1.s_h = s_h;
+      a1.hmax = reinterpret_cast<unsigned*>(hsync);
+      a1.rsync = reinterpret_cast<int*>(hsync + align256((size_t)E * (size_t)C * 4));
+      if ((rc = launch_gemm<kEpiSwigluRq, true>(x_g, w_gu, E, C, 2 * f, d, f, a1, st, true)) !=
+          CONVROT_OK)
+        return rc;
+    } else {
+      // 5. gate/up GEMM with dequant + SwiGLU
+      a1.out = h;
+      if ((rc = launch_gemm<kEpiSwiglu, true>(x_g, w_gu, E, C, 2 * f, d, f, a1, st, true)) !=
+          CONVROT_OK)
+        return rc;
+      // 6. rotate (g_d) + requantise h per row
+      if ((rc = rotquant_impl(h, CONVROT_DTYPE_F32, (int64_t)E * C, f, g_d, h_q, s_h, st,
+                              RqOut{0, 1, 1, 1}, true)) != CONVROT_OK)
+        return rc;
+    }
     // 7. down GEMM with dequant to the experts' BF16 outputs
     GemmArgs a2{};
     a2.s_a = s_h;

@@ -364,18 +364,24 @@ __global__ void __launch_bounds__(kTopcThreads) topc_reg_kernel(const float* __r
 
 // ----------------------------------------------------------------- gather --
 // dst[r, :] = src[idx[r], :], s_dst[r] = s_src[idx[r]]; one warp per row.
+// Also clears `zero` [n_zero] words (the synchronisation scratch of the GEMM
+// that reads dst next), if given.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const int8_t* __restrict__ src,
                                                           const float* __restrict__ s_src,
                                                           int64_t n_src,
                                                           const int32_t* __restrict__ idx,
                                                           int64_t n_rows, int K,
                                                           int8_t* __restrict__ dst,
-                                                          float* __restrict__ s_dst) {
+                                                          float* __restrict__ s_dst,
+                                                          uint32_t* __restrict__ zero,
+                                                          int64_t n_zero) {
   griddep_launch_dependents();
   griddep_wait();
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= n_rows) return;
+  if (zero != nullptr && lane == 0)
+    for (int64_t i = r; i < n_zero; i += n_rows) zero[i] = 0u;
   const int t = __ldg(idx + r);
   if (t < 0 || t >= n_src) {
     if (lane == 0) atomicOr(&g_device_error, kErrBadIndex);
