@@ -489,6 +489,7 @@ int launch_gemm(const int8_t* a, const int8_t* b, int64_t G, int64_t M, int64_t 
   }
   args.m_blocks = (int)cdiv(M, gemm::BM);
   args.slabs = args.m_blocks;
+  args.a_lane0 = M <= 64 ? 64 : 0;
   const int64_t tiles = G * args.m_blocks * args.n_blocks;
   if (tiles >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
   args.num_tiles = (int)tiles;
