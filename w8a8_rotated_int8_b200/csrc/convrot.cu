@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "convrot.h"
@@ -536,13 +537,28 @@ int topc_impl(const float* s_t, int64_t T, int E, int64_t C, int32_t* idx, float
 template <int NJ>
 int launch_combine(const void* z, const float* s_t, const int32_t* slot, int E, int64_t T,
                    int64_t C, int64_t d, void* y, int sms, cudaStream_t st, bool pdl) {
-  // tokens per CTA: a power of two in [1, 32] that leaves about eight CTAs
-  // per SM, so every SM streams rows while each CTA's slot tiles stay
-  // coalesced
-  int tpc = 32;
-  while (tpc > 1 && T < (int64_t)tpc * 8 * std::max(sms, 1)) tpc >>= 1;
-  const size_t smem = combine_tokens_smem(E, tpc);
   auto kern = combine_tokens_kernel<NJ>;
+  // tokens per CTA: the smallest power of two in [1, 32] for which the whole
+  // grid is resident at once (measured on B200 at T = 2048: one wave of 4
+  // tokens per CTA beats 3.5 waves of single tokens by 4 us, as every later
+  // wave would repeat the list building after the GEMM has finished)
+  static std::atomic<int> resident[kMaxDevices][4];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CONVROT_ERR_CUDA;
+  std::atomic<int>& cached = resident[dev][NJ == 1 ? 0 : NJ == 2 ? 1 : NJ == 4 ? 2 : 3];
+  int per_sm = cached.load(std::memory_order_relaxed);
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCombThreads,
+                                                      combine_tokens_smem(E, 1)) != cudaSuccess) {
+      cudaGetLastError();
+      return CONVROT_ERR_CUDA;
+    }
+    cached.store(per_sm, std::memory_order_relaxed);
+  }
+  const int64_t capacity = std::max<int64_t>(1, (int64_t)std::max(per_sm, 1) * std::max(sms, 1));
+  int tpc = 1;
+  while (tpc < 32 && cdiv(T, tpc) > capacity) tpc <<= 1;
+  const size_t smem = combine_tokens_smem(E, tpc);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
           cudaSuccess)
