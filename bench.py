@@ -36,9 +36,11 @@ from synthetic import MOE_CONFIGS, moe_inputs  # noqa: E402
 METRIC = "W8A8 ConvRot MoE block tokens/s"
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
 # kernel (the gate/up GEMM with the requantising SwiGLU epilogue), from the
-# ncu captures summarised in profiles/; to be dropped whenever that kernel
+# ncu captures summarised in profiles/block_kernels_moe_T8192.md and
+# profiles/gemm_s8_tcgen05_moe_T2048.md; to be dropped whenever that kernel
 # changes
-DOMINANT_TRAFFIC_BYTES = {}
+DOMINANT_TRAFFIC_BYTES = {"moe_T8192": 437.2e6 + 4.3e6,
+                          "moe_T2048": 411.9e6 + 4.9e6}
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 
