@@ -245,9 +245,12 @@ int encode_rows_sw128(CUtensorMap* map, const void* base, uint64_t row_bytes, ui
   return r == CUDA_SUCCESS ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
+// grid_cap > 0: when the rows need more CTAs than fit on the device at once,
+// run at most grid_cap persistent CTAs (the MoE call keeps SMs free for the
+// routing kernels that run beside the activation rotation).
 template <typename InT, int G, int SEG>
 int launch_rq_tma(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
-                   cudaStream_t st, bool pdl) {
+                   cudaStream_t st, bool pdl, int64_t grid_cap) {
   constexpr int kRowsPerWarp = 32 / SEG;
   const uint64_t row_bytes = (uint64_t)K * sizeof(InT);
   CUtensorMap tm;
@@ -268,24 +271,25 @@ int launch_rq_tma(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut
   device_setup(&sms);
   const int64_t units = (rows + kRowsPerWarp - 1) / kRowsPerWarp;
   const int64_t ctas = (units + kRqTmaWarps - 1) / kRqTmaWarps;
-  const int64_t grid = std::min<int64_t>(ctas, (int64_t)per_sm * std::max(sms, 1));
+  int64_t grid = std::min<int64_t>(ctas, (int64_t)per_sm * std::max(sms, 1));
+  if (grid_cap > 0 && ctas > grid) grid = std::min(grid, grid_cap);
   return launch_kernel(kern, dim3((unsigned)grid), dim3(kRqTmaWarps * 32), smem, st, pdl, 1, tm,
                        rows, K, slots, slot_bytes, q, s, out);
 }
 
 template <typename InT, int G>
 int launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
-               cudaStream_t st, bool pdl) {
+               cudaStream_t st, bool pdl, int64_t grid_cap) {
   // K % 64 == 0, K <= 2048: one warp segment of SEG lanes per row, 64
   // elements per lane (G = 256 needs at least the four lanes of one group)
   if (K % 64 == 0 && K <= 2048) {
     const int lanes = K / 64;
-    if (lanes <= 1 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 1 : 4)>(x, rows, K, q, s, out, st, pdl);
-    if (lanes <= 2 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 2 : 4)>(x, rows, K, q, s, out, st, pdl);
-    if (lanes <= 4) return launch_rq_tma<InT, G, 4>(x, rows, K, q, s, out, st, pdl);
-    if (lanes <= 8) return launch_rq_tma<InT, G, 8>(x, rows, K, q, s, out, st, pdl);
-    if (lanes <= 16) return launch_rq_tma<InT, G, 16>(x, rows, K, q, s, out, st, pdl);
-    return launch_rq_tma<InT, G, 32>(x, rows, K, q, s, out, st, pdl);
+    if (lanes <= 1 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 1 : 4)>(x, rows, K, q, s, out, st, pdl, grid_cap);
+    if (lanes <= 2 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 2 : 4)>(x, rows, K, q, s, out, st, pdl, grid_cap);
+    if (lanes <= 4) return launch_rq_tma<InT, G, 4>(x, rows, K, q, s, out, st, pdl, grid_cap);
+    if (lanes <= 8) return launch_rq_tma<InT, G, 8>(x, rows, K, q, s, out, st, pdl, grid_cap);
+    if (lanes <= 16) return launch_rq_tma<InT, G, 16>(x, rows, K, q, s, out, st, pdl, grid_cap);
+    return launch_rq_tma<InT, G, 32>(x, rows, K, q, s, out, st, pdl, grid_cap);
   }
   const int nch = K / 16;
   int tpr;
@@ -314,13 +318,13 @@ int launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out
 
 template <typename InT>
 int dispatch_rq(int group, const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
-                cudaStream_t st, bool pdl) {
+                cudaStream_t st, bool pdl, int64_t grid_cap) {
   switch (group) {
-    case 1: return launch_rq<InT, 1>(x, rows, K, q, s, out, st, pdl);
-    case 4: return launch_rq<InT, 4>(x, rows, K, q, s, out, st, pdl);
-    case 16: return launch_rq<InT, 16>(x, rows, K, q, s, out, st, pdl);
-    case 64: return launch_rq<InT, 64>(x, rows, K, q, s, out, st, pdl);
-    default: return launch_rq<InT, 256>(x, rows, K, q, s, out, st, pdl);
+    case 1: return launch_rq<InT, 1>(x, rows, K, q, s, out, st, pdl, grid_cap);
+    case 4: return launch_rq<InT, 4>(x, rows, K, q, s, out, st, pdl, grid_cap);
+    case 16: return launch_rq<InT, 16>(x, rows, K, q, s, out, st, pdl, grid_cap);
+    case 64: return launch_rq<InT, 64>(x, rows, K, q, s, out, st, pdl, grid_cap);
+    default: return launch_rq<InT, 256>(x, rows, K, q, s, out, st, pdl, grid_cap);
   }
 }
 
@@ -336,11 +340,13 @@ int check_rq_args(const void* x, int x_dtype, int64_t rows, int64_t K, int group
 }
 
 int rotquant_impl(const void* x, int x_dtype, int64_t rows, int64_t K, int group, int8_t* q,
-                  float* s, cudaStream_t st, RqOut out = RqOut{0, 1, 1, 1}, bool pdl = false) {
+                  float* s, cudaStream_t st, RqOut out = RqOut{0, 1, 1, 1}, bool pdl = false,
+                  int64_t grid_cap = 0) {
   if (rows == 0) return CONVROT_OK;
-  const int rc = (x_dtype == CONVROT_DTYPE_BF16)
-                     ? dispatch_rq<__nv_bfloat16>(group, x, rows, (int)K, q, s, out, st, pdl)
-                     : dispatch_rq<float>(group, x, rows, (int)K, q, s, out, st, pdl);
+  const int rc =
+      (x_dtype == CONVROT_DTYPE_BF16)
+          ? dispatch_rq<__nv_bfloat16>(group, x, rows, (int)K, q, s, out, st, pdl, grid_cap)
+          : dispatch_rq<float>(group, x, rows, (int)K, q, s, out, st, pdl, grid_cap);
   if (rc != CONVROT_OK) return rc;
   return launch_status();
 }
@@ -983,8 +989,13 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
   int rc_side = softmax_impl(logits_bf16, T, E, s_t, ss->stream);
   // 3. expert-choice top-C (+ each token's slot per expert)
   if (rc_side == CONVROT_OK) rc_side = topc_impl(s_t, T, E, C, idx, w, slot, ss->stream, true);
-  // 2. rotate + quantise the tokens once (the gate/up rotation is expert-independent)
-  rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, T, d, g_gu, x_q, s_x, st);
+  // 2. rotate + quantise the tokens once (the gate/up rotation is expert-independent);
+  // a rotation longer than one round of resident CTAs runs on about 1.25 CTAs
+  // per SM instead of filling every SM's register file, so the routing kernels
+  // start beside it (measured on B200: -5 us at T=8192; no change when one round
+  // covers the rows, as at T=2048)
+  rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, T, d, g_gu, x_q, s_x, st, RqOut{0, 1, 1, 1},
+                     false, sms + sms / 4);
   // the join is recorded even after a failed launch so the side stream never dangles
   if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess ||
       cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess)
