@@ -65,6 +65,20 @@ def test_argument_checks_need_no_gpu(lib):
     assert lib.convrot_i8_gemm_i32(al, al, 0, 1, 8, 24, 64, al, None) == INVALID
     assert lib.convrot_i8_gemm_i32(al, al, 0, 1, 8, 16, 1 << 20, al, None) == INVALID
     assert lib.convrot_i8_gemm_i32(al, al, 2, 1, 8, 16, 64, al, None) == INVALID  # bad layout
+    # requantising SwiGLU GEMM: a group that does not fit one thread (256), a group that is not
+    # a power of four, F not a multiple of the group, a misaligned output, a scratch too small
+    rq = lib.convrot_i8_gemm_swiglu_rq
+    big = 1 << 20
+    assert rq(al, al, al, al, 1, 2, 64, 256, 256, 256, al, al, al, big, None) == INVALID
+    assert rq(al, al, al, al, 1, 2, 64, 256, 256, 8, al, al, al, big, None) == INVALID
+    assert rq(al, al, al, al, 1, 2, 64, 80, 256, 64, al, al, al, big, None) == INVALID
+    assert rq(al, al, al, al, 1, 2, 64, 256, 256, 64, mis, al, al, big, None) == MISALIGNED
+    assert (rq(al, al, al, al, 1, 2, 64, 256, 256, 64, al, al, al, 64, None)
+            == binding.CONVROT_ERR_WORKSPACE_TOO_SMALL)
+    # its scratch: the row maxima (256-byte aligned), then an arrival counter per 128-row slab
+    # (one spare slab per group) and the abort word
+    assert lib.convrot_swiglu_rq_sync_bytes(64, 256) == 64 * 256 * 4 + (64 * 3 + 1) * 4
+    assert lib.convrot_swiglu_rq_sync_bytes(5, 40) == 1024 + (5 * 2 + 1) * 4
     # tiled weight sizes: 128-row blocks x 128-byte K tiles of 16 KB
     assert lib.convrot_tiled_weight_bytes(2, 300, 200) == 2 * 3 * 2 * 16384
     assert lib.convrot_tiled_weight_bytes(128, 1536, 2048) == 128 * 12 * 16 * 16384
