@@ -6,7 +6,7 @@ h rotate+requantise in its epilogue, down GEMM to bf16, router-weighted
 combine) over one batch of synthetic tokens, through the C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config moe_T8192]
-                    [--impl ours|reference] [--no-cpu-baseline] [--ablation]
+                    [--impl ours|reference] [--no-cpu-baseline] [--ablation] [--sweep]
 
 Multi-GPU (launched by torch.distributed.run): every rank runs its own batch
 of T tokens against the same weights (weak scaling, no data-path
@@ -582,6 +582,8 @@ def main():
                     help="rotation-off ablation: block error with and without ConvRot")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one JSON line per token count T in 512..8192 (C = 2T/64), no CPU baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -596,7 +598,12 @@ def main():
         return
     world, rank, local = dist_setup()
     try:
-        run_ours(args, cfg, world, rank, local)
+        if args.sweep:
+            args.cpu_baseline = False
+            for name in ("moe_T512", "moe_T1024", "moe_T2048", "moe_T4096", "moe_T8192"):
+                run_ours(args, MOE_CONFIGS[name], world, rank, local)
+        else:
+            run_ours(args, cfg, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist
