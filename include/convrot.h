@@ -141,7 +141,8 @@ int convrot_router_softmax(const void* logits_bf16, int64_t T, int E, float* s_t
  *   C     0 <= C <= T
  *   idx   device, [E, C] int32: the C tokens with the largest score, ties to
  *         the lower token index, in ascending token order
- *   w     device, [E, C] fp32: w[e, c] = s_t[e, idx[e, c]]
+ *   w     device, [E, C] fp32: w[e, c] = s_t[e, idx[e, c]] (a -0 score
+ *         compares equal to +0 and comes back as +0)
  *   slot  device, [E, T] int32 or NULL: slot[e, t] = c where idx[e, c] = t,
  *         or -1 if expert e did not pick token t (the inverse of idx)
  * ------------------------------------------------------------------------- */
