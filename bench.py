@@ -35,10 +35,9 @@ from synthetic import MOE_CONFIGS, moe_inputs  # noqa: E402
 
 METRIC = "W8A8 ConvRot MoE block tokens/s"
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
-# kernel (the gate/up GEMM with the requantising SwiGLU epilogue), from the
-# ncu captures summarised in profiles/block_kernels_moe_T8192.md and
-# profiles/gemm_s8_tcgen05_moe_T2048.md; to be dropped whenever that kernel
-# changes
+# kernel (the gate/up GEMM with the requantising SwiGLU epilogue), from ncu
+# captures of the block call at T=8192 and T=2048 (their summaries are under
+# profiles/); to be dropped whenever that kernel changes
 DOMINANT_TRAFFIC_BYTES = {"moe_T8192": 437.2e6 + 5.5e6,
                           "moe_T2048": 411.9e6 + 7.0e6}
 UNIT = "tokens/s"
