@@ -162,6 +162,44 @@ def test_topc_slot_table_inverts_idx(t, c):
     assert np.array_equal(slot, expect)
 
 
+def _degenerate_scores(kind, t, e, gen):
+    if kind == "equal":  # every token ties: the first C tokens win
+        return np.full((t, e), 0.25, np.float32)
+    if kind == "signed_zero":  # -0 and +0 compare equal
+        z = np.where(torch.rand(t, e, generator=gen).numpy() < 0.5, -0.0, 0.0).astype(np.float32)
+        z[::7] = 1e-3
+        return z
+    if kind == "signed":  # negative scores, +-inf and subnormals order by value
+        s = torch.randn(t, e, generator=gen).numpy().astype(np.float32)
+        s[::5] = np.float32(1e-40) * np.sign(s[::5])
+        s[3::11] = np.inf
+        s[4::13] = -np.inf
+        return s
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("kind", ["equal", "signed_zero", "signed"])
+@pytest.mark.parametrize("t", [1, 31, 1000, 4096, 16384])
+def test_topc_degenerate_scores(kind, t):
+    """Degenerate score columns: all equal, signed zeros, negatives, +-inf,
+    subnormals; C in {0, 1, T // 3, T}. The picks equal the oracle's and the
+    slot table inverts them."""
+    e = 3
+    gen = torch.Generator().manual_seed(t + len(kind))
+    s = _degenerate_scores(kind, t, e, gen)
+    s_dev = torch.from_numpy(np.ascontiguousarray(s.T)).cuda()
+    for c in sorted({0, 1, t // 3, t}):
+        idx, w, slot = W.convrot_topc(s_dev, c, with_slot=True)
+        idx_ref, w_ref = O.expert_choice_topc(s, c)
+        idx, w, slot = idx.cpu().numpy(), w.cpu().numpy(), slot.cpu().numpy()
+        assert np.array_equal(idx, idx_ref), (kind, t, c)
+        assert np.array_equal(w, w_ref), (kind, t, c)  # by value: a -0 pick comes back as +0
+        expect = np.full((e, t), -1, np.int32)
+        for x in range(e):
+            expect[x, idx[x]] = np.arange(c)
+        assert np.array_equal(slot, expect), (kind, t, c)
+
+
 def test_gather_rows():
     src = torch.randint(-127, 128, (100, 64), dtype=torch.int8)
     s_src = torch.rand(100)
