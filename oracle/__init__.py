@@ -6,18 +6,20 @@ This package is TEST INFRASTRUCTURE. Only the test suite, the smoke check in
 binding) never imports, links or executes anything in here, and nothing in
 here imports the product package.
 
-Everything is plain NumPy: the rotation and rounding in fp32 (with an exact
-fp64 matrix form of the rotation kept for the pins), exact integer GEMMs,
-fp64 for the router softmax, fp32 for the scales, dequantised outputs,
-SwiGLU and the router-weighted combine.
+Everything is plain NumPy: the rotation as an explicit fp64 Sylvester
+Hadamard matrix, the quantiser's quotient in fp64, exact integer GEMMs, fp64
+for the router softmax, fp32 for the scales, dequantised outputs, SwiGLU and
+the router-weighted combine.
 """
 
 from .convrot_oracle import (  # noqa: F401
     bf16_round,
     block_rotate,
+    combine,
+    combine_f32,
     dequant,
+    down_from_codes,
     expert_choice_topc,
-    fwht_f32,
     hadamard,
     int_gemm,
     moe_block,
@@ -26,5 +28,7 @@ from .convrot_oracle import (  # noqa: F401
     rotquant,
     router_softmax,
     silu_f32,
+    swiglu_from_codes,
     w8a8_linear,
+    w8a8_linear_from_codes,
 )

@@ -22,20 +22,17 @@ Readings of what the pages leave open (each is fixed here once):
 
 * Hadamard: Sylvester construction in natural order, no sign flips,
   normalised by 1/sqrt(g); applied block-diagonally along K (contiguous
-  groups of g). Only g in {1, 4, 16, 64, 256} (powers of four) are accepted,
-  so 1/sqrt(g) is a power of two.
-* Precision of rotation and rounding: fp32, as the NitroFusion2 page states
-  for its conversions ("How they were made": the rotation and rounding in
-  fp32). The rotation is the fast Walsh-Hadamard butterfly (a+b, a-b) in
-  fp32 with the stage spans in increasing order 1, 2, ..., g/2, then the
-  exact scaling by 1/sqrt(g); block_rotate (fp64 matrix product) is its
-  exact mathematical counterpart.
-* Symmetric INT8 of a rotated fp32 row v: a = max|v|, s = fp32(a / 127),
-  r = fp32(127 / a), q = clamp(rint(fp32(v * r)), -127, 127) with ties to
-  even. A row with a < 2^-120 (zero, or too small for r to be finite) gets
-  s = 0 and q = 0.
+  groups of g) as an explicit fp64 matrix product. Only g in
+  {1, 4, 16, 64, 256} (powers of four) are accepted, so 1/sqrt(g) is a power
+  of two.
+* Symmetric INT8 with nearest rounding of a rotated row v (fp64):
+  a = max|v|, s = fp32(a / 127) (the fp64 quotient rounded once to fp32),
+  q = clamp(rne(v / s), -127, 127) with the quotient taken in fp64 and ties
+  to even. A row whose s is 0 (an all-zero row, or one too small for fp32)
+  gets all-zero codes.
 * Activations: per-token dynamic scales, the same rotation and quantiser as
-  the weights.
+  the weights; so is the SwiGLU output h before the down projection (g = 64,
+  one scale per (expert, token) row).
 * Router score: per-token softmax over the experts, evaluated in fp64 and
   rounded once to fp32. Top-C ties go to the lower token index; the selected
   indices are stored in ascending token order.
@@ -97,55 +94,30 @@ def block_rotate(v: np.ndarray, g: int) -> np.ndarray:
     return (grouped @ r).reshape(v.shape)
 
 
-def fwht_f32(v: np.ndarray, g: int) -> np.ndarray:
-    """The fp32 rotation: per contiguous group of g along the last axis,
-    butterflies (a + b, a - b) in fp32 with spans 1, 2, ..., g/2 in that
-    order, then multiplication by 1/sqrt(g) (a power of two)."""
-    if g not in ALLOWED_GROUPS:
-        raise ValueError(f"group must be one of {ALLOWED_GROUPS}, got {g}")
-    x = np.array(v, dtype=np.float32)
-    k = x.shape[-1]
-    if k % g != 0:
-        raise ValueError(f"K={k} is not a multiple of the group size {g}")
-    lead = x.shape[:-1]
-    span = 1
-    while span < g:
-        y = x.reshape(lead + (k // (2 * span), 2, span))
-        a = y[..., 0, :].copy()
-        b = y[..., 1, :].copy()
-        y[..., 0, :] = a + b
-        y[..., 1, :] = a - b
-        x = y.reshape(lead + (k,))
-        span *= 2
-    return (x * np.float32(1.0 / np.sqrt(g))).astype(np.float32)
-
-
 # ------------------------------------------------------------ quantisation --
-TINY = np.float32(2.0 ** -120)
-
-
 def quantize_rows(v: np.ndarray):
-    """Symmetric per-row INT8 of an fp32 matrix [rows, K] (see the header).
+    """Symmetric per-row INT8 of a rotated matrix [rows, K] (see the header).
 
     Returns (q int8 [rows, K], s float32 [rows]).
     """
-    v = np.asarray(v, dtype=np.float32)
-    a = np.max(np.abs(v), axis=-1)
-    ok = a >= TINY
-    a_safe = np.where(ok, a, np.float32(1))
-    s = np.where(ok, a_safe / np.float32(QMAX), np.float32(0)).astype(np.float32)
-    r = (np.float32(QMAX) / a_safe).astype(np.float32)
-    prod = (v * r[..., None]).astype(np.float32)
-    q = np.clip(np.rint(prod), -QMAX, QMAX).astype(np.int8)
-    q[~ok] = 0
+    v = np.asarray(v, dtype=np.float64)
+    a = np.max(np.abs(v), axis=-1) if v.shape[-1] else np.zeros(v.shape[:-1])
+    s = (a / np.float64(QMAX)).astype(np.float32)
+    q = np.zeros(v.shape, dtype=np.int8)
+    nz = s != 0
+    if np.any(nz):
+        quot = v[nz] / s[nz].astype(np.float64)[..., None]
+        q[nz] = np.clip(np.rint(quot), -QMAX, QMAX).astype(np.int8)
     return q, s
 
 
 def rotquant(x: np.ndarray, g: int):
-    """Rotate each row in groups of g (fp32 butterflies) and quantise it per
-    row. Serves the weights (offline, per output row), the activations (per
-    token) and the SwiGLU output h before the down projection (g = 64)."""
-    return quantize_rows(fwht_f32(x, g))
+    """Rotate each row by blockdiag(R_g) (fp64) and quantise it per row.
+
+    Serves the weights (offline, per output row), the activations (per
+    token) and the SwiGLU output h before the down projection (g = 64).
+    """
+    return quantize_rows(block_rotate(x, g))
 
 
 # --------------------------------------------------------- integer GEMM -----
@@ -190,13 +162,18 @@ def bf16_round(x: np.ndarray) -> np.ndarray:
     return rounded.view(np.float32)
 
 
+def w8a8_linear_from_codes(x_q, s_x, w_q, s_w) -> np.ndarray:
+    """The linear given quantised inputs: Y = bf16(fp32(acc) * (s_w * s_x))."""
+    return bf16_round(dequant(int_gemm(x_q, w_q), s_w, s_x))
+
+
 def w8a8_linear(x: np.ndarray, w_q: np.ndarray, s_w: np.ndarray, g: int) -> np.ndarray:
     """W8A8 ConvRot linear: Y = bf16(fp32(acc) * (s_w * s_x)).
 
     x: [M, K] bf16 values; w_q: [N, K] int8 rotated codes; s_w: [N] fp32.
     """
     x_q, s_x = rotquant(x, g)
-    return bf16_round(dequant(int_gemm(x_q, w_q), s_w, s_x))
+    return w8a8_linear_from_codes(x_q, s_x, w_q, s_w)
 
 
 # --------------------------------------------------------------- routing ----
@@ -238,6 +215,44 @@ def silu_f32(g: np.ndarray) -> np.ndarray:
     return (g32 / (np.float32(1) + e)).astype(np.float32)
 
 
+def swiglu_from_codes(x_q, s_x, wgu_q, s_gu) -> np.ndarray:
+    """One expert's gate/up linear given quantised inputs, then SwiGLU:
+    y = fp32(acc) * (s_gu * s_x); h = silu(y[:, :f]) * y[:, f:] (fp32)."""
+    y = dequant(int_gemm(x_q, wgu_q), s_gu, s_x)
+    f = y.shape[1] // 2
+    return (silu_f32(y[:, :f]) * y[:, f:]).astype(np.float32)
+
+
+def down_from_codes(h_q, s_h, wd_q, s_d) -> np.ndarray:
+    """One expert's down projection given quantised inputs: a W8A8 linear
+    with BF16 output, z = bf16(fp32(acc) * (s_d * s_h))."""
+    return w8a8_linear_from_codes(h_q, s_h, wd_q, s_d)
+
+
+# --------------------------------------------------------------- combine ----
+def combine_f32(t: int, idx: np.ndarray, w: np.ndarray, z: dict) -> np.ndarray:
+    """Router-weighted sum before the final rounding: out32[idx[e, c]] +=
+    fp32(w[e, c] * z[e][c]) in fp32, experts in ascending order.
+
+    z maps expert e to its [C, d] bf16 outputs (as fp32); experts missing
+    from z contribute nothing. Returns out32 [t, d] fp32.
+    """
+    d = next(iter(z.values())).shape[1] if z else 0
+    out32 = np.zeros((t, d), dtype=np.float32)
+    for e in sorted(z):
+        rows = idx[e]
+        # rows are distinct within an expert, so fancy-index += is exact;
+        # the product w*z is rounded to fp32, then added in fp32
+        out32[rows] = out32[rows] + (w[e][:, None] * z[e]).astype(np.float32)
+    return out32
+
+
+def combine(t: int, idx: np.ndarray, w: np.ndarray, z: dict) -> np.ndarray:
+    """The router-weighted combine with its one bf16 rounding: Y [t, d] as
+    fp32 holding bf16 values (see combine_f32)."""
+    return bf16_round(combine_f32(t, idx, w, z))
+
+
 # -------------------------------------------------------------- MoE block ---
 def moe_block(x, logits, wgu_q, s_gu, wd_q, s_d, c, g_gu=256, g_d=64,
               experts=None, keep=False, out_tokens=None):
@@ -248,40 +263,37 @@ def moe_block(x, logits, wgu_q, s_gu, wd_q, s_d, c, g_gu=256, g_d=64,
     wd_q: [E, d, f] int8, s_d: [E, d]; c: tokens per expert.
     ``experts`` restricts the combine to a subset of experts (used to time a
     bounded sample); ``out_tokens`` evaluates only the output rows of those
-    tokens (each row depends only on its own token, so the others are simply
-    skipped and left 0); ``keep`` returns the intermediates as a dict.
+    tokens (each row depends only on its own token, so the expert rows of
+    other tokens are left 0 and so are their outputs); ``keep`` returns the
+    intermediates as a dict.
 
     Returns Y as fp32 holding bf16 values [T, d] (and the dict if keep).
     """
     x = np.asarray(x, dtype=np.float32)
     t, d = x.shape
-    n_exp, two_f, _ = wgu_q.shape
-    f = two_f // 2
+    n_exp = wgu_q.shape[0]
     x_q, s_x = rotquant(x, g_gu)
     scores = router_softmax(logits)
     idx, w = expert_choice_topc(scores, c)
-    out32 = np.zeros((t, d), dtype=np.float32)
     inter = {"x_q": x_q, "s_x": s_x, "scores": scores, "idx": idx, "w": w,
              "h": {}, "h_q": {}, "s_h": {}, "z": {}}
+    z_all = {}
     for e in (range(n_exp) if experts is None else experts):
-        rows = idx[e]
+        sel = np.arange(c)
         if out_tokens is not None:
-            rows = rows[np.isin(rows, out_tokens)]
-            if rows.size == 0:
+            sel = np.nonzero(np.isin(idx[e], out_tokens))[0]
+            if sel.size == 0:
                 continue
-        sel = np.searchsorted(idx[e], rows)
-        y = dequant(int_gemm(x_q[rows], wgu_q[e]), s_gu[e], s_x[rows])
-        gate, up = y[:, :f], y[:, f:]
-        h = (silu_f32(gate) * up).astype(np.float32)
+        rows = idx[e][sel]
+        h = swiglu_from_codes(x_q[rows], s_x[rows], wgu_q[e], s_gu[e])
         h_q, s_h = rotquant(h, g_d)
-        # the down projection is a W8A8 linear with BF16 output
-        z = bf16_round(dequant(int_gemm(h_q, wd_q[e]), s_d[e], s_h))
-        # rows are distinct within an expert, so fancy-index += is exact;
-        # the product w*z is rounded to fp32, then added in fp32
-        out32[rows] = out32[rows] + (w[e][sel][:, None] * z).astype(np.float32)
+        z = np.zeros((c, d), dtype=np.float32)
+        z[sel] = down_from_codes(h_q, s_h, wd_q[e], s_d[e])
+        z_all[e] = z
         if keep:
             inter["h"][e], inter["h_q"][e], inter["s_h"][e] = h, h_q, s_h
             inter["z"][e] = z
+    out32 = combine_f32(t, idx, w, z_all) if z_all else np.zeros((t, d), np.float32)
     y_out = bf16_round(out32)
     if keep:
         inter["out32"] = out32

@@ -11,8 +11,10 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import (bf16_round, block_rotate, dequant, fwht_f32, int_gemm, quantize_rows,
-                    rotquant, w8a8_linear)
+from fractions import Fraction
+
+from oracle import (bf16_round, block_rotate, dequant, int_gemm, quantize_rows, rotquant,
+                    w8a8_linear, w8a8_linear_from_codes)
 from tests.golden import read_fixture
 
 
@@ -34,48 +36,85 @@ def test_worked_rotated_codes_g4():
     assert s[0] == np.float32(13) / np.float32(127)
 
 
+def _nearest_f32(x: Fraction) -> np.float32:
+    """The fp32 value nearest to the exact rational x (ties to even), found
+    by comparing the neighbours of a candidate in exact arithmetic."""
+    c = np.float32(float(x))
+    best = None
+    for cand in (np.nextafter(c, np.float32(-np.inf)), c, np.nextafter(c, np.float32(np.inf))):
+        d = abs(Fraction(float(cand)) - x)
+        even = (int(np.float32(cand).view(np.uint32)) & 1) == 0
+        if best is None or d < best[0] or (d == best[0] and even):
+            best = (d, cand)
+    return np.float32(best[1])
+
+
+def test_quantiser_scale_is_fp32_of_absmax_over_127(rng):
+    """s is the fp32 value nearest to the exact absmax / 127."""
+    v = rng.standard_normal((40, 96)) * 10.0 ** rng.integers(-20, 20, (40, 1))
+    _, s = quantize_rows(v)
+    for i in range(v.shape[0]):
+        a = max(Fraction(abs(float(x))) for x in v[i])
+        assert s[i] == _nearest_f32(a / 127)
+
+
 def test_quantiser_bounds(rng):
-    v = (rng.standard_normal((64, 256)) * rng.uniform(0.01, 50, size=(64, 1))).astype(np.float32)
+    v = rng.standard_normal((64, 256)) * rng.uniform(0.01, 50, size=(64, 1))
     q, s = quantize_rows(v)
     s64 = s.astype(np.float64)[:, None]
     assert np.all(np.abs(q.astype(np.int64)) <= 127)
-    # nearest code up to the fp32 reciprocal: |v - s q| <= s (1/2 + 1e-4)
-    assert np.all(np.abs(v - s64 * q) <= s64 * (0.5 + 1e-4))
+    # nearest code of the fp64 quotient: |v - s q| <= s (1/2 + 127 * 2^-53)
+    assert np.all(np.abs(v - s64 * q) <= s64 * (0.5 + 2.0 ** -46))
     # the absmax element of every row gets a full-scale code
     j = np.argmax(np.abs(v), axis=1)
     assert np.all(np.abs(q[np.arange(64), j]) == 127)
-    # the scale is absmax/127 as one fp32 division
-    assert np.array_equal(s, np.max(np.abs(v), axis=1) / np.float32(127))
 
 
-def test_quantiser_nearest_code_property(rng):
-    """Every code is the nearest integer to the exact v / s, ties to even,
-    except where v / s lies within 1e-4 of a half-integer (the fp32
-    reciprocal may tip it); there it is one of the two neighbours."""
-    v = rng.standard_normal((16, 64)).astype(np.float32)
+def test_quantiser_nearest_code_brute_force(rng):
+    """Every code is the integer in [-127, 127] nearest to the exact v / s
+    (ties to even), found by trying all 255 codes in exact arithmetic. The
+    only allowed exception is a quotient within 127 * 2^-53 of a half-integer
+    (the fp64 division may tip it); none occurs in these rows."""
+    v = rng.standard_normal((12, 48))
     v[1, 3] = 0.0
-    v[2, :8] = np.float32(127) * np.array([1, 0.5, 2.5, -2.5, 3.5, 1.5, -0.5, 126.5], np.float32) / 127
+    # exact half-integer quotients: the row's absmax is 127, so s = 1
+    v[2, :9] = [127, 0.5, 2.5, -2.5, 3.5, 1.5, -0.5, 126.5, -126.5]
+    # a row with absmax 1, so s = fp32(1/127) != 1/127: between
+    # (k + 1/2) * s and (k + 1/2) / 127 the quotient by s and the quotient by
+    # the unrounded absmax / 127 fall on different sides of k + 1/2
+    v[3, :] = 0.0
+    v[3, 0] = 1.0
+    s_f32 = Fraction(float(np.float32(1.0 / 127.0)))
+    for j, k in enumerate((100, 57, 3), start=1):
+        lo, hi = sorted((Fraction(2 * k + 1, 2) * s_f32, Fraction(2 * k + 1, 2) / 127))
+        v[3, j] = float((lo + hi) / 2)
+        v[3, j + 3] = -float((lo + hi) / 2)
     q, s = quantize_rows(v)
-    codes = np.arange(-127, 128)
+    codes = range(-127, 128)
     for i in range(v.shape[0]):
+        si = Fraction(float(s[i]))
         for j in range(v.shape[1]):
-            x = float(v[i, j]) / float(s[i])
-            dist = np.abs(x - codes)
-            best = codes[dist == dist.min()]
-            frac = abs(abs(x - np.floor(x)) - 0.5)
-            if frac > 1e-4:
-                assert q[i, j] == (best[0] if len(best) == 1 else best[best % 2 == 0][0])
-            else:
-                assert q[i, j] in (np.floor(x), np.ceil(x))
+            x = Fraction(float(v[i, j])) / si
+            dist = {c: abs(x - c) for c in codes}
+            m = min(dist.values())
+            best = [c for c in codes if dist[c] == m]
+            want = best[0] if len(best) == 1 else [c for c in best if c % 2 == 0][0]
+            assert q[i, j] == want, (i, j, float(x))
 
 
 def test_zero_and_tiny_rows():
-    v = np.zeros((3, 8), np.float32)
-    v[1, 2] = np.float32(2.0 ** -121)   # below the 2^-120 floor: treated as zero
-    v[2, 2] = np.float32(2.0 ** -119)
+    """s = fp32(a / 127) may be subnormal or 0 for a tiny row. Worked by hand:
+    row 1: a = 2^-140, a / 127 = 2^-149 * 512/127 = 2^-149 * 4.03.. -> the
+    subnormal s = 4 * 2^-149 = 2^-147; codes 2^-140 / s = 128 -> clamped to 127,
+    2^-141 / s = 64, -2^-140 / s = -128 -> clamped to -127. Row 2: a = 2^-145, a / 127 = 2^-149 * 0.126 -> s = 0, codes 0."""
+    v = np.zeros((3, 8))
+    v[1, 2], v[1, 5], v[1, 6] = 2.0 ** -140, -(2.0 ** -141), -(2.0 ** -140)
+    v[2, 0] = 2.0 ** -145
     q, s = quantize_rows(v)
-    assert np.all(q[:2] == 0) and np.all(s[:2] == 0)
-    assert q[2, 2] == 127 and s[2] == np.float32(2.0 ** -119) / np.float32(127)
+    assert np.all(q[0] == 0) and s[0] == 0
+    assert s[1] == np.float32(2.0 ** -147)
+    assert q[1].tolist() == [0, 0, 127, 0, 0, -64, -127, 0]  # +-128 clamped to +-127
+    assert np.all(q[2] == 0) and s[2] == 0
 
 
 def test_int_gemm_triple_loop(rng):
@@ -118,21 +157,17 @@ def test_bf16_round_matches_library(rng):
 
 def _linear_error_bound(x, w, g, y):
     """Rigorous bound on |Y - X W^T| for the W8A8 ConvRot linear."""
-    xr, wr = fwht_f32(x, g).astype(np.float64), fwht_f32(w, g).astype(np.float64)
+    xr, wr = block_rotate(x, g), block_rotate(w, g)
     xq, sx = quantize_rows(xr)
     wq, sw = quantize_rows(wr)
     w_hat = wq * sw.astype(np.float64)[:, None]
-    half = 0.5 + 1e-4
+    half = 0.5 + 2.0 ** -46
     # quantisation: |x'.w' - x_hat.w_hat| <= sum|x'| |w' - w_hat| + sum |w_hat| |x' - x_hat|
     bound = (np.abs(xr).sum(1)[:, None] * (sw.astype(np.float64)[None, :] * half)
              + (sx.astype(np.float64)[:, None] * half) * np.abs(w_hat).sum(1)[None, :])
-    # fp32 rotation of x and w: log2(g) roundings of at most the group's |.|-sum
-    st = max(int(np.log2(g)), 0) * 2.0 ** -24 / np.sqrt(g)
-    ex = st * np.abs(x.astype(np.float64)).reshape(x.shape[0], -1, g).sum(-1).max(-1)
-    ew = st * np.abs(w.astype(np.float64)).reshape(w.shape[0], -1, g).sum(-1).max(-1)
-    bound += (ex[:, None] * np.abs(wr).sum(1)[None, :] + np.abs(xr).sum(1)[:, None] * ew[None, :])
     ref = x.astype(np.float64) @ w.astype(np.float64).T
-    # fp32 dequant (3 roundings) and the final bf16 rounding
+    # fp64 rotation of bf16 data is exact up to fp64 rounding; fp32 dequant
+    # (3 roundings) and the final bf16 rounding
     slack = np.abs(ref + bound) * (2.0 ** -8 + 4 * 2.0 ** -24) + 1e-30
     return np.abs(y - ref), bound + slack
 
@@ -163,3 +198,11 @@ def test_rotation_reduces_outlier_error(rng):
         wq, sw = rotquant(w, g)
         errs[g] = np.linalg.norm(w8a8_linear(x, wq, sw, g) - ref)
     assert errs[256] < 0.5 * errs[1]
+
+
+def test_linear_from_codes_is_the_linear(rng):
+    x = _bf16(rng.standard_normal((8, 256)))
+    w = _bf16(rng.standard_normal((12, 256)) * 0.02)
+    wq, sw = rotquant(w, 64)
+    xq, sx = rotquant(x, 64)
+    assert np.array_equal(w8a8_linear(x, wq, sw, 64), w8a8_linear_from_codes(xq, sx, wq, sw))
