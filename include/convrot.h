@@ -18,8 +18,14 @@
  * Readings fixed by this library where the pages are silent:
  *  - rotation: Sylvester Hadamard in natural order, normalised by 1/sqrt(g),
  *    applied to contiguous groups of g along K; g in {1, 4, 16, 64, 256};
- *  - quantiser: s = fp32(absmax / 127), q = clamp(rint(v / s), -127, 127)
- *    (ties to even), codes and scale 0 for an all-zero row;
+ *  - quantiser (the definition): v' = v . blockdiag(H_g / sqrt(g)),
+ *    s = fp32(max|v'| / 127), q = clamp(rne(v' / s), -127, 127), ties to
+ *    even; all-zero codes when s is 0. The offline weight quantisers compute
+ *    exactly this (fp64 rotation and quotients). The run-time activation and
+ *    h quantisers rotate in fp32 and take q = rint(v'_32 * fp32(127 / a_32))
+ *    (rows with absmax below 2^-100 divide by their scale instead): their
+ *    codes can differ from the definition's by one where v'/s lies within the
+ *    fp32 rounding error of a half-integer;
  *  - activations (and the SwiGLU output h) use per-row dynamic scales;
  *  - router score: per-token softmax over the experts (fp64, rounded to
  *    fp32); top-C ties go to the lower token index; each expert's tokens are
@@ -96,9 +102,10 @@ int convrot_check_device_error(void* stream, unsigned* flags);
 int convrot_wait_selftest(unsigned long long limit_ns, int* result_dev, void* stream);
 
 /* ---------------------------------------------------------------------------
- * Rotate + quantise rows (offline weights, run-time activations, and the
- * SwiGLU output h before the down projection). "Nucleus-Image INT8 Convrot
- * Experts + FP8 Text Encoder", section "Quantization".
+ * Rotate + quantise rows at run time (activations per token, and the SwiGLU
+ * output h before the down projection). "Nucleus-Image INT8 Convrot Experts +
+ * FP8 Text Encoder", section "Quantization". fp32 arithmetic (see the
+ * quantiser note at the top): within one code of the definition.
  *   x      device, [rows, K] bf16 (x_dtype = CONVROT_DTYPE_BF16) or fp32
  *   rows   >= 0;  K: multiple of 16 and of `group`, 16 <= K <= 8192
  *   group  rotation group g in {1, 4, 16, 64, 256}
@@ -109,9 +116,13 @@ int convrot_wait_selftest(unsigned long long limit_ns, int* result_dev, void* st
 int convrot_rotquant(const void* x, int x_dtype, int64_t rows, int64_t K, int group, int8_t* q,
                      float* scale, void* stream);
 
-/* Offline weight quantisation: the same operation on bf16 weight rows. A
- * stack of expert matrices [E, N, K] is passed as rows = E * N (the rotation
- * is per row, so the 3-D packed layout needs no other entry point). */
+/* Offline weight quantisation of bf16 weight rows, exactly the definition:
+ * fp64 rotation (exact sums of bf16 values while a group's exponent spread
+ * stays under ~37 bits), s = fp32 of the fp64 quotient absmax / 127, codes
+ * rne of correctly rounded fp64 quotients. Same sizes and arguments as
+ * convrot_rotquant with bf16 input. A stack of expert matrices [E, N, K] is
+ * passed as rows = E * N (the rotation is per row, so the 3-D packed layout
+ * needs no other entry point). */
 int convrot_quantize_weights(const void* w_bf16, int64_t rows, int64_t K, int group,
                              int8_t* w_q, float* row_scale, void* stream);
 
@@ -257,8 +268,12 @@ int w8a8_convrot_linear(const void* x_bf16, int64_t M, int64_t K, const int8_t* 
  * library (CONVROT_NOALLOC_MAX_CODES code bytes + CONVROT_NOALLOC_MAX_ROWS
  * fp32 scales, about 8.1 MiB), which every GPU that loads the library keeps
  * until the process exits.
- *  - M * K > CONVROT_NOALLOC_MAX_CODES or M > CONVROT_NOALLOC_MAX_ROWS:
- *    returns CONVROT_ERR_WORKSPACE_TOO_SMALL and launches nothing.
+ *  - Invalid sizes, groups or pointers are reported as by w8a8_convrot_linear
+ *    first; then M * K > CONVROT_NOALLOC_MAX_CODES or
+ *    M > CONVROT_NOALLOC_MAX_ROWS returns CONVROT_ERR_WORKSPACE_TOO_SMALL and
+ *    launches nothing.
+ *  - The array belongs to the current device: x and y must be memory of that
+ *    device (or managed memory), else CONVROT_ERR_INVALID_ARG.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress, no allocation) with that device current; make
  *    that first call before any stream capture.

@@ -90,7 +90,7 @@ def block_rotate(v: np.ndarray, g: int) -> np.ndarray:
     if k % g != 0:
         raise ValueError(f"K={k} is not a multiple of the group size {g}")
     r = rotation_matrix(g)
-    grouped = v.reshape(v.shape[:-1] + (k // g, g))
+    grouped = v.reshape(-1, g)  # every contiguous group of g as one row
     return (grouped @ r).reshape(v.shape)
 
 

@@ -1,10 +1,13 @@
 """GPU parity: every stage of the CUDA path through the C ABI against the oracle.
 
-Bar: bit-exact codes, scales, int32 accumulators, top-C index sets and
-dequantised outputs and the router-weighted combine; the SwiGLU output and the
-atomic scatter epilogue within the bounds their arithmetic allows (CUDA expf vs
-a correctly rounded exp; atomic accumulation order); the block output within
-the 1e-2 max-relative budget.
+Bar: bit-exact weight codes and scales (fp64 offline quantiser), int32
+accumulators, top-C index sets, dequantised outputs and the router-weighted
+combine, each given the same quantised inputs; the run-time activation and h
+codes (fp32 rotation) within the budget of tests/code_budget.py (at most 1e-4
+of the codes one off, only next to a half-integer, none further); the SwiGLU
+output and the atomic scatter epilogue within the bounds their arithmetic
+allows (CUDA expf vs a correctly rounded exp; atomic accumulation order); the
+block output within the 1e-2 max-relative budget.
 """
 
 import numpy as np
@@ -13,6 +16,7 @@ import torch
 
 import oracle as O
 from synthetic import LINEAR_CONFIGS, MOE_CONFIGS, linear_inputs, moe_inputs
+from tests.code_budget import check_codes
 from tests.golden import read_fixture
 
 pytestmark = pytest.mark.gpu
@@ -58,20 +62,19 @@ def bf16_activations(rows, k, seed, outliers=True):
     (100, 1536, 64), (77, 512, 16), (50, 256, 4), (40, 64, 1), (3, 16, 16), (1, 4096, 64),
     (20000, 2048, 256),  # many more row groups than resident CTAs (persistent loop)
 ])
-def test_rotquant_bf16_bit_exact(rows, k, g):
+def test_rotquant_bf16_within_budget(rows, k, g):
     x = bf16_activations(rows, k, seed=rows * 7 + k)
     q, s = W.convrot_rotquant(x.cuda(), g)
-    q_ref, s_ref = O.rotquant(np32(x), g)
-    assert np.array_equal(s.cpu().numpy(), s_ref)
-    assert np.array_equal(q.cpu().numpy(), q_ref)
+    check_codes(q.cpu().numpy(), s.cpu().numpy(), np32(x), g)
 
 
 @pytest.mark.parametrize("rows,k,g", [(160, 320, 64), (513, 1536, 64), (64, 2048, 256),
                                       (9001, 1536, 64), (3, 192, 64), (11, 8192 - 64, 64)])
-def test_rotquant_f32_bit_exact(rows, k, g):
+def test_rotquant_f32_within_budget(rows, k, g):
     """fp32 rows (the SwiGLU output); K = 320, 1536, 192, 8128 have group
     counts that are not powers of two (one thread per group); the first row
-    is zero and the second below the 2^-120 threshold."""
+    is zero and the second tiny (absmax about 1e-38, below the reciprocal's
+    range: its codes come from the subnormal-capable scale)."""
     gen = torch.Generator().manual_seed(k)
     a = torch.randn(rows, k, generator=gen)
     b = torch.randn(rows, k, generator=gen)
@@ -80,9 +83,25 @@ def test_rotquant_f32_bit_exact(rows, k, g):
     if rows > 1:
         h[1] = h[1] * 1e-38
     q, s = W.convrot_rotquant(h.cuda(), g)
-    q_ref, s_ref = O.rotquant(h.numpy(), g)
-    assert np.array_equal(s.cpu().numpy(), s_ref)
-    assert np.array_equal(q.cpu().numpy(), q_ref)
+    check_codes(q.cpu().numpy(), s.cpu().numpy(), h.numpy(), g)
+    assert float(s[0]) == 0.0 and int(q[0].abs().sum()) == 0
+
+
+def test_rotquant_subnormal_scale_worked_example():
+    """The oracle's hand-worked tiny row (g = 1): a = 2^-140 gives the
+    subnormal s = 2^-147, and the codes 2^-140 / s = 128 and -128 clamp to
+    +-127 while -2^-141 / s = -64; a = 2^-145 gives s = 0 and zero codes."""
+    v = torch.zeros(3, 16)
+    v[1, 2], v[1, 5], v[1, 6] = 2.0 ** -140, -(2.0 ** -141), -(2.0 ** -140)
+    v[2, 0] = 2.0 ** -145
+    q, s = W.convrot_rotquant(v.cuda(), 1)
+    q, s = q.cpu(), s.cpu()
+    assert float(s[1]) == 2.0 ** -147
+    assert q[1, :8].tolist() == [0, 0, 127, 0, 0, -64, -127, 0]
+    assert float(s[0]) == 0.0 and float(s[2]) == 0.0
+    assert int(q[0].abs().sum()) == 0 and int(q[2].abs().sum()) == 0
+    q_ref, s_ref = O.rotquant(v.numpy(), 1)
+    assert np.array_equal(q.numpy(), q_ref) and np.array_equal(s.numpy(), s_ref)
 
 
 def test_rotquant_worked_examples_and_degenerate_rows():
@@ -100,6 +119,19 @@ def test_rotquant_worked_examples_and_degenerate_rows():
     assert q4[1, :8].tolist() == rot["codes"][0]
     assert s4[1].item() == np.float32(13.0 / 127.0)
     assert q4[2].abs().sum().item() == 0
+
+
+@pytest.mark.parametrize("rows,k,g", [(300, 768, 256), (64, 8192, 256), (1000, 1536, 64),
+                                      (77, 512, 16), (50, 256, 4), (40, 64, 1), (3, 16, 16)])
+def test_weight_quantisation_bit_exact(rows, k, g):
+    """The offline quantiser (fp64 rotation and quotients) equals the
+    definition bit for bit: codes and scales, on outlier-laden rows too."""
+    w = bf16_activations(rows, k, seed=rows + 3 * k)
+    w = (w.float() * 0.02).to(torch.bfloat16)
+    q, s = W.convrot_quantize_weights(w.cuda(), g)
+    q_ref, s_ref = O.rotquant(np32(w), g)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
 
 
 def test_weight_quantisation_3d_stack():
@@ -314,7 +346,8 @@ def test_gemm_swiglu(g, m, f, k, layout):
 ])
 def test_gemm_swiglu_rq_matches_two_step(g, m, f, k, g_h, layout):
     """Codes and scales equal the SwiGLU GEMM followed by the rotation kernel
-    bit for bit, and the oracle's rotation + quantiser of that same h."""
+    bit for bit (the same fp32 arithmetic), and the definition's codes of
+    that same h within the budget."""
     a = _codes((g, m, k), 7 + m)
     b = _codes((g, 2 * f, k), 8 + f)
     s_a = (torch.rand(g, m) * 0.05 + 1e-3).cuda()
@@ -327,9 +360,9 @@ def test_gemm_swiglu_rq_matches_two_step(g, m, f, k, g_h, layout):
     assert torch.equal(q1.view(-1, f), q2)
     assert torch.equal(s1.view(-1), s2)
     assert float(s1[0, 3]) == 0.0 and int(q1[0, 3].abs().sum()) == 0
-    q_ref, s_ref = O.rotquant(h.view(-1, f).cpu().numpy(), g_h)
-    assert np.array_equal(q1.view(-1, f).cpu().numpy(), q_ref)
-    assert np.array_equal(s1.view(-1).cpu().numpy(), s_ref)
+    # and the definition's codes of that same h within the budget
+    check_codes(q1.view(-1, f).cpu().numpy(), s1.view(-1).cpu().numpy(),
+                h.view(-1, f).cpu().numpy(), g_h)
 
 
 def test_gemm_swiglu_rq_repeated_calls_reuse_nothing():
@@ -420,31 +453,54 @@ def test_combine_sums_in_expert_order(e_n, t, c, d):
 
 
 # ------------------------------------------------------------------ linear --
+def _linear_with_codes(x, w_q, s_w, g):
+    """The linear through its C-ABI entry, plus the activation codes and
+    scales it left in its workspace."""
+    m, k = x.shape
+    ws = torch.empty(max(W.convrot_linear_workspace_size(m, k), 16), dtype=torch.uint8,
+                     device="cuda")
+    y = W.w8a8_convrot_linear(x, w_q, s_w, g, workspace=ws)
+    torch.cuda.synchronize()
+    x_q = ws[:m * k].view(torch.int8).view(m, k)
+    off = (m * k + 255) // 256 * 256
+    s_x = ws[off:off + 4 * m].view(torch.float32)
+    return y, x_q, s_x
+
+
 @pytest.mark.parametrize("name", ["linear_64x256x256", "gateup_4096x3072x2048",
                                   "down_4096x2048x1536"])
-def test_w8a8_linear_bit_exact(name):
+def test_w8a8_linear_parity(name):
+    """Weights bit-exact; the output bit-exact given the GPU's activation codes;
+    those codes within the budget; the output within 1e-2 of the oracle's."""
     cfg = LINEAR_CONFIGS[name]
     x, w = linear_inputs(cfg)
     w_q, s_w = W.convrot_quantize_weights(w.cuda(), cfg.group)
-    y = W.w8a8_convrot_linear(x.cuda(), w_q, s_w, cfg.group).cpu()
+    y, x_q, s_x = _linear_with_codes(x.cuda(), w_q, s_w, cfg.group)
     w_q_ref, s_w_ref = O.rotquant(np32(w), cfg.group)
     assert np.array_equal(w_q.cpu().numpy(), w_q_ref) and np.array_equal(s_w.cpu().numpy(), s_w_ref)
+    x_q, s_x = x_q.cpu().numpy(), s_x.cpu().numpy()
+    assert np.array_equal(np32(y), O.w8a8_linear_from_codes(x_q, s_x, w_q_ref, s_w_ref))
+    check_codes(x_q, s_x, np32(x), cfg.group)
     y_ref = O.w8a8_linear(np32(x), w_q_ref, s_w_ref, cfg.group)
-    assert np.array_equal(np32(y), y_ref)
+    assert _max_rel(np32(y), y_ref) <= 1e-2
 
 
 @pytest.mark.parametrize("g", [1, 16, 256])
 def test_linear_rotation_off_ablation(g):
     """The rotation-off ablation (g = 1: per-token / per-channel INT8 with no
-    Hadamard) runs through the same kernels, bit-exact with the oracle; on the
-    outlier-laden gate|up inputs the rotation lowers the error against the
-    exact product (the reason for ConvRot)."""
+    Hadamard) runs through the same kernels, with the parity of the ConvRot
+    linear; on the outlier-laden gate|up inputs the rotation lowers the error
+    against the exact product (the reason for ConvRot)."""
     x, w = linear_inputs(LINEAR_CONFIGS["gateup_4096x3072x2048"])
     x, w = x[:256], w[:512]
     w_q, s_w = W.convrot_quantize_weights(w.cuda(), g)
-    y = np32(W.w8a8_convrot_linear(x.cuda(), w_q, s_w, g))
+    y, x_q, s_x = _linear_with_codes(x.cuda(), w_q, s_w, g)
+    y = np32(y)
     w_q_ref, s_w_ref = O.rotquant(np32(w), g)
-    assert np.array_equal(y, O.w8a8_linear(np32(x), w_q_ref, s_w_ref, g))
+    assert np.array_equal(w_q.cpu().numpy(), w_q_ref)
+    x_q, s_x = x_q.cpu().numpy(), s_x.cpu().numpy()
+    assert np.array_equal(y, O.w8a8_linear_from_codes(x_q, s_x, w_q_ref, s_w_ref))
+    check_codes(x_q, s_x, np32(x), g)
     exact = np32(x).astype(np.float64) @ np32(w).astype(np.float64).T
     rel = np.linalg.norm(y - exact) / np.linalg.norm(exact)
     assert rel < {1: 0.06, 16: 0.02, 256: 0.014}[g]
@@ -461,7 +517,7 @@ def test_moe_block_rotation_off():
     ow = _oracle_weights(inp, cfg, range(cfg.n_exp))
     y_ref, it = O.moe_block(np32(inp["x"]), np32(inp["logits"]), *ow, c=cfg.c, g_gu=1, g_d=1,
                             keep=True)
-    assert np.array_equal(v["x_q"].cpu().numpy(), it["x_q"])
+    check_codes(v["x_q"].cpu().numpy(), v["s_x"].cpu().numpy(), np32(inp["x"]), 1)
     assert np.array_equal(v["idx"].cpu().numpy(), it["idx"])
     assert _max_rel(np32(y), y_ref) <= 1e-2
 
@@ -510,6 +566,35 @@ def _max_rel(y, ref):
     return float(np.max(np.abs(y - ref)) / max(np.max(np.abs(ref)), 1e-30))
 
 
+def _check_block_stages(v, inp, cfg, it, experts, wq_ref):
+    """Stage by stage, each GPU stage against the oracle given the GPU's own
+    inputs to it: x codes (budget), routing (exact), h codes (budget, from the
+    oracle's SwiGLU of the GPU's gathered codes), z (bit-exact given the GPU's
+    h codes). Returns the h-code flips and the number of h codes checked."""
+    x_q = v["x_q"].cpu().numpy()
+    s_x = v["s_x"].cpu().numpy()
+    wgu_q, s_gu, wd_q, s_d = wq_ref
+    idx = v["idx"].cpu().numpy()
+    assert np.array_equal(idx, it["idx"])
+    assert np.array_equal(v["w"].cpu().numpy(), it["w"])
+    assert np.array_equal(v["x_g"].cpu().numpy(), x_q[idx])
+    assert np.array_equal(v["s_g"].cpu().numpy(), s_x[idx])
+    flips = codes = 0
+    for e in experts:
+        rows = idx[e]
+        h = O.swiglu_from_codes(x_q[rows], s_x[rows], wgu_q[e], s_gu[e])
+        if cfg.g_d == 256:  # stored fp32 h: SwiGLU within CUDA expf's few ulp
+            assert _fp32_ulps(v["h"][e].cpu().numpy(), h).max() <= 4
+        h_q = v["h_q"][e].cpu().numpy()
+        s_h = v["s_h"][e].cpu().numpy()
+        n, c, _, _ = check_codes(h_q, s_h, h, cfg.g_d, input_err=8.0)
+        flips += n
+        codes += c
+        z = O.down_from_codes(h_q, s_h, wd_q[e], s_d[e])
+        assert np.array_equal(np32(v["z"][e]), z)
+    return flips, codes
+
+
 # g_d = 256 takes the fp32 h + rotation-kernel path (a group of 256 spans
 # four epilogue threads); g_d <= 64 rotates and requantises h in the gate/up
 # GEMM's epilogue and stores no fp32 h.
@@ -528,41 +613,21 @@ def test_moe_block_small_end_to_end(name):
     inp = moe_inputs(cfg)
     y, v, wq = _run_moe(inp, cfg)
     ow = _oracle_weights(inp, cfg, range(cfg.n_exp))
-    for got, ref in zip(wq, ow):
+    for got, ref in zip(wq, ow):  # offline weights: bit-exact
         assert np.array_equal(got.cpu().numpy(), ref)
     y_ref, it = O.moe_block(np32(inp["x"]), np32(inp["logits"]), *ow, c=cfg.c, g_gu=cfg.g_gu,
                             g_d=cfg.g_d, keep=True)
-    # stage by stage
-    assert np.array_equal(v["x_q"].cpu().numpy(), it["x_q"])
-    assert np.array_equal(v["s_x"].cpu().numpy(), it["s_x"])
+    check_codes(v["x_q"].cpu().numpy(), v["s_x"].cpu().numpy(), np32(inp["x"]), cfg.g_gu)
     assert _ulp_diff(v["s_t"].cpu().numpy(), it["scores"].T).max() <= 1
-    assert np.array_equal(v["idx"].cpu().numpy(), it["idx"])
-    assert np.array_equal(v["w"].cpu().numpy(), it["w"])
-    h_q_diff = 0
-    n_codes = 0
-    for e in range(cfg.n_exp):
-        if cfg.g_d == 256:
-            assert _fp32_ulps(v["h"][e].cpu().numpy(), it["h"][e]).max() <= 4
-        dq = np.abs(v["h_q"][e].cpu().numpy().astype(np.int32) - it["h_q"][e].astype(np.int32))
-        assert dq.max() <= 1
-        h_q_diff += int((dq != 0).sum())
-        n_codes += dq.size
-    assert h_q_diff <= max(2, 1e-4 * n_codes)
+    _check_block_stages(v, inp, cfg, it, range(cfg.n_exp), ow)
+    # the combine, bit-exact given the GPU's expert outputs
+    z = {e: np32(v["z"][e]) for e in range(cfg.n_exp)}
     y_np = np32(y)
+    assert np.array_equal(y_np, O.combine(cfg.t, it["idx"], it["w"], z))
+    # and the whole block against the oracle's
     assert _max_rel(y_np, y_ref) <= 1e-2
     unchosen = np.setdiff1d(np.arange(cfg.t), np.unique(it["idx"]))
     assert np.all(y_np[unchosen] == 0)
-    # tokens whose experts' h codes all agree with the oracle come out bit-exact
-    # (same fp32 sum order); only the rare expf-driven code flips can differ
-    touched = set()
-    for e in range(cfg.n_exp):
-        bad = (np.any(v["h_q"][e].cpu().numpy() != it["h_q"][e], axis=1)
-               | (v["s_h"][e].cpu().numpy() != it["s_h"][e]))
-        touched.update(it["idx"][e][bad].tolist())
-        # the experts' bf16 outputs of the rows whose codes agree are bit-exact
-        assert np.array_equal(np32(v["z"][e])[~bad], it["z"][e][~bad])
-    clean = np.setdiff1d(np.arange(cfg.t), np.array(sorted(touched), dtype=np.int64))
-    assert np.array_equal(y_np[clean], y_ref[clean])
 
 
 def test_moe_block_graph_capture_matches_eager():
@@ -609,29 +674,35 @@ def test_moe_block_capacity_extremes():
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name", ["moe_T8192", "moe_T2048"])
-def test_moe_block_full_size_sampled_rows(name):
-    """Full-size block as the bench runs it; the oracle evaluates sampled rows."""
+def test_moe_block_full_size(name):
+    """The full-size block as the bench runs it, every stage at full size:
+    weights bit-exact; all T rows of x codes and all E*C rows of h codes within
+    the budget (h from the oracle's SwiGLU of the GPU's gathered codes); routing
+    exact; every expert output z bit-exact given the GPU's h codes; every
+    output row bit-exact given z; sampled rows within 1e-2 of the oracle's
+    whole block."""
     cfg = MOE_CONFIGS[name]
     inp = moe_inputs(cfg)
     y, v, wq = _run_moe(inp, cfg)
     x_np, logits_np = np32(inp["x"]), np32(inp["logits"])
-    scores = O.router_softmax(logits_np)
-    idx_ref, _ = O.expert_choice_topc(scores, cfg.c)
-    assert np.array_equal(v["idx"].cpu().numpy(), idx_ref)
+    ow = _oracle_weights(inp, cfg, range(cfg.n_exp))
+    for got, ref in zip(wq, ow):
+        assert np.array_equal(got.cpu().numpy(), ref)
+    idx_ref, w_ref = O.expert_choice_topc(O.router_softmax(logits_np), cfg.c)
+    fx, nx, _, _ = check_codes(v["x_q"].cpu().numpy(), v["s_x"].cpu().numpy(), x_np, cfg.g_gu)
+    fh, nh = _check_block_stages(v, inp, cfg, {"idx": idx_ref, "w": w_ref}, range(cfg.n_exp), ow)
+    print(f"\n{name}: x codes off by one {fx} of {nx} ({fx / nx:.2e}); "
+          f"h codes off by one {fh} of {nh} ({fh / nh:.2e})")
+    z = {e: np32(v["z"][e]) for e in range(cfg.n_exp)}
+    y_np = np32(y)
+    assert np.array_equal(y_np, O.combine(cfg.t, idx_ref, w_ref, z))
     counts = np.bincount(idx_ref.ravel(), minlength=cfg.t)
     rng = np.random.default_rng(0)
     busy = np.argsort(-counts, kind="stable")[:8]
     sample = np.unique(np.concatenate([np.arange(8), rng.choice(cfg.t, 16, replace=False), busy]))
-    experts = sorted({e for e in range(cfg.n_exp) if np.isin(idx_ref[e], sample).any()})
-    ow = _oracle_weights(inp, cfg, experts)
-    for e in experts[:4]:
-        assert np.array_equal(wq[0][e].cpu().numpy(), ow[0][e])
-        assert np.array_equal(wq[2][e].cpu().numpy(), ow[2][e])
     y_ref = O.moe_block(x_np, logits_np, *ow, c=cfg.c, g_gu=cfg.g_gu, g_d=cfg.g_d,
                         out_tokens=sample)
-    y_np = np32(y)
     assert _max_rel(y_np[sample], y_ref[sample]) <= 1e-2
-    assert np.array_equal(v["x_q"].cpu().numpy()[sample], O.rotquant(x_np[sample], cfg.g_gu)[0])
 
 
 # ---------------------------------------------------------- failure path --

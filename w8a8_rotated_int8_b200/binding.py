@@ -120,9 +120,21 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream=None):
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+def _stream(stream=None, like=None):
+    """The given stream, else the current stream of `like`'s device (else of
+    the current device)."""
+    if stream is None:
+        stream = torch.cuda.current_stream(None if like is None else like.device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _invoke(t, name, *args, stream=None):
+    """Calls the C entry `name` with `t`'s device current (the library works on
+    the current device) and that device's current stream (or `stream`) as the
+    last argument; raises on a non-OK status."""
+    with torch.cuda.device(t.device):
+        rc = getattr(lib(), name)(*args, _stream(stream, t))
+    _check(rc, name)
 
 
 def _need(t, dtype, name):
@@ -151,7 +163,7 @@ def convrot_check_device_error(stream=None) -> int:
 def convrot_wait_selftest(limit_ns: int, stream=None) -> int:
     """Runs the bounded-wait self-test; returns 0 when the wait gave up."""
     res = torch.full((1,), -1, dtype=torch.int32, device="cuda")
-    _check(lib().convrot_wait_selftest(limit_ns, _p(res), _stream(stream)), "convrot_wait_selftest")
+    _invoke(res, "convrot_wait_selftest", limit_ns, _p(res), stream=stream)
     return int(res.item())
 
 
@@ -166,8 +178,7 @@ def convrot_rotquant(x, group, q=None, scale=None, stream=None):
     q = torch.empty((rows, k), dtype=torch.int8, device=x.device) if q is None else q
     scale = torch.empty((rows,), dtype=torch.float32, device=x.device) if scale is None else scale
     dt = DTYPE_BF16 if x.dtype == torch.bfloat16 else DTYPE_F32
-    _check(lib().convrot_rotquant(_p(x), dt, rows, k, group, _p(q), _p(scale), _stream(stream)),
-           "convrot_rotquant")
+    _invoke(x, "convrot_rotquant", _p(x), dt, rows, k, group, _p(q), _p(scale), stream=stream)
     return q, scale
 
 
@@ -178,8 +189,7 @@ def convrot_quantize_weights(w, group, stream=None):
     rows = w.numel() // k
     q = torch.empty(w.shape, dtype=torch.int8, device=w.device)
     s = torch.empty(w.shape[:-1], dtype=torch.float32, device=w.device)
-    _check(lib().convrot_quantize_weights(_p(w), rows, k, group, _p(q), _p(s), _stream(stream)),
-           "convrot_quantize_weights")
+    _invoke(w, "convrot_quantize_weights", _p(w), rows, k, group, _p(q), _p(s), stream=stream)
     return q, s
 
 
@@ -205,8 +215,8 @@ def convrot_quantize_weights_tiled(w, group, n_mats, stream=None):
     rows = total // n_mats
     data = torch.empty((tiled_weight_bytes(n_mats, rows, k),), dtype=torch.int8, device=w.device)
     scale = torch.empty((total,), dtype=torch.float32, device=w.device)
-    _check(lib().convrot_quantize_weights_tiled(_p(w), n_mats, rows, k, group, _p(data), _p(scale),
-                                                _stream(stream)), "convrot_quantize_weights_tiled")
+    _invoke(w, "convrot_quantize_weights_tiled", _p(w),
+            n_mats, rows, k, group, _p(data), _p(scale), stream=stream)
     return TiledWeights(data, scale, n_mats, rows, k)
 
 
@@ -224,8 +234,7 @@ def convrot_router_softmax(logits, stream=None):
     _need(logits, torch.bfloat16, "logits")
     t, e = logits.shape
     s_t = torch.empty((e, t), dtype=torch.float32, device=logits.device)
-    _check(lib().convrot_router_softmax(_p(logits), t, e, _p(s_t), _stream(stream)),
-           "convrot_router_softmax")
+    _invoke(logits, "convrot_router_softmax", _p(logits), t, e, _p(s_t), stream=stream)
     return s_t
 
 
@@ -237,8 +246,7 @@ def convrot_topc(s_t, c, with_slot=False, stream=None):
     idx = torch.empty((e, c), dtype=torch.int32, device=s_t.device)
     w = torch.empty((e, c), dtype=torch.float32, device=s_t.device)
     slot = torch.empty((e, t), dtype=torch.int32, device=s_t.device) if with_slot else None
-    _check(lib().convrot_topc(_p(s_t), t, e, c, _p(idx), _p(w), _p(slot), _stream(stream)),
-           "convrot_topc")
+    _invoke(s_t, "convrot_topc", _p(s_t), t, e, c, _p(idx), _p(w), _p(slot), stream=stream)
     return (idx, w, slot) if with_slot else (idx, w)
 
 
@@ -252,8 +260,7 @@ def convrot_combine_rows(z, s_t, slot, c, stream=None):
     e, t = slot.shape
     d = z.shape[-1]
     y = torch.empty((t, d), dtype=torch.bfloat16, device=slot.device)
-    _check(lib().convrot_combine_rows(_p(z), _p(s_t), _p(slot), e, t, c, d, _p(y),
-                                      _stream(stream)), "convrot_combine_rows")
+    _invoke(z, "convrot_combine_rows", _p(z), _p(s_t), _p(slot), e, t, c, d, _p(y), stream=stream)
     return y
 
 
@@ -265,8 +272,8 @@ def convrot_gather_rows(src, s_src, idx, stream=None):
     n = idx.numel()
     dst = torch.empty((n, k), dtype=torch.int8, device=src.device)
     s_dst = torch.empty((n,), dtype=torch.float32, device=src.device)
-    _check(lib().convrot_gather_rows(_p(src), _p(s_src), n_src, _p(idx), n, k, _p(dst), _p(s_dst),
-                                     _stream(stream)), "convrot_gather_rows")
+    _invoke(src, "convrot_gather_rows", _p(src),
+            _p(s_src), n_src, _p(idx), n, k, _p(dst), _p(s_dst), stream=stream)
     return dst, s_dst
 
 
@@ -295,8 +302,7 @@ def convrot_i8_gemm_i32(a, b, stream=None):
     """Exact int32 acc[g, m, n] = sum_k a[g, m, k] b[g, n, k]."""
     g, m, n, k, bt, lay = _gemm_dims(a, b)
     d = torch.empty((g, m, n), dtype=torch.int32, device=a.device)
-    _check(lib().convrot_i8_gemm_i32(_p(a), _p(bt), lay, g, m, n, k, _p(d), _stream(stream)),
-           "convrot_i8_gemm_i32")
+    _invoke(a, "convrot_i8_gemm_i32", _p(a), _p(bt), lay, g, m, n, k, _p(d), stream=stream)
     return d if a.dim() == 3 else d[0]
 
 
@@ -305,8 +311,8 @@ def convrot_i8_gemm_bf16(a, s_a, b, s_b, stream=None):
     _need(s_a, torch.float32, "s_a")
     _need(s_b, torch.float32, "s_b")
     y = torch.empty((g, m, n), dtype=torch.bfloat16, device=a.device)
-    _check(lib().convrot_i8_gemm_bf16(_p(a), _p(s_a), _p(bt), _p(s_b), lay, g, m, n, k, _p(y),
-                                      _stream(stream)), "convrot_i8_gemm_bf16")
+    _invoke(a, "convrot_i8_gemm_bf16", _p(a),
+            _p(s_a), _p(bt), _p(s_b), lay, g, m, n, k, _p(y), stream=stream)
     return y if a.dim() == 3 else y[0]
 
 
@@ -318,8 +324,8 @@ def convrot_i8_gemm_swiglu(a, s_a, b, s_b, stream=None):
     _need(s_b, torch.float32, "s_b")
     f = n2 // 2
     h = torch.empty((g, m, f), dtype=torch.float32, device=a.device)
-    _check(lib().convrot_i8_gemm_swiglu(_p(a), _p(s_a), _p(bt), _p(s_b), lay, g, m, f, k, _p(h),
-                                        _stream(stream)), "convrot_i8_gemm_swiglu")
+    _invoke(a, "convrot_i8_gemm_swiglu", _p(a),
+            _p(s_a), _p(bt), _p(s_b), lay, g, m, f, k, _p(h), stream=stream)
     return h if a.dim() == 3 else h[0]
 
 
@@ -334,9 +340,8 @@ def convrot_i8_gemm_swiglu_rq(a, s_a, b, s_b, g_h=64, stream=None):
     s_h = torch.empty((g, m), dtype=torch.float32, device=a.device)
     nbytes = lib().convrot_swiglu_rq_sync_bytes(g, m)
     sync = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=a.device)
-    _check(lib().convrot_i8_gemm_swiglu_rq(_p(a), _p(s_a), _p(bt), _p(s_b), lay, g, m, f, k, g_h,
-                                           _p(h_q), _p(s_h), _p(sync), nbytes, _stream(stream)),
-           "convrot_i8_gemm_swiglu_rq")
+    _invoke(a, "convrot_i8_gemm_swiglu_rq", _p(a), _p(s_a), _p(bt), _p(s_b), lay, g, m, f, k,
+            g_h, _p(h_q), _p(s_h), _p(sync), nbytes, stream=stream)
     return (h_q, s_h) if a.dim() == 3 else (h_q[0], s_h[0])
 
 
@@ -346,17 +351,15 @@ def convrot_i8_gemm_scatter(a, s_a, b, s_b, idx, w, out32, stream=None):
     for t, nm in ((s_a, "s_a"), (s_b, "s_b"), (w, "w"), (out32, "out32")):
         _need(t, torch.float32, nm)
     _need(idx, torch.int32, "idx")
-    _check(lib().convrot_i8_gemm_scatter(_p(a), _p(s_a), _p(bt), _p(s_b), lay, _p(idx), _p(w), g, m,
-                                         n, k, _p(out32), out32.shape[0], _stream(stream)),
-           "convrot_i8_gemm_scatter")
+    _invoke(a, "convrot_i8_gemm_scatter", _p(a), _p(s_a), _p(bt), _p(s_b), lay, _p(idx),
+            _p(w), g, m, n, k, _p(out32), out32.shape[0], stream=stream)
     return out32
 
 
 def convrot_f32_to_bf16(x, stream=None):
     _need(x, torch.float32, "x")
     y = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
-    _check(lib().convrot_f32_to_bf16(_p(x), x.numel(), _p(y), _stream(stream)),
-           "convrot_f32_to_bf16")
+    _invoke(x, "convrot_f32_to_bf16", _p(x), x.numel(), _p(y), stream=stream)
     return y
 
 
@@ -377,9 +380,8 @@ def w8a8_convrot_linear(x, w_q, w_scale, group, y=None, workspace=None, stream=N
         workspace = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=x.device)
     if y is None:
         y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
-    _check(lib().w8a8_convrot_linear(_p(x), m, k, _p(w_q), _p(w_scale), n, group, _p(y),
-                                     _p(workspace), workspace.numel(), _stream(stream)),
-           "w8a8_convrot_linear")
+    _invoke(x, "w8a8_convrot_linear", _p(x), m, k, _p(w_q), _p(w_scale), n, group, _p(y),
+            _p(workspace), workspace.numel(), stream=stream)
     return y
 
 
@@ -395,8 +397,8 @@ def w8a8_convrot_linear_noalloc(x, w_q, w_scale, group, y=None, stream=None):
     n = w_q.shape[0]
     if y is None:
         y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
-    _check(lib().w8a8_convrot_linear_noalloc(_p(x), m, k, _p(w_q), _p(w_scale), n, group, _p(y),
-                                             _stream(stream)), "w8a8_convrot_linear_noalloc")
+    _invoke(x, "w8a8_convrot_linear_noalloc", _p(x),
+            m, k, _p(w_q), _p(w_scale), n, group, _p(y), stream=stream)
     return y
 
 
@@ -437,10 +439,9 @@ def moe_expert_choice_forward(x, logits, w_gu, w_d, c, g_gu=256, g_d=64, y=None,
         workspace = torch.empty((max(size, 16),), dtype=torch.uint8, device=x.device)
     if y is None:
         y = torch.empty((t, d), dtype=torch.bfloat16, device=x.device)
-    _check(lib().moe_expert_choice_forward(_p(x), _p(logits), _p(w_gu), _p(s_gu), _p(w_d), _p(s_d),
-                                           t, d, f, e, c, g_gu, g_d, _p(y), _p(workspace),
-                                           workspace.numel(), _stream(stream)),
-           "moe_expert_choice_forward")
+    _invoke(x, "moe_expert_choice_forward", _p(x), _p(logits), _p(w_gu), _p(s_gu), _p(w_d),
+            _p(s_d), t, d, f, e, c, g_gu, g_d, _p(y), _p(workspace), workspace.numel(),
+            stream=stream)
     return y
 
 

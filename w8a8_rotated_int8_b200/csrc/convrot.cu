@@ -353,6 +353,43 @@ int rotquant_impl(const void* x, int x_dtype, int64_t rows, int64_t K, int group
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// The offline weight quantiser: fp64 rotation and quotients (the definition
+// exactly), one persistent CTA per row at a time, the row in shared memory.
+template <int G>
+int launch_rq_f64(const void* w, int64_t rows, int K, int8_t* q, float* s, RqOut out,
+                  cudaStream_t st) {
+  auto kern = rotquant_f64_kernel<G>;
+  const size_t smem = (size_t)K * sizeof(double);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRq64Threads, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  int sms = 0;
+  device_setup(&sms);
+  const int64_t grid = std::min<int64_t>(rows, (int64_t)per_sm * std::max(sms, 1));
+  return launch_kernel(kern, dim3((unsigned)grid), dim3(kRq64Threads), smem, st, false, 1,
+                       reinterpret_cast<const __nv_bfloat16*>(w), rows, K, q, s, out);
+}
+
+int quantize_weights_impl(const void* w, int64_t rows, int64_t K, int group, int8_t* q, float* s,
+                          cudaStream_t st, RqOut out) {
+  if (rows == 0) return CONVROT_OK;
+  int rc;
+  switch (group) {
+    case 1: rc = launch_rq_f64<1>(w, rows, (int)K, q, s, out, st); break;
+    case 4: rc = launch_rq_f64<4>(w, rows, (int)K, q, s, out, st); break;
+    case 16: rc = launch_rq_f64<16>(w, rows, (int)K, q, s, out, st); break;
+    case 64: rc = launch_rq_f64<64>(w, rows, (int)K, q, s, out, st); break;
+    default: rc = launch_rq_f64<256>(w, rows, (int)K, q, s, out, st); break;
+  }
+  if (rc != CONVROT_OK) return rc;
+  return launch_status();
+}
+
 // Bytes of the tiled weight format for n_mats matrices of `rows` x K.
 int64_t tiled_bytes(int64_t n_mats, int64_t rows, int64_t K) {
   return n_mats * cdiv(rows, 128) * cdiv(K, 128) * 16384;
@@ -689,7 +726,11 @@ int convrot_rotquant(const void* x, int x_dtype, int64_t rows, int64_t K, int gr
 
 int convrot_quantize_weights(const void* w_bf16, int64_t rows, int64_t K, int group, int8_t* w_q,
                              float* row_scale, void* stream) {
-  return convrot_rotquant(w_bf16, CONVROT_DTYPE_BF16, rows, K, group, w_q, row_scale, stream);
+  int rc = check_rq_args(w_bf16, CONVROT_DTYPE_BF16, rows, K, group, w_q, row_scale);
+  if (rc != CONVROT_OK) return rc;
+  if ((rc = device_setup(nullptr)) != CONVROT_OK) return rc;
+  return quantize_weights_impl(w_bf16, rows, K, group, w_q, row_scale, as_stream(stream),
+                               RqOut{0, 1, 1, 1});
 }
 
 int64_t convrot_tiled_weight_bytes(int64_t n_mats, int64_t rows, int64_t K) {
@@ -709,8 +750,7 @@ int convrot_quantize_weights_tiled(const void* w_bf16, int64_t n_mats, int64_t r
   if (cudaMemsetAsync(w_tiled, 0, (size_t)tiled_bytes(n_mats, rows, K), st) != cudaSuccess)
     return CONVROT_ERR_CUDA;
   const RqOut out{1, rows, (int)cdiv(rows, 128), (int)cdiv(K, 128)};
-  return rotquant_impl(w_bf16, CONVROT_DTYPE_BF16, n_mats * rows, K, group, w_tiled, row_scale, st,
-                       out);
+  return quantize_weights_impl(w_bf16, n_mats * rows, K, group, w_tiled, row_scale, st, out);
 }
 
 int convrot_router_softmax(const void* logits_bf16, int64_t T, int E, float* s_t, void* stream) {
@@ -1069,6 +1109,19 @@ struct NoAllocSlot {
 NoAllocSlot g_noalloc_slot[kMaxDevices];
 std::mutex g_noalloc_mu;
 
+// Whether p is device (or managed) memory that the current device can use as
+// its own: allocated on it, or managed.
+bool on_current_device(const void* p) {
+  int dev = 0;
+  cudaPointerAttributes at;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (at.type == cudaMemoryTypeManaged) return true;
+  return at.type == cudaMemoryTypeDevice && at.device == dev;
+}
+
 // Device address of the scratch array for the current device, looked up once
 // per device (host code cannot use the array's name as a device pointer).
 int noalloc_scratch(void** out) {
@@ -1097,15 +1150,18 @@ int noalloc_scratch(void** out) {
 extern "C" int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_t K,
                                            const int8_t* w_q, const float* w_scale, int64_t N,
                                            int group, void* y_bf16, void* stream) {
-  if (M < 0 || K < 0) return CONVROT_ERR_INVALID_ARG;
-  if (M > CONVROT_NOALLOC_MAX_ROWS || M * K > (int64_t)CONVROT_NOALLOC_MAX_CODES)
-    return CONVROT_ERR_WORKSPACE_TOO_SMALL;
   int rc = check_rq_args(x_bf16, CONVROT_DTYPE_BF16, M, K, group, w_q, w_scale);
   if (rc != CONVROT_OK) return rc;
   if ((rc = check_gemm_shape(w_q, w_q, 1, M, N, K)) != CONVROT_OK) return rc;
   if (M > 0 && N > 0 && (!w_scale || !y_bf16)) return CONVROT_ERR_INVALID_ARG;
   if (!al16(w_scale) || !al16(y_bf16)) return CONVROT_ERR_MISALIGNED;
+  // K <= 8192 and M < 2^31 hold here, so M * K cannot overflow
+  if (M > CONVROT_NOALLOC_MAX_ROWS || M * K > (int64_t)CONVROT_NOALLOC_MAX_CODES)
+    return CONVROT_ERR_WORKSPACE_TOO_SMALL;
   if ((rc = device_setup(nullptr)) != CONVROT_OK) return rc;
+  // the scratch is the current device's: the caller's buffers must be there too
+  if (M > 0 && N > 0 && (!on_current_device(x_bf16) || !on_current_device(y_bf16)))
+    return CONVROT_ERR_INVALID_ARG;
   void* scratch = nullptr;
   if ((rc = noalloc_scratch(&scratch)) != CONVROT_OK) return rc;
   if (M == 0 || N == 0) return CONVROT_OK;

@@ -5,24 +5,35 @@
 // (ConvRot) and quantised to symmetric INT8 with nearest rounding and one
 // FP32 scale per row. "NitroFusion2 for ComfyUI: int8, W6A8, W4A8", section
 // "How they were made": block Hadamard rotation, one scale per row, 8-bit
-// activations, with the rotation and rounding done in fp32. The same
-// operation serves the weights (offline, per output row), the activations
-// (per token) and the SwiGLU output before the down projection.
+// activations. The definition (Sylvester Hadamard, natural order):
+//   v' = v . blockdiag(H_g / sqrt(g)),  a = max|v'|,
+//   s  = fp32(a / 127),  q = clamp(rne(v' / s), -127, 127)  (s = 0: q = 0).
 //
-// Arithmetic (fp32, IEEE, no contraction):
-//   rotation  fast Walsh-Hadamard butterflies (a + b, a - b) with spans
-//             1, 2, ..., g/2 in that order, then v' = v * (1/sqrt(g)) (a
-//             power of two for g a power of four);
-//   scale     a = max|v'|, s = a / 127, r = 127 / a (one IEEE division each);
-//   codes     q = rint(v' * r), ties to even (|v' * r| <= 127 (1 + 2^-24), so
-//             the code never leaves [-127, 127]);
-//   a row with a < 2^-120 gets s = 0 and all-zero codes.
+// Two implementations:
+//  * rotquant_f64_kernel (offline weights): the rotation and the quotient in
+//    fp64, which reproduces the definition exactly: the butterflies of bf16
+//    values are exact sums (while a group's exponent spread stays under ~37
+//    bits), the scale is the fp64 quotient rounded once to fp32, and every
+//    code is rne of a correctly rounded fp64 quotient.
+//  * rotquant_kernel / rotquant_tma_kernel (activations and h, on the hot
+//    path): fp32 arithmetic, IEEE, no contraction --
+//      rotation  butterflies (a + b, a - b), spans 1, 2, ..., g/2, then
+//                v' = v * (1/sqrt(g)) (a power of two for g a power of four);
+//      scale     s = a / 127 (one IEEE division; subnormal or 0 for tiny a);
+//      codes     q = rint(v' * r) with r = 127 / a while a >= 2^-100 (then
+//                |v' r| <= 127 (1 + 2^-23): the code never leaves
+//                [-127, 127]); below that q = clamp(rint(v' / s)) through an
+//                exactly rescaled reciprocal, so a subnormal s is honoured;
+//                s = 0 gives all-zero codes.
+//    These codes differ from the definition's only where v'/s lies within
+//    the fp32 rounding error of a half-integer (a flip of one, at most).
 //
-// Layout: each thread owns 16 consecutive elements of a row (one 32-byte bf16
-// or 64-byte fp32 load, one 16-byte code store). Spans 1..8 are butterflies
-// in registers; the larger spans pair 16-element chunks held by lanes whose
-// indices differ in one bit, exchanged with warp shuffles (a row's chunks sit
-// in consecutive lanes, so chunk i and chunk i ^ d are lane and lane ^ d).
+// Layout of the fp32 forms: each thread owns 16 consecutive elements of a
+// row (one 32-byte bf16 or 64-byte fp32 load, one 16-byte code store). Spans
+// 1..8 are butterflies in registers; the larger spans pair 16-element chunks
+// held by lanes whose indices differ in one bit, exchanged with warp shuffles
+// (a row's chunks sit in consecutive lanes, so chunk i and chunk i ^ d are
+// lane and lane ^ d).
 #pragma once
 
 #include "common.cuh"
@@ -74,6 +85,29 @@ struct RqTraits {
   static constexpr int kLaneSpanEnd = G >= 16 ? G / 16 : 1;  // lane distances 1 .. kLaneSpanEnd/2
   static constexpr float kInvSqrt = G == 1 ? 1.0f : G == 4 ? 0.5f : G == 16 ? 0.25f : G == 64 ? 0.125f : 0.0625f;
 };
+
+// Rows whose absmax a is at least this use the reciprocal r = 127 / a (finite
+// and normal); the codes of smaller rows come from their (possibly subnormal)
+// scale s: q = clamp(rint((v * 2^100) * r2)), r2 = 1 / (s * 2^100), where both
+// products by 2^100 are exact and s * 2^100 is a normal number.
+constexpr float kRqRecipMin = 7.888609052210118e-31f;  // 2^-100
+constexpr float kRqTinyLift = 1.2676506002282294e+30f;  // 2^100
+
+// r2 of a tiny row (0 when s is 0: every code is then 0).
+__device__ __forceinline__ float rq_tiny_recip(float s) {
+  return s == 0.0f ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(s, kRqTinyLift));
+}
+
+__device__ __forceinline__ int rq_code_tiny(float v, float r2) {
+  const int c = __float2int_rn(__fmul_rn(__fmul_rn(v, kRqTinyLift), r2));
+  return c > 127 ? 127 : (c < -127 ? -127 : c);
+}
+
+// Bits of the rounding add whose low byte is the code rint(v * r) (|v r| <=
+// 127.5): v r + 1.5 * 2^23 rounds to nearest even at the unit.
+__device__ __forceinline__ uint32_t rq_code_bits(float v, float r) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(v, r), 12582912.0f));
+}
 
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
   return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
@@ -194,15 +228,19 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x
     }
     m = rq_row_max(m, tpr, red[it & 1]);
 
-    const bool nonzero = m >= 7.52316384526264e-37f;  // 2^-120
-    const float s = nonzero ? __fdiv_rn(m, 127.0f) : 0.0f;
-    const float r = nonzero ? __fdiv_rn(127.0f, m) : 0.0f;
+    const float s = __fdiv_rn(m, 127.0f);
+    const bool recip = m >= kRqRecipMin;
+    const float r = recip ? __fdiv_rn(127.0f, m) : 0.0f;
     if (active) {
-      // rint by adding 1.5 * 2^23 (the fp32 add rounds to nearest even)
       int k[16];
+      if (recip) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
-        k[j] = __float_as_int(__fadd_rn(__fmul_rn(v[j], r), 12582912.0f)) - 0x4B400000;
+        for (int j = 0; j < 16; ++j) k[j] = (int)rq_code_bits(v[j], r) - 0x4B400000;
+      } else {
+        const float r2 = rq_tiny_recip(s);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) k[j] = rq_code_tiny(v[j], r2);
+      }
       uint4 c;
       c.x = pack4(k[0], k[1], k[2], k[3]);
       c.y = pack4(k[4], k[5], k[6], k[7]);
@@ -298,24 +336,35 @@ __device__ __forceinline__ void rq_lane64(unsigned long long (&p)[32], bool acti
 #pragma unroll
   for (int off = SEG >> 1; off > 0; off >>= 1)
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  const bool nonzero = mx >= 7.52316384526264e-37f;  // 2^-120
-  const float sc = nonzero ? __fdiv_rn(mx, 127.0f) : 0.0f;
-  const float r = nonzero ? __fdiv_rn(127.0f, mx) : 0.0f;
+  const float sc = __fdiv_rn(mx, 127.0f);
+  const bool recip = mx >= kRqRecipMin;
+  const float r = recip ? __fdiv_rn(127.0f, mx) : 0.0f;
   if (active) {
     // rint by adding 1.5 * 2^23: the code is the low byte of the sum's bits.
     // Scalar intrinsics on purpose: a packed mul.rn.f32x2 followed by a
     // packed add.rn.f32x2 was contracted into one fma (the product then is
     // not rounded to fp32 before the rint).
     uint32_t cw[16];
+    if (recip) {
 #pragma unroll
-    for (int m = 0; m < 32; m += 2) {
-      const float2 a = f2_unpack(p[m]);
-      const float2 b = f2_unpack(p[m + 1]);
-      const uint32_t c0 = __float_as_uint(__fadd_rn(__fmul_rn(a.x, r), 12582912.0f));
-      const uint32_t c1 = __float_as_uint(__fadd_rn(__fmul_rn(a.y, r), 12582912.0f));
-      const uint32_t c2 = __float_as_uint(__fadd_rn(__fmul_rn(b.x, r), 12582912.0f));
-      const uint32_t c3 = __float_as_uint(__fadd_rn(__fmul_rn(b.y, r), 12582912.0f));
-      cw[m >> 1] = __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
+      for (int m = 0; m < 32; m += 2) {
+        const float2 a = f2_unpack(p[m]);
+        const float2 b = f2_unpack(p[m + 1]);
+        const uint32_t c0 = rq_code_bits(a.x, r);
+        const uint32_t c1 = rq_code_bits(a.y, r);
+        const uint32_t c2 = rq_code_bits(b.x, r);
+        const uint32_t c3 = rq_code_bits(b.y, r);
+        cw[m >> 1] = __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
+      }
+    } else {
+      const float r2 = rq_tiny_recip(sc);
+#pragma unroll
+      for (int m = 0; m < 32; m += 2) {
+        const float2 a = f2_unpack(p[m]);
+        const float2 b = f2_unpack(p[m + 1]);
+        cw[m >> 1] = pack4(rq_code_tiny(a.x, r2), rq_code_tiny(a.y, r2), rq_code_tiny(b.x, r2),
+                           rq_code_tiny(b.y, r2));
+      }
     }
 #pragma unroll
     for (int c = 0; c < 4; ++c)
@@ -434,6 +483,85 @@ __global__ void __launch_bounds__(kRqTmaWarps * 32, 2) rotquant_tma_kernel(
       }
     }
     __syncwarp();
+  }
+}
+
+// ------------------------------------------------------ fp64 (offline) --
+// The definition exactly, for bf16 weight rows (see the top of this file):
+// one CTA per row at a time (persistent over rows b, b + gridDim.x, ...), the
+// row held in shared memory as fp64, butterflies stage by stage over the
+// whole row (spans 1 .. G/2 stay inside each contiguous group of G), the
+// exact scaling by 1/sqrt(G), a block maximum, s = fp32(a / 127) from the
+// correctly rounded fp64 quotient, codes rne(v' / s) from correctly rounded
+// fp64 quotients, clamped to [-127, 127]. K % 16 == 0; dynamic shared memory
+// K * 8 bytes.
+constexpr int kRq64Threads = 256;
+
+template <int G>
+__global__ void __launch_bounds__(kRq64Threads) rotquant_f64_kernel(
+    const __nv_bfloat16* __restrict__ x, int64_t rows, int K, int8_t* __restrict__ q,
+    float* __restrict__ scales, RqOut out) {
+  extern __shared__ double row_s[];
+  __shared__ double red[kRq64Threads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const double inv = (double)RqTraits<G>::kInvSqrt;  // 1/sqrt(G), a power of two
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + row * K);
+    for (int i = tid; i < K / 8; i += kRq64Threads) {
+      const uint4 u = __ldg(src + i);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        row_s[8 * i + 2 * k] = (double)__uint_as_float(w[k] << 16);
+        row_s[8 * i + 2 * k + 1] = (double)__uint_as_float(w[k] & 0xFFFF0000u);
+      }
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int span = 1; span < G; span <<= 1) {
+      for (int p = tid; p < K / 2; p += kRq64Threads) {
+        const int i = ((p & ~(span - 1)) << 1) | (p & (span - 1));
+        const double a = row_s[i], b = row_s[i + span];
+        row_s[i] = __dadd_rn(a, b);
+        row_s[i + span] = __dsub_rn(a, b);
+      }
+      __syncthreads();
+    }
+    double m = 0.0;
+    for (int i = tid; i < K; i += kRq64Threads) {
+      const double v = __dmul_rn(row_s[i], inv);
+      row_s[i] = v;
+      m = fmax(m, fabs(v));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    m = 0.0;
+#pragma unroll
+    for (int w = 0; w < kRq64Threads / 32; ++w) m = fmax(m, red[w]);
+    const float s = __double2float_rn(__ddiv_rn(m, 127.0));
+    const double sd = (double)s;
+    for (int c = tid; c < K / 16; c += kRq64Threads) {
+      int k[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        int code = 0;
+        if (s != 0.0f) {
+          code = __double2int_rn(__ddiv_rn(row_s[16 * c + j], sd));
+          code = code > 127 ? 127 : (code < -127 ? -127 : code);
+        }
+        k[j] = code;
+      }
+      uint4 cv;
+      cv.x = pack4(k[0], k[1], k[2], k[3]);
+      cv.y = pack4(k[4], k[5], k[6], k[7]);
+      cv.z = pack4(k[8], k[9], k[10], k[11]);
+      cv.w = pack4(k[12], k[13], k[14], k[15]);
+      *reinterpret_cast<uint4*>(q + rq_dst(out, row, K, 16 * c)) = cv;
+    }
+    if (tid == 0) scales[row] = s;
+    __syncthreads();  // the row buffer and red[] are reused by the next row
   }
 }
 
