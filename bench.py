@@ -6,7 +6,15 @@ h rotate+requantise in its epilogue, down GEMM to bf16, router-weighted
 combine) over one batch of synthetic tokens, through the C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config moe_T8192]
-                    [--impl ours|reference] [--no-cpu-baseline] [--ablation] [--sweep]
+                    [--impl ours|reference] [--no-cpu-baseline] [--no-extras]
+                    [--ablation] [--sweep]
+
+The JSON line reports the configured block (default T=8192), and under
+"workloads" the same block at T=2048 (the weight-bound regime, with its
+fraction of HBM bandwidth) and at every T of the 512..8192 sweep, the single
+W8A8 ConvRot linears (gate|up 4096x3072x2048, down 4096x2048x1536, and
+64x256x256) with their fraction of the INT8 tensor peak, and a dense INT8
+GEMM probe of the tensor peak this library's own kernel reaches.
 
 Multi-GPU (launched by torch.distributed.run): every rank runs its own batch
 of T tokens against the same weights (weak scaling, no data-path
@@ -31,17 +39,50 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synthetic import MOE_CONFIGS, moe_inputs  # noqa: E402
+from synthetic import LINEAR_CONFIGS, MOE_CONFIGS, linear_inputs, moe_inputs  # noqa: E402
 
 METRIC = "W8A8 ConvRot MoE block tokens/s"
-# dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
-# kernel (the gate/up GEMM with the requantising SwiGLU epilogue), from ncu
-# captures of the block call at T=8192 and T=2048 (their summaries are under
-# profiles/); to be dropped whenever that kernel changes
-DOMINANT_TRAFFIC_BYTES = {"moe_T8192": 437.2e6 + 5.5e6,
-                          "moe_T2048": 411.9e6 + 7.0e6}
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
+INT8_DATASHEET_TOPS = 4500.0  # B200 dense INT8, nominal (context only)
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+def source_sha16():
+    """Hash of the CUDA sources and the ABI header: a traffic figure captured
+    by ncu on other sources no longer describes the kernel."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "w8a8_rotated_int8_b200", "csrc")
+    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    for path in files + [os.path.join(ROOT, "include", "convrot.h")]:
+        with open(path, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel, workload):
+    """dram__bytes_read.sum + dram__bytes_write.sum per launch of `kernel` on
+    `workload`, from a record line of a summary under profiles/:
+        traffic-record: kernel=<k> workload=<w> bytes_per_launch=<n> source_sha16=<h>
+    Returns (bytes or None, note)."""
+    if not os.path.isdir(PROFILES):
+        return None, "no profiles directory"
+    sha = source_sha16()
+    found = None
+    for name in sorted(os.listdir(PROFILES)):
+        with open(os.path.join(PROFILES, name)) as fh:
+            for line in fh:
+                if not line.startswith("traffic-record:"):
+                    continue
+                kv = dict(part.split("=", 1) for part in line.split()[1:] if "=" in part)
+                if kv.get("kernel") == kernel and kv.get("workload") == workload:
+                    found = (float(kv["bytes_per_launch"]), kv.get("source_sha16"), name)
+    if found is None:
+        return None, "no ncu capture of this kernel on this workload"
+    if found[1] != sha:
+        return None, f"kernel sources changed since the capture in profiles/{found[2]}"
+    return found[0], f"ncu capture, profiles/{found[2]}"
 
 
 def load_peaks():
@@ -57,7 +98,12 @@ def load_peaks():
 
 
 def algorithmic_work(cfg, t):
-    """Ops and compulsory bytes of one block call and of its two GEMM launches."""
+    """Ops and compulsory bytes of one block call and of its two GEMM launches.
+
+    The roofline bytes of a GEMM (``*_alg``) are its weights once plus their
+    scales: gathered and intermediate copies are not algorithmic traffic.
+    ``gateup``/``gateup_rq``/``down`` also count what the launch reads and
+    writes of its activations (as-built bytes, for context)."""
     e, c, d, f = cfg.n_exp, cfg.c, cfg.d, cfg.f
     w_bytes = e * (2 * f * d + d * f)
     s_bytes = e * (2 * f + d) * 4
@@ -78,8 +124,26 @@ def algorithmic_work(cfg, t):
         # weights + scales + h codes and scales in + bf16 rows out
         "bytes": e * d * f + e * d * 4 + e * c * (f + 4) + e * c * d * 2,
     }
+    gateup_alg = {"ops": gateup["ops"], "bytes": e * 2 * f * d + e * 2 * f * 4}
+    down_alg = {"ops": down["ops"], "bytes": e * d * f + e * d * 4}
     return {"ops": ops, "block_bytes": block_bytes, "gateup": gateup, "gateup_rq": gateup_rq,
-            "down": down}
+            "down": down, "gateup_alg": gateup_alg, "down_alg": down_alg}
+
+
+def roofline_of(ops, nbytes, seconds, peaks):
+    """Both fractions of one launch (or call): achieved bytes/s against the
+    measured HBM copy bandwidth and ops/s against the INT8 tensor peak (2 x
+    the measured bf16 burst, the nominal int8:bf16 ratio); the bound is the
+    larger of the two ideal times."""
+    int8 = 2.0 * peaks["bf16_tflops"]
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = ops / (int8 * 1e12)
+    gbs = nbytes / seconds / 1e9
+    tops = ops / seconds / 1e12
+    return {"bound": "hbm" if t_hbm >= t_tc else "tensor",
+            "ideal_us": max(t_hbm, t_tc) * 1e6, "roofline_frac": max(t_hbm, t_tc) / seconds,
+            "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+            "tops": tops, "tensor_frac": tops / int8, "tensor_frac_datasheet": tops / INT8_DATASHEET_TOPS}
 
 
 def fused_h(cfg):
@@ -90,7 +154,7 @@ def fused_h(cfg):
 
 class ClockSampler:
     """SM clock and clock-event reasons sampled (read-only, NVML) by a thread
-    every ~2 ms while the timed region runs; nvidia-smi if NVML is missing."""
+    every ~0.5 ms while the timed region runs."""
 
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
@@ -126,7 +190,7 @@ class ClockSampler:
                 self.samples.append((mhz, rs))
             except Exception:  # noqa: BLE001 - sampling is best effort
                 pass
-            self.stop_evt.wait(0.002)
+            self.stop_evt.wait(0.0005)
 
     def start(self):
         import threading
@@ -378,7 +442,91 @@ def stage_times(W, ws_views, inp_dev, wq, cfg, t, reps, flush_buf):
     return out
 
 
-def run_ours(args, cfg, world, rank, local):
+def timed(fn, steps, flush_buf, stream):
+    """Device seconds of each of `steps` calls of fn (L2 flushed before each,
+    outside the events; CUDA events on the launching stream)."""
+    out = []
+    for _ in range(steps):
+        flush_buf.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        out.append(a.elapsed_time(b) * 1e-3)
+    return out
+
+
+def block_workload(W, cfg, wq, ws, flush_buf, steps, warmup, dev, stream):
+    """The block at cfg's T on cfg's own tokens and logits, with the weights
+    wq (the same model at every T). Returns its measurements."""
+    inp = moe_inputs(cfg, weights=False)
+    x, logits = inp["x"].to(dev), inp["logits"].to(dev)
+    y = torch.empty((cfg.t, cfg.d), dtype=torch.bfloat16, device=dev)
+    gu, dn = wq
+
+    def step():
+        W.moe_expert_choice_forward(x, logits, gu, dn, cfg.c, cfg.g_gu, cfg.g_d, y=y, workspace=ws)
+
+    timed(step, warmup, flush_buf, stream)
+    st = statistics.mean(timed(step, steps, flush_buf, stream))
+    work = algorithmic_work(cfg, cfg.t)
+    return {"tokens": cfg.t, "capacity": cfg.c, "ms_per_step": st * 1e3, "tokens_per_s": cfg.t / st,
+            "block": roofline_of(work["ops"], work["block_bytes"], st, load_peaks())}
+
+
+def linear_workloads(W, flush_buf, reps, dev, stream):
+    """The single W8A8 ConvRot linears through w8a8_convrot_linear (rotation +
+    GEMM), and the GEMM alone on the same codes (convrot_i8_gemm_bf16)."""
+    peaks = load_peaks()
+    out = {}
+    for name, cfg in LINEAR_CONFIGS.items():
+        x, w = linear_inputs(cfg)
+        x, w = x.to(dev), w.to(dev)
+        w_q, s_w = W.convrot_quantize_weights(w, cfg.group)
+        ws = torch.empty(max(W.convrot_linear_workspace_size(cfg.m, cfg.k), 16), dtype=torch.uint8,
+                         device=dev)
+        y = torch.empty((cfg.m, cfg.n), dtype=torch.bfloat16, device=dev)
+        lin = lambda: W.w8a8_convrot_linear(x, w_q, s_w, cfg.group, y=y, workspace=ws)  # noqa: E731
+        timed(lin, 3, flush_buf, stream)
+        t_lin = statistics.median(timed(lin, reps, flush_buf, stream))
+        x_q = ws[:cfg.m * cfg.k].view(torch.int8).view(cfg.m, cfg.k)
+        off = (cfg.m * cfg.k + 255) // 256 * 256
+        s_x = ws[off:off + 4 * cfg.m].view(torch.float32)
+        gemm = lambda: W.convrot_i8_gemm_bf16(x_q, s_x, w_q, s_w)  # noqa: E731
+        timed(gemm, 3, flush_buf, stream)
+        t_gemm = statistics.median(timed(gemm, reps, flush_buf, stream))
+        ops = 2 * cfg.m * cfg.n * cfg.k
+        # the linear's algorithmic bytes: X in (bf16), codes and scales of W, Y out (bf16)
+        nbytes = cfg.m * cfg.k * 2 + cfg.n * cfg.k + cfg.n * 4 + cfg.m * cfg.n * 2
+        gemm_bytes = cfg.m * cfg.k + cfg.m * 4 + cfg.n * cfg.k + cfg.n * 4 + cfg.m * cfg.n * 2
+        out[name] = {"m": cfg.m, "n": cfg.n, "k": cfg.k, "group": cfg.group,
+                     "linear_us": t_lin * 1e6, "linear": roofline_of(ops, nbytes, t_lin, peaks),
+                     "gemm_us": t_gemm * 1e6, "gemm": roofline_of(ops, gemm_bytes, t_gemm, peaks)}
+    return out
+
+
+def int8_peak_probe(W, flush_buf, dev, stream, n=8192, reps=10):
+    """Dense INT8 tensor throughput this library's own GEMM reaches: one
+    n x n x n product of random codes with the bf16 epilogue (the output is
+    1/n of the work), best of `reps`. A lower bound on the hardware's peak."""
+    gen = torch.Generator(device=dev).manual_seed(0)
+    a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=gen)
+    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=gen)
+    s_a = torch.full((n,), 1e-3, device=dev)
+    s_b = torch.full((n,), 1e-3, device=dev)
+    fn = lambda: W.convrot_i8_gemm_bf16(a, s_a, b, s_b)  # noqa: E731
+    timed(fn, 3, flush_buf, stream)
+    best = min(timed(fn, reps, flush_buf, stream))
+    tops = 2.0 * n ** 3 / best / 1e12
+    peaks = load_peaks()
+    return {"shape": f"{n}x{n}x{n}", "us": best * 1e6, "tops": tops,
+            "of_2x_bf16_measured": tops / (2.0 * peaks["bf16_tflops"]),
+            "of_datasheet": tops / INT8_DATASHEET_TOPS}
+
+
+def run_ours(args, cfg, world, rank, local, extras=True):
     import w8a8_rotated_int8_b200 as W
     W.load_library()
     W.convrot_device_check()
@@ -430,27 +578,16 @@ def run_ours(args, cfg, world, rank, local):
     x_h = inp["x"].pin_memory()
     l_h = inp["logits"].pin_memory()
     y_h = torch.empty((t, cfg.d), dtype=torch.bfloat16).pin_memory()
-    for _ in range(2):
-        flush_buf.zero_()
+
+    def e2e_step():
         x.copy_(x_h, non_blocking=True)
         logits.copy_(l_h, non_blocking=True)
         step(x, logits, y)
         y_h.copy_(y, non_blocking=True)
-    torch.cuda.synchronize()
-    e2e_t = []
-    for _ in range(args.steps):
-        flush_buf.zero_()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        x.copy_(x_h, non_blocking=True)
-        logits.copy_(l_h, non_blocking=True)
-        step(x, logits, y)
-        y_h.copy_(y, non_blocking=True)
-        b.record(stream)
-        b.synchronize()
-        e2e_t.append(a.elapsed_time(b) * 1e-3)
-    e2e_step = max_over_ranks(statistics.mean(e2e_t), world)
+
+    timed(e2e_step, 2, flush_buf, stream)
+    e2e_step_s = max_over_ranks(statistics.mean(timed(e2e_step, args.steps, flush_buf, stream)),
+                                world)
 
     # per-stage device times (dominant kernel for the roofline)
     views = W.moe_stage_views(ws, t, cfg.d, cfg.f, cfg.n_exp, cfg.c)
@@ -459,32 +596,52 @@ def run_ours(args, cfg, world, rank, local):
     if flags != 0:
         raise RuntimeError(f"device error flags {flags:#x}")
 
+    # the other workloads of the same model, on rank 0 only (N = 1 lines)
+    workloads = {}
+    if extras and world == 1:
+        big = torch.empty(W.moe_workspace_size(8192, cfg.d, cfg.f, cfg.n_exp, 256),
+                          dtype=torch.uint8, device=dev) if t < 8192 else ws
+        for name in ("moe_T512", "moe_T1024", "moe_T2048", "moe_T4096", "moe_T8192"):
+            other = MOE_CONFIGS[name]
+            if other.t == t:
+                continue
+            workloads[name] = block_workload(W, other, wq, big, flush_buf, 20, 3, dev, stream)
+        del big
+        workloads["linears"] = linear_workloads(W, flush_buf, 10, dev, stream)
+        workloads["int8_gemm_probe"] = int8_peak_probe(W, flush_buf, dev, stream)
+        flags = W.convrot_check_device_error()
+        if flags != 0:
+            raise RuntimeError(f"device error flags {flags:#x}")
+
     if rank != 0:
         return
     peaks = load_peaks()
     work = algorithmic_work(cfg, t)
     gateup_stage = "gemm_gateup_swiglu_rq" if fused_h(cfg) else "gemm_gateup_swiglu"
     dom = max((gateup_stage, "gemm_down_bf16"), key=lambda k: st[k])
-    dk = {"gemm_gateup_swiglu_rq": work["gateup_rq"], "gemm_gateup_swiglu": work["gateup"],
-          "gemm_down_bf16": work["down"]}[dom]
-    int8_peak_tops = 2.0 * peaks["bf16_tflops"]  # int8 dense = 2x bf16 dense (nominal ratio)
-    t_hbm = dk["bytes"] / (peaks["hbm_gbs"] * 1e9)
-    t_tc = dk["ops"] / (int8_peak_tops * 1e12)
-    if t_hbm >= t_tc:
-        achieved = dk["bytes"] / st[dom] / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    dk = work["down_alg"] if dom == "gemm_down_bf16" else work["gateup_alg"]
+    kr = roofline_of(dk["ops"], dk["bytes"], st[dom], peaks)
+    int8_peak = 2.0 * peaks["bf16_tflops"]
+    if kr["bound"] == "hbm":
+        roof = {"bound": "hbm", "achieved": kr["hbm_gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": kr["hbm_frac"]}
     else:
-        achieved = dk["ops"] / st[dom] / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak_tops, "unit": "TOPS"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel"] = dom
-    roof["algorithmic_bytes"] = dk["bytes"]
-    roof["algorithmic_ops"] = dk["ops"]
-    roof["peak_source"] = (f"{peaks['source']} (HBM copy; int8 = 2 x measured bf16 burst)")
-    roof["traffic"] = (args.traffic_bytes if args.traffic_bytes is not None
-                       else DOMINANT_TRAFFIC_BYTES.get(cfg.name))
-    block_roof_t = max(work["block_bytes"] / (peaks["hbm_gbs"] * 1e9),
-                       work["ops"] / (int8_peak_tops * 1e12))
+        roof = {"bound": "tensor", "achieved": kr["tops"], "peak": int8_peak, "unit": "TOPS",
+                "frac": kr["tensor_frac"]}
+    traffic, traffic_note = profile_traffic(dom, cfg.name)
+    if args.traffic_bytes is not None:
+        traffic, traffic_note = args.traffic_bytes, "given on the command line"
+    roof.update({
+        "scope": f"dominant kernel ({dom}); the whole block is under block_roofline",
+        "traffic": traffic, "traffic_source": traffic_note,
+        "hbm_frac": kr["hbm_frac"], "tensor_frac": kr["tensor_frac"],
+        "tensor_frac_datasheet": kr["tensor_frac_datasheet"],
+        "kernel_us": st[dom] * 1e6, "algorithmic_bytes": dk["bytes"], "algorithmic_ops": dk["ops"],
+        "bytes_rule": "expert weights once + their scales (gathered and intermediate copies excluded)",
+        "peak_source": (f"{peaks['source']}: HBM copy {peaks['hbm_gbs']} GB/s; INT8 "
+                        f"{int8_peak:.0f} TOPS = 2 x measured bf16 burst"),
+    })
+    block = roofline_of(work["ops"], work["block_bytes"], mean_step, peaks)
 
     value = job_throughput(t, world, mean_step)
     # softmax, rotation, top-C, [gather, GEMM, (h rotation,) GEMM], combine
@@ -498,18 +655,19 @@ def run_ours(args, cfg, world, rank, local):
                    "f": cfg.f, "capacity": cfg.c, "g_gu": cfg.g_gu, "g_d": cfg.g_d,
                    "parallelism": f"replicas x{world} (independent batches)",
                    "l2": "flushed before every step (256 MiB write + 256 MiB read, outside the timed events)"},
+        "roofline_block_frac": block["roofline_frac"],
         "gpu_launches": launches_per_step * args.steps,
-        "e2e": {"value": job_throughput(t, world, e2e_step), "unit": UNIT,
+        "e2e": {"value": job_throughput(t, world, e2e_step_s), "unit": UNIT,
                 "h2d_bytes_per_step": int(x_h.numel() * 2 + l_h.numel() * 2),
                 "d2h_bytes_per_step": int(y_h.numel() * 2)},
         "roofline": roof,
-        "block_roofline": {"time_us": block_roof_t * 1e6, "frac": block_roof_t / mean_step,
-                           "algorithmic_bytes": work["block_bytes"], "ops": work["ops"],
-                           "effective_tops": work["ops"] / mean_step / 1e12},
+        "block_roofline": {**block, "algorithmic_bytes": work["block_bytes"], "ops": work["ops"]},
         "stage_us": {k: v * 1e6 for k, v in st.items()},
         "clocks": clk,
         "wall_s": wall,
     }
+    if workloads:
+        line["workloads"] = workloads
     if args.cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(cfg, inp)
     print(json.dumps(line), flush=True)
@@ -577,6 +735,8 @@ def main():
     ap.add_argument("--config", default="moe_T8192", choices=sorted(MOE_CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-extras", dest="extras", action="store_false",
+                    help="only the configured block (no other T, linears or INT8 probe)")
     ap.add_argument("--ablation", action="store_true",
                     help="rotation-off ablation: block error with and without ConvRot")
     ap.add_argument("--traffic-bytes", type=float, default=None,
@@ -600,9 +760,9 @@ def main():
         if args.sweep:
             args.cpu_baseline = False
             for name in ("moe_T512", "moe_T1024", "moe_T2048", "moe_T4096", "moe_T8192"):
-                run_ours(args, MOE_CONFIGS[name], world, rank, local)
+                run_ours(args, MOE_CONFIGS[name], world, rank, local, extras=False)
         else:
-            run_ours(args, cfg, world, rank, local)
+            run_ours(args, cfg, world, rank, local, extras=args.extras)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -99,16 +99,19 @@ def linear_inputs(cfg: LinearConfig):
     return x, w
 
 
-def moe_inputs(cfg: MoEConfig, t: int | None = None):
+def moe_inputs(cfg: MoEConfig, t: int | None = None, weights: bool = True):
     """Returns dict of CPU tensors: x [T,d], logits [T,E] (bf16),
     wgu [E,2f,d] (bf16; rows 0..f-1 gate, f..2f-1 up), wd [E,d,f] (bf16).
 
-    ``t`` overrides the token count (the weights do not depend on it).
+    ``t`` overrides the token count (the weights do not depend on it);
+    ``weights=False`` draws only x and the logits (the same values).
     """
     t = cfg.t if t is None else t
     gen = torch.Generator().manual_seed(cfg.seed)
     x = _activations(t, cfg.d, gen)
     logits = torch.randn(t, cfg.n_exp, generator=gen, dtype=torch.float32).to(torch.bfloat16)
+    if not weights:
+        return {"x": x, "logits": logits}
     wgu = torch.empty(cfg.n_exp, 2 * cfg.f, cfg.d, dtype=torch.bfloat16)
     for e in range(cfg.n_exp):
         wgu[e] = _weights(2 * cfg.f, cfg.d, gen)

@@ -39,3 +39,37 @@ def test_requantising_gemm_bytes():
 def test_fused_h_follows_the_down_group():
     assert bench.fused_h(MOE_CONFIGS["moe_T8192"])
     assert bench.fused_h(MOE_CONFIGS["moe_T2048"])
+
+
+def test_gemm_roofline_bytes_are_weights_and_scales():
+    """The roofline of a GEMM counts its weights once plus their scales; the
+    gathered activation codes and the h codes are not algorithmic traffic."""
+    cfg = MOE_CONFIGS["moe_T8192"]
+    w = bench.algorithmic_work(cfg, cfg.t)
+    assert w["gateup_alg"]["bytes"] == 402_653_184 + 786_432
+    assert w["down_alg"]["bytes"] == 201_326_592 + 524_288
+    assert w["gateup_alg"]["ops"] == w["gateup"]["ops"]
+
+
+def test_roofline_fractions():
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 500.0}  # int8 peak = 1000 TOPS
+    r = bench.roofline_of(ops=2e12, nbytes=1e9, seconds=4e-3, peaks=peaks)
+    assert r["bound"] == "tensor"                      # 2 ms of tensor work > 1 ms of HBM
+    assert abs(r["hbm_gbs"] - 250.0) < 1e-9 and abs(r["hbm_frac"] - 0.25) < 1e-12
+    assert abs(r["tops"] - 500.0) < 1e-9 and abs(r["tensor_frac"] - 0.5) < 1e-12
+    assert abs(r["roofline_frac"] - 0.5) < 1e-12 and abs(r["ideal_us"] - 2000.0) < 1e-6
+
+
+def test_traffic_record_needs_the_current_sources(tmp_path, monkeypatch):
+    """A traffic figure counts only while the kernel sources are those it was
+    captured on."""
+    monkeypatch.setattr(bench, "PROFILES", str(tmp_path))
+    (tmp_path / "k.md").write_text(
+        "# summary\ntraffic-record: kernel=gemm_x workload=moe_T8192 bytes_per_launch=4.5e8 "
+        f"source_sha16={bench.source_sha16()}\n"
+        "traffic-record: kernel=gemm_y workload=moe_T8192 bytes_per_launch=1e8 "
+        "source_sha16=0000000000000000\n")
+    assert bench.profile_traffic("gemm_x", "moe_T8192")[0] == 4.5e8
+    got, note = bench.profile_traffic("gemm_y", "moe_T8192")
+    assert got is None and "changed" in note
+    assert bench.profile_traffic("gemm_x", "moe_T2048")[0] is None
