@@ -101,6 +101,25 @@ int convrot_check_device_error(void* stream, unsigned* flags);
  * up. Used to test the failure path without faulting the GPU. */
 int convrot_wait_selftest(unsigned long long limit_ns, int* result_dev, void* stream);
 
+/* Diagnostic: one thread clears the two ints at words_dev (a counter and an
+ * abort word), then waits up to `limit_ns` for the counter to reach 1 through
+ * the bounded cross-CTA wait the requantising GEMM uses between tiles;
+ * nothing raises it, so the wait gives up, records a flag (reported by
+ * convrot_check_device_error) and sets *result_dev (device int) to 0. */
+int convrot_count_wait_selftest(unsigned long long limit_ns, int* words_dev, int* result_dev,
+                                void* stream);
+
+/* Host rule of the requantising SwiGLU GEMM (convrot_i8_gemm_swiglu_rq, and
+ * the MoE call's gate/up step): how many co-resident CTAs (or CTA pairs) it
+ * runs `tiles` tiles on, n_blocks tiles per row block, when `capacity` of
+ * them fit on the device at once. The tiles of a row block wait for one
+ * another, so the answer is `tiles` when they all fit, else a whole number
+ * of row blocks, and 0 when not even one row block's tiles fit together: the
+ * library then takes the two-step path (fp32 h, rotation kernel) instead of
+ * launching a kernel whose waits could not end. Pure host arithmetic;
+ * returns -1 for negative arguments. */
+int64_t convrot_swiglu_rq_units(int64_t tiles, int64_t n_blocks, int64_t capacity);
+
 /* ---------------------------------------------------------------------------
  * Rotate + quantise rows at run time (activations per token, and the SwiGLU
  * output h before the down projection). "Nucleus-Image INT8 Convrot Experts +
@@ -316,6 +335,14 @@ int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const 
  * library keeps per device, forked from and joined back to `stream` with
  * events, so it overlaps the activation rotation; the call as a whole is
  * still ordered on `stream` (and can be captured on it).
+ * Failure of a device-side wait: the call is asynchronous, so a kernel that
+ * gives up on a bounded wait (the gate/up GEMM's cross-tile wait gives up
+ * after 100 ms, e.g. when another workload holds some of the SMs and the
+ * GEMM's CTAs cannot all be resident; the pipeline waits after 2 s) cannot
+ * change the returned status. The kernels then stop early and y is invalid;
+ * a caller that may share the device checks convrot_check_device_error(stream)
+ * after the call (it synchronises) and treats CONVROT_ERR_TIMEOUT as a
+ * failed call.
  * ------------------------------------------------------------------------- */
 typedef struct {
   size_t x_q;      /* [T, d] int8     rotated activation codes      */

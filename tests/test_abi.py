@@ -105,3 +105,19 @@ def test_workspace_layout_is_disjoint_and_aligned(lib):
     assert all(o % 256 == 0 for o in offs)
     assert len(set(offs)) == len(offs)
     assert lay["total"] >= lay["z"] + 64 * 256 * 2048 * 2
+
+
+def test_requantising_gemm_plan_falls_back_when_too_few_ctas_fit(lib):
+    """The host rule for the requantising gate/up GEMM: its tiles of one row
+    block wait for one another, so it runs only on a capacity that holds a
+    whole row block's tiles at once; with less (a share of the SMs) the plan
+    is 0 and the library takes the two-step path instead of launching waits
+    that could not end."""
+    units = binding.convrot_swiglu_rq_units
+    # T=8192: 64 experts x 1 pair m-block x 12 n-blocks = 768 tiles, 74 pairs fit
+    assert units(768, 12, 74) == 72            # six whole row blocks per wave
+    assert units(768, 12, 11) == 0             # one row block cannot meet: fall back
+    assert units(768, 12, 12) == 12
+    assert units(30, 12, 74) == 30             # every tile fits at once
+    assert units(0, 12, 74) == 0
+    assert units(-1, 12, 74) == -1

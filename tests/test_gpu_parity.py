@@ -711,3 +711,16 @@ def test_bounded_wait_gives_up_and_reports():
     flags = W.convrot_check_device_error()
     assert flags & (1 << 5)
     assert W.convrot_check_device_error() == 0       # cleared by the read
+
+
+def test_cross_tile_wait_gives_up_and_reports():
+    """The bounded counter wait between the requantising GEMM's tiles, on a
+    counter nothing raises: it gives up after its limit and the host reads
+    CONVROT_ERR_TIMEOUT (the self-test bit); the context stays usable."""
+    assert W.convrot_count_wait_selftest(2_000_000) == 0   # 2 ms limit
+    flags = W.convrot_check_device_error()
+    assert flags & (1 << 5)
+    assert W.convrot_check_device_error() == 0
+    # the device still runs work afterwards
+    q, s = W.convrot_rotquant(torch.ones(4, 256, dtype=torch.bfloat16, device="cuda"), 256)
+    assert float(s[0]) > 0

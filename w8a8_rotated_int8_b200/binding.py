@@ -57,6 +57,8 @@ _SIGNATURES = {
     "convrot_device_check": (_I, []),
     "convrot_check_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "convrot_wait_selftest": (_I, [ctypes.c_ulonglong, _P, _P]),
+    "convrot_count_wait_selftest": (_I, [ctypes.c_ulonglong, _P, _P, _P]),
+    "convrot_swiglu_rq_units": (_I64, [_I64, _I64, _I64]),
     "convrot_rotquant": (_I, [_P, _I, _I64, _I64, _I, _P, _P, _P]),
     "convrot_quantize_weights": (_I, [_P, _I64, _I64, _I, _P, _P, _P]),
     "convrot_tiled_weight_bytes": (_I64, [_I64, _I64, _I64]),
@@ -165,6 +167,21 @@ def convrot_wait_selftest(limit_ns: int, stream=None) -> int:
     res = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     _invoke(res, "convrot_wait_selftest", limit_ns, _p(res), stream=stream)
     return int(res.item())
+
+
+def convrot_count_wait_selftest(limit_ns: int, stream=None) -> int:
+    """Runs the bounded cross-CTA counter wait on a counter nothing raises;
+    returns 0 when the wait gave up."""
+    res = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    words = torch.empty((2,), dtype=torch.int32, device="cuda")
+    _invoke(res, "convrot_count_wait_selftest", limit_ns, _p(words), _p(res), stream=stream)
+    return int(res.item())
+
+
+def convrot_swiglu_rq_units(tiles: int, n_blocks: int, capacity: int) -> int:
+    """Host rule: co-resident units the requantising GEMM runs on (0 = it
+    cannot run, the two-step path is used instead)."""
+    return int(lib().convrot_swiglu_rq_units(tiles, n_blocks, capacity))
 
 
 # ------------------------------------------------------------------ stages --

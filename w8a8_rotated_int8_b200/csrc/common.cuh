@@ -30,6 +30,10 @@ enum DeviceErrorBits : unsigned {
 
 __device__ unsigned int g_device_error = 0;
 __device__ unsigned long long g_wait_limit_ns = 2000000000ull;  // 2 s
+// The cross-CTA wait of a GEMM tile for the other tiles of its rows: they run
+// side by side, so this wait normally lasts microseconds; a launch whose
+// CTAs are not all resident (too few SMs granted) gives up after this.
+__device__ unsigned long long g_rowsync_limit_ns = 100000000ull;  // 100 ms
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
@@ -116,11 +120,12 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint6
 }
 
 // Waits until *count >= target (a counter other CTAs of the same grid raise),
-// bounded like mbar_wait. `grid_abort` is a word of the same launch that a
+// for at most limit_ns. `grid_abort` is a word of the same launch that a
 // CTA which gave up sets, so the others stop waiting for it at once. On
 // giving up the CTA's abort flag is raised too. Returns false then.
 __device__ __forceinline__ bool wait_count_geq(const int* count, int target, int* grid_abort,
-                                               volatile int* abort_flag, unsigned err_bit) {
+                                               volatile int* abort_flag, unsigned err_bit,
+                                               uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
   while (true) {
@@ -134,7 +139,7 @@ __device__ __forceinline__ bool wait_count_geq(const int* count, int target, int
         *abort_flag = 1;
         return false;
       }
-      if (global_timer_ns() - t0 > g_wait_limit_ns) {
+      if (global_timer_ns() - t0 > limit_ns) {
         atomicOr(&g_device_error, err_bit);
         atomicExch(grid_abort, 1);
         *abort_flag = 1;

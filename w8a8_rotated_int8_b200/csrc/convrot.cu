@@ -440,13 +440,19 @@ int encode_tiled_b(CUtensorMap* map, const void* base, uint64_t kb_count, uint64
 // Units (CTAs, or CTA pairs) the requantising SwiGLU GEMM runs `tiles` tiles
 // on, n_blocks of them per row block; 0 when the device cannot keep enough of
 // them resident for the tiles of a row block to meet.
-int64_t swiglu_rq_units(int64_t tiles, int64_t n_blocks, bool pairs, int sms) {
-  int64_t cap = std::min<int64_t>(pairs ? sms / 2 : sms, swiglu_rq_capacity(pairs));
+// The same for a given capacity of co-resident units (a pure host rule).
+int64_t rq_units_for(int64_t tiles, int64_t n_blocks, int64_t cap) {
+  if (tiles <= 0 || n_blocks <= 0) return 0;
   if (tiles <= cap) return tiles;
   if (cap < n_blocks) return 0;
   // a whole number of row blocks per wave: the tiles of a row block then run
   // side by side instead of one wave apart
   return cap / n_blocks * n_blocks;
+}
+
+int64_t swiglu_rq_units(int64_t tiles, int64_t n_blocks, bool pairs, int sms) {
+  const int64_t cap = std::min<int64_t>(pairs ? sms / 2 : sms, swiglu_rq_capacity(pairs));
+  return rq_units_for(tiles, n_blocks, cap);
 }
 
 // Whether the gate/up GEMM over G groups of M rows (tiled weights, F h
@@ -714,6 +720,20 @@ int convrot_wait_selftest(unsigned long long limit_ns, int* result_dev, void* st
   if (!result_dev || limit_ns > 10000000000ull) return CONVROT_ERR_INVALID_ARG;
   wait_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(limit_ns, result_dev);
   return launch_status();
+}
+
+int convrot_count_wait_selftest(unsigned long long limit_ns, int* words_dev, int* result_dev,
+                                void* stream) {
+  int rc = device_setup(nullptr);
+  if (rc != CONVROT_OK) return rc;
+  if (!words_dev || !result_dev || limit_ns > 10000000000ull) return CONVROT_ERR_INVALID_ARG;
+  count_wait_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(limit_ns, words_dev, result_dev);
+  return launch_status();
+}
+
+int64_t convrot_swiglu_rq_units(int64_t tiles, int64_t n_blocks, int64_t capacity) {
+  if (tiles < 0 || n_blocks < 0 || capacity < 0) return -1;
+  return rq_units_for(tiles, n_blocks, capacity);
 }
 
 int convrot_rotquant(const void* x, int x_dtype, int64_t rows, int64_t K, int group, int8_t* q,

@@ -619,4 +619,19 @@ __global__ void wait_selftest_kernel(unsigned long long limit_ns, int* result) {
   }
 }
 
+// The cross-CTA counter wait of the requantising GEMM, alone: thread 0
+// clears the counter and the abort word at `words` (two ints), then waits for
+// the counter to reach 1, which nothing does; *result = 0 once it gave up.
+__global__ void count_wait_selftest_kernel(unsigned long long limit_ns, int* words, int* result) {
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    words[0] = 0;
+    words[1] = 0;
+    __threadfence();
+    const bool ok = wait_count_geq(words, 1, words + 1, &abort_flag, kErrSelfTest, limit_ns);
+    *result = ok ? 1 : 0;
+  }
+}
+
 }  // namespace convrot
