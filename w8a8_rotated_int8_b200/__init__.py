@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     LIB_PATH,
     convrot_check_device_error,
     convrot_combine_rows,
+    convrot_count_wait_selftest,
     convrot_device_check,
     convrot_f32_to_bf16,
     convrot_gather_rows,
@@ -24,6 +25,7 @@ from .binding import (  # noqa: F401
     convrot_quantize_weights_tiled,
     convrot_rotquant,
     convrot_router_softmax,
+    convrot_swiglu_rq_units,
     convrot_topc,
     convrot_wait_selftest,
     load_library,
