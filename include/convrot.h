@@ -331,10 +331,9 @@ int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const 
  * resident, as convrot_i8_gemm_swiglu_rq needs) h is rotated and requantised
  * in the gate/up GEMM's epilogue and the fp32 h region is left untouched;
  * with g_d = 256 h is stored in fp32 and rotated by a separate kernel.
- * Inside the call the routing (softmax, top-C) runs on a second stream the
- * library keeps per device, forked from and joined back to `stream` with
- * events, so it overlaps the activation rotation; the call as a whole is
- * still ordered on `stream` (and can be captured on it).
+ * Every kernel of the call runs on `stream` (so the call can be captured in a
+ * CUDA graph on it); they are chained with programmatic dependent launch, and
+ * the activation rotation runs beside the routing kernels.
  * Failure of a device-side wait: the call is asynchronous, so a kernel that
  * gives up on a bounded wait (the gate/up GEMM's cross-tile wait gives up
  * after 100 ms, e.g. when another workload holds some of the SMs and the

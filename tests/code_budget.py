@@ -7,7 +7,7 @@ Convrot Experts + FP8 Text Encoder", section "Quantization": symmetric INT8
 with nearest rounding, one FP32 scale per row). A GPU code may therefore
 differ from the definition's by one, and only where the exact quotient v'/s
 lies within the fp32 error of a half-integer. The budget: at most 1e-4 of the
-codes off by one, none off by more.
+codes off by one (at least 8 allowed in small cases), none off by more.
 
 The error bound per row: the fp32 butterflies of a group add at most
 log2(g) roundings of 2^-24 times the group's |.|-sum / sqrt(g) to each
@@ -62,5 +62,8 @@ def check_codes(q_gpu: np.ndarray, s_gpu: np.ndarray, x: np.ndarray, g: int,
         assert not far.any(), (f"{int(far.sum())} codes differ from the definition away from a "
                                f"half-integer (first at row {r[far][0]}, col {c[far][0]})")
     flips = int(r.size)
-    assert flips <= max(2, budget * q_gpu.size), f"{flips} flips in {q_gpu.size} codes"
+    # the budget is a rate; small cases get a floor of 8 (one row whose absmax
+    # makes many quotients exact half-integers can flip several codes, each of
+    # them checked above to sit at a half-integer)
+    assert flips <= max(8, budget * q_gpu.size), f"{flips} flips in {q_gpu.size} codes"
     return flips, q_gpu.size, q_ref, s_ref

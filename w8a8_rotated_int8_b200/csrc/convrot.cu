@@ -37,43 +37,6 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
-// Second stream of a device for work of one call that can run beside the
-// caller's stream (joined back with events before its results are used).
-// Created once per device; `mu` serialises the fork/join of concurrent calls.
-struct SideStream {
-  bool ready = false;
-  cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr;
-  cudaEvent_t join = nullptr;
-  std::mutex mu;
-};
-SideStream g_side[kMaxDevices];
-
-int side_stream(SideStream** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    cudaGetLastError();
-    return CONVROT_ERR_UNSUPPORTED_DEVICE;
-  }
-  SideStream& ss = g_side[dev];
-  std::lock_guard<std::mutex> lock(g_dev_mu);
-  if (!ss.ready) {
-    // highest priority: the routing chain is the longer branch of the fork,
-    // so its CTAs should take SMs first as they free up
-    int least = 0, greatest = 0;
-    cudaDeviceGetStreamPriorityRange(&least, &greatest);
-    if (cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, greatest) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
-      cudaGetLastError();
-      return CONVROT_ERR_CUDA;
-    }
-    ss.ready = true;
-  }
-  *out = &ss;
-  return CONVROT_OK;
-}
-
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -250,7 +213,7 @@ int encode_rows_sw128(CUtensorMap* map, const void* base, uint64_t row_bytes, ui
 // routing kernels that run beside the activation rotation).
 template <typename InT, int G, int SEG>
 int launch_rq_tma(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
-                   cudaStream_t st, bool pdl, int64_t grid_cap) {
+                   cudaStream_t st, bool pdl, int64_t grid_cap, bool wait_at_end) {
   constexpr int kRowsPerWarp = 32 / SEG;
   const uint64_t row_bytes = (uint64_t)K * sizeof(InT);
   CUtensorMap tm;
@@ -261,35 +224,55 @@ int launch_rq_tma(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut
   slots = std::max(2, std::min(kRqMaxSlots, slots));
   const size_t smem = 1024 + (size_t)kRqTmaWarps * slots * (slot_bytes + 8) + kRqTmaWarps * 4;
   auto kern = rotquant_tma_kernel<InT, G, SEG>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRqTmaWarps * 32, smem) !=
-          cudaSuccess ||
-      per_sm < 1)
-    per_sm = 1;
   int sms = 0;
   device_setup(&sms);
+  // the attribute and the occupancy for this shared-memory size, once per device
+  struct Residency {
+    size_t smem = 0;
+    int per_sm = 0;
+  };
+  static Residency cached[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CONVROT_ERR_CUDA;
+  int per_sm = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    Residency& r = cached[dev];
+    if (r.smem != smem) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kRqTmaWarps * 32, smem) !=
+              cudaSuccess ||
+          n < 1) {
+        cudaGetLastError();
+        n = 1;
+      }
+      r.smem = smem;
+      r.per_sm = n;
+    }
+    per_sm = r.per_sm;
+  }
   const int64_t units = (rows + kRowsPerWarp - 1) / kRowsPerWarp;
   const int64_t ctas = (units + kRqTmaWarps - 1) / kRqTmaWarps;
   int64_t grid = std::min<int64_t>(ctas, (int64_t)per_sm * std::max(sms, 1));
   if (grid_cap > 0 && ctas > grid) grid = std::min(grid, grid_cap);
   return launch_kernel(kern, dim3((unsigned)grid), dim3(kRqTmaWarps * 32), smem, st, pdl, 1, tm,
-                       rows, K, slots, slot_bytes, q, s, out);
+                       rows, K, slots, slot_bytes, q, s, out, wait_at_end ? 1 : 0);
 }
 
 template <typename InT, int G>
 int launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
-               cudaStream_t st, bool pdl, int64_t grid_cap) {
+               cudaStream_t st, bool pdl, int64_t grid_cap, bool wait_at_end) {
   // K % 64 == 0, K <= 2048: one warp segment of SEG lanes per row, 64
   // elements per lane (G = 256 needs at least the four lanes of one group)
   if (K % 64 == 0 && K <= 2048) {
     const int lanes = K / 64;
-    if (lanes <= 1 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 1 : 4)>(x, rows, K, q, s, out, st, pdl, grid_cap);
-    if (lanes <= 2 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 2 : 4)>(x, rows, K, q, s, out, st, pdl, grid_cap);
-    if (lanes <= 4) return launch_rq_tma<InT, G, 4>(x, rows, K, q, s, out, st, pdl, grid_cap);
-    if (lanes <= 8) return launch_rq_tma<InT, G, 8>(x, rows, K, q, s, out, st, pdl, grid_cap);
-    if (lanes <= 16) return launch_rq_tma<InT, G, 16>(x, rows, K, q, s, out, st, pdl, grid_cap);
-    return launch_rq_tma<InT, G, 32>(x, rows, K, q, s, out, st, pdl, grid_cap);
+    if (lanes <= 1 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 1 : 4)>(x, rows, K, q, s, out, st, pdl, grid_cap, wait_at_end);
+    if (lanes <= 2 && G < 256) return launch_rq_tma<InT, G, (G < 256 ? 2 : 4)>(x, rows, K, q, s, out, st, pdl, grid_cap, wait_at_end);
+    if (lanes <= 4) return launch_rq_tma<InT, G, 4>(x, rows, K, q, s, out, st, pdl, grid_cap, wait_at_end);
+    if (lanes <= 8) return launch_rq_tma<InT, G, 8>(x, rows, K, q, s, out, st, pdl, grid_cap, wait_at_end);
+    if (lanes <= 16) return launch_rq_tma<InT, G, 16>(x, rows, K, q, s, out, st, pdl, grid_cap, wait_at_end);
+    return launch_rq_tma<InT, G, 32>(x, rows, K, q, s, out, st, pdl, grid_cap, wait_at_end);
   }
   const int nch = K / 16;
   int tpr;
@@ -318,13 +301,13 @@ int launch_rq(const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out
 
 template <typename InT>
 int dispatch_rq(int group, const void* x, int64_t rows, int K, int8_t* q, float* s, RqOut out,
-                cudaStream_t st, bool pdl, int64_t grid_cap) {
+                cudaStream_t st, bool pdl, int64_t grid_cap, bool wait_at_end) {
   switch (group) {
-    case 1: return launch_rq<InT, 1>(x, rows, K, q, s, out, st, pdl, grid_cap);
-    case 4: return launch_rq<InT, 4>(x, rows, K, q, s, out, st, pdl, grid_cap);
-    case 16: return launch_rq<InT, 16>(x, rows, K, q, s, out, st, pdl, grid_cap);
-    case 64: return launch_rq<InT, 64>(x, rows, K, q, s, out, st, pdl, grid_cap);
-    default: return launch_rq<InT, 256>(x, rows, K, q, s, out, st, pdl, grid_cap);
+    case 1: return launch_rq<InT, 1>(x, rows, K, q, s, out, st, pdl, grid_cap, wait_at_end);
+    case 4: return launch_rq<InT, 4>(x, rows, K, q, s, out, st, pdl, grid_cap, wait_at_end);
+    case 16: return launch_rq<InT, 16>(x, rows, K, q, s, out, st, pdl, grid_cap, wait_at_end);
+    case 64: return launch_rq<InT, 64>(x, rows, K, q, s, out, st, pdl, grid_cap, wait_at_end);
+    default: return launch_rq<InT, 256>(x, rows, K, q, s, out, st, pdl, grid_cap, wait_at_end);
   }
 }
 
@@ -341,12 +324,13 @@ int check_rq_args(const void* x, int x_dtype, int64_t rows, int64_t K, int group
 
 int rotquant_impl(const void* x, int x_dtype, int64_t rows, int64_t K, int group, int8_t* q,
                   float* s, cudaStream_t st, RqOut out = RqOut{0, 1, 1, 1}, bool pdl = false,
-                  int64_t grid_cap = 0) {
+                  int64_t grid_cap = 0, bool wait_at_end = false) {
   if (rows == 0) return CONVROT_OK;
-  const int rc =
-      (x_dtype == CONVROT_DTYPE_BF16)
-          ? dispatch_rq<__nv_bfloat16>(group, x, rows, (int)K, q, s, out, st, pdl, grid_cap)
-          : dispatch_rq<float>(group, x, rows, (int)K, q, s, out, st, pdl, grid_cap);
+  const int rc = (x_dtype == CONVROT_DTYPE_BF16)
+                     ? dispatch_rq<__nv_bfloat16>(group, x, rows, (int)K, q, s, out, st, pdl,
+                                                  grid_cap, wait_at_end)
+                     : dispatch_rq<float>(group, x, rows, (int)K, q, s, out, st, pdl, grid_cap,
+                                          wait_at_end);
   if (rc != CONVROT_OK) return rc;
   return launch_status();
 }
@@ -661,11 +645,12 @@ int softmax_impl(const void* logits, int64_t T, int E, float* s_t, cudaStream_t 
 
 int gather_impl(const int8_t* src, const float* s_src, int64_t n_src, const int32_t* idx,
                 int64_t n_rows, int64_t K, int8_t* dst, float* s_dst, cudaStream_t st,
-                uint32_t* zero = nullptr, int64_t n_zero = 0) {
+                uint32_t* zero = nullptr, int64_t n_zero = 0, bool pdl = false) {
   if (n_rows == 0) return CONVROT_OK;
   const int64_t grid = (n_rows + 7) / 8;
-  gather_rows_kernel<<<(unsigned)grid, 256, 0, st>>>(src, s_src, n_src, idx, n_rows, (int)K, dst,
-                                                      s_dst, zero, n_zero);
+  const int rc = launch_kernel(gather_rows_kernel, dim3((unsigned)grid), dim3(256), 0, st, pdl, 1,
+                               src, s_src, n_src, idx, n_rows, (int)K, dst, s_dst, zero, n_zero);
+  if (rc != CONVROT_OK) return rc;
   return launch_status();
 }
 
@@ -1034,34 +1019,24 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
   int32_t* slot = reinterpret_cast<int32_t*>(ws + lay.slot);
   void* z = ws + lay.z;
 
-  // Routing (1, 3) runs on the side stream while the caller's stream rotates
-  // and quantises the tokens (2); the streams join before the gather. The
-  // kernels after the gather (and top-C after the softmax) are launched with
-  // programmatic stream serialization: each starts while its predecessor
-  // finishes and waits for it (griddepcontrol.wait) before reading its output.
-  SideStream* ss = nullptr;
-  if ((rc = side_stream(&ss)) != CONVROT_OK) return rc;
-  std::lock_guard<std::mutex> side_lock(ss->mu);
-  if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
-      cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
-    return CONVROT_ERR_CUDA;
+  // One stream, every kernel after the first launched with programmatic
+  // stream serialization, in the order 1. softmax, 2. top-C, 3. x rotation,
+  // 4. gather, ...: top-C waits for the softmax before reading its scores;
+  // the x rotation reads only X, so it runs beside the routing from the start
+  // and waits for top-C only before it exits (its completion implies top-C's);
+  // the gather then waits for the rotation and has both its inputs.
   // 1. router softmax
-  int rc_side = softmax_impl(logits_bf16, T, E, s_t, ss->stream);
-  // 3. expert-choice top-C (+ each token's slot per expert)
-  if (rc_side == CONVROT_OK) rc_side = topc_impl(s_t, T, E, C, idx, w, slot, ss->stream, true);
-  // 2. rotate + quantise the tokens once (the gate/up rotation is expert-independent);
-  // a rotation longer than one round of resident CTAs runs on about 1.25 CTAs
-  // per SM instead of filling every SM's register file, so the routing kernels
-  // start beside it (measured on B200: -5 us at T=8192; no change when one round
-  // covers the rows, as at T=2048)
-  rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, T, d, g_gu, x_q, s_x, st, RqOut{0, 1, 1, 1},
-                     false, sms + sms / 4);
-  // the join is recorded even after a failed launch so the side stream never dangles
-  if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess ||
-      cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess)
-    return CONVROT_ERR_CUDA;
-  if (rc_side != CONVROT_OK) return rc_side;
-  if (rc != CONVROT_OK) return rc;
+  if ((rc = softmax_impl(logits_bf16, T, E, s_t, st)) != CONVROT_OK) return rc;
+  // 2. expert-choice top-C (+ each token's slot per expert)
+  if ((rc = topc_impl(s_t, T, E, C, idx, w, slot, st, true)) != CONVROT_OK) return rc;
+  // 3. rotate + quantise the tokens once (the gate/up rotation is expert-independent);
+  // a rotation longer than one round of resident CTAs runs on at most 1.5
+  // CTAs per SM, which the top-C CTAs beside it leave room for (measured on
+  // B200 at T=8192: -6 us against two CTAs per SM, whose last CTAs start
+  // only as top-C ends)
+  if ((rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, T, d, g_gu, x_q, s_x, st, RqOut{0, 1, 1, 1},
+                          true, sms + sms / 2, true)) != CONVROT_OK)
+    return rc;
   if (C > 0) {
     // h is rotated and requantised inside the gate/up GEMM's epilogue when its
     // groups fit one thread (g_d <= 64) and the device holds enough of the
@@ -1073,7 +1048,8 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
     // synchronisation words)
     if ((rc = gather_impl(x_q, s_x, T, idx, (int64_t)E * C, d, x_g, s_g, st,
                           fused_h ? reinterpret_cast<uint32_t*>(hsync) : nullptr,
-                          fused_h ? (int64_t)(swiglu_rq_sync_bytes(E, C) / 4) : 0)) != CONVROT_OK)
+                          fused_h ? (int64_t)(swiglu_rq_sync_bytes(E, C) / 4) : 0, true)) !=
+        CONVROT_OK)
       return rc;
     GemmArgs a1{};
     a1.s_a = s_g;

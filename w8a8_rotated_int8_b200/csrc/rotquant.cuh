@@ -17,11 +17,15 @@
 //    code is rne of a correctly rounded fp64 quotient.
 //  * rotquant_kernel / rotquant_tma_kernel (activations and h, on the hot
 //    path): fp32 arithmetic, IEEE, no contraction --
-//      rotation  butterflies (a + b, a - b), spans 1, 2, ..., g/2, then
-//                v' = v * (1/sqrt(g)) (a power of two for g a power of four);
-//      scale     s = a / 127 (one IEEE division; subnormal or 0 for tiny a);
-//      codes     q = rint(v' * r) with r = 127 / a while a >= 2^-100 (then
-//                |v' r| <= 127 (1 + 2^-23): the code never leaves
+//      rotation  butterflies (a + b, a - b), spans 1, 2, ..., g/2, giving
+//                u = v' * sqrt(g); v' = u * (1/sqrt(g)) (a power of two for g
+//                a power of four, so the scaling is exact and commutes with
+//                fp32 rounding);
+//      scale     a = max|v'| = max|u| / sqrt(g), s = a / 127 (one IEEE
+//                division; subnormal or 0 for tiny a);
+//      codes     while a >= 2^-100: q = rne(u * (127 / max|u|)), the product
+//                exact inside one fma with the rounding constant 1.5 * 2^23
+//                (|u r| <= 127 (1 + 2^-24): the code never leaves
 //                [-127, 127]); below that q = clamp(rint(v' / s)) through an
 //                exactly rescaled reciprocal, so a subnormal s is honoured;
 //                s = 0 gives all-zero codes.
@@ -103,10 +107,26 @@ __device__ __forceinline__ int rq_code_tiny(float v, float r2) {
   return c > 127 ? 127 : (c < -127 ? -127 : c);
 }
 
-// Bits of the rounding add whose low byte is the code rint(v * r) (|v r| <=
-// 127.5): v r + 1.5 * 2^23 rounds to nearest even at the unit.
-__device__ __forceinline__ uint32_t rq_code_bits(float v, float r) {
-  return __float_as_uint(__fadd_rn(__fmul_rn(v, r), 12582912.0f));
+// Bits whose low byte is the code rne(u * r) (|u r| <= 127.5): the exact
+// product plus 1.5 * 2^23, rounded once (one fma), lands in [2^23, 2^24)
+// where fp32 has unit spacing, so the rounding is to the nearest integer,
+// ties to even.
+constexpr float kRqMagic = 12582912.0f;  // 1.5 * 2^23
+__device__ __forceinline__ uint32_t rq_code_bits(float u, float r) {
+  return __float_as_uint(__fmaf_rn(u, r, kRqMagic));
+}
+
+// Two codes at once from a packed pair (fma.rn.f32x2): the bits of both.
+__device__ __forceinline__ unsigned long long rq_code_bits2(unsigned long long u2,
+                                                            unsigned long long r2,
+                                                            unsigned long long magic2) {
+  return f2_fma(u2, r2, magic2);
+}
+
+// Low bytes of four code bit patterns (c0 lowest) as one word.
+__device__ __forceinline__ uint32_t rq_pack_bytes(uint32_t c0, uint32_t c1, uint32_t c2,
+                                                  uint32_t c3) {
+  return __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
 }
 
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
@@ -220,17 +240,15 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x
         v[j] = __fmaf_rn(sgn, v[j], p);
       }
     }
-    float m = 0.0f;
+    float mu = 0.0f;  // max |u| (unscaled)
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      v[j] = __fmul_rn(v[j], Tr::kInvSqrt);
-      m = fmaxf(m, fabsf(v[j]));
-    }
-    m = rq_row_max(m, tpr, red[it & 1]);
+    for (int j = 0; j < 16; ++j) mu = fmaxf(mu, fabsf(v[j]));
+    mu = rq_row_max(mu, tpr, red[it & 1]);
 
+    const float m = __fmul_rn(mu, Tr::kInvSqrt);
     const float s = __fdiv_rn(m, 127.0f);
     const bool recip = m >= kRqRecipMin;
-    const float r = recip ? __fdiv_rn(127.0f, m) : 0.0f;
+    const float r = recip ? __fdiv_rn(127.0f, mu) : 0.0f;
     if (active) {
       int k[16];
       if (recip) {
@@ -239,7 +257,7 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x
       } else {
         const float r2 = rq_tiny_recip(s);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) k[j] = rq_code_tiny(v[j], r2);
+        for (int j = 0; j < 16; ++j) k[j] = rq_code_tiny(__fmul_rn(v[j], Tr::kInvSqrt), r2);
       }
       uint4 c;
       c.x = pack4(k[0], k[1], k[2], k[3]);
@@ -325,36 +343,31 @@ __device__ __forceinline__ void rq_lane64(unsigned long long (&p)[32], bool acti
       }
     }
   }
-  const unsigned long long inv2 = f2_pack(Tr::kInvSqrt, Tr::kInvSqrt);
-  float mx = 0.0f;
+  // max |u| of the unscaled butterfly outputs (v' = u / sqrt(g) is never formed)
+  float mu = 0.0f;
 #pragma unroll
   for (int m = 0; m < 32; ++m) {
-    p[m] = f2_mul(p[m], inv2);
     const float2 t = f2_unpack(p[m]);
-    mx = fmaxf(mx, fmaxf(fabsf(t.x), fabsf(t.y)));
+    mu = fmaxf(mu, fmaxf(fabsf(t.x), fabsf(t.y)));
   }
 #pragma unroll
   for (int off = SEG >> 1; off > 0; off >>= 1)
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    mu = fmaxf(mu, __shfl_xor_sync(0xffffffffu, mu, off));
+  const float mx = __fmul_rn(mu, Tr::kInvSqrt);
   const float sc = __fdiv_rn(mx, 127.0f);
   const bool recip = mx >= kRqRecipMin;
-  const float r = recip ? __fdiv_rn(127.0f, mx) : 0.0f;
+  const float r = recip ? __fdiv_rn(127.0f, mu) : 0.0f;
   if (active) {
-    // rint by adding 1.5 * 2^23: the code is the low byte of the sum's bits.
-    // Scalar intrinsics on purpose: a packed mul.rn.f32x2 followed by a
-    // packed add.rn.f32x2 was contracted into one fma (the product then is
-    // not rounded to fp32 before the rint).
     uint32_t cw[16];
     if (recip) {
+      const unsigned long long r2 = f2_pack(r, r);
+      const unsigned long long magic2 = f2_pack(kRqMagic, kRqMagic);
 #pragma unroll
       for (int m = 0; m < 32; m += 2) {
-        const float2 a = f2_unpack(p[m]);
-        const float2 b = f2_unpack(p[m + 1]);
-        const uint32_t c0 = rq_code_bits(a.x, r);
-        const uint32_t c1 = rq_code_bits(a.y, r);
-        const uint32_t c2 = rq_code_bits(b.x, r);
-        const uint32_t c3 = rq_code_bits(b.y, r);
-        cw[m >> 1] = __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
+        const float2 a = f2_unpack(rq_code_bits2(p[m], r2, magic2));
+        const float2 b = f2_unpack(rq_code_bits2(p[m + 1], r2, magic2));
+        cw[m >> 1] = rq_pack_bytes(__float_as_uint(a.x), __float_as_uint(a.y),
+                                   __float_as_uint(b.x), __float_as_uint(b.y));
       }
     } else {
       const float r2 = rq_tiny_recip(sc);
@@ -362,8 +375,10 @@ __device__ __forceinline__ void rq_lane64(unsigned long long (&p)[32], bool acti
       for (int m = 0; m < 32; m += 2) {
         const float2 a = f2_unpack(p[m]);
         const float2 b = f2_unpack(p[m + 1]);
-        cw[m >> 1] = pack4(rq_code_tiny(a.x, r2), rq_code_tiny(a.y, r2), rq_code_tiny(b.x, r2),
-                           rq_code_tiny(b.y, r2));
+        cw[m >> 1] = pack4(rq_code_tiny(__fmul_rn(a.x, Tr::kInvSqrt), r2),
+                           rq_code_tiny(__fmul_rn(a.y, Tr::kInvSqrt), r2),
+                           rq_code_tiny(__fmul_rn(b.x, Tr::kInvSqrt), r2),
+                           rq_code_tiny(__fmul_rn(b.y, Tr::kInvSqrt), r2));
       }
     }
 #pragma unroll
@@ -384,12 +399,16 @@ __device__ __forceinline__ void rq_lane64(unsigned long long (&p)[32], bool acti
 constexpr int kRqTmaWarps = 8;
 constexpr int kRqMaxSlots = 4;  // ring depth per warp
 
+// wait_at_end: the kernel reads nothing its predecessor on the stream writes
+// (it runs beside it) and waits for that predecessor only before it exits, so
+// that its completion implies the predecessor's (the MoE call's schedule);
+// otherwise it waits for the predecessor before reading anything.
 template <typename InT, int G, int SEG>
 __global__ void __launch_bounds__(kRqTmaWarps * 32, 2) rotquant_tma_kernel(
     const __grid_constant__ CUtensorMap tm, int64_t rows, int K, int slots, int slot_bytes,
-    int8_t* __restrict__ q, float* __restrict__ scales, RqOut out) {
+    int8_t* __restrict__ q, float* __restrict__ scales, RqOut out, int wait_at_end) {
   griddep_launch_dependents();
-  griddep_wait();
+  if (!wait_at_end) griddep_wait();
   static_assert(SEG >= 1 && SEG <= 32 && (SEG & (SEG - 1)) == 0, "segment of 2^k lanes");
   static_assert(G != 256 || SEG >= 4, "a 256-group spans four lanes");
   constexpr int kRowsPerWarp = 32 / SEG;
@@ -484,6 +503,7 @@ __global__ void __launch_bounds__(kRqTmaWarps * 32, 2) rotquant_tma_kernel(
     }
     __syncwarp();
   }
+  if (wait_at_end) griddep_wait();
 }
 
 // ------------------------------------------------------ fp64 (offline) --
