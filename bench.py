@@ -13,8 +13,10 @@ The JSON line reports the configured block (default T=8192), and under
 "workloads" the same block at T=2048 (the weight-bound regime, with its
 fraction of HBM bandwidth) and at every T of the 512..8192 sweep, the single
 W8A8 ConvRot linears (gate|up 4096x3072x2048, down 4096x2048x1536, and
-64x256x256) with their fraction of the INT8 tensor peak, and a dense INT8
-GEMM probe of the tensor peak this library's own kernel reaches.
+64x256x256) with their fraction of the INT8 tensor peak, the six linears of
+one dense-DiT block (4096 tokens, hidden 3840, feed-forward 10240, all with
+the 256-group rotation), and a dense INT8 GEMM probe of the tensor peak this
+library's own kernel reaches.
 
 Multi-GPU (launched by torch.distributed.run): every rank runs its own batch
 of T tokens against the same weights (weak scaling, no data-path
@@ -39,7 +41,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synthetic import LINEAR_CONFIGS, MOE_CONFIGS, linear_inputs, moe_inputs  # noqa: E402
+from synthetic import (DIT_LINEARS, LINEAR_CONFIGS, MOE_CONFIGS, linear_inputs,  # noqa: E402
+                       moe_inputs)
 
 METRIC = "W8A8 ConvRot MoE block tokens/s"
 UNIT = "tokens/s"
@@ -476,12 +479,12 @@ def block_workload(W, cfg, wq, ws, flush_buf, steps, warmup, dev, stream):
             "block": roofline_of(work["ops"], work["block_bytes"], st, load_peaks())}
 
 
-def linear_workloads(W, flush_buf, reps, dev, stream):
+def linear_workloads(W, flush_buf, reps, dev, stream, configs=None):
     """The single W8A8 ConvRot linears through w8a8_convrot_linear (rotation +
     GEMM), and the GEMM alone on the same codes (convrot_i8_gemm_bf16)."""
     peaks = load_peaks()
     out = {}
-    for name, cfg in LINEAR_CONFIGS.items():
+    for name, cfg in (LINEAR_CONFIGS if configs is None else configs).items():
         x, w = linear_inputs(cfg)
         x, w = x.to(dev), w.to(dev)
         w_q, s_w = W.convrot_quantize_weights(w, cfg.group)
@@ -552,6 +555,16 @@ def run_ours(args, cfg, world, rank, local, extras=True):
     torch.cuda.synchronize()
     if W.convrot_check_device_error() != 0:
         raise RuntimeError("device-side wait timed out during warm-up")
+    # the timed steps replay one call captured in a CUDA graph (what a serving
+    # loop does; the host's launch work then stays out of the device timing)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(x, logits, y)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        flush_buf.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
 
     clocks = ClockSampler(dev)
     barrier(world)
@@ -564,13 +577,14 @@ def run_ours(args, cfg, world, rank, local, extras=True):
     for i in range(args.steps):
         flush_buf.zero_()  # L2 flush (write, then read), outside the timed events
         starts[i].record(stream)
-        step(x, logits, y)
+        graph.replay()
         ends[i].record(stream)
     nvtx_pop()
     torch.cuda.synchronize()
     barrier(world)
     wall = time.perf_counter() - wall0
     clk = clocks.stop()
+    del graph
     step_s = [s.elapsed_time(e) * 1e-3 for s, e in zip(starts, ends)]
     mean_step = max_over_ranks(statistics.mean(step_s), world)
 
@@ -608,6 +622,13 @@ def run_ours(args, cfg, world, rank, local, extras=True):
             workloads[name] = block_workload(W, other, wq, big, flush_buf, 20, 3, dev, stream)
         del big
         workloads["linears"] = linear_workloads(W, flush_buf, 10, dev, stream)
+        dit = linear_workloads(W, flush_buf, 5, dev, stream, DIT_LINEARS)
+        tot_us = sum(v["linear_us"] for v in dit.values())
+        tot_ops = sum(2 * v["m"] * v["n"] * v["k"] for v in dit.values())
+        dit["block"] = {"linears": len(DIT_LINEARS), "linear_us_sum": tot_us,
+                        "tops": tot_ops / tot_us / 1e6,
+                        "tensor_frac": tot_ops / tot_us / 1e6 / (2.0 * load_peaks()["bf16_tflops"])}
+        workloads["dense_dit_block"] = dit
         workloads["int8_gemm_probe"] = int8_peak_probe(W, flush_buf, dev, stream)
         flags = W.convrot_check_device_error()
         if flags != 0:
@@ -654,6 +675,7 @@ def run_ours(args, cfg, world, rank, local, extras=True):
         "config": {"workload": cfg.name, "tokens_per_gpu": t, "d": cfg.d, "experts": cfg.n_exp,
                    "f": cfg.f, "capacity": cfg.c, "g_gu": cfg.g_gu, "g_d": cfg.g_d,
                    "parallelism": f"replicas x{world} (independent batches)",
+                   "launch": "timed steps replay one captured CUDA graph of the call; e2e calls it eagerly",
                    "l2": "flushed before every step (256 MiB write + 256 MiB read, outside the timed events)"},
         "roofline_block_frac": block["roofline_frac"],
         "gpu_launches": launches_per_step * args.steps,

@@ -126,7 +126,7 @@ int64_t convrot_swiglu_rq_units(int64_t tiles, int64_t n_blocks, int64_t capacit
  * FP8 Text Encoder", section "Quantization". fp32 arithmetic (see the
  * quantiser note at the top): within one code of the definition.
  *   x      device, [rows, K] bf16 (x_dtype = CONVROT_DTYPE_BF16) or fp32
- *   rows   >= 0;  K: multiple of 16 and of `group`, 16 <= K <= 8192
+ *   rows   >= 0;  K: multiple of 16 and of `group`, 16 <= K <= 16384
  *   group  rotation group g in {1, 4, 16, 64, 256}
  *   q      device, [rows, K] int8 codes (K-contiguous)
  *   scale  device, [rows] fp32 per-row scales

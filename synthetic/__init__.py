@@ -5,6 +5,7 @@ method's arithmetic (no rotation, quantisation, routing or GEMM).
 """
 
 from .workloads import (  # noqa: F401
+    DIT_LINEARS,
     LINEAR_CONFIGS,
     MOE_CONFIGS,
     LinearConfig,

@@ -52,6 +52,26 @@ LINEAR_CONFIGS = {
                                         swiglu_input=True),
 }
 
+# The dense-DiT W8A8 ConvRot linears of one transformer block (the int8
+# ConvRot files of "NitroFusion2 for ComfyUI: int8, W6A8, W4A8", section "How
+# they were made": all linears of the main and refiner blocks -- attention qkv
+# and out, the three feed-forward layers, adaLN -- with a block Hadamard of
+# 256). The page gives 202 linears and 6.142B quantised weights, not their
+# shapes; assumed here: 34 blocks of six linears, hidden size 3840, a SwiGLU
+# feed-forward of 10240 and an adaLN projection of a 256-wide conditioning
+# vector to four modulation vectors, which gives 6.15B weights. Tokens: a
+# 1024x1024 image as 4096 tokens (the one-step model runs without CFG); the
+# adaLN input is one row per image.
+DIT_D, DIT_F = 3840, 10240
+DIT_LINEARS = {
+    "dit_qkv": LinearConfig("dit_qkv", 4096, 3 * DIT_D, DIT_D, 256, 21),
+    "dit_out": LinearConfig("dit_out", 4096, DIT_D, DIT_D, 256, 22),
+    "dit_ffn_gate": LinearConfig("dit_ffn_gate", 4096, DIT_F, DIT_D, 256, 23),
+    "dit_ffn_up": LinearConfig("dit_ffn_up", 4096, DIT_F, DIT_D, 256, 24),
+    "dit_ffn_down": LinearConfig("dit_ffn_down", 4096, DIT_D, DIT_F, 256, 25, swiglu_input=True),
+    "dit_adaln": LinearConfig("dit_adaln", 1, 4 * DIT_D, 256, 256, 26),
+}
+
 MOE_CONFIGS = {
     # 1024x1024 image with batched CFG: 8192 tokens, capacity factor 2
     "moe_T8192": MoEConfig("moe_T8192", 8192, 2048, 64, 1536, 256, 3),

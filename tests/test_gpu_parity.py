@@ -485,6 +485,30 @@ def test_w8a8_linear_parity(name):
     assert _max_rel(np32(y), y_ref) <= 1e-2
 
 
+@pytest.mark.parametrize("name", ["dit_qkv", "dit_out", "dit_ffn_gate", "dit_ffn_down",
+                                  "dit_adaln"])
+def test_dense_dit_linear_parity(name):
+    """The dense-DiT ConvRot linears at full size (K = 3840 and 10240 take the
+    general rotation kernel): weights bit-exact; all activation codes within
+    the budget; 64 sampled output rows bit-exact given the GPU's codes and
+    within 1e-2 of the oracle's linear."""
+    from synthetic import DIT_LINEARS
+    cfg = DIT_LINEARS[name]
+    x, w = linear_inputs(cfg)
+    w_q, s_w = W.convrot_quantize_weights(w.cuda(), cfg.group)
+    y, x_q, s_x = _linear_with_codes(x.cuda(), w_q, s_w, cfg.group)
+    w_q_ref, s_w_ref = O.rotquant(np32(w), cfg.group)
+    assert np.array_equal(w_q.cpu().numpy(), w_q_ref) and np.array_equal(s_w.cpu().numpy(), s_w_ref)
+    x_q, s_x = x_q.cpu().numpy(), s_x.cpu().numpy()
+    check_codes(x_q, s_x, np32(x), cfg.group)
+    rows = np.unique(np.random.default_rng(0).integers(0, cfg.m, 64))
+    y_np = np32(y)
+    assert np.array_equal(y_np[rows], O.w8a8_linear_from_codes(x_q[rows], s_x[rows], w_q_ref,
+                                                                s_w_ref))
+    y_ref = O.w8a8_linear(np32(x)[rows], w_q_ref, s_w_ref, cfg.group)
+    assert _max_rel(y_np[rows], y_ref) <= 1e-2
+
+
 @pytest.mark.parametrize("g", [1, 16, 256])
 def test_linear_rotation_off_ablation(g):
     """The rotation-off ablation (g = 1: per-token / per-channel INT8 with no

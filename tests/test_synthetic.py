@@ -31,3 +31,15 @@ def test_moe_small_shapes():
     assert inp["wgu"].shape == (cfg.n_exp, 2 * cfg.f, cfg.d)
     assert inp["wd"].shape == (cfg.n_exp, cfg.d, cfg.f)
     assert abs(float(inp["wgu"].float().std()) - 0.02) < 0.002
+
+
+def test_dense_dit_block_matches_the_pages_weight_count():
+    """The assumed dense-DiT block: 34 blocks of its six linears hold the
+    6.142B quantised weights of the NitroFusion2 int8 files within 0.2%, and
+    every K is a multiple of the rotation group 256."""
+    from synthetic import DIT_LINEARS
+    per_block = sum(c.n * c.k for c in DIT_LINEARS.values())
+    assert abs(34 * per_block / 6.142e9 - 1) < 2e-3
+    assert len(DIT_LINEARS) * 34 == 204  # the page counts 202 quantised linears
+    for c in DIT_LINEARS.values():
+        assert c.k % 256 == 0 and c.group == 256

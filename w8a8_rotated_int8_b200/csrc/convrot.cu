@@ -316,7 +316,7 @@ int check_rq_args(const void* x, int x_dtype, int64_t rows, int64_t K, int group
   if (x_dtype != CONVROT_DTYPE_BF16 && x_dtype != CONVROT_DTYPE_F32) return CONVROT_ERR_INVALID_ARG;
   if (rows < 0 || rows >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
   if (!valid_group(group)) return CONVROT_ERR_INVALID_ARG;
-  if (K < 16 || K > 8192 || K % 16 != 0 || K % group != 0) return CONVROT_ERR_INVALID_ARG;
+  if (K < 16 || K > 16384 || K % 16 != 0 || K % group != 0) return CONVROT_ERR_INVALID_ARG;
   if (rows > 0 && (!x || !q || !s)) return CONVROT_ERR_INVALID_ARG;
   if (!al16(x) || !al16(q) || !al16(s)) return CONVROT_ERR_MISALIGNED;
   return CONVROT_OK;
@@ -1151,7 +1151,7 @@ extern "C" int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_
   if ((rc = check_gemm_shape(w_q, w_q, 1, M, N, K)) != CONVROT_OK) return rc;
   if (M > 0 && N > 0 && (!w_scale || !y_bf16)) return CONVROT_ERR_INVALID_ARG;
   if (!al16(w_scale) || !al16(y_bf16)) return CONVROT_ERR_MISALIGNED;
-  // K <= 8192 and M < 2^31 hold here, so M * K cannot overflow
+  // K <= 16384 and M < 2^31 hold here, so M * K cannot overflow
   if (M > CONVROT_NOALLOC_MAX_ROWS || M * K > (int64_t)CONVROT_NOALLOC_MAX_CODES)
     return CONVROT_ERR_WORKSPACE_TOO_SMALL;
   if ((rc = device_setup(nullptr)) != CONVROT_OK) return rc;

@@ -181,13 +181,13 @@ __device__ __forceinline__ int64_t rq_dst(const RqOut& o, int64_t row, int K, in
 // rows_per_cta consecutive rows) and loads its next group's chunk before
 // computing the current one.
 template <typename InT, int G>
-__global__ void __launch_bounds__(512) rotquant_kernel(const InT* __restrict__ x, int64_t rows,
+__global__ void __launch_bounds__(1024) rotquant_kernel(const InT* __restrict__ x, int64_t rows,
                                                       int K, int tpr, int8_t* __restrict__ q,
                                                       float* __restrict__ scales, RqOut out) {
   griddep_launch_dependents();
   griddep_wait();
   using Tr = RqTraits<G>;
-  __shared__ float red[2][16];  // per-warp maxima (512 threads at most), by iteration parity
+  __shared__ float red[2][32];  // per-warp maxima (1024 threads at most), by iteration parity
   const int lane = threadIdx.x & 31;
   const int rows_per_cta = blockDim.x / tpr;
   const int r_local = threadIdx.x / tpr;
