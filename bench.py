@@ -759,6 +759,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-extras", dest="extras", action="store_false",
                     help="only the configured block (no other T, linears or INT8 probe)")
+    ap.add_argument("--only-linears", action="store_true",
+                    help="only the single W8A8 ConvRot linears and the dense-DiT block's linears "
+                         "(one JSON line; used to profile the linear GEMMs)")
     ap.add_argument("--ablation", action="store_true",
                     help="rotation-off ablation: block error with and without ConvRot")
     ap.add_argument("--traffic-bytes", type=float, default=None,
@@ -771,6 +774,18 @@ def main():
     cfg = MOE_CONFIGS[args.config]
     if args.ablation:
         run_ablation(args, cfg)
+        return
+    if args.only_linears:
+        import w8a8_rotated_int8_b200 as W
+        W.load_library()
+        dev = torch.device("cuda", 0)
+        flush_buf = L2Flush(dev)
+        stream = torch.cuda.current_stream()
+        line = {"metric": "W8A8 ConvRot linears", "data": "synthetic (seeded)",
+                "linears": linear_workloads(W, flush_buf, args.steps, dev, stream),
+                "dense_dit_block": linear_workloads(W, flush_buf, args.steps, dev, stream,
+                                                    DIT_LINEARS)}
+        print(json.dumps(line), flush=True)
         return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
