@@ -479,6 +479,87 @@ def block_workload(W, cfg, wq, ws, flush_buf, steps, warmup, dev, stream):
             "block": roofline_of(work["ops"], work["block_bytes"], st, load_peaks())}
 
 
+def lowbit_work(cfg, t, bits):
+    """Ops and compulsory bytes of the block with b-bit expert weights: the
+    packed codes (bits/8 bytes per weight), one E4M3 byte per 16 weights and
+    the FP32 row scales once, X and logits in, Y out; and of its two GEMMs
+    (weights + scales)."""
+    e, c, d, f = cfg.n_exp, cfg.c, cfg.d, cfg.f
+
+    def wbytes(n_w, rows):
+        return n_w * bits // 8 + n_w // 16 + rows * 4
+
+    gu = wbytes(e * 2 * f * d, e * 2 * f)
+    dn = wbytes(e * d * f, e * d)
+    return {"ops": 2 * e * c * (d * 2 * f + f * d),
+            "block_bytes": gu + dn + t * d * 2 + t * e * 2 + t * d * 2,
+            "gateup_alg": {"ops": 2 * e * c * d * 2 * f, "bytes": gu},
+            "down_alg": {"ops": 2 * e * c * f * d, "bytes": dn}}
+
+
+def roofline_f16(ops, nbytes, seconds, peaks):
+    """Both fractions for the low-bit path, whose contraction runs on the
+    kind::f16 tensor cores: the tensor peak is the measured bf16 burst (f16
+    and bf16 have the same dense rate)."""
+    tc = peaks["bf16_tflops"]
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = ops / (tc * 1e12)
+    gbs = nbytes / seconds / 1e9
+    tops = ops / seconds / 1e12
+    return {"bound": "hbm" if t_hbm >= t_tc else "tensor",
+            "ideal_us": max(t_hbm, t_tc) * 1e6, "roofline_frac": max(t_hbm, t_tc) / seconds,
+            "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+            "tflops": tops, "tensor_frac": tops / tc}
+
+
+def lowbit_workloads(W, wgu, wd, g_gu, g_d, flush_buf, steps, dev, stream,
+                     names=("moe_T512", "moe_T2048", "moe_T8192")):
+    """The MoE block with W4A8 and W6A8 expert weights (the same bf16 model
+    quantised to the b-bit formats) at several T, and its two GEMMs alone on
+    the call's own intermediates."""
+    peaks = load_peaks()
+    out = {}
+    for bits in (4, 6):
+        gu, dn = W.quantize_moe_weights_lowbit(wgu, wd, bits, g_gu, g_d)
+        for name in names:
+            cfg = MOE_CONFIGS[name]
+            inp = moe_inputs(cfg, weights=False)
+            x, logits = inp["x"].to(dev), inp["logits"].to(dev)
+            y = torch.empty((cfg.t, cfg.d), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(W.moe_workspace_size(cfg.t, cfg.d, cfg.f, cfg.n_exp, cfg.c),
+                             dtype=torch.uint8, device=dev)
+
+            def step():
+                W.moe_expert_choice_forward_lowbit(x, logits, gu, dn, cfg.c, g_gu, g_d, y=y,
+                                                   workspace=ws)
+
+            timed(step, 3, flush_buf, stream)
+            st = statistics.mean(timed(step, steps, flush_buf, stream))
+            v = W.moe_stage_views(ws, cfg.t, cfg.d, cfg.f, cfg.n_exp, cfg.c)
+            g1 = lambda: W.convrot_lowbit_gemm(v["x_g"], v["s_g"], gu, W.CONVROT_LOWBIT_SWIGLU,  # noqa: E731
+                                               out=v["h"])
+            g2 = lambda: W.convrot_lowbit_gemm(v["h_q"], v["s_h"], dn, W.CONVROT_LOWBIT_BF16,  # noqa: E731
+                                               out=v["z"])
+            timed(g1, 3, flush_buf, stream)
+            t1 = statistics.median(timed(g1, steps, flush_buf, stream))
+            timed(g2, 3, flush_buf, stream)
+            t2 = statistics.median(timed(g2, steps, flush_buf, stream))
+            work = lowbit_work(cfg, cfg.t, bits)
+            out[f"w{bits}a8_{name}"] = {
+                "bits": bits, "tokens": cfg.t, "capacity": cfg.c,
+                "ms_per_step": st * 1e3, "tokens_per_s": cfg.t / st,
+                "block": roofline_f16(work["ops"], work["block_bytes"], st, peaks),
+                "gemm_gateup_swiglu_us": t1 * 1e6,
+                "gemm_gateup_swiglu": roofline_f16(work["gateup_alg"]["ops"],
+                                                   work["gateup_alg"]["bytes"], t1, peaks),
+                "gemm_down_bf16_us": t2 * 1e6,
+                "gemm_down_bf16": roofline_f16(work["down_alg"]["ops"], work["down_alg"]["bytes"],
+                                               t2, peaks)}
+            del ws
+        del gu, dn
+    return out
+
+
 def linear_workloads(W, flush_buf, reps, dev, stream, configs=None):
     """The single W8A8 ConvRot linears through w8a8_convrot_linear (rotation +
     GEMM), and the GEMM alone on the same codes (convrot_i8_gemm_bf16)."""
@@ -630,6 +711,8 @@ def run_ours(args, cfg, world, rank, local, extras=True):
                         "tensor_frac": tot_ops / tot_us / 1e6 / (2.0 * load_peaks()["bf16_tflops"])}
         workloads["dense_dit_block"] = dit
         workloads["int8_gemm_probe"] = int8_peak_probe(W, flush_buf, dev, stream)
+        workloads["lowbit"] = lowbit_workloads(W, inp["wgu"].to(dev), inp["wd"].to(dev), cfg.g_gu,
+                                               cfg.g_d, flush_buf, 10, dev, stream)
         flags = W.convrot_check_device_error()
         if flags != 0:
             raise RuntimeError(f"device error flags {flags:#x}")
@@ -762,6 +845,8 @@ def main():
     ap.add_argument("--only-linears", action="store_true",
                     help="only the single W8A8 ConvRot linears and the dense-DiT block's linears "
                          "(one JSON line; used to profile the linear GEMMs)")
+    ap.add_argument("--only-lowbit", action="store_true",
+                    help="only the W4A8 / W6A8 blocks and their GEMMs (one JSON line)")
     ap.add_argument("--ablation", action="store_true",
                     help="rotation-off ablation: block error with and without ConvRot")
     ap.add_argument("--traffic-bytes", type=float, default=None,
@@ -785,6 +870,19 @@ def main():
                 "linears": linear_workloads(W, flush_buf, args.steps, dev, stream),
                 "dense_dit_block": linear_workloads(W, flush_buf, args.steps, dev, stream,
                                                     DIT_LINEARS)}
+        print(json.dumps(line), flush=True)
+        return
+    if args.only_lowbit:
+        import w8a8_rotated_int8_b200 as W
+        W.load_library()
+        dev = torch.device("cuda", 0)
+        inp = moe_inputs(cfg)
+        line = {"metric": "W4A8 / W6A8 ConvRot MoE block", "data": "synthetic (seeded)",
+                "lowbit": lowbit_workloads(W, inp["wgu"].to(dev), inp["wd"].to(dev), cfg.g_gu,
+                                           cfg.g_d, L2Flush(dev), args.steps, dev,
+                                           torch.cuda.current_stream())}
+        if W.convrot_check_device_error() != 0:
+            raise RuntimeError("device error flags set")
         print(json.dumps(line), flush=True)
         return
     if args.impl == "reference":

@@ -351,7 +351,8 @@ typedef struct {
   size_t w;        /* [E, C] fp32     router weights of the choices */
   size_t x_g;      /* [E, C, d] int8  gathered codes                */
   size_t s_g;      /* [E, C] fp32     gathered scales               */
-  size_t h;        /* [E, C, f] fp32  silu(gate) * up (g_d = 256 only) */
+  size_t h;        /* [E, C, f] fp32  silu(gate) * up (g_d = 256, and the
+                      low-bit block)                                */
   size_t h_q;      /* [E, C, f] int8  rotated, requantised h        */
   size_t s_h;      /* [E, C] fp32     scales of h                   */
   size_t hsync;    /* convrot_swiglu_rq_sync_bytes(E, C) bytes: scratch of
@@ -368,6 +369,88 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
                               const float* s_gu, const int8_t* w_d, const float* s_d, int64_t T,
                               int64_t d, int64_t f, int E, int64_t C, int g_gu, int g_d,
                               void* y_bf16, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * W4A8 / W6A8 in the rotated basis.
+ * "NitroFusion2 for ComfyUI: int8, W6A8, W4A8", section "How they were made":
+ * 6-bit or 4-bit weights in the rotated basis with an FP8 scale per group of
+ * 16, 8-bit activations. Readings fixed by this library:
+ *  - the rotation is the int8 format's (same groups);
+ *  - codes q in [-qmax, qmax], qmax = 7 (bits = 4) or 31 (bits = 6), nearest
+ *    rounding, ties to even;
+ *  - FP8 = E4M3 (bias 7, 3 mantissa bits, subnormals, largest value 448);
+ *  - two scale levels per weight row v' (rotated, fp64): s_r = fp32(a /
+ *    (qmax * 448)) with a = max|v'|; for each group j of 16 consecutive
+ *    elements sigma_j = e4m3(a_j / (qmax * s_r)) (nearest, ties to the even
+ *    code, saturating at 448); q = clamp(rne(v' / (s_r * sigma_j))); a zero
+ *    row or a group with sigma 0 has zero codes. A weight decodes to
+ *    s_r * sigma_j * q;
+ *  - activations: per-token INT8 as in the int8 format; the linear is
+ *    y = fp32(acc) * (s_x * s_r), acc = sum_k x_q * sigma * q.
+ * The quantiser computes the definition exactly (fp64 rotation and
+ * quotients). The GEMM accumulates acc in fp32 on the tensor cores (kind::f16
+ * over exact fp16 operands), so acc differs from the exact sum by fp32
+ * rounding only: |error| <= K * 2^-23 * sum_k |x_q * sigma * q|.
+ *
+ * Packed format of `rows` x K weights (rows % 128 == 0, K % 64 == 0),
+ * convrot_lowbit_weight_bytes(rows, K, bits) bytes: tiles of 128 rows x 64
+ * codes, tile (row block rb, k-block kb) at (rb * K/64 + kb) * T bytes with
+ * T = 4608 (bits = 4) or 6656 (bits = 6), holding bits/2 planes of
+ * [128 rows][16 bytes] (plane c = bytes 16c .. 16c+15 of each row's packed
+ * codes) and then [128 rows][4 bytes] of E4M3 scales (the row's four groups
+ * of the k-block, lowest group in the lowest byte). A row's packed codes
+ * store u = q + 2^(bits-1): 32-bit words w_0 .. w_7 hold the low four bits,
+ * code 8i+2j in bits 4j..4j+3 of w_i and code 8i+2j+1 in bits 16+4j..19+4j
+ * (j = 0..3); for bits = 6 words w_8 .. w_11 hold the top two bits, code
+ * 16i+2j in bits 2j..2j+1 of w_{8+i} and code 16i+2j+1 in bits 16+2j..17+2j
+ * (j = 0..7). Row blocks of consecutive matrices follow each other.
+ * ------------------------------------------------------------------------- */
+/* Bytes of the packed format; -1 for bits not 4 / 6, rows % 128 or K % 64. */
+int64_t convrot_lowbit_weight_bytes(int64_t rows, int64_t K, int bits);
+
+/* Offline: rotate bf16 weight rows [rows, K] (device) with `group` and
+ * quantise them to the b-bit format: w_packed (device) as above, row_scale
+ * (device) [rows] fp32. 64 <= K <= 16384, K % group == 0. */
+int convrot_quantize_weights_lowbit(const void* w_bf16, int64_t rows, int64_t K, int group,
+                                    int bits, void* w_packed, float* row_scale, void* stream);
+
+/* Grouped low-bit GEMM stage: for every group g,
+ *   acc[g, m, n] = sum_k x_q[g, m, k] * sigma[g, n, k/16] * q[g, n, k]
+ * with x_q (device) [G, M, K] int8, s_x (device) [G*M] fp32, w_packed
+ * (device) G matrices of N rows in the packed format, row_scale (device)
+ * [G*N] fp32. epilogue:
+ *   CONVROT_LOWBIT_F32     out fp32 [G, M, N] = acc (s_x unused)
+ *   CONVROT_LOWBIT_BF16    out bf16 [G, M, N] = bf16(acc * (s_x * s_r))
+ *   CONVROT_LOWBIT_SWIGLU  out fp32 [G, M, N/2] = silu(y[:, f]) * y[:, N/2 + f]
+ *                          with y = acc * (s_x * s_r) (gate rows first)
+ * N % 256 == 0; 64 <= K <= 16384, K % 64 == 0. tile_tokens = tokens per
+ * tile (a multiple of 16, at most 128), 0 = chosen by the library. */
+enum { CONVROT_LOWBIT_F32 = 0, CONVROT_LOWBIT_BF16 = 1, CONVROT_LOWBIT_SWIGLU = 2 };
+int convrot_lowbit_gemm(const int8_t* x_q, const float* s_x, const void* w_packed,
+                        const float* row_scale, int64_t G, int64_t M, int64_t N, int64_t K,
+                        int bits, int epilogue, int tile_tokens, void* out, void* stream);
+
+/* WbA8 ConvRot linear: x (device) [M, K] bf16 rotated with `group` and
+ * quantised per token to INT8, then y (device) [M, N] bf16 =
+ * bf16(acc * (s_x * s_r)) against b-bit weights. Workspace (device):
+ * convrot_linear_workspace_size(M, K) bytes. N % 256 == 0, K % 64 == 0. */
+int lowbit_convrot_linear(const void* x_bf16, int64_t M, int64_t K, const void* w_packed,
+                          const float* row_scale, int64_t N, int group, int bits, void* y_bf16,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* The expert-choice MoE block of moe_expert_choice_forward with b-bit expert
+ * weights: w_gu (device) E matrices of 2f rows x d in the packed format (gate
+ * rows then up rows per expert), s_gu [E, 2f]; w_d (device) E matrices of d
+ * rows x f, s_d [E, d]. Routing, the activation and h quantisation and the
+ * combine are the int8 block's; h goes through the workspace's fp32 region.
+ * The workspace and its layout are moe_workspace_layout's. d % 256 == 0,
+ * f % 128 == 0 (besides d % g_gu == 0, f % g_d == 0). Failure of a
+ * device-side wait as for moe_expert_choice_forward. */
+int moe_expert_choice_forward_lowbit(const void* x_bf16, const void* logits_bf16,
+                                     const void* w_gu, const float* s_gu, const void* w_d,
+                                     const float* s_d, int64_t T, int64_t d, int64_t f, int E,
+                                     int64_t C, int g_gu, int g_d, int bits, void* y_bf16,
+                                     void* workspace, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -121,3 +121,41 @@ def test_requantising_gemm_plan_falls_back_when_too_few_ctas_fit(lib):
     assert units(30, 12, 74) == 30             # every tile fits at once
     assert units(0, 12, 74) == 0
     assert units(-1, 12, 74) == -1
+
+
+def test_lowbit_argument_checks_need_no_gpu(lib):
+    """W4A8 / W6A8 entry points: format sizes and host-side rejections."""
+    al = ctypes.c_void_p(4096)
+    mis = ctypes.c_void_p(4096 + 8)
+    INVALID, MISALIGNED = binding.CONVROT_ERR_INVALID_ARG, binding.CONVROT_ERR_MISALIGNED
+    # tiles of 128 rows x 64 codes: 2 planes + 512 scale bytes (4-bit), 3 planes (6-bit)
+    assert lib.convrot_lowbit_weight_bytes(128, 64, 4) == 4608
+    assert lib.convrot_lowbit_weight_bytes(6144, 2048, 6) == 48 * 32 * 6656
+    assert lib.convrot_lowbit_weight_bytes(128, 64, 8) == -1
+    assert lib.convrot_lowbit_weight_bytes(200, 64, 4) == -1
+    assert lib.convrot_lowbit_weight_bytes(128, 96, 4) == -1
+    q = lib.convrot_quantize_weights_lowbit
+    assert q(al, 128, 256, 256, 5, al, al, None) == INVALID       # bits
+    assert q(al, 100, 256, 256, 4, al, al, None) == INVALID       # rows % 128
+    assert q(al, 128, 320, 256, 4, al, al, None) == INVALID       # K % group
+    assert q(al, 128, 96, 16, 4, al, al, None) == INVALID         # K % 64
+    assert q(al, 128, 256, 128, 4, al, al, None) == INVALID       # group not a power of four
+    assert q(mis, 128, 256, 256, 4, al, al, None) == MISALIGNED
+    g = lib.convrot_lowbit_gemm
+    assert g(al, al, al, al, 1, 64, 128, 256, 4, 1, 0, al, None) == INVALID   # N % 256
+    assert g(al, al, al, al, 1, 64, 256, 96, 4, 1, 0, al, None) == INVALID    # K % 64
+    assert g(al, al, al, al, 1, 64, 256, 256, 4, 3, 0, al, None) == INVALID   # epilogue
+    assert g(al, al, al, al, 1, 64, 256, 256, 4, 1, 24, al, None) == INVALID  # tile tokens
+    assert g(al, al, al, al, 1, 64, 256, 256, 4, 1, 144, al, None) == INVALID
+    assert g(mis, al, al, al, 1, 64, 256, 256, 4, 1, 0, al, None) == MISALIGNED
+    lin = lib.lowbit_convrot_linear
+    assert lin(al, 64, 256, al, al, 256, 256, 4, al, al, 16, None) == \
+        binding.CONVROT_ERR_WORKSPACE_TOO_SMALL
+    assert lin(al, 64, 256, al, al, 384, 256, 4, al, al, 1 << 20, None) == INVALID
+    m = lib.moe_expert_choice_forward_lowbit
+    args = [al] * 6
+    assert m(*args, 8, 256, 192, 4, 2, 256, 64, 4, al, al, 1 << 30, None) == INVALID  # f % 128
+    assert m(*args, 8, 320, 128, 4, 2, 64, 64, 4, al, al, 1 << 30, None) == INVALID   # d % 256
+    assert m(*args, 8, 256, 128, 4, 2, 256, 64, 5, al, al, 1 << 30, None) == INVALID  # bits
+    assert (m(*args, 8, 256, 128, 4, 2, 256, 64, 4, al, al, 16, None)
+            == binding.CONVROT_ERR_WORKSPACE_TOO_SMALL)

@@ -83,6 +83,12 @@ _SIGNATURES = {
     "moe_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I64]),
     "moe_expert_choice_forward": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I64, _I, _I,
                                        _P, _P, _SZ, _P]),
+    "convrot_lowbit_weight_bytes": (_I64, [_I64, _I64, _I]),
+    "convrot_quantize_weights_lowbit": (_I, [_P, _I64, _I64, _I, _I, _P, _P, _P]),
+    "convrot_lowbit_gemm": (_I, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _I, _P, _P]),
+    "lowbit_convrot_linear": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _I, _P, _P, _SZ, _P]),
+    "moe_expert_choice_forward_lowbit": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I, _I64,
+                                              _I, _I, _I, _P, _P, _SZ, _P]),
 }
 
 
@@ -487,3 +493,117 @@ def moe_stage_views(workspace, t, d, f, e, c) -> dict:
         "slot": view("slot", torch.int32, (e, t)),
         "z": view("z", torch.bfloat16, (e, c, d)),
     }
+
+
+# ------------------------------------------------------- W4A8 / W6A8 --------
+CONVROT_LOWBIT_F32, CONVROT_LOWBIT_BF16, CONVROT_LOWBIT_SWIGLU = 0, 1, 2
+
+
+def lowbit_weight_bytes(rows, k, bits) -> int:
+    return int(lib().convrot_lowbit_weight_bytes(rows, k, bits))
+
+
+class LowbitWeights:
+    """Weights in the packed b-bit format (uint8 bytes) plus their FP32 row
+    scales; `rows` rows of each of `n_mats` matrices, K columns."""
+
+    def __init__(self, data, scale, n_mats, rows, k, bits):
+        self.data, self.scale = data, scale
+        self.n_mats, self.rows, self.k, self.bits = n_mats, rows, k, bits
+
+
+def convrot_quantize_weights_lowbit(w, group, bits, n_mats=1, stream=None):
+    """Offline: bf16 weight rows [..., K] (n_mats matrices stacked along the
+    rows, each a multiple of 128 rows) -> LowbitWeights."""
+    _need(w, torch.bfloat16, "w")
+    k = w.shape[-1]
+    total = w.numel() // k
+    if total % n_mats:
+        raise ValueError("rows must split evenly into n_mats matrices")
+    nbytes = lowbit_weight_bytes(total, k, bits)
+    if nbytes < 0:
+        raise ValueError("rows must be a multiple of 128 and K of 64; bits 4 or 6")
+    data = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=w.device)
+    scale = torch.empty((total,), dtype=torch.float32, device=w.device)
+    _invoke(w, "convrot_quantize_weights_lowbit", _p(w), total, k, group, bits, _p(data),
+            _p(scale), stream=stream)
+    return LowbitWeights(data, scale, n_mats, total // n_mats, k, bits)
+
+
+def convrot_lowbit_gemm(a, s_a, w: LowbitWeights, epilogue=CONVROT_LOWBIT_BF16, tile_tokens=0,
+                        out=None, stream=None):
+    """Grouped low-bit GEMM: a [G, M, K] int8 codes (s_a [G, M] fp32) against
+    the G matrices of w. epilogue F32 -> acc [G, M, N] fp32; BF16 -> y bf16;
+    SWIGLU -> h [G, M, N/2] fp32."""
+    _need(a, torch.int8, "a")
+    if s_a is not None:
+        _need(s_a, torch.float32, "s_a")
+    g, m, k = a.shape
+    if w.n_mats != g or w.k != k:
+        raise ValueError("weights do not match a")
+    n = w.rows
+    if epilogue == CONVROT_LOWBIT_BF16:
+        shape, dtype = (g, m, n), torch.bfloat16
+    elif epilogue == CONVROT_LOWBIT_SWIGLU:
+        shape, dtype = (g, m, n // 2), torch.float32
+    else:
+        shape, dtype = (g, m, n), torch.float32
+    if out is None:
+        out = torch.empty(shape, dtype=dtype, device=a.device)
+    elif out.numel() != g * m * (n // 2 if epilogue == CONVROT_LOWBIT_SWIGLU else n):
+        raise ValueError("out has the wrong size")
+    else:
+        _need(out, dtype, "out")
+    _invoke(a, "convrot_lowbit_gemm", _p(a), _p(s_a), _p(w.data), _p(w.scale), g, m, n, k,
+            w.bits, epilogue, tile_tokens, _p(out), stream=stream)
+    return out
+
+
+def lowbit_convrot_linear(x, w: LowbitWeights, group, y=None, workspace=None, stream=None):
+    """Y[M, N] bf16 = WbA8 ConvRot linear of x [M, K] bf16 against b-bit weights."""
+    _need(x, torch.bfloat16, "x")
+    m, k = x.shape
+    if w.n_mats != 1 or w.k != k:
+        raise ValueError("weights do not match x")
+    n = w.rows
+    ws_bytes = convrot_linear_workspace_size(m, k)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=x.device)
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    _invoke(x, "lowbit_convrot_linear", _p(x), m, k, _p(w.data), _p(w.scale), n, group, w.bits,
+            _p(y), _p(workspace), workspace.numel(), stream=stream)
+    return y
+
+
+def quantize_moe_weights_lowbit(wgu, wd, bits, g_gu=256, g_d=64, stream=None):
+    """Offline: bf16 wgu [E, 2f, d] and wd [E, d, f] -> LowbitWeights (E matrices each)."""
+    e = wgu.shape[0]
+    gu = convrot_quantize_weights_lowbit(wgu.reshape(-1, wgu.shape[-1]), g_gu, bits, e,
+                                         stream=stream)
+    dn = convrot_quantize_weights_lowbit(wd.reshape(-1, wd.shape[-1]), g_d, bits, e,
+                                         stream=stream)
+    return gu, dn
+
+
+def moe_expert_choice_forward_lowbit(x, logits, w_gu: LowbitWeights, w_d: LowbitWeights, c,
+                                     g_gu=256, g_d=64, y=None, workspace=None, stream=None):
+    """The expert-choice MoE block with b-bit expert weights (from
+    quantize_moe_weights_lowbit); x [T, d] bf16, logits [T, E] bf16 -> y."""
+    _need(x, torch.bfloat16, "x")
+    _need(logits, torch.bfloat16, "logits")
+    t, d = x.shape
+    e = logits.shape[1]
+    f = w_gu.rows // 2
+    if (w_gu.n_mats != e or w_gu.k != d or w_d.n_mats != e or w_d.rows != d or w_d.k != f
+            or w_gu.bits != w_d.bits):
+        raise ValueError("weights do not match x / logits")
+    size = moe_workspace_size(t, d, f, e, c)
+    if workspace is None:
+        workspace = torch.empty((max(size, 16),), dtype=torch.uint8, device=x.device)
+    if y is None:
+        y = torch.empty((t, d), dtype=torch.bfloat16, device=x.device)
+    _invoke(x, "moe_expert_choice_forward_lowbit", _p(x), _p(logits), _p(w_gu.data),
+            _p(w_gu.scale), _p(w_d.data), _p(w_d.scale), t, d, f, e, c, g_gu, g_d, w_gu.bits,
+            _p(y), _p(workspace), workspace.numel(), stream=stream)
+    return y

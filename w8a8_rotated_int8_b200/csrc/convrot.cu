@@ -14,6 +14,7 @@
 #include "convrot.h"
 #include "common.cuh"
 #include "gemm_tcgen05.cuh"
+#include "lowbit.cuh"
 #include "rotquant.cuh"
 #include "routing.cuh"
 
@@ -62,6 +63,19 @@ void set_gemm_attr() {
                        cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<EPI>::kSmem1);
   cudaFuncSetAttribute(gemm_s8_tcgen05_pair_kernel<EPI, BT>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<EPI>::kSmem2);
+}
+
+template <int BITS, int EPI>
+void set_lowbit_attr() {
+  cudaFuncSetAttribute(gemm_lowbit_tcgen05_kernel<BITS, EPI>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, lb::smem_bytes<BITS>());
+}
+
+template <int BITS>
+void set_lowbit_attrs() {
+  set_lowbit_attr<BITS, kLbF32>();
+  set_lowbit_attr<BITS, kLbBf16>();
+  set_lowbit_attr<BITS, kLbSwiglu>();
 }
 
 // every GEMM instantiation the entry points launch
@@ -125,6 +139,8 @@ int device_setup(int* sm_count) {
     if (d.supported) {
       set_gemm_attrs<false>();
       set_gemm_attrs<true>();
+      set_lowbit_attrs<4>();
+      set_lowbit_attrs<6>();
       if (cudaGetLastError() != cudaSuccess) return CONVROT_ERR_CUDA;
       if (swiglu_rq_residency(sms, &d.rq_ctas, &d.rq_pairs) != CONVROT_OK) {
         cudaGetLastError();
@@ -663,6 +679,136 @@ int convert_impl(const float* x, int64_t n, void* y, int sms, cudaStream_t st) {
   return launch_status();
 }
 
+// ---------------------------------------------------------------- low-bit --
+inline bool valid_bits(int bits) { return bits == 4 || bits == 6; }
+
+int lowbit_tile_bytes(int bits) {
+  return bits == 4 ? LbFmt<4>::kTileBytes : LbFmt<6>::kTileBytes;
+}
+
+// Bytes of the b-bit weight format for `rows` x K (rows % 128 == 0, K % 64 == 0).
+int64_t lowbit_bytes(int64_t rows, int64_t K, int bits) {
+  return (rows / 128) * (K / 64) * (int64_t)lowbit_tile_bytes(bits);
+}
+
+template <int G, int BITS>
+int launch_lowbit_quant(const void* w, int64_t rows, int K, uint8_t* out, float* s,
+                        cudaStream_t st) {
+  auto kern = lowbit_quant_f64_kernel<G, BITS>;
+  const size_t smem = (size_t)K * sizeof(double);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLbQuantThreads, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  int sms = 0;
+  device_setup(&sms);
+  const int64_t grid = std::min<int64_t>(rows, (int64_t)per_sm * std::max(sms, 1));
+  return launch_kernel(kern, dim3((unsigned)grid), dim3(kLbQuantThreads), smem, st, false, 1,
+                       reinterpret_cast<const __nv_bfloat16*>(w), rows, K, out, s);
+}
+
+template <int BITS>
+int lowbit_quant_group(const void* w, int64_t rows, int K, int group, uint8_t* out, float* s,
+                       cudaStream_t st) {
+  switch (group) {
+    case 1: return launch_lowbit_quant<1, BITS>(w, rows, K, out, s, st);
+    case 4: return launch_lowbit_quant<4, BITS>(w, rows, K, out, s, st);
+    case 16: return launch_lowbit_quant<16, BITS>(w, rows, K, out, s, st);
+    case 64: return launch_lowbit_quant<64, BITS>(w, rows, K, out, s, st);
+    default: return launch_lowbit_quant<256, BITS>(w, rows, K, out, s, st);
+  }
+}
+
+// 3-D view {K, rows, groups} of int8 activation codes, box {64 codes,
+// box_rows rows, 1}, no swizzle (the converters read it row by row).
+int encode_act_i8(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint64_t groups,
+                  uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return CONVROT_ERR_CUDA;
+  const cuuint64_t dims[3] = {K, rows, groups};
+  const cuuint64_t strides[2] = {K, K * rows};
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+// Tokens per tile when the caller leaves it open: one tile of all the tokens
+// up to 64 (two accumulator buffers), else 128 (one).
+int lowbit_auto_nt(int64_t M) {
+  return M <= 64 ? (int)std::max<int64_t>(16, cdiv(M, 16) * 16) : lb::kMaxNt;
+}
+
+int check_lowbit_gemm(const int8_t* x, const void* wq, int64_t G, int64_t M, int64_t N,
+                      int64_t K, int bits, int tile_tokens) {
+  if (!valid_bits(bits)) return CONVROT_ERR_INVALID_ARG;
+  if (G < 0 || M < 0 || N < 0 || K < 64 || K > 16384 || K % 64 != 0 || N % 256 != 0)
+    return CONVROT_ERR_INVALID_ARG;
+  if (G >= ((int64_t)1 << 31) || M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) ||
+      G * M >= ((int64_t)1 << 31) || G * N >= ((int64_t)1 << 31))
+    return CONVROT_ERR_INVALID_ARG;
+  if (tile_tokens != 0 && (tile_tokens < 16 || tile_tokens > lb::kMaxNt || tile_tokens % 16))
+    return CONVROT_ERR_INVALID_ARG;
+  if (G * M > 0 && N > 0 && (!x || !wq)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(x) || !al16(wq)) return CONVROT_ERR_MISALIGNED;
+  return CONVROT_OK;
+}
+
+template <int BITS, int EPI>
+int launch_lowbit_gemm(const int8_t* x, const float* s_x, const uint8_t* wq, const float* s_w,
+                       int64_t G, int64_t M, int64_t N, int64_t K, int tile_tokens, void* out,
+                       cudaStream_t st, bool pdl = false) {
+  int sms = 0;
+  int rc = device_setup(&sms);
+  if (rc != CONVROT_OK) return rc;
+  if (G == 0 || M == 0 || N == 0) return CONVROT_OK;
+  LowbitArgs a{};
+  a.G = (int)G;
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.n_out = (int)(EPI == kLbSwiglu ? N / 2 : N);
+  a.nt = tile_tokens > 0 ? tile_tokens : lowbit_auto_nt(M);
+  a.box_rows = (int)std::min<int64_t>(a.nt, M);
+  a.t_blocks = (int)cdiv(M, a.nt);
+  a.w_blocks = (int)(N / 256);
+  a.k_blocks = (int)(K / 64);
+  const int64_t tiles = G * a.w_blocks * a.t_blocks;
+  if (tiles >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
+  a.num_tiles = (int)tiles;
+  a.n_acc = 4 * a.nt <= 256 ? 2 : 1;
+  a.wq = wq;
+  a.s_w = s_w;
+  a.s_x = s_x;
+  a.out = out;
+  CUtensorMap tx;
+  if ((rc = encode_act_i8(&tx, x, (uint64_t)K, (uint64_t)M, (uint64_t)G, (uint32_t)a.box_rows)) !=
+      CONVROT_OK)
+    return rc;
+  const int grid = (int)std::min<int64_t>(tiles, sms);
+  if ((rc = launch_kernel(gemm_lowbit_tcgen05_kernel<BITS, EPI>, dim3(grid), dim3(lb::kThreads),
+                          lb::smem_bytes<BITS>(), st, pdl, 1, tx, a)) != CONVROT_OK)
+    return rc;
+  return launch_status();
+}
+
+template <int EPI>
+int launch_lowbit_bits(int bits, const int8_t* x, const float* s_x, const void* wq,
+                       const float* s_w, int64_t G, int64_t M, int64_t N, int64_t K,
+                       int tile_tokens, void* out, cudaStream_t st, bool pdl = false) {
+  const uint8_t* w = reinterpret_cast<const uint8_t*>(wq);
+  if (bits == 4)
+    return launch_lowbit_gemm<4, EPI>(x, s_x, w, s_w, G, M, N, K, tile_tokens, out, st, pdl);
+  return launch_lowbit_gemm<6, EPI>(x, s_x, w, s_w, G, M, N, K, tile_tokens, out, st, pdl);
+}
+
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 }  // namespace
@@ -1085,6 +1231,141 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
   }
   // 8. per token: router-weighted fp32 sum over its experts in ascending
   // order, one bf16 rounding
+  return combine_impl(z, s_t, slot, E, T, C, d, y_bf16, sms, st, C > 0);
+}
+
+// ---------------------------------------------------------------- low-bit --
+int64_t convrot_lowbit_weight_bytes(int64_t rows, int64_t K, int bits) {
+  if (!valid_bits(bits) || rows < 0 || K < 0 || rows % 128 != 0 || K % 64 != 0) return -1;
+  return lowbit_bytes(rows, K, bits);
+}
+
+int convrot_quantize_weights_lowbit(const void* w_bf16, int64_t rows, int64_t K, int group,
+                                    int bits, void* w_packed, float* row_scale, void* stream) {
+  if (!valid_bits(bits) || !valid_group(group)) return CONVROT_ERR_INVALID_ARG;
+  if (rows < 0 || rows >= ((int64_t)1 << 31) || rows % 128 != 0) return CONVROT_ERR_INVALID_ARG;
+  if (K < 64 || K > 16384 || K % 64 != 0 || K % group != 0) return CONVROT_ERR_INVALID_ARG;
+  if (rows > 0 && (!w_bf16 || !w_packed || !row_scale)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(w_bf16) || !al16(w_packed)) return CONVROT_ERR_MISALIGNED;
+  int rc = device_setup(nullptr);
+  if (rc != CONVROT_OK) return rc;
+  if (rows == 0) return CONVROT_OK;
+  cudaStream_t st = as_stream(stream);
+  uint8_t* out = reinterpret_cast<uint8_t*>(w_packed);
+  rc = bits == 4 ? lowbit_quant_group<4>(w_bf16, rows, (int)K, group, out, row_scale, st)
+                 : lowbit_quant_group<6>(w_bf16, rows, (int)K, group, out, row_scale, st);
+  if (rc != CONVROT_OK) return rc;
+  return launch_status();
+}
+
+int convrot_lowbit_gemm(const int8_t* x_q, const float* s_x, const void* w_packed,
+                        const float* row_scale, int64_t G, int64_t M, int64_t N, int64_t K,
+                        int bits, int epilogue, int tile_tokens, void* out, void* stream) {
+  int rc = check_lowbit_gemm(x_q, w_packed, G, M, N, K, bits, tile_tokens);
+  if (rc != CONVROT_OK) return rc;
+  if (epilogue < CONVROT_LOWBIT_F32 || epilogue > CONVROT_LOWBIT_SWIGLU)
+    return CONVROT_ERR_INVALID_ARG;
+  if (G * M > 0 && N > 0 && (!row_scale || !out || (epilogue != CONVROT_LOWBIT_F32 && !s_x)))
+    return CONVROT_ERR_INVALID_ARG;
+  if (!al16(out)) return CONVROT_ERR_MISALIGNED;
+  cudaStream_t st = as_stream(stream);
+  switch (epilogue) {
+    case CONVROT_LOWBIT_F32:
+      return launch_lowbit_bits<kLbF32>(bits, x_q, s_x, w_packed, row_scale, G, M, N, K,
+                                        tile_tokens, out, st);
+    case CONVROT_LOWBIT_BF16:
+      return launch_lowbit_bits<kLbBf16>(bits, x_q, s_x, w_packed, row_scale, G, M, N, K,
+                                         tile_tokens, out, st);
+    default:
+      return launch_lowbit_bits<kLbSwiglu>(bits, x_q, s_x, w_packed, row_scale, G, M, N, K,
+                                           tile_tokens, out, st);
+  }
+}
+
+int lowbit_convrot_linear(const void* x_bf16, int64_t M, int64_t K, const void* w_packed,
+                          const float* row_scale, int64_t N, int group, int bits, void* y_bf16,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_rq_args(x_bf16, CONVROT_DTYPE_BF16, M, K, group, (const int8_t*)workspace,
+                         (const float*)workspace);
+  if (rc != CONVROT_OK) return rc;
+  if ((rc = check_lowbit_gemm((const int8_t*)workspace, w_packed, 1, M, N, K, bits, 0)) !=
+      CONVROT_OK)
+    return rc;
+  if (M > 0 && N > 0 && (!row_scale || !y_bf16 || !workspace)) return CONVROT_ERR_INVALID_ARG;
+  if (!al16(y_bf16) || !al16(workspace)) return CONVROT_ERR_MISALIGNED;
+  if (ws_bytes < convrot_linear_workspace_size(M, K)) return CONVROT_ERR_WORKSPACE_TOO_SMALL;
+  if ((rc = device_setup(nullptr)) != CONVROT_OK) return rc;
+  if (M == 0 || N == 0) return CONVROT_OK;
+  cudaStream_t st = as_stream(stream);
+  int8_t* x_q = reinterpret_cast<int8_t*>(workspace);
+  float* s_x = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
+                                        align256((size_t)M * (size_t)K));
+  if ((rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, M, K, group, x_q, s_x, st)) != CONVROT_OK)
+    return rc;
+  return launch_lowbit_bits<kLbBf16>(bits, x_q, s_x, w_packed, row_scale, 1, M, N, K, 0, y_bf16,
+                                     st, true);
+}
+
+int moe_expert_choice_forward_lowbit(const void* x_bf16, const void* logits_bf16,
+                                     const void* w_gu, const float* s_gu, const void* w_d,
+                                     const float* s_d, int64_t T, int64_t d, int64_t f, int E,
+                                     int64_t C, int g_gu, int g_d, int bits, void* y_bf16,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  if (!valid_bits(bits)) return CONVROT_ERR_INVALID_ARG;
+  if (T < 0 || T >= ((int64_t)1 << 31) || E < 1 || E > 256 || C < 0 || C > T)
+    return CONVROT_ERR_INVALID_ARG;
+  if (!valid_group(g_gu) || !valid_group(g_d)) return CONVROT_ERR_INVALID_ARG;
+  if (d < 256 || d > 8192 || d % 256 != 0 || d % g_gu != 0) return CONVROT_ERR_INVALID_ARG;
+  if (f < 128 || f > 8192 || f % 128 != 0 || f % g_d != 0) return CONVROT_ERR_INVALID_ARG;
+  if ((int64_t)E * C >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
+  if (T > 0 && (!x_bf16 || !logits_bf16 || !w_gu || !s_gu || !w_d || !s_d || !y_bf16 ||
+                !workspace))
+    return CONVROT_ERR_INVALID_ARG;
+  if (!al16(x_bf16) || !al16(logits_bf16) || !al16(w_gu) || !al16(s_gu) || !al16(w_d) ||
+      !al16(s_d) || !al16(y_bf16) || !al16(workspace))
+    return CONVROT_ERR_MISALIGNED;
+  convrot_moe_layout_t lay;
+  moe_workspace_layout(T, d, f, E, C, &lay);
+  if (ws_bytes < lay.total) return CONVROT_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  int rc = device_setup(&sms);
+  if (rc != CONVROT_OK) return rc;
+  if (T == 0) return CONVROT_OK;
+  cudaStream_t st = as_stream(stream);
+  char* ws = reinterpret_cast<char*>(workspace);
+  int8_t* x_q = reinterpret_cast<int8_t*>(ws + lay.x_q);
+  float* s_x = reinterpret_cast<float*>(ws + lay.s_x);
+  float* s_t = reinterpret_cast<float*>(ws + lay.s_t);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + lay.idx);
+  float* w = reinterpret_cast<float*>(ws + lay.w);
+  int8_t* x_g = reinterpret_cast<int8_t*>(ws + lay.x_g);
+  float* s_g = reinterpret_cast<float*>(ws + lay.s_g);
+  float* h = reinterpret_cast<float*>(ws + lay.h);
+  int8_t* h_q = reinterpret_cast<int8_t*>(ws + lay.h_q);
+  float* s_h = reinterpret_cast<float*>(ws + lay.s_h);
+  int32_t* slot = reinterpret_cast<int32_t*>(ws + lay.slot);
+  void* z = ws + lay.z;
+  // the int8 block's schedule (see moe_expert_choice_forward) with the
+  // low-bit GEMMs and h through HBM in fp32 and the rotation kernel
+  if ((rc = softmax_impl(logits_bf16, T, E, s_t, st)) != CONVROT_OK) return rc;
+  if ((rc = topc_impl(s_t, T, E, C, idx, w, slot, st, true)) != CONVROT_OK) return rc;
+  if ((rc = rotquant_impl(x_bf16, CONVROT_DTYPE_BF16, T, d, g_gu, x_q, s_x, st, RqOut{0, 1, 1, 1},
+                          true, sms + sms / 2, true)) != CONVROT_OK)
+    return rc;
+  if (C > 0) {
+    if ((rc = gather_impl(x_q, s_x, T, idx, (int64_t)E * C, d, x_g, s_g, st, nullptr, 0, true)) !=
+        CONVROT_OK)
+      return rc;
+    if ((rc = launch_lowbit_bits<kLbSwiglu>(bits, x_g, s_g, w_gu, s_gu, E, C, 2 * f, d, 0, h, st,
+                                            true)) != CONVROT_OK)
+      return rc;
+    if ((rc = rotquant_impl(h, CONVROT_DTYPE_F32, (int64_t)E * C, f, g_d, h_q, s_h, st,
+                            RqOut{0, 1, 1, 1}, true)) != CONVROT_OK)
+      return rc;
+    if ((rc = launch_lowbit_bits<kLbBf16>(bits, h_q, s_h, w_d, s_d, E, C, d, f, 0, z, st, true)) !=
+        CONVROT_OK)
+      return rc;
+  }
   return combine_impl(z, s_t, slot, E, T, C, d, y_bf16, sms, st, C > 0);
 }
 
