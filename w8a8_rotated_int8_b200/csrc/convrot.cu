@@ -68,7 +68,7 @@ void set_gemm_attr() {
 template <int BITS, int EPI>
 void set_lowbit_attr() {
   cudaFuncSetAttribute(gemm_lowbit_tcgen05_kernel<BITS, EPI>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, lb::smem_bytes<BITS>());
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, lb::kSmemMax);
 }
 
 template <int BITS>
@@ -783,7 +783,14 @@ int launch_lowbit_gemm(const int8_t* x, const float* s_x, const uint8_t* wq, con
   const int64_t tiles = G * a.w_blocks * a.t_blocks;
   if (tiles >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
   a.num_tiles = (int)tiles;
-  a.n_acc = 4 * a.nt <= 256 ? 2 : 1;
+  // accumulator columns (256 beside the A stages): 2 blocks x ks sets x nt
+  // columns x n_acc buffers. Two buffers whenever they fit (the epilogue then
+  // overlaps the next tile); then as many sets as fit, up to two (one MMA
+  // issuer per accumulator).
+  const int per = 256 / (2 * a.nt);  // ks * n_acc that fit
+  a.n_acc = per >= 2 ? 2 : 1;
+  a.ks = per / a.n_acc >= 2 ? 2 : 1;
+  a.raw_stages = lb::raw_stages<BITS>(a.nt);
   a.wq = wq;
   a.s_w = s_w;
   a.s_x = s_x;
@@ -794,7 +801,7 @@ int launch_lowbit_gemm(const int8_t* x, const float* s_x, const uint8_t* wq, con
     return rc;
   const int grid = (int)std::min<int64_t>(tiles, sms);
   if ((rc = launch_kernel(gemm_lowbit_tcgen05_kernel<BITS, EPI>, dim3(grid), dim3(lb::kThreads),
-                          lb::smem_bytes<BITS>(), st, pdl, 1, tx, a)) != CONVROT_OK)
+                          lb::smem_bytes<BITS>(a.nt), st, pdl, 1, tx, a)) != CONVROT_OK)
     return rc;
   return launch_status();
 }

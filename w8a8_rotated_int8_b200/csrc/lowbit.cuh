@@ -192,25 +192,40 @@ enum LowbitEpilogue : int {
 };
 
 namespace lb {
-constexpr int kRawStages = 6;    // packed weights + int8 activation codes, per K-step of 64
-constexpr int kCvStages = 4;     // decoded: A in TMEM (64 columns), B in shared memory
-constexpr int kMaxNt = 128;      // tokens per tile
-constexpr int kConvWarps = 8;    // two per TMEM lane quadrant, one per half of the K-step
+constexpr int kMaxRawStages = 16;  // packed weights + int8 activation codes, per K-step of 64
+constexpr int kCvStages = 4;       // decoded: A in TMEM (64 columns), B in shared memory
+constexpr int kMaxNt = 128;        // tokens per tile
+constexpr int kConvGroups = 4;     // = kCvStages: group g decodes the K-steps j with j % 4 == g
+constexpr int kConvWarps = 4 * kConvGroups;  // one warp per TMEM lane quadrant in each group
 constexpr int kEpiWarps = 4;
-constexpr int kThreads = 32 * (2 + kConvWarps + kEpiWarps);
-constexpr int kActRawBytes = kMaxNt * 64;
-constexpr int kBStageBytes = kMaxNt * 128;
+constexpr int kMmaWarps = 4;      // MMA issuers: one per accumulator (2 blocks x ks sets)
+constexpr int kConvWarp0 = 1 + kMmaWarps;
+constexpr int kEpiWarp0 = kConvWarp0 + kConvWarps;
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAccCol0 = kCvStages * 64;  // accumulators after the A stages
+constexpr int kBarBytes = 512;
+constexpr int kSmemMax = 232448;          // the opt-in limit per CTA
+// Shared memory of one raw stage for nt tokens (the two weight tiles, then
+// the activation box), rounded to 1024 bytes.
 template <int BITS>
-constexpr int raw_stage_bytes() {
-  return (2 * LbFmt<BITS>::kTileBytes + kActRawBytes + 1023) / 1024 * 1024;
+__host__ __device__ constexpr int raw_stage_bytes(int nt) {
+  return (2 * LbFmt<BITS>::kTileBytes + nt * 64 + 1023) / 1024 * 1024;
+}
+// As many raw stages as fit beside the decoded-B ring (the weight stream is
+// compressed, so a deep ring is what keeps enough bytes in flight).
+template <int BITS>
+__host__ __device__ constexpr int raw_stages(int nt) {
+  const int room = kSmemMax - 1024 - kBarBytes - kCvStages * nt * 128;
+  const int r = room / raw_stage_bytes<BITS>(nt);
+  return r > kMaxRawStages ? kMaxRawStages : r;
 }
 template <int BITS>
-constexpr int smem_bytes() {
-  return kRawStages * raw_stage_bytes<BITS>() + kCvStages * kBStageBytes + 256 + 1024;
+__host__ __device__ constexpr int smem_bytes(int nt) {
+  return raw_stages<BITS>(nt) * raw_stage_bytes<BITS>(nt) + kCvStages * nt * 128 + kBarBytes +
+         1024;
 }
-static_assert(smem_bytes<6>() <= 232448, "shared memory per CTA");
+static_assert(raw_stages<6>(kMaxNt) >= 6 && smem_bytes<6>(kMaxNt) <= kSmemMax, "shared memory");
 }  // namespace lb
 
 struct LowbitArgs {
@@ -219,7 +234,13 @@ struct LowbitArgs {
   int nt;               // tokens per tile: a multiple of 16, at most 128
   int box_rows;         // rows of the activation box: min(nt, M)
   int t_blocks, w_blocks, k_blocks, num_tiles;
-  int n_acc;            // accumulator buffers: 2 when 4 * nt <= 256
+  int n_acc;            // accumulator buffers (1 or 2)
+  int ks;               // accumulator sets per weight block (1, 2 or 4): K-slice k of every
+                        // K-step accumulates into set k % ks, and the epilogue adds the
+                        // sets; consecutive MMAs then write different accumulators, so
+                        // their latency overlaps (small-N MMAs into one accumulator
+                        // serialise on it). 2 * ks * nt * n_acc <= 256 columns.
+  int raw_stages;       // depth of the raw ring (lb::raw_stages)
   const uint8_t* wq;    // packed weight tiles (see the top of this file)
   const float* s_w;     // [G*N] row scales
   const float* s_x;     // [G*M] token scales
@@ -353,57 +374,64 @@ __device__ __forceinline__ int64_t lb_row_block(const LowbitArgs& a, int g, int 
 // weight tiles through L2.
 //   warp 0      producer: per K-step one bulk copy per weight tile and a 3-D
 //               TMA box {64 codes, box_rows tokens} of the activation codes
-//   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
-//               kind::f16 M=128 N=nt K=16 (A from TMEM) into two accumulators
-//               (one per weight block), four K-slices per K-step
-//   warps 2-9   converters: warp w decodes half (w-2)/4 of the K-step for the
-//               rows of TMEM lane quadrant w % 4 of both weight blocks into
-//               the A stage (tcgen05.st), and widens a share of the
-//               activation codes to the fp16 B stage
-//   warps 10-13 epilogue: tcgen05.ld of the quadrant's rows, 16 tokens at a
+//   warps 1-4   MMA issuers (warp 1 also allocates 512 TMEM columns): one
+//               lane each issues tcgen05.mma kind::f16 M=128 N=nt K=16 (A
+//               from TMEM) into its own accumulator (weight block, set);
+//               2 * ks of them are active
+//   warps 5-20  converters in four groups of four warps; group g takes the
+//               K-steps j with j % 4 == g (decoded stage g), so four K-steps
+//               are decoded at once: warp w decodes the rows of TMEM lane
+//               quadrant w % 4 of both weight blocks into the A stage
+//               (tcgen05.st) and widens a quarter of the activation codes to
+//               the fp16 B stage (one K-step's decode is a chain of dependent
+//               loads, conversions and tensor-memory stores: several in
+//               flight keep the tensor cores fed)
+//   warps 21-24 epilogue: tcgen05.ld of the quadrant's rows, 16 tokens at a
 //               time; lanes hold consecutive weight rows, so each token's
 //               outputs are one contiguous store per warp
 template <int BITS, int EPI>
 __global__ void __launch_bounds__(lb::kThreads, 1)
     gemm_lowbit_tcgen05_kernel(const __grid_constant__ CUtensorMap tmX, const LowbitArgs args) {
   using F = LbFmt<BITS>;
-  constexpr int R = lb::kRawStages, S = lb::kCvStages;
-  constexpr int RAW = lb::raw_stage_bytes<BITS>();
+  constexpr int S = lb::kCvStages;
   constexpr bool kSwiglu = EPI == kLbSwiglu;
+  const int nt = args.nt;
+  const int R = args.raw_stages;
+  const int RAW = lb::raw_stage_bytes<BITS>(nt);
+  const int BST = nt * 128;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t rawp = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((rawp + 1023u) & ~1023u) - rawp);
   uint8_t* raw = smem;
   uint8_t* bst = smem + R * RAW;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(bst + S * lb::kBStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(bst + S * BST);
   uint64_t* raw_full = bars;
-  uint64_t* raw_empty = bars + R;
-  uint64_t* cv_full = bars + 2 * R;
-  uint64_t* cv_empty = bars + 2 * R + S;
-  uint64_t* tfull = bars + 2 * R + 2 * S;
+  uint64_t* raw_empty = bars + lb::kMaxRawStages;
+  uint64_t* cv_full = bars + 2 * lb::kMaxRawStages;
+  uint64_t* cv_empty = cv_full + S;
+  uint64_t* tfull = cv_empty + S;
   uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = tempty + 2;  // one per MMA issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + lb::kMmaWarps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int nt = args.nt;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < R; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], lb::kConvWarps);
+      mbar_init(&raw_empty[s], 4);
     }
     for (int s = 0; s < S; ++s) {
-      mbar_init(&cv_full[s], lb::kConvWarps);
-      mbar_init(&cv_empty[s], 1);
+      mbar_init(&cv_full[s], 4);
+      mbar_init(&cv_empty[s], 2 * args.ks);   // every issuer commits
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
+      mbar_init(&tfull[a], 2 * args.ks);
       mbar_init(&tempty[a], lb::kEpiWarps);
     }
-    mbar_init(drain, 1);
+    for (int i = 0; i < lb::kMmaWarps; ++i) mbar_init(&drain[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -482,8 +510,17 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
         if (!ok) break;
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
+  } else if (warp < lb::kConvWarp0) {
+    // MMA issuers: issuer i owns accumulator (block i / ks, set i % ks) and
+    // issues its MMAs (the K-slices k of every K-step with k % ks == i % ks).
+    // A thread waits about 120 cycles on every tcgen05.mma it issues (measured
+    // on B200, independent of N up to 128), so short MMAs need several
+    // issuers to keep the tensor pipe busy; they write different
+    // accumulators, so their order does not matter.
+    const int issuer = warp - 1;
+    const int ks = args.ks;
+    if (lane == 0 && issuer < 2 * ks) {
+      const int b = issuer / ks, q = issuer % ks;
       const uint32_t idesc = idesc_f16_f32(128, nt);
       int s = 0;
       uint32_t ph = 0;
@@ -493,8 +530,9 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
         const uint32_t acc_phase = (uint32_t)(args.n_acc == 2 ? (it >> 1) : it) & 1u;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, kErrTimeoutTmemEmpty)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + (uint32_t)(lb::kAccCol0 + acc * 2 * nt);
-        const uint32_t d1 = d0 + (uint32_t)nt;
+        // accumulator (block b, set q) at column base + (b * ks + q) * nt
+        const uint32_t d = tmem_base + (uint32_t)(lb::kAccCol0 + acc * 2 * ks * nt +
+                                                  (b * ks + q) * nt);
         bool ok = true;
         for (int kb = 0; kb < args.k_blocks; ++kb) {
           if (!mbar_wait(&cv_full[s], ph, abort_flag, kErrTimeoutFull)) {
@@ -502,14 +540,11 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t b_addr = smem_u32(bst + s * lb::kBStageBytes);
-          const uint32_t a_col = tmem_base + (uint32_t)(s * 64);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t bd = sdesc_k_sw128(b_addr + 32 * k);
-            const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
-            umma_f16_ts(d0, a_col + 8 * k, bd, idesc, accum);
-            umma_f16_ts(d1, a_col + 32 + 8 * k, bd, idesc, accum);
+          const uint32_t b_addr = smem_u32(bst + s * BST);
+          const uint32_t a_col = tmem_base + (uint32_t)(s * 64 + b * 32);
+          for (int k = q; k < 4; k += ks) {
+            const uint32_t accum = (kb > 0 || k >= ks) ? 1u : 0u;
+            umma_f16_ts(d, a_col + 8 * k, sdesc_k_sw128(b_addr + 32 * k), idesc, accum);
           }
           mma_issued = true;
           umma_commit(&cv_empty[s]);
@@ -522,60 +557,52 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
         umma_commit(&tfull[acc]);
       }
     }
-  } else if (warp < 2 + lb::kConvWarps) {
+  } else if (warp < lb::kEpiWarp0) {
     // ---------------------------------------------------------- converters --
-    const int cw = warp - 2;
+    const int cg = (warp - lb::kConvWarp0) >> 2;   // group = decoded stage
     const int quad = warp & 3;
-    const int half = cw >> 2;
     const int r = quad * 32 + lane;
-    const int ct = cw * 32 + lane;
+    const int ct = ((warp - lb::kConvWarp0) & 3) * 32 + lane;
     const uint32_t t_lane = (uint32_t)(quad * 32) << 16;
-    int rs = 0, cs = 0;
-    uint32_t rph = 0, cph = 0;
-    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
-      bool ok = true;
-      for (int kb = 0; kb < args.k_blocks; ++kb) {
-        bool w_ok = mbar_wait(&raw_full[rs], rph, abort_flag, kErrTimeoutFull);
-        w_ok = w_ok && mbar_wait(&cv_empty[cs], cph ^ 1u, abort_flag, kErrTimeoutEmpty);
-        if (__any_sync(0xffffffffu, !w_ok)) {
-          ok = false;
-          break;
-        }
-        const uint8_t* st = raw + rs * RAW;
-        uint32_t a0[16], a1[16];
-        lb_decode_row<BITS>(st, r, half, a0);
-        lb_decode_row<BITS>(st + F::kTileBytes, r, half, a1);
-        const uint32_t tcol = tmem_base + t_lane + (uint32_t)(cs * 64 + half * 16);
-        tmem_st16(tcol, a0);
-        tmem_st16(tcol + 32, a1);
-        const uint8_t* act = st + 2 * F::kTileBytes;
-        uint8_t* bt = bst + cs * lb::kBStageBytes;
-        for (int u = ct; u < nt * 8; u += 32 * lb::kConvWarps) {
-          const int row = u >> 3, ch = u & 7;
-          const uint2 xv = *reinterpret_cast<const uint2*>(act + row * 64 + ch * 8);
-          uint4 o;
-          i8x4_to_h2x2(xv.x, o.x, o.y);
-          i8x4_to_h2x2(xv.y, o.z, o.w);
-          *reinterpret_cast<uint4*>(bt + row * 128 + ((ch ^ (row & 7)) << 4)) = o;
-        }
-        tmem_wait_st();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&cv_full[cs]);
-          mbar_arrive(&raw_empty[rs]);
-        }
-        if (++rs == R) {
-          rs = 0;
-          rph ^= 1u;
-        }
-        if (++cs == S) {
-          cs = 0;
-          cph ^= 1u;
+    const int my_tiles = (int)blockIdx.x < args.num_tiles
+                             ? (args.num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1
+                             : 0;
+    const int steps = my_tiles * args.k_blocks;
+    const uint32_t tcol = tmem_base + t_lane + (uint32_t)(cg * 64);
+    uint8_t* bt = bst + cg * BST;
+    for (int j = cg; j < steps; j += lb::kConvGroups) {
+      const int rs = j % R;
+      bool w_ok = mbar_wait(&raw_full[rs], (uint32_t)(j / R) & 1u, abort_flag, kErrTimeoutFull);
+      w_ok = w_ok && mbar_wait(&cv_empty[cg], ((uint32_t)(j / lb::kConvGroups) & 1u) ^ 1u,
+                               abort_flag, kErrTimeoutEmpty);
+      if (__any_sync(0xffffffffu, !w_ok)) break;
+      const uint8_t* st = raw + rs * RAW;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t a[16];
+          lb_decode_row<BITS>(st + which * F::kTileBytes, r, half, a);
+          tmem_st16(tcol + (uint32_t)(which * 32 + half * 16), a);
         }
       }
-      if (!ok) break;
+      const uint8_t* act = st + 2 * F::kTileBytes;
+      for (int u = ct; u < nt * 8; u += 128) {
+        const int row = u >> 3, ch = u & 7;
+        const uint2 xv = *reinterpret_cast<const uint2*>(act + row * 64 + ch * 8);
+        uint4 o;
+        i8x4_to_h2x2(xv.x, o.x, o.y);
+        i8x4_to_h2x2(xv.y, o.z, o.w);
+        *reinterpret_cast<uint4*>(bt + row * 128 + ((ch ^ (row & 7)) << 4)) = o;
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&cv_full[cg]);
+        mbar_arrive(&raw_empty[rs]);
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue --
@@ -584,13 +611,13 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t t_lane = (uint32_t)(quad * 32) << 16;
+    const int ks = args.ks;
     int it = 0;
     for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
       const int acc = args.n_acc == 2 ? (it & 1) : 0;
       const uint32_t acc_phase = (uint32_t)(args.n_acc == 2 ? (it >> 1) : it) & 1u;
-      const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrTimeoutTmemFull);
-      if (__any_sync(0xffffffffu, !ok)) break;
-      tc_fence_after();
+      // the tile's scales are requested before the wait for its accumulators:
+      // lane l holds the token scales of tokens t0 + l + 32 i
       int g, wb, tb;
       lb_decode_tile(args, tile, g, wb, tb);
       const int t0 = tb * nt;
@@ -598,22 +625,51 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
       const int n1 = kSwiglu ? args.n_out + n0 : n0 + 128;
       const float sw0 = __ldg(args.s_w + (int64_t)g * args.N + n0);
       const float sw1 = __ldg(args.s_w + (int64_t)g * args.N + n1);
-      const uint32_t d0 = tmem_base + t_lane + (uint32_t)(lb::kAccCol0 + acc * 2 * nt);
-      const uint32_t d1 = d0 + (uint32_t)nt;
+      static_assert(lb::kMaxNt == 128, "four token-scale registers per lane");
+      auto sx_at = [&](int i) {
+        const int t = t0 + 32 * i + lane;
+        return (EPI != kLbF32 && 32 * i < nt && t < args.M)
+                   ? __ldg(args.s_x + (int64_t)g * args.M + t) : 0.0f;
+      };
+      const float sx0 = sx_at(0), sx1 = sx_at(1), sx2 = sx_at(2), sx3 = sx_at(3);
+      const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrTimeoutTmemFull);
+      if (__any_sync(0xffffffffu, !ok)) break;
+      tc_fence_after();
+      const uint32_t dbase = tmem_base + t_lane + (uint32_t)(lb::kAccCol0 + acc * 2 * ks * nt);
       for (int c0 = 0; c0 < nt; c0 += 16) {
-        uint32_t v0[16], v1[16];
-        tmem_ld16(d0 + c0, v0);
-        tmem_ld16(d1 + c0, v1);
-        tmem_wait_ld();
-        const int tl = t0 + c0 + (lane & 15);
-        const float sx_l = (EPI != kLbF32 && tl < args.M) ? __ldg(args.s_x + (int64_t)g * args.M + tl) : 0.0f;
+        // each block's accumulator sets, added in set order
+        float v0[16], v1[16];
+        {
+          uint32_t u0[16], u1[16];
+          tmem_ld16(dbase + c0, u0);
+          tmem_ld16(dbase + (uint32_t)(ks * nt) + c0, u1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            v0[i] = __uint_as_float(u0[i]);
+            v1[i] = __uint_as_float(u1[i]);
+          }
+        }
+        for (int q = 1; q < ks; ++q) {
+          uint32_t u[16];
+          tmem_ld16(dbase + (uint32_t)(q * nt) + c0, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v0[i] = __fadd_rn(v0[i], __uint_as_float(u[i]));
+          tmem_ld16(dbase + (uint32_t)((ks + q) * nt) + c0, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v1[i] = __fadd_rn(v1[i], __uint_as_float(u[i]));
+        }
+        // the register holding this chunk's token scales
+        const float sx_src = c0 < 32 ? sx0 : c0 < 64 ? sx1 : c0 < 96 ? sx2 : sx3;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int t = t0 + c0 + i;
-          const float sx = __shfl_sync(0xffffffffu, sx_l, i);
+          const float sx = __shfl_sync(0xffffffffu, sx_src, (c0 & 16) + i);
           if (t >= args.M) continue;
-          const float a0 = __fmul_rn(__uint_as_float(v0[i]), 16.0f);
-          const float a1 = __fmul_rn(__uint_as_float(v1[i]), 16.0f);
+          const float a0 = __fmul_rn(v0[i], 16.0f);
+          const float a1 = __fmul_rn(v1[i], 16.0f);
           const int64_t orow = (int64_t)g * args.M + t;
           if constexpr (EPI == kLbF32) {
             float* out = reinterpret_cast<float*>(args.out) + orow * args.N;
@@ -648,9 +704,9 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
           mbar_wait_limit(&raw_full[s], (issued_parity >> s) & 1u, &never, kErrTimeoutTeardown,
                           100000000ull);
     }
-    if (warp == 1 && lane == 0 && mma_issued) {
-      umma_commit(drain);
-      mbar_wait_limit(drain, 0, &never, kErrTimeoutTeardown, 100000000ull);
+    if (warp >= 1 && warp < lb::kConvWarp0 && lane == 0 && mma_issued) {
+      umma_commit(&drain[warp - 1]);
+      mbar_wait_limit(&drain[warp - 1], 0, &never, kErrTimeoutTeardown, 100000000ull);
     }
     __syncthreads();
   }
