@@ -85,6 +85,10 @@ int convrot_abi_version(void);
 /* Static description of a status code. Never NULL. */
 const char* convrot_status_string(int status);
 
+/* Name of the last CUDA error (cudaGetErrorName) an entry point saw on the
+ * calling host thread, for a CONVROT_ERR_CUDA status; "none" before any. */
+const char* convrot_last_cuda_error(void);
+
 /* Checks that the current device is an sm_100 part the kernels were built for.
  * Returns CONVROT_OK or CONVROT_ERR_UNSUPPORTED_DEVICE. */
 int convrot_device_check(void);
@@ -236,7 +240,8 @@ int convrot_i8_gemm_swiglu(const int8_t* a, const float* s_a, const int8_t* b, c
  *   The results equal convrot_i8_gemm_swiglu followed by convrot_rotquant
  *   (CONVROT_DTYPE_F32, group g_h) bit for bit.
  *   sync    device scratch of at least convrot_swiglu_rq_sync_bytes(G, M)
- *           bytes (the rows' running maxima and the tiles' arrival counters);
+ *           bytes (the rows' running maxima, the tiles' arrival counters, an
+ *           abort word and a count of published tiles per group);
  *           the call clears it on `stream` before the GEMM, so calls sharing
  *           one scratch must be ordered on one stream.
  * The tiles of a row wait for one another (bounded; a wait that runs out sets
@@ -333,7 +338,10 @@ int w8a8_convrot_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const 
  * with g_d = 256 h is stored in fp32 and rotated by a separate kernel.
  * Every kernel of the call runs on `stream` (so the call can be captured in a
  * CUDA graph on it); they are chained with programmatic dependent launch, and
- * the activation rotation runs beside the routing kernels.
+ * the activation rotation runs beside the routing kernels. After the fused
+ * requantisation the down projection is streamed per expert: its tiles for
+ * expert e start once every gate/up tile of e has published its h codes (a
+ * count in the hsync scratch), not after the whole gate/up GEMM.
  * Failure of a device-side wait: the call is asynchronous, so a kernel that
  * gives up on a bounded wait (the gate/up GEMM's cross-tile wait gives up
  * after 100 ms, e.g. when another workload holds some of the SMs and the

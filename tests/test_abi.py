@@ -42,7 +42,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_strings(lib):
-    assert lib.convrot_abi_version() == 2
+    assert lib.convrot_abi_version() == 3
     for code in range(7):
         assert binding.status_string(code)
     assert binding.status_string(99) == "unknown status"
@@ -76,9 +76,9 @@ def test_argument_checks_need_no_gpu(lib):
     assert (rq(al, al, al, al, 1, 2, 64, 256, 256, 64, al, al, al, 64, None)
             == binding.CONVROT_ERR_WORKSPACE_TOO_SMALL)
     # its scratch: the row maxima (256-byte aligned), then an arrival counter per 128-row slab
-    # (one spare slab per group) and the abort word
-    assert lib.convrot_swiglu_rq_sync_bytes(64, 256) == 64 * 256 * 4 + (64 * 3 + 1) * 4
-    assert lib.convrot_swiglu_rq_sync_bytes(5, 40) == 1024 + (5 * 2 + 1) * 4
+    # (one spare slab per group), the abort word and a published-tile count per group
+    assert lib.convrot_swiglu_rq_sync_bytes(64, 256) == 64 * 256 * 4 + (64 * 3 + 1 + 64) * 4
+    assert lib.convrot_swiglu_rq_sync_bytes(5, 40) == 1024 + (5 * 2 + 1 + 5) * 4
     # tiled weight sizes: 128-row blocks x 128-byte K tiles of 16 KB
     assert lib.convrot_tiled_weight_bytes(2, 300, 200) == 2 * 3 * 2 * 16384
     assert lib.convrot_tiled_weight_bytes(128, 1536, 2048) == 128 * 12 * 16 * 16384

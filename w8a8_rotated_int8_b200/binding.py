@@ -34,7 +34,10 @@ LAYOUT_TILES = 1
 class ConvrotError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        extra = ""
+        if status == CONVROT_ERR_CUDA:
+            extra = f": {lib().convrot_last_cuda_error().decode()}"
+        super().__init__(f"{where}: {status_string(status)}{extra} (status {status})")
 
 
 class MoeLayout(ctypes.Structure):
@@ -54,6 +57,7 @@ _SZ = ctypes.c_size_t
 _SIGNATURES = {
     "convrot_abi_version": (_I, []),
     "convrot_status_string": (ctypes.c_char_p, [_I]),
+    "convrot_last_cuda_error": (ctypes.c_char_p, []),
     "convrot_device_check": (_I, []),
     "convrot_check_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "convrot_wait_selftest": (_I, [ctypes.c_ulonglong, _P, _P]),

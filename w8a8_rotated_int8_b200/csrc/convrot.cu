@@ -167,9 +167,18 @@ inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) 
 inline bool valid_group(int g) { return g == 1 || g == 4 || g == 16 || g == 64 || g == 256; }
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// The name of the last CUDA error an entry point of this thread saw.
+thread_local const char* g_last_cuda_error = "none";
+
+int cuda_failed(cudaError_t e) {
+  g_last_cuda_error = cudaGetErrorName(e);
+  cudaGetLastError();
+  return CONVROT_ERR_CUDA;
+}
+
 int launch_status() {
   const cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+  return e == cudaSuccess ? CONVROT_OK : cuda_failed(e);
 }
 
 // Launches `kern` on `st`; `pdl` adds programmatic stream serialization (the
@@ -199,10 +208,8 @@ int launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   }
   lc.attrs = attr;
   lc.numAttrs = n;
-  if (cudaLaunchKernelEx(&lc, kern, args...) != cudaSuccess) {
-    cudaGetLastError();
-    return CONVROT_ERR_CUDA;
-  }
+  const cudaError_t e = cudaLaunchKernelEx(&lc, kern, args...);
+  if (e != cudaSuccess) return cuda_failed(e);
   return CONVROT_OK;
 }
 
@@ -466,12 +473,20 @@ bool swiglu_rq_fits(int64_t G, int64_t M, int64_t F, int sms) {
 
 // Bytes of the fused h requantisation's synchronisation scratch for G groups
 // of M rows: the row maxima [G*M] (fp32 bits), then at a 256-byte boundary
-// the tile arrivals of every 128-row slab [G*(ceil(M/128)+1)] and one abort
-// word. All zero before the GEMM starts.
+// the tile arrivals of every 128-row slab [G*(ceil(M/128)+1)], one abort
+// word, and each group's count of published tiles [G] (read by a streamed
+// down GEMM). All zero before the GEMM starts.
 size_t swiglu_rq_sync_bytes(int64_t G, int64_t M) {
   const size_t rows = (size_t)G * (size_t)M;
-  const size_t counters = (size_t)G * (size_t)(cdiv(M, 128) + 1) + 1;
+  const size_t counters = (size_t)G * (size_t)(cdiv(M, 128) + 1) + 1 + (size_t)G;
   return ((rows * 4 + 255) & ~(size_t)255) + counters * 4;
+}
+
+// The published-tile counters of that scratch.
+int* swiglu_rq_done_words(char* sync, int64_t G, int64_t M) {
+  const size_t rows = (size_t)G * (size_t)M;
+  return reinterpret_cast<int*>(sync + ((rows * 4 + 255) & ~(size_t)255)) +
+         G * (cdiv(M, 128) + 1) + 1;
 }
 
 // NB = rows of one B matrix per group (2F for SwiGLU). With BT the B operand
@@ -823,7 +838,9 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // ===================================================================== ABI ==
 extern "C" {
 
-int convrot_abi_version(void) { return 2; }
+int convrot_abi_version(void) { return 3; }
+
+const char* convrot_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char* convrot_status_string(int status) {
   switch (status) {
@@ -1207,13 +1224,25 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
     GemmArgs a1{};
     a1.s_a = s_g;
     a1.s_b = s_gu;
+    GemmArgs a2{};  // the down projection to the experts' BF16 outputs
+    a2.s_a = s_h;
+    a2.s_b = s_d;
+    a2.out = z;
     if (fused_h) {
-      // 5 + 6. gate/up GEMM: dequant, SwiGLU, rotation (g_d) and requantisation
+      // 5 + 6. gate/up GEMM: dequant, SwiGLU, rotation (g_d) and requantisation;
+      // each tile publishes its expert's h codes (done) for the down GEMM
       a1.out = h_q;
       a1.g_h = g_d;
       a1.s_h = s_h;
       a1.hmax = reinterpret_cast<unsigned*>(hsync);
       a1.rsync = reinterpret_cast<int*>(hsync + align256((size_t)E * (size_t)C * 4));
+      a1.done = swiglu_rq_done_words(hsync, E, C);
+      const bool pairs1 = C > gemm::BM && sms >= 2;  // as launch_gemm decides
+      const int64_t mb1 = cdiv(C, pairs1 ? gemm2::BM : gemm::BM);
+      const int64_t slabs1 = pairs1 ? 2 * mb1 : mb1;
+      a2.done = a1.done;
+      a2.done_target = (int)((pairs1 ? 2 : 1) * mb1 * cdiv(f, gemm::BN / 2));
+      a2.done_abort = a1.rsync + E * slabs1;
       if ((rc = launch_gemm<kEpiSwigluRq, true>(x_g, w_gu, E, C, 2 * f, d, f, a1, st, true)) !=
           CONVROT_OK)
         return rc;
@@ -1228,11 +1257,10 @@ int moe_expert_choice_forward(const void* x_bf16, const void* logits_bf16, const
                               RqOut{0, 1, 1, 1}, true)) != CONVROT_OK)
         return rc;
     }
-    // 7. down GEMM with dequant to the experts' BF16 outputs
-    GemmArgs a2{};
-    a2.s_a = s_h;
-    a2.s_b = s_d;
-    a2.out = z;
+    // 7. down GEMM; after the fused requantisation it is streamed: each
+    // expert's tiles start once that expert's h codes are published, so the
+    // down GEMM's CTAs take over SMs as the gate/up GEMM's CTAs leave instead
+    // of after its last tile
     if ((rc = launch_gemm<kEpiBf16, true>(h_q, w_d, E, C, d, f, d, a2, st, true)) != CONVROT_OK)
       return rc;
   }
