@@ -443,13 +443,16 @@ def test_combine_sums_in_expert_order(e_n, t, c, d):
         toks = torch.randperm(t, generator=gen)[:c].sort().values
         slot[e, toks] = torch.arange(c, dtype=torch.int32)
     y = W.convrot_combine_rows(z.cuda(), s_t.cuda(), slot.cuda(), c).cpu()
-    ref = np.zeros((t, d), np.float32)
-    zf, sf = np32(z), s_t.numpy()
-    for e in range(e_n):       # fp32 products, fp32 sums, ascending expert order
-        toks = np.nonzero(slot[e].numpy() >= 0)[0]
-        rows = e * c + slot[e].numpy()[toks]
-        ref[toks] = ref[toks] + (sf[e, toks][:, None] * zf[rows]).astype(np.float32)
-    assert np.array_equal(np32(y), O.bf16_round(ref))
+    # the same choices in the oracle's terms: each expert's tokens (ascending,
+    # the slot order) and their router weights, and its rows of z
+    idx = np.zeros((e_n, c), np.int32)
+    zf, sf, sl = np32(z), s_t.numpy(), slot.numpy()
+    for e in range(e_n):
+        toks = np.nonzero(sl[e] >= 0)[0]
+        idx[e, sl[e, toks]] = toks
+    w = np.take_along_axis(sf, idx, axis=1).astype(np.float32)
+    zd = {e: zf[e * c:(e + 1) * c] for e in range(e_n)}
+    assert np.array_equal(np32(y), O.combine(t, idx, w, zd))
 
 
 # ------------------------------------------------------------------ linear --
