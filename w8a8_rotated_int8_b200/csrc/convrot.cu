@@ -756,7 +756,8 @@ int encode_act_i8(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows,
 }
 
 // Tokens per tile when the caller leaves it open: one tile of all the tokens
-// up to 64 (two accumulator buffers), else 128 (one).
+// up to 64, else 128 (the MMA's M; rows past the tile's tokens are not
+// widened and their accumulator rows are not read).
 int lowbit_auto_nt(int64_t M) {
   return M <= 64 ? (int)std::max<int64_t>(16, cdiv(M, 16) * 16) : lb::kMaxNt;
 }
@@ -798,13 +799,6 @@ int launch_lowbit_gemm(const int8_t* x, const float* s_x, const uint8_t* wq, con
   const int64_t tiles = G * a.w_blocks * a.t_blocks;
   if (tiles >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
   a.num_tiles = (int)tiles;
-  // accumulator columns (256 beside the A stages): 2 blocks x ks sets x nt
-  // columns x n_acc buffers. Two buffers whenever they fit (the epilogue then
-  // overlaps the next tile); then as many sets as fit, up to two (one MMA
-  // issuer per accumulator).
-  const int per = 256 / (2 * a.nt);  // ks * n_acc that fit
-  a.n_acc = per >= 2 ? 2 : 1;
-  a.ks = per / a.n_acc >= 2 ? 2 : 1;
   a.raw_stages = lb::raw_stages<BITS>(a.nt);
   a.wq = wq;
   a.s_w = s_w;
@@ -1302,7 +1296,7 @@ int convrot_lowbit_gemm(const int8_t* x_q, const float* s_x, const void* w_packe
     return CONVROT_ERR_INVALID_ARG;
   if (G * M > 0 && N > 0 && (!row_scale || !out || (epilogue != CONVROT_LOWBIT_F32 && !s_x)))
     return CONVROT_ERR_INVALID_ARG;
-  if (!al16(out)) return CONVROT_ERR_MISALIGNED;
+  if (!al16(out) || !al16(row_scale)) return CONVROT_ERR_MISALIGNED;
   cudaStream_t st = as_stream(stream);
   switch (epilogue) {
     case CONVROT_LOWBIT_F32:
@@ -1327,7 +1321,7 @@ int lowbit_convrot_linear(const void* x_bf16, int64_t M, int64_t K, const void* 
       CONVROT_OK)
     return rc;
   if (M > 0 && N > 0 && (!row_scale || !y_bf16 || !workspace)) return CONVROT_ERR_INVALID_ARG;
-  if (!al16(y_bf16) || !al16(workspace)) return CONVROT_ERR_MISALIGNED;
+  if (!al16(y_bf16) || !al16(workspace) || !al16(row_scale)) return CONVROT_ERR_MISALIGNED;
   if (ws_bytes < convrot_linear_workspace_size(M, K)) return CONVROT_ERR_WORKSPACE_TOO_SMALL;
   if ((rc = device_setup(nullptr)) != CONVROT_OK) return rc;
   if (M == 0 || N == 0) return CONVROT_OK;

@@ -28,13 +28,15 @@
 // and INT8 activation codes are not representable in FP8, so the contraction
 // runs on tcgen05 kind::f16 with fp32 accumulation over exact fp16 operands:
 // an activation code (|x| <= 127) is an exact fp16, and so is q * sigma / 16
-// (at most 9 significant bits, between 2^-13 and 28 * 31). The weights are
-// the A operand, decoded by converter warps straight into tensor memory
-// (tcgen05.st), so no decoded weight passes through shared memory; the
-// activation codes are the B operand, widened to fp16 in shared memory with
-// the 128-byte swizzle. D[weight row, token] = sum_k A[row, k] * B[token, k]
-// accumulates sum_k q * sigma / 16 * x; the epilogue multiplies by 16
-// (exact) and dequantises y = acc * (s_x * s_r).
+// (at most 9 significant bits, between 2^-13 and 28 * 31). Converter warps
+// decode the weights into shared memory as the N = 256 operand (two 128-row
+// blocks, the 128-byte swizzle) and widen the activation codes into the
+// M = 128 operand (the tile's tokens), so every MMA is M=128 N=256 K=16
+// whatever the token count: a thread issuing tcgen05.mma waits about 120
+// cycles per instruction (measured on B200) whether N is 16 or 128, so short
+// instructions cannot keep the tensor core busy. D[token, weight row]
+// accumulates sum_k x * q * sigma / 16; the epilogue multiplies by 16 (exact)
+// and dequantises y = acc * (s_x * s_r).
 #pragma once
 
 #include "common.cuh"
@@ -192,40 +194,40 @@ enum LowbitEpilogue : int {
 };
 
 namespace lb {
-constexpr int kMaxRawStages = 16;  // packed weights + int8 activation codes, per K-step of 64
-constexpr int kCvStages = 4;       // decoded: A in TMEM (64 columns), B in shared memory
-constexpr int kMaxNt = 128;        // tokens per tile
-constexpr int kConvGroups = 4;     // = kCvStages: group g decodes the K-steps j with j % 4 == g
-constexpr int kConvWarps = 4 * kConvGroups;  // one warp per TMEM lane quadrant in each group
+constexpr int kMaxRawStages = 8;        // packed weights + int8 activation codes, per K-step of 64
+constexpr int kDecStages = 3;           // decoded stages: fp16 weights (N) and tokens (M)
+constexpr int kConvGroups = kDecStages; // group g decodes the K-steps j with j % 3 == g
+constexpr int kConvWarps = 4 * kConvGroups;
 constexpr int kEpiWarps = 4;
-constexpr int kMmaWarps = 4;      // MMA issuers: one per accumulator (2 blocks x ks sets)
-constexpr int kConvWarp0 = 1 + kMmaWarps;
+constexpr int kConvWarp0 = 2;
 constexpr int kEpiWarp0 = kConvWarp0 + kConvWarps;
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
-constexpr uint32_t kTmemCols = 512;
-constexpr int kAccCol0 = kCvStages * 64;  // accumulators after the A stages
+constexpr int kMaxNt = 128;             // tokens per tile (the MMA's M)
+constexpr int kBBytes = 256 * 128;      // decoded weights: 256 rows x 64 codes, fp16
+constexpr int kABytes = kMaxNt * 128;   // widened tokens: 128 rows x 64 codes, fp16
+constexpr int kDecBytes = kBBytes + kABytes;
+constexpr uint32_t kTmemCols = 512;     // two accumulators of 256 columns
 constexpr int kBarBytes = 512;
-constexpr int kSmemMax = 232448;          // the opt-in limit per CTA
+constexpr int kSmemMax = 232448;        // the opt-in limit per CTA
 // Shared memory of one raw stage for nt tokens (the two weight tiles, then
 // the activation box), rounded to 1024 bytes.
 template <int BITS>
 __host__ __device__ constexpr int raw_stage_bytes(int nt) {
   return (2 * LbFmt<BITS>::kTileBytes + nt * 64 + 1023) / 1024 * 1024;
 }
-// As many raw stages as fit beside the decoded-B ring (the weight stream is
-// compressed, so a deep ring is what keeps enough bytes in flight).
+// As many raw stages as fit beside the decoded stages.
 template <int BITS>
 __host__ __device__ constexpr int raw_stages(int nt) {
-  const int room = kSmemMax - 1024 - kBarBytes - kCvStages * nt * 128;
+  const int room = kSmemMax - 1024 - kBarBytes - kDecStages * kDecBytes;
   const int r = room / raw_stage_bytes<BITS>(nt);
   return r > kMaxRawStages ? kMaxRawStages : r;
 }
 template <int BITS>
 __host__ __device__ constexpr int smem_bytes(int nt) {
-  return raw_stages<BITS>(nt) * raw_stage_bytes<BITS>(nt) + kCvStages * nt * 128 + kBarBytes +
+  return kDecStages * kDecBytes + raw_stages<BITS>(nt) * raw_stage_bytes<BITS>(nt) + kBarBytes +
          1024;
 }
-static_assert(raw_stages<6>(kMaxNt) >= 6 && smem_bytes<6>(kMaxNt) <= kSmemMax, "shared memory");
+static_assert(raw_stages<6>(kMaxNt) >= 3 && smem_bytes<6>(kMaxNt) <= kSmemMax, "shared memory");
 }  // namespace lb
 
 struct LowbitArgs {
@@ -234,12 +236,6 @@ struct LowbitArgs {
   int nt;               // tokens per tile: a multiple of 16, at most 128
   int box_rows;         // rows of the activation box: min(nt, M)
   int t_blocks, w_blocks, k_blocks, num_tiles;
-  int n_acc;            // accumulator buffers (1 or 2)
-  int ks;               // accumulator sets per weight block (1, 2 or 4): K-slice k of every
-                        // K-step accumulates into set k % ks, and the epilogue adds the
-                        // sets; consecutive MMAs then write different accumulators, so
-                        // their latency overlaps (small-N MMAs into one accumulator
-                        // serialise on it). 2 * ks * nt * n_acc <= 256 columns.
   int raw_stages;       // depth of the raw ring (lb::raw_stages)
   const uint8_t* wq;    // packed weight tiles (see the top of this file)
   const float* s_w;     // [G*N] row scales
@@ -279,16 +275,14 @@ __device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t&
   hi = h2_sub(__byte_perm(u, 0x64646464u, 0x4342), 0x64806480u);
 }
 
-// Row r's half (32 codes, two groups) of one k-block of a weight tile, decoded
-// to 16 fp16 pairs q * sigma / 16 in K order.
+// Half `half` (32 codes, two groups) of one row of a weight tile's k-block,
+// from the row's words (lw: the half's plane, hw: its top-bit words for six
+// bits, sw: the row's four E4M3 group scales), to 16 fp16 pairs
+// q * sigma / 16 in K order.
 template <int BITS>
-__device__ __forceinline__ void lb_decode_row(const uint8_t* tile, int r, int half,
-                                              uint32_t (&o)[16]) {
+__device__ __forceinline__ void lb_decode_words(uint4 lw, uint2 hw, uint32_t sw, int half,
+                                                uint32_t (&o)[16]) {
   using F = LbFmt<BITS>;
-  const uint4 lw = *reinterpret_cast<const uint4*>(tile + half * 2048 + r * 16);
-  uint2 hw = make_uint2(0u, 0u);
-  if (BITS == 6) hw = *reinterpret_cast<const uint2*>(tile + 4096 + r * 16 + half * 8);
-  const uint32_t sw = *reinterpret_cast<const uint32_t*>(tile + F::kScaleOff + r * 4);
   const uint32_t sp = h2_mul(e4m3x2_to_h2(sw >> (16 * half)), 0x2C002C00u);  // sigma / 16
   const uint32_t s_a = __byte_perm(sp, 0u, 0x1010), s_b = __byte_perm(sp, 0u, 0x3232);
   const uint32_t c_a = h2_mul(s_a, F::kNegMagic2), c_b = h2_mul(s_b, F::kNegMagic2);
@@ -306,21 +300,6 @@ __device__ __forceinline__ void lb_decode_row(const uint8_t* tile, int r, int ha
   }
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-
 // generic-proxy shared-memory writes made visible to the tensor core (async proxy)
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -332,14 +311,14 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int m, int n) {
   return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T, f16 x f16 -> f32, issued by one thread.
-__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+// D[tmem] (+)= A[smem] * B[smem]^T, f16 x f16 -> f32, issued by one thread.
+__device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -364,45 +343,38 @@ __device__ __forceinline__ int64_t lb_row_block(const LowbitArgs& a, int g, int 
 // weight tiles through L2.
 //   warp 0      producer: per K-step one bulk copy per weight tile and a 3-D
 //               TMA box {64 codes, box_rows tokens} of the activation codes
-//   warps 1-4   MMA issuers (warp 1 also allocates 512 TMEM columns): one
-//               lane each issues tcgen05.mma kind::f16 M=128 N=nt K=16 (A
-//               from TMEM) into its own accumulator (weight block, set);
-//               2 * ks of them are active
-//   warps 5-20  converters in four groups of four warps; group g takes the
-//               K-steps j with j % 4 == g (decoded stage g), so four K-steps
-//               are decoded at once: warp w decodes the rows of TMEM lane
-//               quadrant w % 4 of both weight blocks into the A stage
-//               (tcgen05.st) and widens a quarter of the activation codes to
-//               the fp16 B stage (one K-step's decode is a chain of dependent
-//               loads, conversions and tensor-memory stores: several in
-//               flight keep the tensor cores fed)
-//   warps 21-24 epilogue: tcgen05.ld of the quadrant's rows, 16 tokens at a
-//               time; lanes hold consecutive weight rows, so each token's
-//               outputs are one contiguous store per warp
+//   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
+//               kind::f16 M=128 N=256 K=16, four per K-step, into one of two
+//               256-column accumulators
+//   warps 2-13  converters in three groups of four warps; group g takes the
+//               K-steps j with j % 3 == g (decoded stage g): thread i decodes
+//               rows i and 128 + i of the K-step's weights into the N operand
+//               and widens a share of the activation codes into the M operand
+//   warps 14-17 epilogue: tcgen05.ld of the quadrant's token rows, 16
+//               columns at a time; each lane writes its row's outputs
 template <int BITS, int EPI>
 __global__ void __launch_bounds__(lb::kThreads, 1)
     gemm_lowbit_tcgen05_kernel(const __grid_constant__ CUtensorMap tmX, const LowbitArgs args) {
   using F = LbFmt<BITS>;
-  constexpr int S = lb::kCvStages;
+  constexpr int S = lb::kDecStages;
   constexpr bool kSwiglu = EPI == kLbSwiglu;
   const int nt = args.nt;
   const int R = args.raw_stages;
   const int RAW = lb::raw_stage_bytes<BITS>(nt);
-  const int BST = nt * 128;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t rawp = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((rawp + 1023u) & ~1023u) - rawp);
-  uint8_t* raw = smem;
-  uint8_t* bst = smem + R * RAW;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(bst + S * BST);
+  uint8_t* dec = smem;                               // S x (B 32 KB, A 16 KB)
+  uint8_t* raw = smem + S * lb::kDecBytes;           // R raw stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(raw + R * RAW);
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = bars + lb::kMaxRawStages;
   uint64_t* cv_full = bars + 2 * lb::kMaxRawStages;
   uint64_t* cv_empty = cv_full + S;
   uint64_t* tfull = cv_empty + S;
   uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;  // one per MMA issuer
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + lb::kMmaWarps);
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -415,13 +387,13 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
     }
     for (int s = 0; s < S; ++s) {
       mbar_init(&cv_full[s], 4);
-      mbar_init(&cv_empty[s], 2 * args.ks);   // every issuer commits
+      mbar_init(&cv_empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 2 * args.ks);
+      mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], lb::kEpiWarps);
     }
-    for (int i = 0; i < lb::kMmaWarps; ++i) mbar_init(&drain[i], 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -500,29 +472,18 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
         if (!ok) break;
       }
     }
-  } else if (warp < lb::kConvWarp0) {
-    // MMA issuers: issuer i owns accumulator (block i / ks, set i % ks) and
-    // issues its MMAs (the K-slices k of every K-step with k % ks == i % ks).
-    // A thread waits about 120 cycles on every tcgen05.mma it issues (measured
-    // on B200, independent of N up to 128), so short MMAs need several
-    // issuers to keep the tensor pipe busy; they write different
-    // accumulators, so their order does not matter.
-    const int issuer = warp - 1;
-    const int ks = args.ks;
-    if (lane == 0 && issuer < 2 * ks) {
-      const int b = issuer / ks, q = issuer % ks;
-      const uint32_t idesc = idesc_f16_f32(128, nt);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(128, 256);
       int s = 0;
       uint32_t ph = 0;
       int it = 0;
       for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
-        const int acc = args.n_acc == 2 ? (it & 1) : 0;
-        const uint32_t acc_phase = (uint32_t)(args.n_acc == 2 ? (it >> 1) : it) & 1u;
+        const int acc = it & 1;
+        const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, kErrTimeoutTmemEmpty)) break;
         tc_fence_after();
-        // accumulator (block b, set q) at column base + (b * ks + q) * nt
-        const uint32_t d = tmem_base + (uint32_t)(lb::kAccCol0 + acc * 2 * ks * nt +
-                                                  (b * ks + q) * nt);
+        const uint32_t d = tmem_base + (uint32_t)(acc * 256);
         bool ok = true;
         for (int kb = 0; kb < args.k_blocks; ++kb) {
           if (!mbar_wait(&cv_full[s], ph, abort_flag, kErrTimeoutFull)) {
@@ -530,12 +491,12 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t b_addr = smem_u32(bst + s * BST);
-          const uint32_t a_col = tmem_base + (uint32_t)(s * 64 + b * 32);
-          for (int k = q; k < 4; k += ks) {
-            const uint32_t accum = (kb > 0 || k >= ks) ? 1u : 0u;
-            umma_f16_ts(d, a_col + 8 * k, sdesc_k_sw128(b_addr + 32 * k), idesc, accum);
-          }
+          const uint32_t b_addr = smem_u32(dec + s * lb::kDecBytes);
+          const uint32_t a_addr = b_addr + lb::kBBytes;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_f16_ss(d, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k), idesc,
+                        (kb | k) != 0 ? 1u : 0u);
           mma_issued = true;
           umma_commit(&cv_empty[s]);
           if (++s == S) {
@@ -550,130 +511,182 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
   } else if (warp < lb::kEpiWarp0) {
     // ---------------------------------------------------------- converters --
     const int cg = (warp - lb::kConvWarp0) >> 2;   // group = decoded stage
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;
-    const int ct = ((warp - lb::kConvWarp0) & 3) * 32 + lane;
-    const uint32_t t_lane = (uint32_t)(quad * 32) << 16;
+    const int ti = ((warp - lb::kConvWarp0) & 3) * 32 + lane;  // 0..127
     const int my_tiles = (int)blockIdx.x < args.num_tiles
                              ? (args.num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1
                              : 0;
     const int steps = my_tiles * args.k_blocks;
-    const uint32_t tcol = tmem_base + t_lane + (uint32_t)(cg * 64);
-    uint8_t* bt = bst + cg * BST;
+    uint8_t* bt = dec + cg * lb::kDecBytes;   // weights: rows 0..255 x 128 bytes
+    uint8_t* at = bt + lb::kBBytes;            // tokens: rows 0..nt-1 x 128 bytes
     for (int j = cg; j < steps; j += lb::kConvGroups) {
       const int rs = j % R;
-      bool w_ok = mbar_wait(&raw_full[rs], (uint32_t)(j / R) & 1u, abort_flag, kErrTimeoutFull);
-      w_ok = w_ok && mbar_wait(&cv_empty[cg], ((uint32_t)(j / lb::kConvGroups) & 1u) ^ 1u,
-                               abort_flag, kErrTimeoutEmpty);
-      if (__any_sync(0xffffffffu, !w_ok)) break;
+      const bool r_ok =
+          mbar_wait(&raw_full[rs], (uint32_t)(j / R) & 1u, abort_flag, kErrTimeoutFull);
+      if (__any_sync(0xffffffffu, !r_ok)) break;
+      // the K-step's words into registers, then the raw stage goes back to
+      // the producer: its next copy is in flight while this group decodes
       const uint8_t* st = raw + rs * RAW;
+      uint4 lw[2][2];
+      uint2 hw[2][2];
+      uint32_t sw[2];
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
+        const uint8_t* tile = st + which * F::kTileBytes;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          uint32_t a[16];
-          lb_decode_row<BITS>(st + which * F::kTileBytes, r, half, a);
-          tmem_st16(tcol + (uint32_t)(which * 32 + half * 16), a);
+          lw[which][half] = *reinterpret_cast<const uint4*>(tile + half * 2048 + ti * 16);
+          hw[which][half] =
+              BITS == 6 ? *reinterpret_cast<const uint2*>(tile + 4096 + ti * 16 + half * 8)
+                        : make_uint2(0u, 0u);
+        }
+        sw[which] = *reinterpret_cast<const uint32_t*>(tile + F::kScaleOff + ti * 4);
+      }
+      constexpr int kXChunks = lb::kMaxNt * 8 / 128;  // 8-byte chunks of codes per thread
+      uint2 xv[kXChunks];
+      const uint8_t* act = st + 2 * F::kTileBytes;
+#pragma unroll
+      for (int m = 0; m < kXChunks; ++m) {
+        const int u = ti + 128 * m;
+        xv[m] = u < nt * 8 ? *reinterpret_cast<const uint2*>(act + u * 8) : make_uint2(0u, 0u);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&raw_empty[rs]);
+      const bool d_ok = mbar_wait(&cv_empty[cg], ((uint32_t)(j / lb::kConvGroups) & 1u) ^ 1u,
+                                  abort_flag, kErrTimeoutEmpty);
+      if (__any_sync(0xffffffffu, !d_ok)) break;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const int row = which * 128 + ti;
+        uint8_t* dst = bt + row * 128;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[16];
+          lb_decode_words<BITS>(lw[which][half], hw[which][half], sw[which], half, o);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(dst + (((4 * half + c) ^ (row & 7)) << 4)) =
+                make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
         }
       }
-      const uint8_t* act = st + 2 * F::kTileBytes;
-      for (int u = ct; u < nt * 8; u += 128) {
-        const int row = u >> 3, ch = u & 7;
-        const uint2 xv = *reinterpret_cast<const uint2*>(act + row * 64 + ch * 8);
-        uint4 o;
-        i8x4_to_h2x2(xv.x, o.x, o.y);
-        i8x4_to_h2x2(xv.y, o.z, o.w);
-        *reinterpret_cast<uint4*>(bt + row * 128 + ((ch ^ (row & 7)) << 4)) = o;
+#pragma unroll
+      for (int m = 0; m < kXChunks; ++m) {
+        const int u = ti + 128 * m;
+        if (u < nt * 8) {
+          const int row = u >> 3, ch = u & 7;
+          uint4 o;
+          i8x4_to_h2x2(xv[m].x, o.x, o.y);
+          i8x4_to_h2x2(xv[m].y, o.z, o.w);
+          *reinterpret_cast<uint4*>(at + row * 128 + ((ch ^ (row & 7)) << 4)) = o;
+        }
       }
-      tmem_wait_st();
       fence_proxy_async_smem();
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&cv_full[cg]);
-        mbar_arrive(&raw_empty[rs]);
-      }
+      if (lane == 0) mbar_arrive(&cv_full[cg]);
     }
   } else {
     // ------------------------------------------------------------ epilogue --
     griddep_wait();  // the token scales come from the previous kernel
     griddep_launch_dependents();
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;
     const uint32_t t_lane = (uint32_t)(quad * 32) << 16;
-    const int ks = args.ks;
     int it = 0;
     for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
-      const int acc = args.n_acc == 2 ? (it & 1) : 0;
-      const uint32_t acc_phase = (uint32_t)(args.n_acc == 2 ? (it >> 1) : it) & 1u;
-      // the tile's scales are requested before the wait for its accumulators:
-      // lane l holds the token scales of tokens t0 + l + 32 i
+      const int acc = it & 1;
+      const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
       int g, wb, tb;
       lb_decode_tile(args, tile, g, wb, tb);
+      // column j of the accumulator is weight row j of the tile's two blocks;
+      // every lane reads the same scales (one broadcast load per warp)
+      const float* sw0 = args.s_w + (int64_t)g * args.N + (kSwiglu ? wb * 128 : wb * 256);
+      const float* sw1 = kSwiglu ? sw0 + args.n_out : sw0 + 128;
       const int t0 = tb * nt;
-      const int n0 = kSwiglu ? wb * 128 + r : wb * 256 + r;
-      const int n1 = kSwiglu ? args.n_out + n0 : n0 + 128;
-      const float sw0 = __ldg(args.s_w + (int64_t)g * args.N + n0);
-      const float sw1 = __ldg(args.s_w + (int64_t)g * args.N + n1);
-      static_assert(lb::kMaxNt == 128, "four token-scale registers per lane");
-      auto sx_at = [&](int i) {
-        const int t = t0 + 32 * i + lane;
-        return (EPI != kLbF32 && 32 * i < nt && t < args.M)
-                   ? __ldg(args.s_x + (int64_t)g * args.M + t) : 0.0f;
-      };
-      const float sx0 = sx_at(0), sx1 = sx_at(1), sx2 = sx_at(2), sx3 = sx_at(3);
+      const int row = quad * 32 + lane;
+      const int t = t0 + row;
+      const bool valid = row < nt && t < args.M;
+      const float sx = (EPI != kLbF32 && valid) ? __ldg(args.s_x + (int64_t)g * args.M + t) : 0.0f;
       const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrTimeoutTmemFull);
       if (__any_sync(0xffffffffu, !ok)) break;
       tc_fence_after();
-      const uint32_t dbase = tmem_base + t_lane + (uint32_t)(lb::kAccCol0 + acc * 2 * ks * nt);
-      for (int c0 = 0; c0 < nt; c0 += 16) {
-        // each block's accumulator sets, added in set order
-        float v0[16], v1[16];
-        {
-          uint32_t u0[16], u1[16];
-          tmem_ld16(dbase + c0, u0);
-          tmem_ld16(dbase + (uint32_t)(ks * nt) + c0, u1);
-          tmem_wait_ld();
+      const uint32_t d = tmem_base + t_lane + (uint32_t)(acc * 256);
+      const bool warp_rows = quad * 32 < nt && t0 + quad * 32 < args.M;  // warp-uniform
+      if (warp_rows) {
+        const int64_t orow = (int64_t)g * args.M + t;
+        if constexpr (kSwiglu) {
+          float* out = reinterpret_cast<float*>(args.out) + orow * args.n_out + wb * 128;
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            __syncwarp();
+            uint32_t gv[16], uv[16];
+            tmem_ld16(d + c * 16, gv);
+            tmem_ld16(d + 128 + c * 16, uv);
+            float sg[16], su[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            v0[i] = __uint_as_float(u0[i]);
-            v1[i] = __uint_as_float(u1[i]);
+            for (int q = 0; q < 4; ++q) {
+              *reinterpret_cast<float4*>(sg + 4 * q) =
+                  __ldg(reinterpret_cast<const float4*>(sw0 + c * 16) + q);
+              *reinterpret_cast<float4*>(su + 4 * q) =
+                  __ldg(reinterpret_cast<const float4*>(sw1 + c * 16) + q);
+            }
+            tmem_wait_ld();
+            float h[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float yg =
+                  __fmul_rn(__fmul_rn(__uint_as_float(gv[i]), 16.0f), __fmul_rn(sx, sg[i]));
+              const float yu =
+                  __fmul_rn(__fmul_rn(__uint_as_float(uv[i]), 16.0f), __fmul_rn(sx, su[i]));
+              h[i] = __fmul_rn(silu_f32(yg), yu);
+            }
+            if (valid) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<float4*>(out + c * 16 + 4 * q) =
+                    make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+            }
           }
-        }
-        for (int q = 1; q < ks; ++q) {
-          uint32_t u[16];
-          tmem_ld16(dbase + (uint32_t)(q * nt) + c0, u);
-          tmem_wait_ld();
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            __syncwarp();
+            uint32_t v[16];
+            tmem_ld16(d + c * 16, v);
+            float sc[16];
+            if constexpr (EPI == kLbBf16) {
+              const float* sp = (c < 8 ? sw0 : sw1) + (c & 7) * 16;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v0[i] = __fadd_rn(v0[i], __uint_as_float(u[i]));
-          tmem_ld16(dbase + (uint32_t)((ks + q) * nt) + c0, u);
-          tmem_wait_ld();
+              for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<float4*>(sc + 4 * q) =
+                    __ldg(reinterpret_cast<const float4*>(sp) + q);
+            }
+            tmem_wait_ld();
+            if (valid) {
+              const int n0 = wb * 256 + c * 16;
+              if constexpr (EPI == kLbF32) {
+                float* out = reinterpret_cast<float*>(args.out) + orow * args.N + n0;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v1[i] = __fadd_rn(v1[i], __uint_as_float(u[i]));
-        }
-        // the register holding this chunk's token scales
-        const float sx_src = c0 < 32 ? sx0 : c0 < 64 ? sx1 : c0 < 96 ? sx2 : sx3;
+                for (int q = 0; q < 4; ++q)
+                  *reinterpret_cast<float4*>(out + 4 * q) =
+                      make_float4(__fmul_rn(__uint_as_float(v[4 * q]), 16.0f),
+                                  __fmul_rn(__uint_as_float(v[4 * q + 1]), 16.0f),
+                                  __fmul_rn(__uint_as_float(v[4 * q + 2]), 16.0f),
+                                  __fmul_rn(__uint_as_float(v[4 * q + 3]), 16.0f));
+              } else {
+                uint32_t w[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int t = t0 + c0 + i;
-          const float sx = __shfl_sync(0xffffffffu, sx_src, (c0 & 16) + i);
-          if (t >= args.M) continue;
-          const float a0 = __fmul_rn(v0[i], 16.0f);
-          const float a1 = __fmul_rn(v1[i], 16.0f);
-          const int64_t orow = (int64_t)g * args.M + t;
-          if constexpr (EPI == kLbF32) {
-            float* out = reinterpret_cast<float*>(args.out) + orow * args.N;
-            out[n0] = a0;
-            out[n1] = a1;
-          } else if constexpr (EPI == kLbBf16) {
-            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.N;
-            out[n0] = __float2bfloat16_rn(__fmul_rn(a0, __fmul_rn(sx, sw0)));
-            out[n1] = __float2bfloat16_rn(__fmul_rn(a1, __fmul_rn(sx, sw1)));
-          } else {
-            const float yg = __fmul_rn(a0, __fmul_rn(sx, sw0));
-            const float yu = __fmul_rn(a1, __fmul_rn(sx, sw1));
-            reinterpret_cast<float*>(args.out)[orow * args.n_out + n0] =
-                __fmul_rn(silu_f32(yg), yu);
+                for (int i = 0; i < 8; ++i) {
+                  const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * i]), 16.0f),
+                                             __fmul_rn(sx, sc[2 * i]));
+                  const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(v[2 * i + 1]), 16.0f),
+                                             __fmul_rn(sx, sc[2 * i + 1]));
+                  const __nv_bfloat162 pr = __floats2bfloat162_rn(y0, y1);
+                  w[i] = *reinterpret_cast<const uint32_t*>(&pr);
+                }
+                uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(args.out) +
+                                                      orow * args.N + n0);
+                out[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                out[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              }
+            }
           }
         }
       }
@@ -694,9 +707,9 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
           mbar_wait_limit(&raw_full[s], (issued_parity >> s) & 1u, &never, kErrTimeoutTeardown,
                           100000000ull);
     }
-    if (warp >= 1 && warp < lb::kConvWarp0 && lane == 0 && mma_issued) {
-      umma_commit(&drain[warp - 1]);
-      mbar_wait_limit(&drain[warp - 1], 0, &never, kErrTimeoutTeardown, 100000000ull);
+    if (warp == 1 && lane == 0 && mma_issued) {
+      umma_commit(drain);
+      mbar_wait_limit(drain, 0, &never, kErrTimeoutTeardown, 100000000ull);
     }
     __syncthreads();
   }
