@@ -836,7 +836,7 @@ def run_ablation(args, cfg):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="moe_T8192", choices=sorted(MOE_CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -432,7 +432,9 @@ int convrot_quantize_weights_lowbit(const void* w_bf16, int64_t rows, int64_t K,
  *   CONVROT_LOWBIT_SWIGLU  out fp32 [G, M, N/2] = silu(y[:, f]) * y[:, N/2 + f]
  *                          with y = acc * (s_x * s_r) (gate rows first)
  * N % 256 == 0; 64 <= K <= 16384, K % 64 == 0. tile_tokens = tokens per
- * tile (a multiple of 16, at most 128), 0 = chosen by the library. */
+ * tile (a multiple of 16, at most 128), 0 = chosen by the library (for
+ * M > 128 CTA pairs of 2 x 128 tokens that share each decoded weight). The
+ * result does not depend on the choice beyond fp32 summation order. */
 enum { CONVROT_LOWBIT_F32 = 0, CONVROT_LOWBIT_BF16 = 1, CONVROT_LOWBIT_SWIGLU = 2 };
 int convrot_lowbit_gemm(const int8_t* x_q, const float* s_x, const void* w_packed,
                         const float* row_scale, int64_t G, int64_t M, int64_t N, int64_t K,

@@ -120,6 +120,9 @@ GEMM_CASES = [  # g, m, n, k, tile_tokens (0 = the library's choice)
     (1, 64, 256, 256, 0), (3, 100, 512, 384, 0), (2, 200, 256, 2048, 0), (2, 200, 256, 512, 64),
     (1, 33, 768, 192, 16), (2, 130, 256, 320, 128), (1, 1, 256, 64, 0), (2, 256, 512, 1536, 0),
     (1, 48, 256, 640, 48),
+    # more than 128 tokens per group with the library's choice: CTA pairs of
+    # 2 x 128 tokens (one over, ragged second CTA, several pair blocks)
+    (3, 129, 256, 128, 0), (2, 300, 768, 640, 0), (1, 520, 512, 256, 0),
 ]
 
 
@@ -158,7 +161,7 @@ def _bf16_ulp(v):
 
 @pytest.mark.parametrize("bits", [4, 6])
 @pytest.mark.parametrize("g,m,n,k,nt", [(2, 200, 512, 1024, 0), (1, 40, 256, 256, 0),
-                                        (3, 77, 256, 384, 32)])
+                                        (3, 77, 256, 384, 32), (1, 390, 768, 512, 0)])
 def test_lowbit_gemm_bf16(bits, g, m, n, k, nt):
     x, s_x, lw, q, sig, s_r = _gemm_case(g, m, n, k, bits, seed=7 * m + n)
     y = W.convrot_lowbit_gemm(x.cuda(), s_x.cuda(), lw, W.CONVROT_LOWBIT_BF16, nt)
@@ -194,7 +197,7 @@ def _check_swiglu(h_gpu, x_q, s_x, q, sig, s_r):
 
 @pytest.mark.parametrize("bits", [4, 6])
 @pytest.mark.parametrize("g,m,f,k,nt", [(2, 160, 256, 768, 0), (1, 64, 1536, 2048, 0),
-                                        (3, 40, 128, 512, 16)])
+                                        (3, 40, 128, 512, 16), (2, 280, 384, 256, 0)])
 def test_lowbit_gemm_swiglu(bits, g, m, f, k, nt):
     x, s_x, lw, q, sig, s_r = _gemm_case(g, m, 2 * f, k, bits, seed=3 * m + f)
     h = W.convrot_lowbit_gemm(x.cuda(), s_x.cuda(), lw, W.CONVROT_LOWBIT_SWIGLU, nt)
@@ -332,12 +335,14 @@ def test_lowbit_moe_block_small(bits, name):
 
 @pytest.mark.slow
 @pytest.mark.parametrize("bits", [4, 6])
-def test_lowbit_moe_block_full_size(bits):
-    """The T=2048 block in the bench's launch configuration: routing exact,
+@pytest.mark.parametrize("name", ["moe_T2048", "moe_T8192"])
+def test_lowbit_moe_block_full_size(bits, name):
+    """The T=2048 and T=8192 blocks in the bench's launch configuration (64
+    and 256 tokens per expert: single CTAs and CTA pairs): routing exact,
     every stage of a spread of experts against the oracle given the GPU's
     inputs to it, every output row given z, and sampled rows within 1e-2 of
     the oracle's whole block."""
-    cfg = MOE_CONFIGS["moe_T2048"]
+    cfg = MOE_CONFIGS[name]
     inp = moe_inputs(cfg)
     y, v, gu, dn = _run_lowbit_moe(inp, cfg, bits)
     gu_ref, dn_ref = _lowbit_moe_weights(gu, dn, cfg)

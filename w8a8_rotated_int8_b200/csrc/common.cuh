@@ -78,17 +78,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same with acquire semantics at cluster scope: for a phase completed by
+// release arrivals from the other CTA of a pair, whose shared-memory writes the
+// waiting thread (or the tensor core it then drives) must see.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+template <bool kCluster>
+__device__ __forceinline__ bool mbar_try_wait_t(uint64_t* bar, uint32_t parity) {
+  if constexpr (kCluster)
+    return mbar_try_wait_cluster(bar, parity);
+  else
+    return mbar_try_wait(bar, parity);
+}
+
 // Waits until the phase with the given parity has completed. Returns false if
 // the CTA's abort flag is raised or `limit_ns` passes (then the error bit is
 // recorded and the abort flag raised so the other warp roles stop too).
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
                                                 volatile int* abort_flag, unsigned err_bit,
                                                 uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_t<kCluster>(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_t<kCluster>(bar, parity)) return true;
     if ((++spins & 15u) == 0) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > limit_ns) {
@@ -100,9 +124,10 @@ __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
   }
 }
 
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned err_bit) {
-  return mbar_wait_limit(bar, parity, abort_flag, err_bit, g_wait_limit_ns);
+  return mbar_wait_limit<kCluster>(bar, parity, abort_flag, err_bit, g_wait_limit_ns);
 }
 
 // Waits (bounded, ignoring any abort flag) for a phase to complete: used on
@@ -363,6 +388,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 // the cluster).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+// The same without release semantics: orders nothing before it.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
 

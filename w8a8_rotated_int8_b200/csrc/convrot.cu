@@ -33,6 +33,8 @@ struct DeviceInfo {
   // them, since its tiles wait for one another
   int rq_ctas = 0;
   int rq_pairs = 0;
+  // CTA pairs of the low-bit GEMM that can be resident at once
+  int lb_pairs = 0;
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -67,7 +69,9 @@ void set_gemm_attr() {
 
 template <int BITS, int EPI>
 void set_lowbit_attr() {
-  cudaFuncSetAttribute(gemm_lowbit_tcgen05_kernel<BITS, EPI>,
+  cudaFuncSetAttribute(gemm_lowbit_tcgen05_kernel<BITS, EPI, false>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, lb::kSmemMax);
+  cudaFuncSetAttribute(gemm_lowbit_tcgen05_kernel<BITS, EPI, true>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, lb::kSmemMax);
 }
 
@@ -116,6 +120,27 @@ int swiglu_rq_residency(int sms, int* ctas, int* pairs) {
   return CONVROT_OK;
 }
 
+// Co-resident CTA pairs of the low-bit GEMM on this device.
+int lowbit_pair_residency(int sms, int* pairs) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(2 * (unsigned)(sms / 2));
+  lc.blockDim = dim3(lb::kThreads);
+  lc.dynamicSmemBytes = lb::kSmemMax;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  lc.attrs = &attr;
+  lc.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, gemm_lowbit_tcgen05_kernel<6, kLbSwiglu, true>,
+                                     &lc) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  *pairs = clusters;
+  return CONVROT_OK;
+}
+
 // Per-device one-time setup: capability check, SM count, kernel attributes.
 int device_setup(int* sm_count) {
   int dev = 0;
@@ -142,7 +167,8 @@ int device_setup(int* sm_count) {
       set_lowbit_attrs<4>();
       set_lowbit_attrs<6>();
       if (cudaGetLastError() != cudaSuccess) return CONVROT_ERR_CUDA;
-      if (swiglu_rq_residency(sms, &d.rq_ctas, &d.rq_pairs) != CONVROT_OK) {
+      if (swiglu_rq_residency(sms, &d.rq_ctas, &d.rq_pairs) != CONVROT_OK ||
+          lowbit_pair_residency(sms, &d.lb_pairs) != CONVROT_OK) {
         cudaGetLastError();
         return CONVROT_ERR_CUDA;
       }
@@ -152,6 +178,15 @@ int device_setup(int* sm_count) {
   if (!d.supported) return CONVROT_ERR_UNSUPPORTED_DEVICE;
   if (sm_count) *sm_count = d.sm_count;
   return CONVROT_OK;
+}
+
+// Co-resident CTA pairs of the low-bit GEMM on the current device; 0 before
+// device_setup.
+int lowbit_pair_capacity() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  return g_dev[dev].lb_pairs;
 }
 
 // Co-resident CTAs (pairs = false) or CTA pairs of the requantising SwiGLU
@@ -785,21 +820,25 @@ int launch_lowbit_gemm(const int8_t* x, const float* s_x, const uint8_t* wq, con
   int rc = device_setup(&sms);
   if (rc != CONVROT_OK) return rc;
   if (G == 0 || M == 0 || N == 0) return CONVROT_OK;
+  // more than one tile of tokens per group: CTA pairs, each decoded weight
+  // serving the 256 tokens of both CTAs
+  const int pairs = lowbit_pair_capacity();
+  const bool pair = tile_tokens == 0 && M > lb::kMaxNt && pairs > 0;
   LowbitArgs a{};
   a.G = (int)G;
   a.M = (int)M;
   a.N = (int)N;
   a.K = (int)K;
   a.n_out = (int)(EPI == kLbSwiglu ? N / 2 : N);
-  a.nt = tile_tokens > 0 ? tile_tokens : lowbit_auto_nt(M);
+  a.nt = pair ? lb::kMaxNt : tile_tokens > 0 ? tile_tokens : lowbit_auto_nt(M);
   a.box_rows = (int)std::min<int64_t>(a.nt, M);
-  a.t_blocks = (int)cdiv(M, a.nt);
+  a.t_blocks = (int)cdiv(M, pair ? 2 * a.nt : a.nt);
   a.w_blocks = (int)(N / 256);
   a.k_blocks = (int)(K / 64);
   const int64_t tiles = G * a.w_blocks * a.t_blocks;
   if (tiles >= ((int64_t)1 << 31)) return CONVROT_ERR_INVALID_ARG;
   a.num_tiles = (int)tiles;
-  a.raw_stages = lb::raw_stages<BITS>(a.nt);
+  a.raw_stages = lb::raw_stages<BITS>(a.nt, pair);
   a.wq = wq;
   a.s_w = s_w;
   a.s_x = s_x;
@@ -808,10 +847,16 @@ int launch_lowbit_gemm(const int8_t* x, const float* s_x, const uint8_t* wq, con
   if ((rc = encode_act_i8(&tx, x, (uint64_t)K, (uint64_t)M, (uint64_t)G, (uint32_t)a.box_rows)) !=
       CONVROT_OK)
     return rc;
-  const int grid = (int)std::min<int64_t>(tiles, sms);
-  if ((rc = launch_kernel(gemm_lowbit_tcgen05_kernel<BITS, EPI>, dim3(grid), dim3(lb::kThreads),
-                          lb::smem_bytes<BITS>(a.nt), st, pdl, 1, tx, a)) != CONVROT_OK)
-    return rc;
+  if (pair) {
+    const int grid = 2 * (int)std::min<int64_t>(tiles, pairs);
+    rc = launch_kernel(gemm_lowbit_tcgen05_kernel<BITS, EPI, true>, dim3(grid), dim3(lb::kThreads),
+                       lb::smem_bytes<BITS>(a.nt, true), st, pdl, 2, tx, a);
+  } else {
+    const int grid = (int)std::min<int64_t>(tiles, sms);
+    rc = launch_kernel(gemm_lowbit_tcgen05_kernel<BITS, EPI, false>, dim3(grid),
+                       dim3(lb::kThreads), lb::smem_bytes<BITS>(a.nt, false), st, pdl, 1, tx, a);
+  }
+  if (rc != CONVROT_OK) return rc;
   return launch_status();
 }
 

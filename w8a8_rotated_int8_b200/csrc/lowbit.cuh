@@ -195,47 +195,54 @@ enum LowbitEpilogue : int {
 
 namespace lb {
 constexpr int kMaxRawStages = 8;        // packed weights + int8 activation codes, per K-step of 64
-constexpr int kDecStages = 3;           // decoded stages: fp16 weights (N) and tokens (M)
-constexpr int kConvGroups = kDecStages; // group g decodes the K-steps j with j % 3 == g
+constexpr int kConvGroups = 3;          // group g decodes the K-steps j with j % 3 == g
 constexpr int kConvWarps = 4 * kConvGroups;
 constexpr int kEpiWarps = 4;
 constexpr int kConvWarp0 = 2;
 constexpr int kEpiWarp0 = kConvWarp0 + kConvWarps;
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
-constexpr int kMaxNt = 128;             // tokens per tile (the MMA's M)
-constexpr int kBBytes = 256 * 128;      // decoded weights: 256 rows x 64 codes, fp16
+constexpr int kMaxNt = 128;             // tokens per tile (per CTA of a pair)
 constexpr int kABytes = kMaxNt * 128;   // widened tokens: 128 rows x 64 codes, fp16
-constexpr int kDecBytes = kBBytes + kABytes;
 constexpr uint32_t kTmemCols = 512;     // two accumulators of 256 columns
 constexpr int kBarBytes = 512;
 constexpr int kSmemMax = 232448;        // the opt-in limit per CTA
-// Shared memory of one raw stage for nt tokens (the two weight tiles, then
+// A CTA decodes both 128-row weight blocks of a tile, or (CTA pair) one.
+__host__ __device__ constexpr int w_tiles(bool pair) { return pair ? 1 : 2; }
+// decoded stages: fp16 weights (the N operand, this CTA's rows) and tokens
+__host__ __device__ constexpr int dec_stages(bool pair) { return pair ? 4 : 3; }
+__host__ __device__ constexpr int b_bytes(bool pair) { return w_tiles(pair) * 128 * 128; }
+__host__ __device__ constexpr int dec_bytes(bool pair) { return b_bytes(pair) + kABytes; }
+// Shared memory of one raw stage for nt tokens (this CTA's weight tiles, then
 // the activation box), rounded to 1024 bytes.
 template <int BITS>
-__host__ __device__ constexpr int raw_stage_bytes(int nt) {
-  return (2 * LbFmt<BITS>::kTileBytes + nt * 64 + 1023) / 1024 * 1024;
+__host__ __device__ constexpr int raw_stage_bytes(int nt, bool pair) {
+  return (w_tiles(pair) * LbFmt<BITS>::kTileBytes + nt * 64 + 1023) / 1024 * 1024;
 }
 // As many raw stages as fit beside the decoded stages.
 template <int BITS>
-__host__ __device__ constexpr int raw_stages(int nt) {
-  const int room = kSmemMax - 1024 - kBarBytes - kDecStages * kDecBytes;
-  const int r = room / raw_stage_bytes<BITS>(nt);
+__host__ __device__ constexpr int raw_stages(int nt, bool pair) {
+  const int room = kSmemMax - 1024 - kBarBytes - dec_stages(pair) * dec_bytes(pair);
+  const int r = room / raw_stage_bytes<BITS>(nt, pair);
   return r > kMaxRawStages ? kMaxRawStages : r;
 }
 template <int BITS>
-__host__ __device__ constexpr int smem_bytes(int nt) {
-  return kDecStages * kDecBytes + raw_stages<BITS>(nt) * raw_stage_bytes<BITS>(nt) + kBarBytes +
-         1024;
+__host__ __device__ constexpr int smem_bytes(int nt, bool pair) {
+  return dec_stages(pair) * dec_bytes(pair) +
+         raw_stages<BITS>(nt, pair) * raw_stage_bytes<BITS>(nt, pair) + kBarBytes + 1024;
 }
-static_assert(raw_stages<6>(kMaxNt) >= 3 && smem_bytes<6>(kMaxNt) <= kSmemMax, "shared memory");
+static_assert(raw_stages<6>(kMaxNt, false) >= 3 && smem_bytes<6>(kMaxNt, false) <= kSmemMax,
+              "shared memory");
+static_assert(raw_stages<6>(kMaxNt, true) >= 4 && smem_bytes<6>(kMaxNt, true) <= kSmemMax,
+              "shared memory");
 }  // namespace lb
 
 struct LowbitArgs {
   int G, M, N, K;       // groups, tokens per group, weight rows per group (2F for SwiGLU), K
   int n_out;            // output columns: N, or F for SwiGLU
-  int nt;               // tokens per tile: a multiple of 16, at most 128
+  int nt;               // tokens per tile (per CTA): a multiple of 16, at most 128
+                        // (128 for CTA pairs, whose tiles hold 2 x 128 tokens)
   int box_rows;         // rows of the activation box: min(nt, M)
-  int t_blocks, w_blocks, k_blocks, num_tiles;
+  int t_blocks, w_blocks, k_blocks, num_tiles;  // token blocks of the tile's tokens
   int raw_stages;       // depth of the raw ring (lb::raw_stages)
   const uint8_t* wq;    // packed weight tiles (see the top of this file)
   const float* s_w;     // [G*N] row scales
@@ -322,6 +329,19 @@ __device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// The CTA-pair form: D (M = 256 over the pair) (+)= A * B^T, each CTA
+// supplying its 128 token rows of A and its 128 of the N = 256 weight rows of
+// B at the same shared-memory offsets; issued by one thread of the leader.
+__device__ __forceinline__ void umma_f16_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void lb_decode_tile(const LowbitArgs& a, int tile, int& g, int& wb,
                                                int& tb) {
   tb = tile % a.t_blocks;
@@ -338,47 +358,64 @@ __device__ __forceinline__ int64_t lb_row_block(const LowbitArgs& a, int g, int 
   return swiglu ? base + wb + (which ? a.n_out / 128 : 0) : base + 2 * wb + which;
 }
 
-// One persistent CTA per SM. Tiles (group, weight block of 2 x 128 rows,
-// token block of nt), token block fastest so CTAs running together share the
-// weight tiles through L2.
+// One persistent CTA per SM, or (PAIR) one CTA pair per two SMs. A tile is
+// (group, weight block of 2 x 128 rows, token block), the token block fastest
+// so CTAs running together share the weight tiles through L2. A single CTA
+// takes nt tokens and decodes both weight blocks; the two CTAs of a pair take
+// 128 tokens each and decode one weight block each (the gate / first block in
+// the leader, rank 0), and the leader's MMAs (M = 256 over the pair) read
+// both CTAs' halves, so each decoded weight serves 256 tokens.
 //   warp 0      producer: per K-step one bulk copy per weight tile and a 3-D
-//               TMA box {64 codes, box_rows tokens} of the activation codes
-//   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
-//               kind::f16 M=128 N=256 K=16, four per K-step, into one of two
-//               256-column accumulators
+//               TMA box {64 codes, box_rows tokens} of the activation codes,
+//               into this CTA's shared memory
+//   warp 1      allocates 512 TMEM columns (in both CTAs of a pair); one lane
+//               (of the leader) issues tcgen05.mma kind::f16 with N = 256 and
+//               K = 16, four per K-step, into one of two 256-column
+//               accumulators; in the other CTA of a pair, lanes 0..S-1 relay
+//               its decoded stages' completion to the leader
 //   warps 2-13  converters in three groups of four warps; group g takes the
-//               K-steps j with j % 3 == g (decoded stage g): thread i decodes
-//               rows i and 128 + i of the K-step's weights into the N operand
-//               and widens a share of the activation codes into the M operand
+//               K-steps j with j % 3 == g: thread i decodes row i of each of
+//               the CTA's weight tiles into the N operand and widens a share
+//               of the activation codes into the M operand, in decoded stage
+//               j % S
 //   warps 14-17 epilogue: tcgen05.ld of the quadrant's token rows, 16
 //               columns at a time; each lane writes its row's outputs
-template <int BITS, int EPI>
+template <int BITS, int EPI, bool PAIR>
 __global__ void __launch_bounds__(lb::kThreads, 1)
     gemm_lowbit_tcgen05_kernel(const __grid_constant__ CUtensorMap tmX, const LowbitArgs args) {
   using F = LbFmt<BITS>;
-  constexpr int S = lb::kDecStages;
+  constexpr int S = lb::dec_stages(PAIR);
+  constexpr int WT = lb::w_tiles(PAIR);
+  constexpr int DEC = lb::dec_bytes(PAIR);
   constexpr bool kSwiglu = EPI == kLbSwiglu;
   const int nt = args.nt;
   const int R = args.raw_stages;
-  const int RAW = lb::raw_stage_bytes<BITS>(nt);
+  const int RAW = lb::raw_stage_bytes<BITS>(nt, PAIR);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t rawp = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((rawp + 1023u) & ~1023u) - rawp);
-  uint8_t* dec = smem;                               // S x (B 32 KB, A 16 KB)
-  uint8_t* raw = smem + S * lb::kDecBytes;           // R raw stages
+  uint8_t* dec = smem;                               // S x (B, then A 16 KB)
+  uint8_t* raw = smem + S * DEC;                     // R raw stages
   uint64_t* bars = reinterpret_cast<uint64_t*>(raw + R * RAW);
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = bars + lb::kMaxRawStages;
   uint64_t* cv_full = bars + 2 * lb::kMaxRawStages;
   uint64_t* cv_empty = cv_full + S;
   uint64_t* tfull = cv_empty + S;
-  uint64_t* tempty = tfull + 2;
+  uint64_t* tempty = tfull + 2;                      // the leader's, for a pair
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* fin = drain + 1;                         // pair teardown handshake
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // CTA or pair
+  const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  // this CTA's first token row within a tile's token block
+  const int row0 = PAIR ? (int)rank * lb::kMaxNt : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < R; ++s) {
@@ -386,24 +423,34 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
       mbar_init(&raw_empty[s], 4);
     }
     for (int s = 0; s < S; ++s) {
-      mbar_init(&cv_full[s], 4);
+      // a pair's leader: its four converter warps and the other CTA's relay
+      mbar_init(&cv_full[s], PAIR && leader ? 5 : 4);
       mbar_init(&cv_empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], lb::kEpiWarps);
+      mbar_init(&tempty[a], (PAIR ? 2 : 1) * lb::kEpiWarps);
     }
     mbar_init(drain, 1);
+    mbar_init(fin, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tmX);
   if (warp == 1) {
-    tmem_alloc(tmem_slot, lb::kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, lb::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, lb::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();  // both CTAs' barriers exist before any remote use
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -414,27 +461,28 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
     if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
-      const uint32_t tx = (uint32_t)(2 * F::kTileBytes + args.box_rows * 64);
+      const uint32_t tx = (uint32_t)(WT * F::kTileBytes + args.box_rows * 64);
       auto load_w = [&](int s, int g, int wb, int kb) {
         uint8_t* dst = raw + s * RAW;
 #pragma unroll
-        for (int which = 0; which < 2; ++which) {
-          const int64_t rb = lb_row_block(args, g, wb, which, kSwiglu);
-          bulk_load_1d(dst + which * F::kTileBytes,
+        for (int i = 0; i < WT; ++i) {
+          const int64_t rb = lb_row_block(args, g, wb, PAIR ? (int)rank : i, kSwiglu);
+          bulk_load_1d(dst + i * F::kTileBytes,
                        args.wq + (rb * args.k_blocks + kb) * (int64_t)F::kTileBytes,
                        (uint32_t)F::kTileBytes, &raw_full[s], pol_w);
         }
       };
+      const int tb_rows = PAIR ? 2 * lb::kMaxNt : nt;  // tokens per token block
       auto load_x = [&](int s, int g, int tb, int kb) {
-        tma_load_3d(raw + s * RAW + 2 * F::kTileBytes, &tmX, &raw_full[s], kb * 64, tb * nt, g,
-                    pol_x);
+        tma_load_3d(raw + s * RAW + WT * F::kTileBytes, &tmX, &raw_full[s], kb * 64,
+                    tb * tb_rows + row0, g, pol_x);
       };
       // the first tile's first stages: weights before the wait for the kernel
       // that wrote the activation codes (they do not depend on it)
       int pre = 0;
-      if ((int)blockIdx.x < args.num_tiles) {
+      if (unit < args.num_tiles) {
         int g, wb, tb;
-        lb_decode_tile(args, blockIdx.x, g, wb, tb);
+        lb_decode_tile(args, unit, g, wb, tb);
         pre = min(args.k_blocks, R);
         for (int kb = 0; kb < pre; ++kb) {
           mbar_arrive_expect_tx(&raw_full[kb], tx);
@@ -450,11 +498,11 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
       }
       int s = pre % R;
       uint32_t ph = pre == R ? 1u : 0u;
-      for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
+      for (int tile = unit; tile < args.num_tiles; tile += n_units) {
         int g, wb, tb;
         lb_decode_tile(args, tile, g, wb, tb);
         bool ok = true;
-        for (int kb = tile == (int)blockIdx.x ? pre : 0; kb < args.k_blocks; ++kb) {
+        for (int kb = tile == unit ? pre : 0; kb < args.k_blocks; ++kb) {
           if (!mbar_wait(&raw_empty[s], ph ^ 1u, abort_flag, kErrTimeoutEmpty)) {
             ok = false;
             break;
@@ -473,77 +521,107 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16_f32(128, 256);
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_f16_f32(PAIR ? 256 : 128, 256);
       int s = 0;
       uint32_t ph = 0;
       int it = 0;
-      for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
+      for (int tile = unit; tile < args.num_tiles; tile += n_units, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, kErrTimeoutTmemEmpty)) break;
+        if (!mbar_wait<PAIR>(&tempty[acc], acc_phase ^ 1u, abort_flag, kErrTimeoutTmemEmpty))
+          break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(acc * 256);
         bool ok = true;
         for (int kb = 0; kb < args.k_blocks; ++kb) {
-          if (!mbar_wait(&cv_full[s], ph, abort_flag, kErrTimeoutFull)) {
+          if (!mbar_wait<PAIR>(&cv_full[s], ph, abort_flag, kErrTimeoutFull)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t b_addr = smem_u32(dec + s * lb::kDecBytes);
-          const uint32_t a_addr = b_addr + lb::kBBytes;
+          const uint32_t b_addr = smem_u32(dec + s * DEC);
+          const uint32_t a_addr = b_addr + lb::b_bytes(PAIR);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_f16_ss(d, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k), idesc,
-                        (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = sdesc_k_sw128(a_addr + 32 * k);
+            const uint64_t bd = sdesc_k_sw128(b_addr + 32 * k);
+            if constexpr (PAIR)
+              umma_f16_ss_pair(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              umma_f16_ss(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
           mma_issued = true;
-          umma_commit(&cv_empty[s]);
+          if constexpr (PAIR)
+            umma_commit_pair(&cv_empty[s], 0x3);
+          else
+            umma_commit(&cv_empty[s]);
           if (++s == S) {
             s = 0;
             ph ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if constexpr (PAIR)
+          umma_commit_pair(&tfull[acc], 0x3);
+        else
+          umma_commit(&tfull[acc]);
+      }
+    } else if (PAIR && !leader && lane < S) {
+      // relay of the other CTA: lane s passes each completed phase of this
+      // CTA's decoded stage s on to the leader's barrier of that stage, off
+      // the converters' path. The converters' shared-memory writes are
+      // complete (and fenced for the async proxy) once the local phase has
+      // completed; the relay observes that before it arrives, and the
+      // leader's MMAs, issued after the leader observes the arrive, read
+      // this CTA's shared memory directly. The arrive is relaxed: a release
+      // at cluster scope costs about a microsecond per K-step here (measured:
+      // 287 against 222 us for a 64 x 3072 x 2048 x 256-token GEMM).
+      const int my_tiles =
+          unit < args.num_tiles ? (args.num_tiles - 1 - unit) / n_units + 1 : 0;
+      const int steps = my_tiles * args.k_blocks;
+      const uint32_t remote = mapa_shared(smem_u32(&cv_full[lane]), 0);
+      for (int j = lane; j < steps; j += S) {
+        if (!mbar_wait(&cv_full[lane], (uint32_t)(j / S) & 1u, abort_flag, kErrTimeoutFull)) break;
+        mbar_arrive_cluster_relaxed(remote);
       }
     }
   } else if (warp < lb::kEpiWarp0) {
     // ---------------------------------------------------------- converters --
-    const int cg = (warp - lb::kConvWarp0) >> 2;   // group = decoded stage
+    const int cg = (warp - lb::kConvWarp0) >> 2;
     const int ti = ((warp - lb::kConvWarp0) & 3) * 32 + lane;  // 0..127
-    const int my_tiles = (int)blockIdx.x < args.num_tiles
-                             ? (args.num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1
-                             : 0;
+    const int my_tiles =
+        unit < args.num_tiles ? (args.num_tiles - 1 - unit) / n_units + 1 : 0;
     const int steps = my_tiles * args.k_blocks;
-    uint8_t* bt = dec + cg * lb::kDecBytes;   // weights: rows 0..255 x 128 bytes
-    uint8_t* at = bt + lb::kBBytes;            // tokens: rows 0..nt-1 x 128 bytes
     for (int j = cg; j < steps; j += lb::kConvGroups) {
       const int rs = j % R;
+      const int ds = j % S;
+      uint8_t* bt = dec + ds * DEC;        // weights: WT x 128 rows x 128 bytes
+      uint8_t* at = bt + lb::b_bytes(PAIR);  // tokens: rows 0..nt-1 x 128 bytes
       const bool r_ok =
           mbar_wait(&raw_full[rs], (uint32_t)(j / R) & 1u, abort_flag, kErrTimeoutFull);
       if (__any_sync(0xffffffffu, !r_ok)) break;
       // the K-step's words into registers, then the raw stage goes back to
       // the producer: its next copy is in flight while this group decodes
       const uint8_t* st = raw + rs * RAW;
-      uint4 lw[2][2];
-      uint2 hw[2][2];
-      uint32_t sw[2];
+      uint4 lw[WT][2];
+      uint2 hw[WT][2];
+      uint32_t sw[WT];
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint8_t* tile = st + which * F::kTileBytes;
+      for (int i = 0; i < WT; ++i) {
+        const uint8_t* tile = st + i * F::kTileBytes;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          lw[which][half] = *reinterpret_cast<const uint4*>(tile + half * 2048 + ti * 16);
-          hw[which][half] =
+          lw[i][half] = *reinterpret_cast<const uint4*>(tile + half * 2048 + ti * 16);
+          hw[i][half] =
               BITS == 6 ? *reinterpret_cast<const uint2*>(tile + 4096 + ti * 16 + half * 8)
                         : make_uint2(0u, 0u);
         }
-        sw[which] = *reinterpret_cast<const uint32_t*>(tile + F::kScaleOff + ti * 4);
+        sw[i] = *reinterpret_cast<const uint32_t*>(tile + F::kScaleOff + ti * 4);
       }
       constexpr int kXChunks = lb::kMaxNt * 8 / 128;  // 8-byte chunks of codes per thread
       uint2 xv[kXChunks];
-      const uint8_t* act = st + 2 * F::kTileBytes;
+      const uint8_t* act = st + WT * F::kTileBytes;
 #pragma unroll
       for (int m = 0; m < kXChunks; ++m) {
         const int u = ti + 128 * m;
@@ -551,17 +629,17 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&raw_empty[rs]);
-      const bool d_ok = mbar_wait(&cv_empty[cg], ((uint32_t)(j / lb::kConvGroups) & 1u) ^ 1u,
-                                  abort_flag, kErrTimeoutEmpty);
+      const bool d_ok =
+          mbar_wait(&cv_empty[ds], ((uint32_t)(j / S) & 1u) ^ 1u, abort_flag, kErrTimeoutEmpty);
       if (__any_sync(0xffffffffu, !d_ok)) break;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const int row = which * 128 + ti;
+      for (int i = 0; i < WT; ++i) {
+        const int row = i * 128 + ti;
         uint8_t* dst = bt + row * 128;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t o[16];
-          lb_decode_words<BITS>(lw[which][half], hw[which][half], sw[which], half, o);
+          lb_decode_words<BITS>(lw[i][half], hw[i][half], sw[i], half, o);
 #pragma unroll
           for (int c = 0; c < 4; ++c)
             *reinterpret_cast<uint4*>(dst + (((4 * half + c) ^ (row & 7)) << 4)) =
@@ -581,7 +659,7 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&cv_full[cg]);
+      if (lane == 0) mbar_arrive(&cv_full[ds]);
     }
   } else {
     // ------------------------------------------------------------ epilogue --
@@ -589,8 +667,9 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
     griddep_launch_dependents();
     const int quad = warp & 3;
     const uint32_t t_lane = (uint32_t)(quad * 32) << 16;
+    const int tb_rows = PAIR ? 2 * lb::kMaxNt : nt;
     int it = 0;
-    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
+    for (int tile = unit; tile < args.num_tiles; tile += n_units, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
       int g, wb, tb;
@@ -599,7 +678,7 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
       // every lane reads the same scales (one broadcast load per warp)
       const float* sw0 = args.s_w + (int64_t)g * args.N + (kSwiglu ? wb * 128 : wb * 256);
       const float* sw1 = kSwiglu ? sw0 + args.n_out : sw0 + 128;
-      const int t0 = tb * nt;
+      const int t0 = tb * tb_rows + row0;   // this CTA's first token
       const int row = quad * 32 + lane;
       const int t = t0 + row;
       const bool valid = row < nt && t < args.M;
@@ -692,31 +771,51 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if constexpr (PAIR)
+          mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+        else
+          mbar_arrive(&tempty[acc]);
+      }
     }
   }
 
   __syncthreads();
+  int never = 0;
   if (*abort_flag) {
     // after a timeout: let every issued copy and MMA land before the shared
     // memory and the TMEM columns are released
-    int never = 0;
     if (warp == 0 && lane == 0) {
       for (int s = 0; s < R; ++s)
         if (issued_mask & (1u << s))
           mbar_wait_limit(&raw_full[s], (issued_parity >> s) & 1u, &never, kErrTimeoutTeardown,
                           100000000ull);
     }
-    if (warp == 1 && lane == 0 && mma_issued) {
-      umma_commit(drain);
+    if (warp == 1 && lane == 0 && leader && mma_issued) {
+      if constexpr (PAIR)
+        umma_commit_pair(drain, 0x1);
+      else
+        umma_commit(drain);
       mbar_wait_limit(drain, 0, &never, kErrTimeoutTeardown, 100000000ull);
+    }
+    __syncthreads();
+  }
+  if constexpr (PAIR) {
+    // neither CTA releases the pair's TMEM or leaves while the other may still
+    // signal its barriers or read its shared memory (bounded)
+    if (threadIdx.x == 0) {
+      mbar_arrive_cluster(mapa_shared(smem_u32(fin), rank ^ 1u));
+      mbar_wait_limit(fin, 0, &never, kErrTimeoutTeardown, 1000000000ull);
     }
     __syncthreads();
   }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, lb::kTmemCols);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, lb::kTmemCols);
+    else
+      tmem_dealloc(tmem_base, lb::kTmemCols);
   }
 }
 
