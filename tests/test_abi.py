@@ -148,10 +148,12 @@ def test_lowbit_argument_checks_need_no_gpu(lib):
     assert g(al, al, al, al, 1, 64, 256, 256, 4, 1, 24, al, None) == INVALID  # tile tokens
     assert g(al, al, al, al, 1, 64, 256, 256, 4, 1, 144, al, None) == INVALID
     assert g(mis, al, al, al, 1, 64, 256, 256, 4, 1, 0, al, None) == MISALIGNED
+    assert g(al, al, al, mis, 1, 64, 256, 256, 4, 1, 0, al, None) == MISALIGNED  # row scales
     lin = lib.lowbit_convrot_linear
     assert lin(al, 64, 256, al, al, 256, 256, 4, al, al, 16, None) == \
         binding.CONVROT_ERR_WORKSPACE_TOO_SMALL
     assert lin(al, 64, 256, al, al, 384, 256, 4, al, al, 1 << 20, None) == INVALID
+    assert lin(al, 64, 256, al, mis, 256, 256, 4, al, al, 1 << 20, None) == MISALIGNED
     m = lib.moe_expert_choice_forward_lowbit
     args = [al] * 6
     assert m(*args, 8, 256, 192, 4, 2, 256, 64, 4, al, al, 1 << 30, None) == INVALID  # f % 128
