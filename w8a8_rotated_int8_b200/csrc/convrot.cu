@@ -69,9 +69,11 @@ void set_gemm_attr() {
 
 template <int BITS, int EPI>
 void set_lowbit_attr() {
-  cudaFuncSetAttribute(gemm_lowbit_tcgen05_kernel<BITS, EPI, false>,
+  cudaFuncSetAttribute(gemm_lowbit_tcgen05_kernel<BITS, EPI, false, false>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, lb::kSmemMax);
-  cudaFuncSetAttribute(gemm_lowbit_tcgen05_kernel<BITS, EPI, true>,
+  cudaFuncSetAttribute(gemm_lowbit_tcgen05_kernel<BITS, EPI, false, true>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, lb::kSmemMax);
+  cudaFuncSetAttribute(gemm_lowbit_tcgen05_kernel<BITS, EPI, true, false>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, lb::kSmemMax);
 }
 
@@ -134,7 +136,8 @@ int lowbit_pair_residency(int sms, int* pairs) {
   lc.attrs = &attr;
   lc.numAttrs = 1;
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, gemm_lowbit_tcgen05_kernel<6, kLbSwiglu, true>,
+  if (cudaOccupancyMaxActiveClusters(&clusters,
+                                     gemm_lowbit_tcgen05_kernel<6, kLbSwiglu, true, false>,
                                      &lc) != cudaSuccess)
     return CONVROT_ERR_CUDA;
   *pairs = clusters;
@@ -849,12 +852,17 @@ int launch_lowbit_gemm(const int8_t* x, const float* s_x, const uint8_t* wq, con
     return rc;
   if (pair) {
     const int grid = 2 * (int)std::min<int64_t>(tiles, pairs);
-    rc = launch_kernel(gemm_lowbit_tcgen05_kernel<BITS, EPI, true>, dim3(grid), dim3(lb::kThreads),
-                       lb::smem_bytes<BITS>(a.nt, true), st, pdl, 2, tx, a);
+    rc = launch_kernel(gemm_lowbit_tcgen05_kernel<BITS, EPI, true, false>, dim3(grid),
+                       dim3(lb::kThreads), lb::smem_bytes<BITS>(a.nt, true), st, pdl, 2, tx, a);
   } else {
+    // up to 64 tokens per tile: M = 64 instructions
     const int grid = (int)std::min<int64_t>(tiles, sms);
-    rc = launch_kernel(gemm_lowbit_tcgen05_kernel<BITS, EPI, false>, dim3(grid),
-                       dim3(lb::kThreads), lb::smem_bytes<BITS>(a.nt, false), st, pdl, 1, tx, a);
+    if (a.nt <= 64)
+      rc = launch_kernel(gemm_lowbit_tcgen05_kernel<BITS, EPI, false, true>, dim3(grid),
+                         dim3(lb::kThreads), lb::smem_bytes<BITS>(a.nt, false), st, pdl, 1, tx, a);
+    else
+      rc = launch_kernel(gemm_lowbit_tcgen05_kernel<BITS, EPI, false, false>, dim3(grid),
+                         dim3(lb::kThreads), lb::smem_bytes<BITS>(a.nt, false), st, pdl, 1, tx, a);
   }
   if (rc != CONVROT_OK) return rc;
   return launch_status();

@@ -380,7 +380,9 @@ __device__ __forceinline__ int64_t lb_row_block(const LowbitArgs& a, int g, int 
 //               j % S
 //   warps 14-17 epilogue: tcgen05.ld of the quadrant's token rows, 16
 //               columns at a time; each lane writes its row's outputs
-template <int BITS, int EPI, bool PAIR>
+// M64 (single CTA, at most 64 tokens per tile): M = 64 instructions, half
+// the tensor work and half the token operand read per instruction.
+template <int BITS, int EPI, bool PAIR, bool M64>
 __global__ void __launch_bounds__(lb::kThreads, 1)
     gemm_lowbit_tcgen05_kernel(const __grid_constant__ CUtensorMap tmX, const LowbitArgs args) {
   using F = LbFmt<BITS>;
@@ -522,7 +524,7 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
-      const uint32_t idesc = idesc_f16_f32(PAIR ? 256 : 128, 256);
+      const uint32_t idesc = idesc_f16_f32(PAIR ? 256 : M64 ? 64 : 128, 256);
       int s = 0;
       uint32_t ph = 0;
       int it = 0;
@@ -679,15 +681,19 @@ __global__ void __launch_bounds__(lb::kThreads, 1)
       const float* sw0 = args.s_w + (int64_t)g * args.N + (kSwiglu ? wb * 128 : wb * 256);
       const float* sw1 = kSwiglu ? sw0 + args.n_out : sw0 + 128;
       const int t0 = tb * tb_rows + row0;   // this CTA's first token
-      const int row = quad * 32 + lane;
+      // M = 64: accumulator row r sits in lane 16 of sub-partition r / 16's
+      // 32 lanes plus r % 16, so lanes 16..31 of each warp hold no row
+      constexpr int kRowsPerQuad = M64 ? 16 : 32;
+      const int row = quad * kRowsPerQuad + (lane & (kRowsPerQuad - 1));
       const int t = t0 + row;
-      const bool valid = row < nt && t < args.M;
+      const bool valid = lane < kRowsPerQuad && row < nt && t < args.M;
       const float sx = (EPI != kLbF32 && valid) ? __ldg(args.s_x + (int64_t)g * args.M + t) : 0.0f;
       const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, kErrTimeoutTmemFull);
       if (__any_sync(0xffffffffu, !ok)) break;
       tc_fence_after();
       const uint32_t d = tmem_base + t_lane + (uint32_t)(acc * 256);
-      const bool warp_rows = quad * 32 < nt && t0 + quad * 32 < args.M;  // warp-uniform
+      const bool warp_rows =
+          quad * kRowsPerQuad < nt && t0 + quad * kRowsPerQuad < args.M;  // warp-uniform
       if (warp_rows) {
         const int64_t orow = (int64_t)g * args.M + t;
         if constexpr (kSwiglu) {
