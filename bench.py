@@ -52,15 +52,21 @@ PROFILES = os.path.join(ROOT, "profiles")
 
 
 def source_sha16():
-    """Hash of the CUDA sources and the ABI header: a traffic figure captured
-    by ncu on other sources no longer describes the kernel."""
+    """Hash of the CUDA sources and the ABI header without their comments and
+    blank lines: a traffic figure captured by ncu on other code no longer
+    describes the kernel (a comment does not change it)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "w8a8_rotated_int8_b200", "csrc")
     files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
     for path in files + [os.path.join(ROOT, "include", "convrot.h")]:
-        with open(path, "rb") as fh:
-            h.update(fh.read())
+        with open(path) as fh:
+            text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+        for line in text.splitlines():
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -30,13 +30,14 @@
 // an activation code (|x| <= 127) is an exact fp16, and so is q * sigma / 16
 // (at most 9 significant bits, between 2^-13 and 28 * 31). Converter warps
 // decode the weights into shared memory as the N = 256 operand (two 128-row
-// blocks, the 128-byte swizzle) and widen the activation codes into the
-// M = 128 operand (the tile's tokens), so every MMA is M=128 N=256 K=16
-// whatever the token count: a thread issuing tcgen05.mma waits about 120
-// cycles per instruction (measured on B200) whether N is 16 or 128, so short
-// instructions cannot keep the tensor core busy. D[token, weight row]
-// accumulates sum_k x * q * sigma / 16; the epilogue multiplies by 16 (exact)
-// and dequantises y = acc * (s_x * s_r).
+// blocks, the 128-byte swizzle) and widen the activation codes into the M
+// operand (the tile's tokens), so every MMA has N = 256 whatever the token
+// count: a thread issuing tcgen05.mma waits about 120 cycles per instruction
+// (measured on B200) whether N is 16 or 128, so short instructions cannot
+// keep the tensor core busy. M is 64 for tiles of up to 64 tokens, 128 up to
+// 128, and 256 over a CTA pair for more (each CTA then decodes one of the two
+// weight blocks). D[token, weight row] accumulates sum_k x * q * sigma / 16;
+// the epilogue multiplies by 16 (exact) and dequantises y = acc * (s_x * s_r).
 #pragma once
 
 #include "common.cuh"
