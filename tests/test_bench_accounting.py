@@ -73,3 +73,22 @@ def test_traffic_record_needs_the_current_sources(tmp_path, monkeypatch):
     got, note = bench.profile_traffic("gemm_y", "moe_T8192")
     assert got is None and "changed" in note
     assert bench.profile_traffic("gemm_x", "moe_T2048")[0] is None
+
+
+def test_source_hash_ignores_comments_not_code(tmp_path, monkeypatch):
+    """The hash that keys the traffic records changes with the code of the
+    CUDA sources or the header, not with their comments or blank lines."""
+    csrc = tmp_path / "w8a8_rotated_int8_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "include").mkdir()
+    kern = csrc / "k.cuh"
+    head = tmp_path / "include" / "convrot.h"
+    kern.write_text("// a kernel\n__global__ void k(int* p) { p[0] = 1; }\n")
+    head.write_text("/* the ABI */\nint f(void);\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    base = bench.source_sha16()
+    kern.write_text("// a kernel, now documented\n\n__global__ void k(int* p) { p[0] = 1; }  // one\n")
+    head.write_text("/* the ABI,\n   in two lines */\nint f(void);  /* f */\n")
+    assert bench.source_sha16() == base
+    kern.write_text("// a kernel\n__global__ void k(int* p) { p[0] = 2; }\n")
+    assert bench.source_sha16() != base
