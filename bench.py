@@ -163,8 +163,10 @@ def fused_h(cfg):
 
 class ClockSampler:
     """SM clock and clock-event reasons sampled (read-only, NVML) by a thread
-    as fast as NVML answers (two queries per sample, ~0.1 ms apart) while the
-    timed region runs."""
+    as fast as NVML answers (two queries per sample). The thread starts before
+    the timed region, so it is already sampling when the region begins; only
+    the samples taken between begin() and end() are reported. `nvml` replaces
+    the pynvml module (a fake, for tests without a GPU)."""
 
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
@@ -172,37 +174,47 @@ class ClockSampler:
                ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
                ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, torch_device):
+    def __init__(self, torch_device, nvml=None):
         import threading
         self.dev = torch_device
-        self.samples = []
+        self.samples = []          # (perf_counter seconds, SM MHz, reason bits)
         self.stop_evt = threading.Event()
         self.thread = None
         self.nvml = None
+        self.fake = nvml
         self.handle = None
         self.max_mhz = None
+        self.window = [None, None]
 
     def _open(self):
-        import pynvml
-        pynvml.nvmlInit()
-        props = torch.cuda.get_device_properties(self.dev)
-        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
-        self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
-        self.nvml = pynvml
+        if self.fake is not None:
+            nv = self.fake
+            nv.nvmlInit()
+            self.handle = nv.nvmlDeviceGetHandleByIndex(0)
+        else:
+            import pynvml as nv
+            nv.nvmlInit()
+            props = torch.cuda.get_device_properties(self.dev)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self.handle = nv.nvmlDeviceGetHandleByPciBusId(bus)
+        self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+        self.nvml = nv
 
     def _loop(self):
         nv = self.nvml
         while not self.stop_evt.is_set():
             try:
+                t = time.perf_counter()
                 mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
                 rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
-                self.samples.append((mhz, rs))
+                self.samples.append((t, mhz, rs))
             except Exception:  # noqa: BLE001 - sampling is best effort
                 pass
             self.stop_evt.wait(0.0001)
 
     def start(self):
+        """Opens NVML and starts sampling; returns once the first sample is in
+        (at most 1 s), so the thread is warm when the timed region begins."""
         import threading
         try:
             self._open()
@@ -211,6 +223,15 @@ class ClockSampler:
             return
         self.thread = threading.Thread(target=self._loop, daemon=True)
         self.thread.start()
+        t0 = time.perf_counter()
+        while not self.samples and time.perf_counter() - t0 < 1.0:
+            time.sleep(0.0005)
+
+    def begin(self):
+        self.window[0] = time.perf_counter()
+
+    def end(self):
+        self.window[1] = time.perf_counter()
 
     def stop(self):
         if self.nvml is None:
@@ -218,12 +239,16 @@ class ClockSampler:
         self.stop_evt.set()
         self.thread.join(timeout=5)
         nv = self.nvml
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"]}
-        reasons = sorted({name for _, rs in self.samples for name, const in self.REASONS
+        lo, hi = self.window
+        inside = [(m, rs) for t, m, rs in self.samples
+                  if (lo is None or t >= lo) and (hi is None or t <= hi)]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz,
+                    "reasons": ["no samples in the timed region"], "samples": 0}
+        reasons = sorted({name for _, rs in inside for name, const in self.REASONS
                           if rs & getattr(nv, const)})
-        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
-                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(m for m, _ in inside),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside)}
 
 
 class L2Flush:
@@ -655,9 +680,10 @@ def run_ours(args, cfg, world, rank, local, extras=True):
     torch.cuda.synchronize()
 
     clocks = ClockSampler(dev)
+    clocks.start()  # sampling from here on; only the timed window below is reported
     barrier(world)
     torch.cuda.synchronize()
-    clocks.start()
+    clocks.begin()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     wall0 = time.perf_counter()
@@ -669,6 +695,7 @@ def run_ours(args, cfg, world, rank, local, extras=True):
         ends[i].record(stream)
     nvtx_pop()
     torch.cuda.synchronize()
+    clocks.end()
     barrier(world)
     wall = time.perf_counter() - wall0
     clk = clocks.stop()

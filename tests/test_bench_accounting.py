@@ -92,3 +92,69 @@ def test_source_hash_ignores_comments_not_code(tmp_path, monkeypatch):
     assert bench.source_sha16() == base
     kern.write_text("// a kernel\n__global__ void k(int* p) { p[0] = 2; }\n")
     assert bench.source_sha16() != base
+
+
+class _FakeNvml:
+    """Stands in for pynvml: the SM clock and reasons change with a phase the
+    test sets (before, during and after the timed region)."""
+
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwPowerBrakeSlowdown = 0x80
+
+    def __init__(self):
+        self.phase = "before"
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return i
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        return 1965 if self.phase == "during" else 900
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.nvmlClocksEventReasonSwPowerCap if self.phase == "during" else \
+            self.nvmlClocksEventReasonHwSlowdown
+
+
+def test_clock_sampler_reports_only_the_timed_window():
+    """Samples taken before begin() or after end() (here: a slow clock and a
+    hardware slowdown) stay out of the record; the window's samples give the
+    median clock and the reasons active in it."""
+    import time
+    nv = _FakeNvml()
+    clk = bench.ClockSampler(None, nvml=nv)
+    clk.start()
+    assert clk.samples, "the sampler is warm when start() returns"
+    time.sleep(0.02)
+    nv.phase = "during"
+    time.sleep(0.002)
+    clk.begin()
+    time.sleep(0.03)
+    clk.end()
+    time.sleep(0.002)
+    nv.phase = "after"
+    time.sleep(0.02)
+    rec = clk.stop()
+    assert rec["sm_mhz"] == 1965 and rec["sm_max_mhz"] == 1965
+    assert rec["reasons"] == ["sw_power_cap"]
+    assert rec["samples"] >= 10
+
+
+def test_clock_sampler_without_nvml():
+    class Broken:
+        def nvmlInit(self):
+            raise RuntimeError("no driver")
+    clk = bench.ClockSampler(None, nvml=Broken())
+    clk.start()
+    clk.begin()
+    clk.end()
+    assert clk.stop()["reasons"] == ["nvml unavailable"]
